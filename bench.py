@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the decode-step hybrid sparse + linear attention on B200.
+
+One step = for every layer of the workload: one decode (block scores, top-k,
+gather, exact softmax part, Taylor linear part by subtraction, merge) and one
+append (cache write, window eviction, linear-state and block-stat update).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
+on a bounded sample of the same workload instead.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of the
+workload's units (independent batches; no collective on the data path) and the
+step time is the max over ranks ("scaling": "weak").
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 512 << 20
+METRIC = "hybrid decode-attn steps/s and achieved HBM GB/s (% of peak) at 32K-256K ctx"
+DEFAULT_WORKLOAD = "llama8b_32k_layer"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- bytes model
+
+def algorithmic_bytes(w, T):
+    """Bytes one decode must move per (layer, b, kv head) at length T, and the
+    append's bytes per unit (the method's minimum: selected/exact tokens, block
+    statistics, linear state, q and out; no unselected token)."""
+    d, G = w.head_dim, w.group
+    per = w.bytes_per_unit(T)
+    decode = sum(per.values())
+    append = (2 * d * 2) + (2 * d * 2) + 2 * d * d * 4 + 2 * 2 * d * 4 + 2 * 2 * d * 4 + 2 * 4
+    attend = per["exact_kv"] + per["q_out"]
+    return decode, append, attend
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- native arm
+
+class Bench:
+    def __init__(self, w, steps, warmup, device):
+        import torch
+        import syngen.device as SD
+        from syngen import host as SH
+        from hybrid_sparse_linear_decode_b200 import HybridAttentionLayer, make_config
+        self.w, self.device = w, device
+        self.n_steps = warmup + steps + 1
+        n_app = self.n_steps
+        cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window,
+                          w.top_k, w.T0 + n_app)
+        ws_bytes = HybridAttentionLayer.workspace_bytes(cfg)
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device)   # shared: one stream
+        self.layers, self.app_k, self.app_v, self.q = [], [], [], []
+        n_q = min(self.n_steps, 8)
+        for l in range(w.layers):
+            L = HybridAttentionLayer(cfg, device, workspace=self.workspace)
+            tb = SD.DeviceTables(w, l, L.device)
+            SD.fill_kv(w, tb, L.k_cache, L.v_cache, 0, w.T0)
+            shp = (w.batch, w.n_kv_heads, n_app, w.head_dim)
+            ak = torch.empty(shp, dtype=torch.bfloat16, device=device)
+            av = torch.empty(shp, dtype=torch.bfloat16, device=device)
+            SD.fill_kv(w, tb, ak, av, w.T0, w.T0 + n_app, t_out0=w.T0)
+            # per-step appended tokens, contiguous [step][B][Hkv][d]
+            self.app_k.append(ak.permute(2, 0, 1, 3).contiguous())
+            self.app_v.append(av.permute(2, 0, 1, 3).contiguous())
+            del ak, av
+            qs = []
+            for s in range(n_q):
+                qb = SH.q_bits(w, l, s)
+                qs.append(torch.from_numpy(qb.view("int16")).to(device).view(torch.bfloat16))
+            self.q.append(qs)
+            L.init(w.T0)
+            self.layers.append(L)
+        self.out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=device)
+        torch.cuda.synchronize()
+        self.step_idx = 0
+
+    def step(self):
+        s = self.step_idx
+        for l, L in enumerate(self.layers):
+            q = self.q[l][s % len(self.q[l])]
+            L.decode(q, out=self.out)
+            L.append(self.app_k[l][s], self.app_v[l][s])
+        self.step_idx += 1
+
+    def launches_per_step(self):
+        return 3 * len(self.layers)   # select, attend, append per layer
+
+
+def run_native(args, rank, world):
+    import torch
+    from syngen import configs as C
+    torch.cuda.set_device(rank % torch.cuda.device_count())
+    device = torch.device("cuda", torch.cuda.current_device())
+    w = C.get_workload(args.workload)
+    K, Wm = args.steps, args.warmup
+    b = Bench(w, K, Wm, device)
+    T_mid = w.T0 + Wm + K // 2
+    dec_b, app_b, att_b = algorithmic_bytes(w, T_mid)
+    units = w.layers * w.units_per_layer
+    step_bytes = units * (dec_b + app_b)
+    flush = step_bytes < 4 * 126e6      # the step's data would otherwise stay in L2
+    scratch = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if flush else None
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(Wm):
+        b.step()
+        if flush:
+            scratch.zero_()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, device time with CUDA events, max over ranks
+    stream = torch.cuda.current_stream()
+    clk = ClockSampler(torch.cuda.current_device())
+    clk.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    if flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            evs[i][0].record(stream)
+            b.step()
+            evs[i][1].record(stream)
+            scratch.zero_()
+        torch.cuda.synchronize()
+        total_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            b.step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total_ms = e0.elapsed_time(e1)
+    barrier()
+    clocks = clk.stop()
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    steps_s = 1e3 / ms_per_step
+
+    # ---- attention-kernel timing (events around the attention launch of every layer)
+    ka, kb_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kern_ms, n_kern = 0.0, 0
+    Kk = min(K, 20)
+    pool = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in b.layers]
+            for _ in range(Kk)]
+    for i in range(Kk):
+        for l, L in enumerate(b.layers):
+            e0, e1 = pool[i][l]
+            e0.record(stream)
+            e1.record(stream)
+            L.set_timing_events(e0, e1)
+        b.step()
+        for L in b.layers:
+            L.set_timing_events(None, None)
+        if flush:
+            scratch.zero_()
+    torch.cuda.synchronize()
+    for i in range(Kk):
+        for e0, e1 in pool[i]:
+            kern_ms += e0.elapsed_time(e1)
+            n_kern += 1
+    attend_ms = kern_ms / n_kern
+    attend_bytes = w.units_per_layer * att_b
+    hbm_peak, peak_kind = peaks()
+    achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
+    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---- e2e through the host-buffer entry point (pinned host q / k / v / out)
+    e2e = None
+    if not args.no_e2e:
+        Ke = min(K, 20)
+        qh = [[t.cpu().pin_memory() for t in qs] for qs in b.q]
+        kh = [t.cpu().pin_memory() for t in b.app_k]
+        vh = [t.cpu().pin_memory() for t in b.app_v]
+        oh = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32).pin_memory()
+        s0 = b.step_idx
+        assert s0 + Ke <= b.n_steps
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+        for i in range(Ke):
+            s = b.step_idx
+            evs[i][0].record(stream)
+            for l, L in enumerate(b.layers):
+                L.step_host(qh[l][s % len(qh[l])], kh[l][s], vh[l][s], oh)
+            evs[i][1].record(stream)
+            b.step_idx += 1
+            if flush:
+                scratch.zero_()
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(c) for a, c in evs) / Ke
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = w.layers * (w.batch * w.n_q_heads * w.head_dim * 2 + 2 * w.batch * w.n_kv_heads * w.head_dim * 2)
+        d2h = w.layers * w.batch * w.n_q_heads * w.head_dim * 4
+        e2e = {"value": round(world * 1e3 / e2e_ms, 3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)}
+
+    status = 0
+    for L in b.layers:
+        status |= L.status()
+    result = {
+        "metric": METRIC,
+        "value": round(world * steps_s, 3),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded counter-based generator; no dataset, no weights)",
+        "config": {
+            "workload": w.name, "layers": w.layers, "batch": w.batch, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context_T0": w.T0, "block": w.block_size,
+            "sinks": w.n_sink, "window": w.window, "top_k": w.top_k,
+            "l2": "flushed between timed steps (512 MB write)" if flush else "step data >> L2 (no flush)",
+            "parallelism": f"replicas x{world} (independent units per GPU)",
+        },
+        "attention_tokens_per_s": round(world * steps_s * w.batch, 3),
+        "context_tokens_per_s": round(world * steps_s * w.batch * w.layers * T_mid, 1),
+        "achieved_gbs_step": round(step_gbs, 1),
+        "pct_of_hbm_peak_step": round(100 * step_gbs / hbm_peak, 2),
+        "bytes_per_step": step_bytes,
+        "roofline": {"bound": "hbm", "kernel": "attend_kernel (exact part + subtraction + merge)",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
+                     "traffic": None, "bytes_per_launch": attend_bytes, "avg_launch_us": round(attend_ms * 1e3, 3)},
+        "e2e": e2e,
+        "gpu_launches": b.launches_per_step() * K,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    return result
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+
+def oracle_sample(w, seconds: float, steps_per_unit: int = 3):
+    """Time the fp64 oracle's decode + append on whole units of the workload
+    (bounded sample); returns seconds per full step and a description."""
+    import numpy as np
+    import oracle as O
+    from syngen import host as SH
+    scale = 1 / math.sqrt(w.head_dim)
+    tb = SH.LayerTables(w, 0)
+    units = [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    spent, n_unit_steps, used = 0.0, 0, 0
+    for (b, h) in units:
+        K, V = SH.kv_f64(w, tb, b, h, 0, w.T0 + steps_per_unit)
+        u = O.OracleUnit(K[:w.T0], V[:w.T0], w.n_sink, w.window, w.block_size, w.top_k, scale,
+                         capacity=w.T0 + steps_per_unit)
+        q = SH.bf16_bits_to_f64(SH.q_bits(w, 0, 0))[b, h * w.group:(h + 1) * w.group]
+        for s in range(steps_per_unit):
+            t0 = time.perf_counter()
+            u.decode(q)
+            u.append(K[w.T0 + s], V[w.T0 + s])
+            spent += time.perf_counter() - t0
+            n_unit_steps += 1
+        used += 1
+        if spent >= seconds:
+            break
+    per_unit_step = spent / n_unit_steps
+    units_per_step = w.layers * w.units_per_layer
+    return per_unit_step * units_per_step, (f"{n_unit_steps} unit-steps (decode+append of one (layer,b,kv-head)) "
+                                            f"over {used} units, scaled x{units_per_step} units per step")
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    from syngen import configs as C
+    w = C.get_workload(args.workload)
+    per_step_s, _ = oracle_sample(w, 0.5, steps_per_unit=1)   # warm numpy / BLAS
+    t_total, samples = 0.0, []
+    for _ in range(args.warmup):
+        oracle_sample(w, 0.1, steps_per_unit=1)
+    for _ in range(args.steps):
+        s, desc = oracle_sample(w, args.cpu_sample_seconds / max(1, args.steps), steps_per_unit=1)
+        samples.append(s)
+    ms = 1e3 * statistics.mean(samples)
+    v = 1e3 / ms
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name},
+        "cpu_baseline": {"value": round(v, 6), "unit": "steps/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(v, 6), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_native(args, rank, world)
+    if rank == 0 and not args.no_cpu_baseline:
+        from syngen import configs as C
+        w = C.get_workload(args.workload)
+        s, desc = oracle_sample(w, args.cpu_sample_seconds)
+        res["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": "steps/s", "cores": cpu_cores(),
+                               "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,468 @@
+// C ABI of the hybrid sparse + linear decode attention: argument checks, the
+// workspace layout, TMA descriptors and kernel launches.  Host code only.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "../../include/hyb_attn.h"
+#include "hyb_internal.h"
+
+using namespace hyb;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct WsLayout {
+  size_t status, tk_sel, tk_att, scores, sel, lin, partials, H64, z64, stage_q, stage_k, stage_v, stage_out, total;
+};
+
+struct Checked {
+  int D, G, units;
+  int64_t max_blocks;
+};
+
+int check_config(const hyb_attn_config* c, Checked* out) {
+  if (c == nullptr) return HYB_EINVAL;
+  if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1) return HYB_EINVAL;
+  if (c->n_q_heads % c->n_kv_heads != 0) return HYB_EINVAL;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4) return HYB_EINVAL;
+  if (c->head_dim != 64 && c->head_dim != 128) return HYB_EINVAL;
+  if (c->block_size < 1 || c->n_sink < 0 || c->window < 0 || c->top_k < 0) return HYB_EINVAL;
+  if (c->capacity < 1) return HYB_EINVAL;
+  if (!(c->scale >= 0.f) || !std::isfinite(c->scale)) return HYB_EINVAL;
+  const int64_t units = (int64_t)c->batch * c->n_kv_heads;
+  if (units > (1 << 20)) return HYB_EINVAL;
+  if (units * c->capacity >= ((int64_t)1 << 31)) return HYB_EINVAL;  // TMA row coordinate is int32
+  if ((int64_t)c->n_sink + c->window + c->top_k * (int64_t)c->block_size >= ((int64_t)1 << 30)) return HYB_EINVAL;
+  const int64_t ev_cap = c->capacity - c->n_sink - c->window;
+  const int64_t mb = ev_cap > 0 ? ceil_div(ev_cap, c->block_size) : 0;
+  if (mb >= ((int64_t)1 << 30)) return HYB_EINVAL;
+  if (out) {
+    out->D = c->head_dim;
+    out->G = G;
+    out->units = (int)units;
+    out->max_blocks = mb;
+  }
+  return HYB_OK;
+}
+
+WsLayout ws_layout(const hyb_attn_config& c, const Checked& k) {
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  const size_t U = (size_t)k.units, D = (size_t)k.D, G = (size_t)k.G;
+  w.status = take(sizeof(uint32_t));
+  w.tk_sel = take(U * sizeof(uint32_t));
+  w.tk_att = take(U * sizeof(uint32_t));
+  w.scores = take(U * (size_t)(k.max_blocks > 0 ? k.max_blocks : 1) * sizeof(float));
+  w.sel = take(U * (size_t)(c.top_k > 0 ? c.top_k : 1) * sizeof(int32_t));
+  w.lin = take(U * G * (D + 1) * sizeof(float));
+  w.partials = take(((size_t)kMaxAttendCtas + U) * (size_t)partial_floats((int)D) * sizeof(float));
+  w.H64 = take(U * D * D * sizeof(double));
+  w.z64 = take(U * 2 * D * sizeof(double));
+  w.stage_q = take(U * G * D * 2);
+  w.stage_k = take(U * D * 2);
+  w.stage_v = take(U * D * 2);
+  w.stage_out = take(U * G * D * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+Geometry geometry(const hyb_attn_config& c, int64_t T) {
+  Geometry g{};
+  const int64_t S = c.n_sink, W = c.window, Bk = c.block_size;
+  g.T = T;
+  g.sink_len = T < S ? T : S;
+  g.win_start = T > S ? (T - W > S ? T - W : S) : T;
+  g.ev_end = T > S + W ? T - W : S;
+  g.nb = g.ev_end > S ? ceil_div(g.ev_end - S, Bk) : 0;
+  g.k_eff = c.top_k < g.nb ? c.top_k : g.nb;
+  g.n_sink_chunks = (int32_t)ceil_div(g.sink_len, kTile);
+  g.n_win_chunks = (int32_t)ceil_div(T - g.win_start, kTile);
+  g.chunks_per_block = (int32_t)ceil_div(Bk, kTile);
+  g.n_sel_chunks = (int32_t)(g.k_eff * g.chunks_per_block);
+  g.chunks_per_unit = g.n_sink_chunks + g.n_win_chunks + g.n_sel_chunks;
+  return g;
+}
+
+int attend_grid(int64_t total_chunks, int n_sm) {
+  int64_t g = total_chunks;
+  if (g > n_sm) g = n_sm;
+  if (g > kMaxAttendCtas) g = kMaxAttendCtas;
+  return (int)(g < 1 ? 1 : g);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// KV cache viewed as [rows = B*Hkv*capacity][D/64][64] bf16; a box is 16 rows x
+// D columns, swizzled 128 B.
+bool make_kv_map(CUtensorMap* m, void* base, int64_t rows, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)(D / 64), (cuuint64_t)rows};
+  cuuint64_t strides[2] = {128, (cuuint64_t)D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)(D / 64), (cuuint32_t)kBoxRows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool is_device_ptr(const void* p, int device) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice && a.device == device;
+}
+
+}  // namespace
+
+struct hyb_attn_ctx {
+  hyb_attn_config cfg;
+  hyb_attn_buffers buf;
+  Checked ck;
+  WsLayout ws;
+  int64_t T;
+  int device, n_sm;
+  float scale;
+  CUtensorMap tmK, tmV;
+  cudaEvent_t ev_begin, ev_end;
+  template <class P>
+  P* w(size_t off) const {
+    return reinterpret_cast<P*>(static_cast<uint8_t*>(buf.workspace) + off);
+  }
+};
+
+namespace {
+
+int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_given, int32_t* sel_out,
+                float* scores_out, cudaStream_t stream) {
+  if (x == nullptr || q == nullptr || out == nullptr) return HYB_EINVAL;
+  if (!aligned16(q) || !aligned16(out)) return HYB_EINVAL;
+  if (sel_given != nullptr && !aligned16(sel_given)) return HYB_EINVAL;
+  if (sel_out != nullptr && (reinterpret_cast<uintptr_t>(sel_out) & 3u)) return HYB_EINVAL;
+  if (scores_out != nullptr && (reinterpret_cast<uintptr_t>(scores_out) & 15u)) return HYB_EINVAL;
+  if (x->T == 0) return HYB_ESTATE;
+  const hyb_attn_config& c = x->cfg;
+  const Checked& k = x->ck;
+  const Geometry g = geometry(c, x->T);
+
+  SelectParams sp{};
+  sp.q = static_cast<const __nv_bfloat16*>(q);
+  sp.mu = x->buf.mu;
+  sp.var = x->buf.var;
+  sp.H = x->buf.H;
+  sp.zk = x->buf.zk;
+  sp.zv = x->buf.zv;
+  sp.n = x->buf.n;
+  sp.scores = scores_out ? scores_out : x->w<float>(x->ws.scores);
+  sp.sel = x->w<int32_t>(x->ws.sel);
+  sp.sel_out = sel_given ? nullptr : sel_out;
+  sp.lin = x->w<float>(x->ws.lin);
+  sp.tickets = x->w<uint32_t>(x->ws.tk_sel);
+  sp.status = x->w<uint32_t>(x->ws.status);
+  sp.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
+  sp.units = k.units;
+  sp.G = k.G;
+  sp.nb = (int32_t)g.nb;
+  sp.top_k = c.top_k;
+  sp.k_eff = (int32_t)g.k_eff;
+  sp.do_select = sel_given ? 0 : 1;
+  const bool need_scores = (sel_given == nullptr) ? (g.nb > 0) : (scores_out != nullptr && g.nb > 0);
+  sp.score_ctas = need_scores ? (int32_t)ceil_div(g.nb, kScoreBlocksPerCta) : 0;
+  sp.lin_ctas = k.D / 32;
+  sp.scale = x->scale;
+  cudaError_t e = launch_select(sp, k.D, sp.score_ctas + sp.lin_ctas, stream);
+  if (e != cudaSuccess) return HYB_ECUDA;
+
+  AttendParams ap{};
+  ap.q = sp.q;
+  ap.sel = sel_given ? sel_given : sp.sel;
+  ap.lin = sp.lin;
+  ap.partials = x->w<float>(x->ws.partials);
+  ap.tickets = x->w<uint32_t>(x->ws.tk_att);
+  ap.status = sp.status;
+  ap.out = out;
+  ap.cap = c.capacity;
+  ap.total_chunks = (int64_t)k.units * g.chunks_per_unit;
+  ap.T = (int32_t)g.T;
+  ap.S = c.n_sink;
+  ap.Bk = c.block_size;
+  ap.top_k = c.top_k;
+  ap.nb = (int32_t)g.nb;
+  ap.k_eff = (int32_t)g.k_eff;
+  ap.sink_len = (int32_t)g.sink_len;
+  ap.win_start = (int32_t)g.win_start;
+  ap.ev_end = (int32_t)g.ev_end;
+  ap.n_sink_chunks = g.n_sink_chunks;
+  ap.n_win_chunks = g.n_win_chunks;
+  ap.chunks_per_block = g.chunks_per_block;
+  ap.chunks_per_unit = g.chunks_per_unit;
+  ap.units = k.units;
+  ap.G = k.G;
+  ap.merge_only = g.chunks_per_unit == 0 ? 1 : 0;
+  ap.grid = ap.merge_only ? k.units : attend_grid(ap.total_chunks, x->n_sm);
+  ap.scale = x->scale;
+  const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
+  if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
+  e = launch_attend(&x->tmK, &x->tmV, ap, k.D, /*pdl=*/!timed, stream);
+  if (e != cudaSuccess) return HYB_ECUDA;
+  if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
+  return HYB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hyb_attn_query_sizes(const hyb_attn_config* cfg, hyb_attn_sizes* out) {
+  Checked k;
+  const int rc = check_config(cfg, &k);
+  if (rc != HYB_OK || out == nullptr) return rc != HYB_OK ? rc : HYB_EINVAL;
+  const int64_t U = k.units, D = k.D;
+  out->kv_cache_elems = U * cfg->capacity * D;
+  out->H_elems = U * D * D;
+  out->z_elems = U * D;
+  out->n_elems = U;
+  out->max_blocks = k.max_blocks;
+  out->stats_elems = U * k.max_blocks * D;
+  out->workspace_bytes = (int64_t)ws_layout(*cfg, k).total;
+  return HYB_OK;
+}
+
+size_t hyb_attn_workspace_size(const hyb_attn_config* cfg) {
+  Checked k;
+  if (check_config(cfg, &k) != HYB_OK) return 0;
+  return ws_layout(*cfg, k).total;
+}
+
+int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_plan_info* out) {
+  Checked k;
+  const int rc = check_config(cfg, &k);
+  if (rc != HYB_OK) return rc;
+  if (out == nullptr || T < 0 || T > cfg->capacity || n_sm < 1) return HYB_EINVAL;
+  const Geometry g = geometry(*cfg, T);
+  out->T = T;
+  out->n_blocks = g.nb;
+  out->k_eff = g.k_eff;
+  out->exact_tokens = g.sink_len + (T - g.win_start) + g.k_eff * cfg->block_size;
+  out->chunks_per_unit = g.chunks_per_unit;
+  const int64_t total = (int64_t)k.units * g.chunks_per_unit;
+  out->attend_ctas = total == 0 ? k.units : attend_grid(total, n_sm);
+  out->partial_slots = total == 0 ? 0 : out->attend_ctas + k.units - 1;
+  out->score_ctas_per_unit = g.nb > 0 ? (int32_t)ceil_div(g.nb, kScoreBlocksPerCta) : 0;
+  out->linear_ctas_per_unit = k.D / 32;
+  return HYB_OK;
+}
+
+int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T0,
+                  cudaStream_t stream) {
+  if (out == nullptr) return HYB_EINVAL;
+  *out = nullptr;
+  Checked k;
+  if (check_config(cfg, &k) != HYB_OK || buf == nullptr) return HYB_EINVAL;
+  if (T0 < 0 || T0 > cfg->capacity) return HYB_EINVAL;
+  const void* ptrs[] = {buf->k_cache, buf->v_cache, buf->H, buf->zk, buf->zv, buf->n, buf->workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return HYB_EINVAL;
+  if (k.max_blocks > 0 && (buf->mu == nullptr || buf->var == nullptr || !aligned16(buf->mu) || !aligned16(buf->var)))
+    return HYB_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(buf->workspace) & (kAlign - 1)) != 0) return HYB_EINVAL;
+  const WsLayout ws = ws_layout(*cfg, k);
+  if (buf->workspace_bytes < ws.total) return HYB_EINVAL;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return HYB_ECUDA;
+  if (!is_device_ptr(buf->k_cache, device) || !is_device_ptr(buf->v_cache, device) ||
+      !is_device_ptr(buf->workspace, device) || !is_device_ptr(buf->H, device))
+    return HYB_EINVAL;
+  int n_sm = 0;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return HYB_ECUDA;
+
+  hyb_attn_ctx* x = new (std::nothrow) hyb_attn_ctx();
+  if (x == nullptr) return HYB_ENOMEM;
+  x->cfg = *cfg;
+  x->buf = *buf;
+  x->ck = k;
+  x->ws = ws;
+  x->T = T0;
+  x->device = device;
+  x->n_sm = n_sm;
+  x->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)k.D);
+  x->ev_begin = x->ev_end = nullptr;
+  const int64_t rows = (int64_t)k.units * cfg->capacity;
+  if (!make_kv_map(&x->tmK, buf->k_cache, rows, k.D) || !make_kv_map(&x->tmV, buf->v_cache, rows, k.D)) {
+    delete x;
+    return HYB_ECUDA;
+  }
+  if (prepare_attend(k.D) != cudaSuccess) {
+    delete x;
+    return HYB_ECUDA;
+  }
+
+  const Geometry g = geometry(*cfg, T0);
+  InitParams ip{};
+  ip.k_cache = static_cast<const __nv_bfloat16*>(buf->k_cache);
+  ip.v_cache = static_cast<const __nv_bfloat16*>(buf->v_cache);
+  ip.H = buf->H;
+  ip.zk = buf->zk;
+  ip.zv = buf->zv;
+  ip.n = buf->n;
+  ip.mu = buf->mu;
+  ip.var = buf->var;
+  ip.H64 = x->w<double>(ws.H64);
+  ip.z64 = x->w<double>(ws.z64);
+  ip.tickets_sel = x->w<uint32_t>(ws.tk_sel);
+  ip.tickets_att = x->w<uint32_t>(ws.tk_att);
+  ip.status = x->w<uint32_t>(ws.status);
+  ip.cap = cfg->capacity;
+  ip.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
+  ip.ev_begin = cfg->n_sink;
+  ip.ev_end = g.ev_end;
+  ip.units = k.units;
+  ip.S = cfg->n_sink;
+  ip.Bk = cfg->block_size;
+  ip.nb = (int32_t)g.nb;
+  ip.tokens_per_cta = 2048;
+  if (cudaMemsetAsync(ip.H64, 0, (size_t)k.units * k.D * k.D * sizeof(double), stream) != cudaSuccess ||
+      cudaMemsetAsync(ip.z64, 0, (size_t)k.units * 2 * k.D * sizeof(double), stream) != cudaSuccess ||
+      launch_init(ip, k.D, stream) != cudaSuccess) {
+    delete x;
+    return HYB_ECUDA;
+  }
+  *out = x;
+  return HYB_OK;
+}
+
+int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaStream_t stream) {
+  if (x == nullptr || k_new == nullptr || v_new == nullptr) return HYB_EINVAL;
+  if (!aligned16(k_new) || !aligned16(v_new)) return HYB_EINVAL;
+  const hyb_attn_config& c = x->cfg;
+  if (x->T >= c.capacity) return HYB_ECAPACITY;
+  AppendParams p{};
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_cache = static_cast<__nv_bfloat16*>(x->buf.k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
+  p.H = x->buf.H;
+  p.zk = x->buf.zk;
+  p.zv = x->buf.zv;
+  p.n = x->buf.n;
+  p.mu = x->buf.mu;
+  p.var = x->buf.var;
+  p.cap = c.capacity;
+  p.T = x->T;
+  p.max_blocks = x->ck.max_blocks > 0 ? x->ck.max_blocks : 1;
+  p.units = x->ck.units;
+  // after the append the window is [T + 1 - W, T + 1): position T - W leaves it
+  p.p = x->T - c.window;
+  p.evict = (p.p >= c.n_sink) ? 1 : 0;
+  if (p.evict) {
+    p.blk = (int32_t)((p.p - c.n_sink) / c.block_size);
+    p.cnt = (int32_t)((p.p - c.n_sink) % c.block_size + 1);
+  }
+  if (launch_append(p, x->ck.D, stream) != cudaSuccess) return HYB_ECUDA;
+  x->T += 1;
+  return HYB_OK;
+}
+
+int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out, float* scores_out,
+                    cudaStream_t stream) {
+  return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, stream);
+}
+
+int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32_t* sel, float* out,
+                                   cudaStream_t stream) {
+  if (sel == nullptr) return HYB_EINVAL;
+  return decode_impl(ctx, q, out, sel, nullptr, nullptr, stream);
+}
+
+int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, const void* v_host,
+                       float* out_host, cudaStream_t stream) {
+  if (x == nullptr || q_host == nullptr || out_host == nullptr) return HYB_EINVAL;
+  if ((k_host == nullptr) != (v_host == nullptr)) return HYB_EINVAL;
+  if (k_host != nullptr && x->T >= x->cfg.capacity) return HYB_ECAPACITY;
+  const size_t U = (size_t)x->ck.units, D = (size_t)x->ck.D, G = (size_t)x->ck.G;
+  void* dq = x->w<void>(x->ws.stage_q);
+  float* dout = x->w<float>(x->ws.stage_out);
+  if (cudaMemcpyAsync(dq, q_host, U * G * D * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess) return HYB_ECUDA;
+  if (k_host != nullptr) {
+    if (cudaMemcpyAsync(x->w<void>(x->ws.stage_k), k_host, U * D * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(x->w<void>(x->ws.stage_v), v_host, U * D * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return HYB_ECUDA;
+  }
+  int rc = decode_impl(x, dq, dout, nullptr, nullptr, nullptr, stream);
+  if (rc != HYB_OK) return rc;
+  if (k_host != nullptr) {
+    rc = hyb_attn_append(x, x->w<void>(x->ws.stage_k), x->w<void>(x->ws.stage_v), stream);
+    if (rc != HYB_OK) return rc;
+  }
+  if (cudaMemcpyAsync(out_host, dout, U * G * D * sizeof(float), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return HYB_ECUDA;
+  return HYB_OK;
+}
+
+int64_t hyb_attn_length(const hyb_attn_ctx* x) { return x ? x->T : -1; }
+
+int hyb_attn_status(hyb_attn_ctx* x, uint32_t* flags, int clear, cudaStream_t stream) {
+  if (x == nullptr || flags == nullptr) return HYB_EINVAL;
+  uint32_t* d = x->w<uint32_t>(x->ws.status);
+  if (cudaMemcpyAsync(flags, d, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return HYB_ECUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HYB_ECUDA;
+  if (clear && cudaMemsetAsync(d, 0, sizeof(uint32_t), stream) != cudaSuccess) return HYB_ECUDA;
+  return HYB_OK;
+}
+
+int hyb_attn_set_timing_events(hyb_attn_ctx* x, cudaEvent_t begin, cudaEvent_t end) {
+  if (x == nullptr || ((begin == nullptr) != (end == nullptr))) return HYB_EINVAL;
+  x->ev_begin = begin;
+  x->ev_end = end;
+  return HYB_OK;
+}
+
+void hyb_attn_destroy(hyb_attn_ctx* x) { delete x; }
+
+const char* hyb_attn_strerror(int code) {
+  switch (code) {
+    case HYB_OK: return "ok";
+    case HYB_EINVAL: return "invalid argument (shape, pointer, alignment or unsupported configuration)";
+    case HYB_ECAPACITY: return "KV cache capacity reached";
+    case HYB_ECUDA: return "CUDA call or kernel launch failed";
+    case HYB_ESTATE: return "call not valid in the current state";
+    case HYB_ENOMEM: return "host allocation failed";
+    default: return "unknown error code";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,231 @@
+// State kernels: the per-token append and the build of the state of a
+// prefilled history.
+//
+// The state of a unit (batch row, KV head) covers the evicted tokens
+// L = [S, T - W) -- past the sinks and out of the sliding window ("SALSA:
+// Training-Consistent Sparse Caching with Sink Preservation for Linearized
+// LLMs", abstract: window + sparse cache + linear-attention hidden state):
+//   H = sum_L k v^T, zk = sum_L k, zv = sum_L v, n = |L|   (the recurrent state
+//   of residual linear attention, "SPLA: Block Sparse Plus Linear Attention for
+//   Long Context Modeling", sections "Residual Linear Attention" / "Recurrence"),
+//   mu_j, var_j = mean and population variance of the keys of block
+//   j = [S + j*Bk, min(S + (j+1)*Bk, T - W))   (the block statistics the
+//   selection metric expands around, SPLA abstract).
+#include "hyb_device.cuh"
+#include "hyb_internal.h"
+
+namespace hyb {
+
+namespace {
+
+// ---------------------------------------------------------------- append
+// Grid (D / RPC, units), 256 threads; CTA x owns rows [x*RPC, (x+1)*RPC) of H.
+// CTA 0 also writes the new token into the caches, folds the evicted token into
+// zk, zv, n and updates its block's mean / population variance with Welford's
+// online recurrence (B. P. Welford, Technometrics 4(3), 1962).
+template <int D>
+__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+  constexpr int RPC = 1024 / D;  // 256 threads x 4 floats
+  __shared__ float kp[D], vp[D];
+  const int unit = blockIdx.y, rg = blockIdx.x, tid = threadIdx.x;
+  const int64_t ub = (int64_t)unit * p.cap;
+  if (p.evict) {
+    if (tid < D) {
+      // W == 0 evicts the token being appended; read it from the input then
+      const bool self = (p.p == p.T);
+      const __nv_bfloat16* ks = self ? p.k_new + (int64_t)unit * D : p.k_cache + (ub + p.p) * D;
+      const __nv_bfloat16* vs = self ? p.v_new + (int64_t)unit * D : p.v_cache + (ub + p.p) * D;
+      kp[tid] = __bfloat162float(ks[tid]);
+      vp[tid] = __bfloat162float(vs[tid]);
+    }
+    __syncthreads();
+    const int r = rg * RPC + tid / (D / 4);
+    const int c = (tid % (D / 4)) * 4;
+    float4* hp = reinterpret_cast<float4*>(p.H + ((int64_t)unit * D + r) * D + c);
+    float4 h = *hp;
+    const float k = kp[r];
+    h.x += k * vp[c];
+    h.y += k * vp[c + 1];
+    h.z += k * vp[c + 2];
+    h.w += k * vp[c + 3];
+    *hp = h;
+    if (rg == 0 && tid < D) {
+      const int64_t zi = (int64_t)unit * D + tid;
+      p.zk[zi] += kp[tid];
+      p.zv[zi] += vp[tid];
+      const int64_t si = ((int64_t)unit * p.max_blocks + p.blk) * D + tid;
+      const float x = kp[tid];
+      if (p.cnt == 1) {
+        p.mu[si] = x;
+        p.var[si] = 0.f;
+      } else {
+        const float cnt = (float)p.cnt;
+        const float mu0 = p.mu[si];
+        const float delta = x - mu0;
+        const float mu1 = mu0 + delta / cnt;
+        p.mu[si] = mu1;
+        p.var[si] = (p.var[si] * (cnt - 1.f) + delta * (x - mu1)) / cnt;
+      }
+      if (tid == 0) p.n[unit] += 1.f;
+    }
+  }
+  if (rg == 0 && tid < D) {
+    p.k_cache[(ub + p.T) * D + tid] = p.k_new[(int64_t)unit * D + tid];
+    p.v_cache[(ub + p.T) * D + tid] = p.v_new[(int64_t)unit * D + tid];
+  }
+}
+
+// ---------------------------------------------------------------- init
+// (1) H, zk, zv over L: grid (ceil(|L| / tokens_per_cta), units).  Each CTA
+//     accumulates its token range in fp32 (thread tile RT x RT of the D x D
+//     outer-product sum, keys/values staged through shared memory 32 tokens at a
+//     time) and adds the result into fp64 accumulators.
+template <int D>
+__global__ void __launch_bounds__(256) init_linear_kernel(const InitParams p) {
+  constexpr int RT = D / 16;
+  __shared__ __align__(16) float ks[32][D];
+  __shared__ __align__(16) float vs[32][D];
+  const int unit = blockIdx.y, tid = threadIdx.x;
+  const int tr = tid / 16, tc = tid % 16;
+  const int64_t t0 = p.ev_begin + (int64_t)blockIdx.x * p.tokens_per_cta;
+  const int64_t t1 = min(t0 + (int64_t)p.tokens_per_cta, p.ev_end);
+  const int64_t ub = (int64_t)unit * p.cap;
+  float acc[RT][RT];
+#pragma unroll
+  for (int i = 0; i < RT; ++i)
+#pragma unroll
+    for (int j = 0; j < RT; ++j) acc[i][j] = 0.f;
+  float zacc = 0.f;
+  for (int64_t tt = t0; tt < t1; tt += 32) {
+    const int n = (int)min((int64_t)32, t1 - tt);
+    for (int e = tid; e < 32 * D; e += 256) {
+      const int r = e / D, c = e % D;
+      float kv = 0.f, vv = 0.f;
+      if (r < n) {
+        kv = __bfloat162float(p.k_cache[(ub + tt + r) * D + c]);
+        vv = __bfloat162float(p.v_cache[(ub + tt + r) * D + c]);
+      }
+      ks[r][c] = kv;
+      vs[r][c] = vv;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < 32; ++r) {
+      float a[RT], b[RT];
+#pragma unroll
+      for (int i = 0; i < RT; ++i) {
+        a[i] = ks[r][tr * RT + i];
+        b[i] = vs[r][tc * RT + i];
+      }
+#pragma unroll
+      for (int i = 0; i < RT; ++i)
+#pragma unroll
+        for (int j = 0; j < RT; ++j) acc[i][j] += a[i] * b[j];
+    }
+    if (tid < D) {
+      for (int r = 0; r < n; ++r) zacc += ks[r][tid];
+    } else if (tid < 2 * D) {
+      for (int r = 0; r < n; ++r) zacc += vs[r][tid - D];
+    }
+    __syncthreads();
+  }
+  double* H64 = p.H64 + (int64_t)unit * D * D;
+#pragma unroll
+  for (int i = 0; i < RT; ++i)
+#pragma unroll
+    for (int j = 0; j < RT; ++j) atomicAdd(H64 + (int64_t)(tr * RT + i) * D + tc * RT + j, (double)acc[i][j]);
+  if (tid < 2 * D) atomicAdd(p.z64 + (int64_t)unit * 2 * D + tid, (double)zacc);
+}
+
+// (2) block statistics: one warp per block, two passes (mean, then the mean
+//     squared deviation) in fp64.
+template <int D>
+__global__ void __launch_bounds__(256) init_stats_kernel(const InitParams p) {
+  constexpr int CPL = D / 32;
+  const int unit = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + warp;
+  if (j >= p.nb) return;
+  const int64_t bs = p.ev_begin + (int64_t)j * p.Bk;
+  const int64_t be = min(bs + (int64_t)p.Bk, p.ev_end);
+  const double cnt = (double)(be - bs);
+  const __nv_bfloat16* kc = p.k_cache + (int64_t)unit * p.cap * D;
+  double s[CPL], q[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) s[i] = q[i] = 0.0;
+  for (int64_t t = bs; t < be; ++t)
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) s[i] += (double)__bfloat162float(kc[t * D + lane + 32 * i]);
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) s[i] /= cnt;
+  for (int64_t t = bs; t < be; ++t)
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const double d = (double)__bfloat162float(kc[t * D + lane + 32 * i]) - s[i];
+      q[i] += d * d;
+    }
+  const int64_t so = ((int64_t)unit * p.max_blocks + j) * D;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    p.mu[so + lane + 32 * i] = (float)s[i];
+    p.var[so + lane + 32 * i] = (float)(q[i] / cnt);
+  }
+}
+
+// (3) fp64 accumulators -> fp32 state; reset the tickets and the status word.
+template <int D>
+__global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) {
+  const int unit = blockIdx.x, tid = threadIdx.x;
+  const double* H64 = p.H64 + (int64_t)unit * D * D;
+  float* H = p.H + (int64_t)unit * D * D;
+  for (int e = tid; e < D * D; e += 256) H[e] = (float)H64[e];
+  if (tid < D) {
+    p.zk[(int64_t)unit * D + tid] = (float)p.z64[(int64_t)unit * 2 * D + tid];
+    p.zv[(int64_t)unit * D + tid] = (float)p.z64[(int64_t)unit * 2 * D + D + tid];
+  }
+  if (tid == 0) {
+    p.n[unit] = (float)(p.ev_end - p.ev_begin);
+    p.tickets_sel[unit] = 0u;
+    p.tickets_att[unit] = 0u;
+    if (unit == 0) *p.status = 0u;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {
+  const dim3 grid(D * D / 1024, p.units);
+  if (D == 128)
+    append_kernel<128><<<grid, 256, 0, s>>>(p);
+  else
+    append_kernel<64><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s) {
+  const int64_t ev = p.ev_end - p.ev_begin;
+  if (ev > 0) {
+    const dim3 g1((unsigned)((ev + p.tokens_per_cta - 1) / p.tokens_per_cta), p.units);
+    if (D == 128)
+      init_linear_kernel<128><<<g1, 256, 0, s>>>(p);
+    else
+      init_linear_kernel<64><<<g1, 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.nb > 0) {
+    const dim3 g2((unsigned)((p.nb + 7) / 8), p.units);
+    if (D == 128)
+      init_stats_kernel<128><<<g2, 256, 0, s>>>(p);
+    else
+      init_stats_kernel<64><<<g2, 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (D == 128)
+    init_finalize_kernel<128><<<p.units, 256, 0, s>>>(p);
+  else
+    init_finalize_kernel<64><<<p.units, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace hyb

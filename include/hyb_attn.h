@@ -1,0 +1,229 @@
+/*
+ * hyb_attn.h -- C ABI of the B200 (sm_100a) decode-step hybrid sparse + linear
+ * attention.
+ *
+ * What one decode step computes, for each batch row b and KV head h (a "unit")
+ * with the G = n_q_heads / n_kv_heads query heads of its group:
+ *
+ *   positions [0, T) of the unit's history split into            (SALSA: Training-
+ *     sinks    [0, min(S, T)),                                    Consistent Sparse
+ *     window   [max(S, T - W), T),                                Caching with Sink
+ *     evicted  L = [S, T - W)  (empty when T <= S + W),           Preservation for
+ *   L tiled into blocks j = [S + j*Bk, min(S + (j+1)*Bk, T - W))  Linearized LLMs,
+ *   from position S; the newest block may be partial.             abstract)
+ *
+ *   block score  score_j = sum_{i in group} q'_i . mu_j + 1/2 sum_c q'_ic^2 var_jc,
+ *   q' = q * scale, mu_j / var_j the block's key mean and population variance
+ *   (SPLA: Block Sparse Plus Linear Attention for Long Context Modeling --
+ *   abstract, and sections "Principled Block Selection via Taylor Expansion" and
+ *   "Grouped Sparsity");
+ *
+ *   the top_k blocks by score (ties to the lower index) are attended exactly
+ *   together with the sinks and the window: weight exp(s_t), s_t = q'.k_t;
+ *   every other evicted token gets the first-order Taylor weight 1 + s_t (SLAKE:
+ *   Softmax-Approximated Training-Free Linear Attention with KV-Cache Eviction
+ *   for Long-Sequence LLMs, abstract, PTAA), computed without reading it as the
+ *   global linear state (H = sum_L k v^T, zk = sum_L k, zv = sum_L v, n = |L|)
+ *   minus the selected blocks' own (1 + s_t) terms (SPLA abstract, section
+ *   "IO-Efficient Implementation");
+ *
+ *   one shared normaliser:
+ *     o_i = [sum_X e^{s_t} v_t + sum_{L\sel} (1 + s_t) v_t] / [sum_X e^{s_t} + sum_{L\sel} (1 + s_t)].
+ *
+ * Conventions for every call:
+ *   - The caller owns all device memory and every stream; the library owns only
+ *     the host-side context.  Pointers are device pointers unless the name ends
+ *     in _host, and must be 16-byte aligned.
+ *   - Calls are asynchronous: they enqueue kernels on `stream` and return.
+ *   - Return value 0 is success; a negative HYB_E* code means nothing was
+ *     enqueued (except HYB_ECUDA, where a launch failed).  No exception or abort
+ *     crosses the ABI.
+ *   - Anomalies found on the device (non-finite output, denominator <= 0, an
+ *     out-of-range block index in a caller-given selection, a timed-out wait)
+ *     set bits in a device status word, read with hyb_attn_status().
+ *   - All batch rows share the length T.  One context holds one layer.
+ *   - Supported: head_dim 64 or 128; group size G in {1, 2, 4};
+ *     batch * n_kv_heads * capacity < 2^31.
+ */
+#ifndef HYB_ATTN_H
+#define HYB_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes -------------------------------------------------------- */
+#define HYB_OK          0
+#define HYB_EINVAL     (-1)  /* bad shape, pointer, alignment or argument */
+#define HYB_ECAPACITY  (-2)  /* append would pass `capacity` tokens */
+#define HYB_ECUDA      (-3)  /* a CUDA call or kernel launch failed */
+#define HYB_ESTATE     (-4)  /* call not valid in the current state (e.g. decode at T = 0) */
+#define HYB_ENOMEM     (-5)  /* host allocation of the context failed */
+
+/* ---- device status bits (hyb_attn_status) -------------------------------- */
+#define HYB_STATUS_NONFINITE     0x1u  /* an output element was NaN or Inf */
+#define HYB_STATUS_DENOMINATOR   0x2u  /* a shared normaliser was <= 0 (no clamp is applied) */
+#define HYB_STATUS_BAD_SELECTION 0x4u  /* a caller-given block index was out of range (skipped) */
+#define HYB_STATUS_TIMEOUT       0x8u  /* a bounded wait inside a kernel gave up */
+#define HYB_STATUS_NAN_SCORE     0x10u /* a block score was NaN (ranked last) */
+
+/* ---- configuration ------------------------------------------------------- */
+typedef struct hyb_attn_config {
+  int32_t batch;       /* B  >= 1 */
+  int32_t n_q_heads;   /* Hq >= 1, a multiple of n_kv_heads; query head i belongs to KV head i / G */
+  int32_t n_kv_heads;  /* Hkv >= 1 */
+  int32_t head_dim;    /* d: 64 or 128 */
+  int32_t block_size;  /* Bk >= 1: tokens per selectable block of the evicted stream */
+  int32_t n_sink;      /* S >= 0: leading positions always attended exactly */
+  int32_t window;      /* W >= 0: trailing positions always attended exactly */
+  int32_t top_k;       /* k >= 0: blocks attended exactly per (b, KV head) */
+  int64_t capacity;    /* rows per (b, KV head) in the KV cache, >= 1 */
+  float   scale;       /* q' = q * scale; 0 selects 1/sqrt(head_dim) */
+} hyb_attn_config;
+
+/* Sizes (in elements, except where noted) of the caller-owned buffers for a
+ * configuration.  max_blocks = ceil(max(0, capacity - S - W) / Bk) is the row
+ * count of the block-statistics arrays per unit. */
+typedef struct hyb_attn_sizes {
+  int64_t kv_cache_elems;   /* B * Hkv * capacity * d   (bf16, each of K and V) */
+  int64_t H_elems;          /* B * Hkv * d * d          (fp32) */
+  int64_t z_elems;          /* B * Hkv * d              (fp32, each of zk and zv) */
+  int64_t n_elems;          /* B * Hkv                  (fp32) */
+  int64_t max_blocks;       /* ceil(max(0, capacity - S - W) / Bk) */
+  int64_t stats_elems;      /* B * Hkv * max_blocks * d (fp32, each of mu and var) */
+  int64_t workspace_bytes;  /* scratch the library uses between and inside calls */
+} hyb_attn_sizes;
+
+/* Caller-owned device buffers of one layer.  Layouts (row-major, unit index
+ * u = b * Hkv + h):
+ *   k_cache, v_cache  bf16 [B][Hkv][capacity][d]   position t of unit u at row u*capacity + t
+ *   H                 fp32 [B][Hkv][d][d]          H[u][r][c] = sum_{t in L} k_t[r] v_t[c]
+ *   zk, zv            fp32 [B][Hkv][d]
+ *   n                 fp32 [B][Hkv]                |L| (exact up to 2^24)
+ *   mu, var           fp32 [B][Hkv][max_blocks][d] key mean / population variance of block j
+ *   workspace         hyb_attn_sizes.workspace_bytes bytes, 256-byte aligned; contents are
+ *                     private to the library.  Contexts whose calls are serialised on one
+ *                     stream may share one workspace.
+ * The state arrays (H, zk, zv, n, mu, var) are written by hyb_attn_init and kept
+ * up to date by hyb_attn_append; copying them together with the caches and T is a
+ * complete checkpoint of the layer. */
+typedef struct hyb_attn_buffers {
+  void*  k_cache;
+  void*  v_cache;
+  float* H;
+  float* zk;
+  float* zv;
+  float* n;
+  float* mu;
+  float* var;
+  void*  workspace;
+  size_t workspace_bytes;
+} hyb_attn_buffers;
+
+typedef struct hyb_attn_ctx hyb_attn_ctx;  /* opaque host-side handle, one per layer */
+
+/* Host-only description of how one decode at length T is split into work
+ * (exposed for tests and tooling; no device access). */
+typedef struct hyb_attn_plan_info {
+  int64_t T;
+  int64_t n_blocks;          /* nb: candidate blocks at T */
+  int64_t k_eff;             /* min(top_k, nb) */
+  int64_t exact_tokens;      /* |sinks| + |window| + tokens of k_eff full blocks (upper bound) */
+  int32_t chunks_per_unit;   /* 64-token pieces of the exact set per unit (fixed for a given T) */
+  int32_t attend_ctas;       /* grid of the attention kernel */
+  int32_t partial_slots;     /* split-K partial records the attention kernel writes */
+  int32_t score_ctas_per_unit;
+  int32_t linear_ctas_per_unit;
+} hyb_attn_plan_info;
+
+/* Fill `out` with the buffer sizes of `cfg`.  Host only; never touches a GPU.
+ * Returns HYB_EINVAL for an unsupported configuration. */
+int hyb_attn_query_sizes(const hyb_attn_config* cfg, hyb_attn_sizes* out);
+
+/* Workspace bytes for `cfg` (0 for an unsupported configuration).  Host only. */
+size_t hyb_attn_workspace_size(const hyb_attn_config* cfg);
+
+/* Work split of a decode at length T on a device with `n_sm` multiprocessors.
+ * Host only. */
+int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_plan_info* out);
+
+/* Create a context for one layer whose caches already hold T0 tokens per unit
+ * (positions [0, T0) of k_cache / v_cache), and build the state of those tokens
+ * on `stream`: the linear state over L = [S, T0 - W) and the statistics of every
+ * block of L, the newest possibly partial (SPLA abstract: block statistics and a
+ * recurrent state of the unselected tokens).  The context records the buffer
+ * pointers; the caller keeps them alive until hyb_attn_destroy.  The current
+ * CUDA device must be the device owning the buffers.
+ * Errors: HYB_EINVAL (cfg, pointers, alignment, T0 outside [0, capacity]),
+ * HYB_ENOMEM, HYB_ECUDA.  On error *out is set to NULL. */
+int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
+                  int64_t T0, cudaStream_t stream);
+
+/* Append one token per unit: k_new, v_new bf16 [B][Hkv][d].  The token is
+ * written at position T; then T += 1, and if the token at position T - W - 1
+ * (after the increment) lies at or past S it leaves the window: it is folded
+ * into H, zk, zv, n (a rank-1 update, SPLA "Recurrence") and into the running
+ * mean / population variance of its block (Welford's update), which opens a new
+ * block when the previous one is full.  Errors: HYB_EINVAL (null or misaligned
+ * pointers), HYB_ECAPACITY (T == capacity), HYB_ECUDA. */
+int hyb_attn_append(hyb_attn_ctx* ctx, const void* k_new, const void* v_new, cudaStream_t stream);
+
+/* One decode step at the current length T for every unit:
+ *   q           bf16 [B][Hq][d]  (input)
+ *   out         fp32 [B][Hq][d]  (output)
+ *   sel_out     int32 [B][Hkv][top_k] or NULL: the selected block indices,
+ *               ascending, -1 padded when nb < top_k
+ *   scores_out  fp32 [B][Hkv][max_blocks] or NULL: the block scores (entries
+ *               [0, nb) of each unit are written)
+ * Kernels: block scoring + top-k + the global linear term phi(q)^T state, then
+ * split-K exact attention over sinks, window and selected blocks with the
+ * selected blocks' (1 + s) subtraction and the shared-normaliser merge.
+ * Errors: HYB_EINVAL (null or misaligned pointers), HYB_ESTATE (T == 0),
+ * HYB_ECUDA. */
+int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out,
+                    float* scores_out, cudaStream_t stream);
+
+/* As hyb_attn_decode, with the block selection given by the caller instead of
+ * the top-k: sel int32 [B][Hkv][top_k], each row ascending and distinct, -1
+ * entries ignored.  Indices outside [0, nb) are skipped and raise
+ * HYB_STATUS_BAD_SELECTION.  Used to compare outputs for a fixed selection. */
+int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32_t* sel,
+                                   float* out, cudaStream_t stream);
+
+/* One decode + append step from host memory, for callers whose inputs and
+ * outputs live on the host: copies q_host (bf16 [B][Hq][d]) and k_host, v_host
+ * (bf16 [B][Hkv][d]) to device staging space in the workspace, runs
+ * hyb_attn_decode then hyb_attn_append, and copies the fp32 output back to
+ * out_host ([B][Hq][d]).  All copies are cudaMemcpyAsync on `stream`; host
+ * buffers should be pinned for the copies to be asynchronous.  k_host / v_host
+ * may be NULL to skip the append.  The call returns after enqueueing; the output
+ * is valid once `stream` has been synchronised. */
+int hyb_attn_step_host(hyb_attn_ctx* ctx, const void* q_host, const void* k_host,
+                       const void* v_host, float* out_host, cudaStream_t stream);
+
+/* Current length T (host mirror; no device access). */
+int64_t hyb_attn_length(const hyb_attn_ctx* ctx);
+
+/* Copy the device status word to *flags (synchronises `stream`); with clear != 0
+ * reset it to zero afterwards.  Returns HYB_OK or HYB_ECUDA. */
+int hyb_attn_status(hyb_attn_ctx* ctx, uint32_t* flags, int clear, cudaStream_t stream);
+
+/* Profiling hook: when both events are non-NULL, every later decode records
+ * `begin` just before and `end` just after the attention kernel on the decode's
+ * stream, so the caller can time that kernel alone.  Pass NULL, NULL to stop. */
+int hyb_attn_set_timing_events(hyb_attn_ctx* ctx, cudaEvent_t begin, cudaEvent_t end);
+
+/* Release the host context (device buffers stay with the caller). */
+void hyb_attn_destroy(hyb_attn_ctx* ctx);
+
+/* Static description of a return code. */
+const char* hyb_attn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYB_ATTN_H */

@@ -1,0 +1,122 @@
+"""The C-ABI library builds, loads and exports every entry point the header
+declares; host-only entry points (sizes, plan, argument checks) work without a
+GPU.  No kernel is launched here."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hyb_attn.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(hyb_attn_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hybrid_sparse_linear_decode_b200 import build
+    build.build()
+    from hybrid_sparse_linear_decode_b200 import _abi
+    return _abi.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ["hyb_attn_init", "hyb_attn_append", "hyb_attn_decode", "hyb_attn_decode_with_selection",
+              "hyb_attn_workspace_size", "hyb_attn_length", "hyb_attn_status", "hyb_attn_destroy",
+              "hyb_attn_strerror", "hyb_attn_query_sizes", "hyb_attn_plan", "hyb_attn_step_host",
+              "hyb_attn_set_timing_events"]:
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from hybrid_sparse_linear_decode_b200 import _abi
+    so = _abi.LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True, check=True).stdout
+    exported = set(l.split()[-1] for l in out.splitlines() if l.strip())
+    for n in _declared_functions():
+        assert n in exported, f"{n} declared in hyb_attn.h but not exported"
+        assert getattr(lib, n) is not None
+    # the binding covers the same set
+    assert set(n for n, _, _ in _abi.SIGNATURES) == set(_declared_functions())
+
+
+def _cfg(**kw):
+    from hybrid_sparse_linear_decode_b200 import make_config
+    base = dict(batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128, block_size=64, n_sink=4, window=1024,
+                top_k=16, capacity=32768 + 64)
+    base.update(kw)
+    return make_config(**base)
+
+
+def test_sizes_and_workspace(lib):
+    import hybrid_sparse_linear_decode_b200 as H
+    c = _cfg()
+    s = H.hyb_attn_query_sizes(c)
+    assert s.kv_cache_elems == 8 * (32768 + 64) * 128
+    assert s.H_elems == 8 * 128 * 128 and s.z_elems == 8 * 128 and s.n_elems == 8
+    assert s.max_blocks == -(-(32768 + 64 - 4 - 1024) // 64)
+    assert s.stats_elems == 8 * s.max_blocks * 128
+    assert s.workspace_bytes == H.hyb_attn_workspace_size(c) > 0
+    # window and sinks covering the whole capacity: no blocks at all
+    s2 = H.hyb_attn_query_sizes(_cfg(capacity=1000))
+    assert s2.max_blocks == 0
+
+
+@pytest.mark.parametrize("bad", [dict(head_dim=96), dict(n_q_heads=24, n_kv_heads=8), dict(n_q_heads=64),
+                                 dict(block_size=0), dict(top_k=-1), dict(capacity=0), dict(window=-1),
+                                 dict(scale=-1.0), dict(batch=4096, capacity=1 << 20)])
+def test_invalid_configs_rejected(lib, bad):
+    import hybrid_sparse_linear_decode_b200 as H
+    with pytest.raises(H.HybAttnError) as e:
+        H.hyb_attn_query_sizes(_cfg(**bad))
+    assert e.value.code == -1
+    assert H.hyb_attn_workspace_size(_cfg(**bad)) == 0
+
+
+def test_init_rejects_bad_arguments_without_touching_a_gpu(lib):
+    import hybrid_sparse_linear_decode_b200 as H
+    c = _cfg()
+    buf = H.hyb_attn_buffers()  # all null
+    with pytest.raises(H.HybAttnError) as e:
+        H.hyb_attn_init(c, buf, 100, 0)
+    assert e.value.code == -1
+    buf2 = H.hyb_attn_buffers(16, 32, 48, 64, 80, 96, 112, 128, 256, 1)  # tiny workspace
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_init(c, buf2, 100, 0)
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_init(c, buf2, c.capacity + 1, 0)
+    # null context handles
+    assert lib.hyb_attn_decode(None, None, None, None, None, None) == -1
+    assert lib.hyb_attn_append(None, None, None, None) == -1
+    assert lib.hyb_attn_length(None) == -1
+    assert H.hyb_attn_strerror(-2).startswith("KV cache capacity")
+
+
+@pytest.mark.parametrize("T", [0, 1, 3, 4, 5, 1027, 1028, 1029, 1092, 1093, 32768, 32768 + 64])
+def test_plan_partition(lib, T):
+    """Chunk counts of the exact set follow the partition: sinks, window, and
+    ceil(Bk/64) chunks per selected block; the grid never exceeds the SM count."""
+    import hybrid_sparse_linear_decode_b200 as H
+    c = _cfg()
+    p = H.hyb_attn_plan(c, T, 148)
+    S, W, Bk = 4, 1024, 64
+    ev = max(0, T - S - W)
+    nb = -(-ev // Bk)
+    assert p.n_blocks == nb and p.k_eff == min(16, nb)
+    sink = min(S, T)
+    win = T - max(S, T - W) if T > S else 0
+    assert p.chunks_per_unit == -(-sink // 64) + -(-win // 64) + p.k_eff
+    total = 8 * p.chunks_per_unit
+    if total:
+        assert p.attend_ctas == min(total, 148)
+        assert p.partial_slots == p.attend_ctas + 8 - 1
+    assert p.score_ctas_per_unit == -(-nb // 64)

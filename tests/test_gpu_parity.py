@@ -1,0 +1,161 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle, at
+sizes the oracle finishes in seconds: several tiles, ragged tails and the
+degenerate cases of the method."""
+
+import math
+
+import numpy as np
+import pytest
+
+from harness import Case, check_outputs, check_selection, check_state, full_check, bits_to_f64
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(**kw):
+    base = dict(B=1, Hq=4, Hkv=1, d=128, T0=600, Bk=32, S=4, W=64, k=4, n_append=0, seed=1)
+    base.update(kw)
+    return Case(**base)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),                                                   # plain
+    dict(d=64),                                               # head dim 64
+    dict(Hq=2, Hkv=1), dict(Hq=8, Hkv=8),                     # G = 2, G = 1
+    dict(B=2, Hq=16, Hkv=4, T0=1500),                         # several units
+    dict(T0=3, S=4, W=16),                                    # T <= S: sinks only
+    dict(T0=15, S=4, W=16),                                   # S < T <= S + W: no evicted token
+    dict(T0=4 + 16 + 30, S=4, W=16, Bk=8, k=8),               # nb <= k: every block selected
+    dict(T0=4 + 64 + 32 * 5 + 1),                             # newest block holds 1 token
+    dict(k=0),                                                # nothing selected
+    dict(W=0),                                                # no window
+    dict(S=0),                                                # no sinks
+    dict(S=0, W=0, k=0, T0=333),                              # empty exact set: pure Taylor
+    dict(Bk=100, k=3, T0=1200),                               # block spans 2 chunks, ragged
+    dict(Bk=128, k=5, T0=2000, W=200),                        # 2 chunks per block
+    dict(Bk=200, k=2, T0=1500, W=70),                         # 4 chunks per block, partial pieces
+    dict(Bk=16, k=30, T0=1000, W=100),                        # many short blocks
+    dict(W=1000, T0=3000, S=7),                               # long unaligned window
+    dict(B=4, Hq=32, Hkv=8, T0=5000, Bk=64, W=1024, k=16),    # 32 units, CTAs span units
+    dict(scale=0.05),                                         # explicit scale
+    dict(k_scale=3.0, T0=900),                                # large scores (max shift matters)
+])
+def test_decode_matches_oracle(kw):
+    c = _case(**kw)
+    q = c.random_q()
+    (mx, rel), _ = full_check(c, q)
+    assert c.layer.status() == 0
+
+
+def test_all_selected_is_softmax_and_q0_is_mean():
+    """Closed-form properties through the GPU: k >= nb gives full softmax;
+    q = 0 gives the mean of V over [0, T)."""
+    c = _case(T0=700, Bk=32, k=1000, W=64)
+    q = c.random_q()
+    out, sel, _ = c.decode(q)
+    Kf, Vf = c.unit_kv(0, 0)
+    ref = O.full_softmax(bits_to_f64(q)[0], Kf, Vf, c.T, c.scale)
+    check_outputs(out[0], ref)
+    out0, _, _ = c.decode(np.zeros_like(q))
+    check_outputs(out0[0], np.broadcast_to(Vf.mean(axis=0), out0[0].shape), max_abs=1e-4, rel_l2=1e-4)
+
+
+@pytest.mark.parametrize("kw,n", [
+    (dict(T0=600, Bk=32, W=64), 40),
+    (dict(T0=4 + 64 + 32 * 3, Bk=32, W=64), 3),               # the first append opens a new block
+    (dict(T0=10, S=4, W=16, Bk=8), 40),                       # grows from sinks-only through eviction
+    (dict(T0=200, W=0, Bk=8), 20),                            # W = 0 evicts the appended token itself
+    (dict(T0=300, S=0, W=5, Bk=7, d=64), 30),
+    (dict(B=2, Hq=8, Hkv=2, T0=900, Bk=100, W=50), 110),      # fills a whole 100-token block
+])
+def test_append_state_and_decode(kw, n):
+    """State after n appends equals the direct definition on the final history,
+    and decode after the appends still matches the oracle."""
+    c = _case(n_append=n, **kw)
+    check_state(c)
+    for i in range(n):
+        c.append()
+        if i % 7 == 0 or i == n - 1:
+            full_check(c, c.random_q())
+    check_state(c)
+
+
+def test_decode_with_given_selection():
+    c = _case(T0=1500, Bk=32, k=6)
+    q = c.random_q()
+    part = O.partition(c.T, c.S, c.W, c.Bk)
+    for trial in range(4):
+        sel = np.sort(c.rng.choice(part.nb, size=c.k, replace=False)).astype(np.int32)
+        if trial == 3:
+            sel[-2:] = -1
+        out = c.decode_with_selection(q, sel.reshape(1, 1, -1))
+        ref, _, _ = c.oracle_unit(q, 0, 0, sel=np.array([j for j in sel if j >= 0]))
+        check_outputs(out[0], ref)
+    assert c.layer.status(clear=True) == 0
+
+
+def test_bad_selection_index_is_reported_and_skipped():
+    from hybrid_sparse_linear_decode_b200 import HYB_STATUS_BAD_SELECTION
+    c = _case(T0=1500, Bk=32, k=4)
+    q = c.random_q()
+    part = O.partition(c.T, c.S, c.W, c.Bk)
+    sel = np.array([[[1, 5, part.nb + 3, 10 ** 6]]], dtype=np.int32)
+    out = c.decode_with_selection(q, sel)
+    assert c.layer.status(clear=True) & HYB_STATUS_BAD_SELECTION
+    ref, _, _ = c.oracle_unit(q, 0, 0, sel=np.array([1, 5]))
+    check_outputs(out[0], ref)
+    assert c.layer.status() == 0
+
+
+def test_ties_go_to_lower_block_index():
+    """Blocks with identical keys have identical scores: the selection must
+    take the lowest indices among them (exact on both sides)."""
+    B, Hkv, d, S, W, Bk = 1, 1, 64, 4, 32, 16
+    nbk = 20
+    T0 = S + nbk * Bk + W
+    rng = np.random.default_rng(3)
+    Kf = rng.standard_normal((B, Hkv, T0, d))
+    Vf = rng.standard_normal((B, Hkv, T0, d))
+    blk = rng.standard_normal((Bk, d))
+    for j in (2, 5, 9, 13, 17):            # five copies of one block
+        Kf[0, 0, S + j * Bk:S + (j + 1) * Bk] = blk * 0.3 + 2.0
+    from harness import bf16_bits
+    c = Case(B, 4, Hkv, d, T0, Bk, S, W, 3, kv_bits=(bf16_bits(Kf), bf16_bits(Vf)))
+    q = bf16_bits(np.abs(rng.standard_normal((1, 4, d))))
+    out, sel, scores = c.decode(q)
+    assert list(sel[0, 0]) == [2, 5, 9]
+    s = scores[0, 0]
+    assert s[2] == s[5] == s[9] == s[13] == s[17]
+
+
+def test_step_host_matches_device_path():
+    """The host-buffer entry point (copies + decode + append) equals the device path."""
+    import torch
+    c1 = _case(T0=1000, n_append=3, seed=5)
+    c2 = _case(T0=1000, n_append=3, seed=5)
+    for i in range(3):
+        q = c1.random_q()
+        c2.rng.standard_normal((c2.B, c2.Hq, c2.d))      # keep the rngs in step
+        out1, _, _ = c1.decode(q, with_scores=False)
+        c1.append()
+        qh = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        kh = torch.from_numpy(np.ascontiguousarray(c2.Kb[:, :, c2.T]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        vh = torch.from_numpy(np.ascontiguousarray(c2.Vb[:, :, c2.T]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        oh = torch.empty((c2.B, c2.Hq, c2.d), dtype=torch.float32).pin_memory()
+        c2.layer.step_host(qh, kh, vh, oh)
+        torch.cuda.synchronize()
+        c2.T += 1
+        np.testing.assert_array_equal(oh.numpy(), out1.astype(np.float32))
+    assert c1.layer.T == c2.layer.T
+
+
+def test_capacity_error():
+    import torch
+    from hybrid_sparse_linear_decode_b200 import HybAttnError
+    c = _case(T0=100, n_append=1)
+    c.append()
+    k = torch.zeros((1, 1, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(HybAttnError) as e:
+        c.layer.append(k, k)
+    assert e.value.code == -2

@@ -1,0 +1,170 @@
+"""Parity at the full sizes of the five synthetic workloads, in the launch
+configuration the benchmark times: device caches are filled by the device
+generator, the oracle regenerates the same units on the host (bit-identical
+generator twins, see test_gpu_syngen.py) for sampled units."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from harness import bits_to_f64, check_outputs, check_selection, to_device_bf16, OUT_MAX_ABS, OUT_REL_L2, STATE_REL
+from syngen import configs as C
+from syngen import host as SH
+
+pytestmark = pytest.mark.gpu
+
+
+class WorkloadLayer:
+    def __init__(self, w: C.Workload, layer: int, device="cuda", n_app=None):
+        import torch
+        import syngen.device as SD
+        from hybrid_sparse_linear_decode_b200 import HybridAttentionLayer, make_config
+        SD.build()
+        self.w, self.l = w, layer
+        self.n_app = w.capacity - w.T0 if n_app is None else n_app
+        cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window,
+                          w.top_k, w.T0 + self.n_app)
+        self.layer = HybridAttentionLayer(cfg, device)
+        self.tables = SD.DeviceTables(w, layer, self.layer.device)
+        SD.fill_kv(w, self.tables, self.layer.k_cache, self.layer.v_cache, 0, w.T0)
+        self.app_k = self.app_v = None
+        if self.n_app:
+            shp = (w.batch, w.n_kv_heads, self.n_app, w.head_dim)
+            self.app_k = torch.empty(shp, dtype=torch.bfloat16, device=self.layer.device)
+            self.app_v = torch.empty(shp, dtype=torch.bfloat16, device=self.layer.device)
+            SD.fill_kv(w, self.tables, self.app_k, self.app_v, w.T0, w.T0 + self.n_app, t_out0=w.T0)
+        self.layer.init(w.T0)
+        self.T = w.T0
+        self.scale = 1 / math.sqrt(w.head_dim)
+        self._host = {}
+
+    def q_bits(self, step):
+        return SH.q_bits(self.w, self.l, step)
+
+    def decode(self, qb):
+        import torch
+        dev = self.layer.device
+        sel = torch.full((self.w.batch, self.w.n_kv_heads, self.w.top_k), -7, dtype=torch.int32, device=dev)
+        out = self.layer.decode(to_device_bf16(qb, dev), sel_out=sel)
+        torch.cuda.synchronize()
+        return out.cpu().numpy().astype(np.float64), sel.cpu().numpy()
+
+    def append(self, i):
+        self.layer.append(self.app_k[:, :, i].contiguous(), self.app_v[:, :, i].contiguous())
+        self.T += 1
+
+    def host_unit(self, b, h):
+        if (b, h) not in self._host:
+            self._host[(b, h)] = SH.kv_f64(self.w, self.tables.host, b, h, 0, self.w.T0 + self.n_app)
+        return self._host[(b, h)]
+
+    def check_units(self, qb, units, out, sel):
+        w = self.w
+        G = w.group
+        part = O.partition(self.T, w.n_sink, w.window, w.block_size)
+        refs, gots, ndiff = [], [], 0
+        for (b, h) in units:
+            K, V = self.host_unit(b, h)
+            K, V = K[:self.T], V[:self.T]
+            q = bits_to_f64(qb)[b, h * G:(h + 1) * G]
+            mu, var = O.block_stats(K, part)
+            scores = O.block_scores(q, mu, var, self.scale)
+            ndiff += check_selection(sel[b, h], scores, w.top_k)
+            gsel = np.array([j for j in sel[b, h] if j >= 0])
+            refs.append(O.hybrid_subtract(q, K, V, part, gsel, self.scale))
+            gots.append(out[b, h * G:(h + 1) * G])
+        return check_outputs(np.array(gots), np.array(refs)), ndiff
+
+    def check_state(self, units):
+        w = self.w
+        part = O.partition(self.T, w.n_sink, w.window, w.block_size)
+        L = self.layer
+        for (b, h) in units:
+            K, V = self.host_unit(b, h)
+            K, V = K[:self.T], V[:self.T]
+            H, zk, zv, n = O.linear_state(K, V, part)
+            mu, var = O.block_stats(K, part)
+            assert float(L.n[b, h]) == n
+            for name, ref, t in (("H", H, L.H[b, h]), ("zk", zk, L.zk[b, h]), ("zv", zv, L.zv[b, h]),
+                                 ("mu", mu, L.mu[b, h, :part.nb]), ("var", var, L.var[b, h, :part.nb])):
+                got = t.cpu().numpy().astype(np.float64)
+                rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+                assert rel <= STATE_REL, (name, (b, h), rel)
+
+
+def test_tiny_workload_decode_appends_state():
+    w = C.get_workload("tiny")
+    wl = WorkloadLayer(w, 0)
+    units = [(0, 0)]
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    (mx, rel), nd = wl.check_units(qb, units, out, sel)
+    planted = set(wl.tables.host.planted[0, 0].tolist())
+    assert planted <= set(sel[0, 0].tolist())
+    for i in range(w.appends_after_decode):
+        wl.append(i)
+    wl.check_state(units)
+    qb = SH.q_bits(w, 0, 1)
+    out, sel = wl.decode(qb)
+    wl.check_units(qb, units, out, sel)
+
+
+def test_llama8b_32k_layer_every_unit():
+    w = C.get_workload("llama8b_32k_layer")
+    wl = WorkloadLayer(w, 0, n_app=0)
+    units = [(0, h) for h in range(w.n_kv_heads)]
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    wl.check_units(qb, units, out, sel)
+    wl.check_state(units[:2])
+    # every planted block is selected
+    for h in range(w.n_kv_heads):
+        assert set(wl.tables.host.planted[0, h].tolist()) <= set(sel[0, h].tolist())
+    # q = 0 at full size: the mean of V over [0, T) for every unit
+    out0, _ = wl.decode(np.zeros_like(qb))
+    for h in range(2):
+        _, V = wl.host_unit(0, h)
+        check_outputs(out0[0, h * w.group:(h + 1) * w.group],
+                      np.broadcast_to(V[:w.T0].mean(axis=0), (w.group, w.head_dim)), max_abs=1e-4, rel_l2=1e-4)
+
+
+@pytest.mark.parametrize("layer", [0, 31])
+def test_llama8b_32layers_b8_32k_sampled(layer):
+    w = C.get_workload("llama8b_32layers_b8_32k")
+    wl = WorkloadLayer(w, layer, n_app=1)
+    units = [(0, 0), (3, 5), (7, 7), (5, 2)]
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    wl.check_units(qb, units, out, sel)
+    wl.append(0)
+    wl.check_state(units[:2])
+
+
+def test_llama8b_32layers_b4_128k_sampled():
+    w = C.get_workload("llama8b_32layers_b4_128k")
+    wl = WorkloadLayer(w, 9, n_app=0)
+    units = [(0, 0), (2, 3), (3, 7)]
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    wl.check_units(qb, units, out, sel)
+
+
+def test_llama8b_256k_256_steps_sampled():
+    w = C.get_workload("llama8b_256k_256steps")
+    wl = WorkloadLayer(w, 0)
+    assert wl.n_app == 256
+    units = [(0, 1), (0, 6)]
+    for step in range(w.steps):
+        qb = wl.q_bits(step)
+        out, sel = wl.decode(qb)
+        if step in (0, 97, 255):
+            wl.check_units(qb, units, out, sel)
+            for h in range(w.n_kv_heads):
+                if step == 0:
+                    assert set(wl.tables.host.planted[0, h].tolist()) <= set(sel[0, h].tolist())
+        wl.append(step)
+    assert wl.layer.T == w.T0 + 256
+    wl.check_state(units)
+    assert wl.layer.status() == 0
