@@ -25,6 +25,7 @@ from ._abi import (  # noqa: F401
     hyb_attn_set_timing_events,
     hyb_attn_destroy,
     hyb_attn_strerror,
+    hyb_attn_last_cuda_error,
     load_library,
     LIB_PATH,
     HYB_STATUS_NONFINITE,

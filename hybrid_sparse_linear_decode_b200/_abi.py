@@ -70,13 +70,17 @@ SIGNATURES = [
     ("hyb_attn_set_timing_events", ctypes.c_int, [c_vp, c_vp, c_vp]),
     ("hyb_attn_destroy", None, [c_vp]),
     ("hyb_attn_strerror", ctypes.c_char_p, [ctypes.c_int]),
+    ("hyb_attn_last_cuda_error", ctypes.c_char_p, []),
 ]
 
 
 class HybAttnError(RuntimeError):
     def __init__(self, fn: str, code: int):
         self.code = code
-        super().__init__(f"{fn} failed: {code} ({strerror(code)})")
+        msg = f"{fn} failed: {code} ({strerror(code)})"
+        if code == HYB_ECUDA:
+            msg += f" [{hyb_attn_last_cuda_error()}]"
+        super().__init__(msg)
 
 
 _lib = None
@@ -108,6 +112,10 @@ def strerror(code: int) -> str:
 
 
 hyb_attn_strerror = strerror
+
+
+def hyb_attn_last_cuda_error() -> str:
+    return load_library().hyb_attn_last_cuda_error().decode()
 
 
 def hyb_attn_query_sizes(cfg: hyb_attn_config) -> hyb_attn_sizes:

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <cstdio>
 #include <cstring>
 #include <new>
 
@@ -107,6 +108,14 @@ int attend_grid(int64_t total_chunks, int n_sm) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Record a failed CUDA call and map it to HYB_ECUDA.
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = e;
+  return HYB_ECUDA;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -205,7 +214,7 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   sp.lin_ctas = k.D / 32;
   sp.scale = x->scale;
   cudaError_t e = launch_select(sp, k.D, sp.score_ctas + sp.lin_ctas, stream);
-  if (e != cudaSuccess) return HYB_ECUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
 
   AttendParams ap{};
   ap.q = sp.q;
@@ -238,7 +247,7 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
   if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
   e = launch_attend(&x->tmK, &x->tmV, ap, k.D, /*pdl=*/!timed, stream);
-  if (e != cudaSuccess) return HYB_ECUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
   return HYB_OK;
 }
@@ -326,9 +335,10 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
     delete x;
     return HYB_ECUDA;
   }
-  if (prepare_attend(k.D) != cudaSuccess) {
+  const cudaError_t pe = prepare_attend(k.D);
+  if (pe != cudaSuccess) {
     delete x;
-    return HYB_ECUDA;
+    return cuda_fail(pe);
   }
 
   const Geometry g = geometry(*cfg, T0);
@@ -392,7 +402,8 @@ int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaS
     p.blk = (int32_t)((p.p - c.n_sink) / c.block_size);
     p.cnt = (int32_t)((p.p - c.n_sink) % c.block_size + 1);
   }
-  if (launch_append(p, x->ck.D, stream) != cudaSuccess) return HYB_ECUDA;
+  const cudaError_t e = launch_append(p, x->ck.D, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
   x->T += 1;
   return HYB_OK;
 }
@@ -452,6 +463,12 @@ int hyb_attn_set_timing_events(hyb_attn_ctx* x, cudaEvent_t begin, cudaEvent_t e
 }
 
 void hyb_attn_destroy(hyb_attn_ctx* x) { delete x; }
+
+const char* hyb_attn_last_cuda_error(void) {
+  static thread_local char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", cudaGetErrorName(g_last_cuda_error), cudaGetErrorString(g_last_cuda_error));
+  return buf;
+}
 
 const char* hyb_attn_strerror(int code) {
   switch (code) {

@@ -13,9 +13,9 @@ namespace hyb {
 constexpr int kTile = 64;             // tokens per attention chunk (one pipeline stage)
 constexpr int kBoxRows = 16;          // rows per TMA box
 constexpr int kStages = 4;            // attention pipeline depth
-constexpr int kConsumerGroups = 2;    // warpgroups consuming alternate stages
+constexpr int kConsumerGroups = 2;    // warp groups consuming alternate chunks
 constexpr int kWarpsPerGroup = 4;     // each consumer warp takes 16 tokens of a 64-token chunk
-constexpr int kAttendThreads = (kConsumerGroups * kWarpsPerGroup + 1) * 32;  // + 1 producer warp
+constexpr int kAttendThreads = kConsumerGroups * kWarpsPerGroup * 32;
 constexpr int kMaxAttendCtas = 1024;  // upper bound of the attention grid (sizes the workspace)
 constexpr int kScoreBlocksPerCta = 64;
 constexpr int kSelectThreads = 256;

@@ -9,10 +9,13 @@
 // partial record, and the last CTA to finish a unit (atomic ticket, no
 // spinning) merges that unit's partials with the global linear term.
 //
-// CTA: 1 producer warp + 2 consumer warpgroups of 4 warps.  The producer fills a
-// 4-stage shared-memory ring with TMA tensor loads (cp.async.bulk.tensor, 128-byte
-// swizzle, 16-row boxes, no multicast) of the chunk's K and V rows; the consumer
-// groups take alternate stages; warp w of a group handles tokens [16w, 16w+16).
+// CTA: 2 groups of 4 warps (8 warps, so two per SM sub-partition and up to 255
+// registers a thread).  A 4-stage shared-memory ring is filled with TMA tensor
+// loads (cp.async.bulk.tensor, 128-byte swizzle, 16-row boxes, no multicast) of
+// each chunk's K and V rows; group g owns the chunks of local index i = g (mod 2)
+// and hence stages g and g + 2: after its 4 warps have consumed chunk i (group
+// barrier), the group's leader thread reuses the stage for chunk i + 4.  Warp w
+// of a group handles tokens [16w, 16w+16) of a chunk.
 //
 // Per warp and 16 tokens, on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
 // accumulate), with the G <= 4 query heads of the KV group packed into the
@@ -49,7 +52,6 @@ struct AttendSmem {
   uint8_t kv[kStages][2][kTileBytes];                   // 1024-byte aligned (base aligned)
   float wpart[kConsumerGroups * kWarpsPerGroup][partial_floats(D)];
   uint64_t full[kStages];
-  uint64_t empty[kStages];
   int4 desc[kStages];                                   // start, len, is_sel, unit
   int abort_flag;
   int last_flag;
@@ -63,8 +65,8 @@ __device__ __forceinline__ uint32_t swz(int t, int C) {
   return (uint32_t)(L * 128 + (((C & 7) ^ (L & 7)) << 4));
 }
 
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+__device__ __forceinline__ void group_sync(int grp) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "n"(kWarpsPerGroup * 32) : "memory");
 }
 
 __device__ __forceinline__ int64_t cta_of_chunk(int64_t c, int64_t total, int grid) {
@@ -121,77 +123,61 @@ __device__ void merge_unit(const AttendParams& p, int unit, int64_t first, int64
   }
 }
 
+// Hand chunk i (local index within this CTA's range) to its pipeline stage:
+// write its descriptor and start the TMA loads of its K and V rows (16-row boxes;
+// rows past the chunk end are read too and ignored).  Called by one thread.
 template <int D>
-__device__ void producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttendParams& p,
-                         AttendSmem<D>& sm, int64_t c_begin, int n_local) {
+__device__ void issue_chunk(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttendParams& p,
+                            AttendSmem<D>& sm, int64_t c_begin, int i, bool& waited) {
   using S = AttendSmem<D>;
-  tma_prefetch_desc(tmK);
-  tma_prefetch_desc(tmV);
-  bool waited = false;
-  int issued = 0;  // chunks [0, issued) have been handed to the ring
+  const int64_t c = c_begin + i;
   const int cpu = p.chunks_per_unit;
-  for (int i = 0; i < n_local; ++i) {
-    const int64_t c = c_begin + i;
-    const int unit = (int)(c / cpu);
-    const int ci = (int)(c % cpu);
-    const int stage = i % kStages;
-    if (i >= kStages) {
-      if (!mbar_wait_bounded(&sm.empty[stage], ((i / kStages) - 1) & 1, kWaitLimit)) {
-        sm.abort_flag = 1;
-        atomicOr(p.status, HYB_STATUS_TIMEOUT);
-      }
+  const int unit = (int)(c / cpu);
+  const int ci = (int)(c % cpu);
+  const int stage = i % kStages;
+  int start = 0, len = 0, is_sel = 0;
+  if (ci < p.n_sink_chunks) {
+    start = ci * kTile;
+    len = min(kTile, p.sink_len - start);
+  } else if (ci < p.n_sink_chunks + p.n_win_chunks) {
+    start = p.win_start + (ci - p.n_sink_chunks) * kTile;
+    len = min(kTile, p.T - start);
+  } else {
+    if (!waited) {  // the selection is written by the preceding select kernel
+      pdl_wait_primary();
+      waited = true;
     }
-    if (*(volatile int*)&sm.abort_flag) break;
-    int start = 0, len = 0, is_sel = 0;
-    if (ci < p.n_sink_chunks) {
-      start = ci * kTile;
-      len = min(kTile, p.sink_len - start);
-    } else if (ci < p.n_sink_chunks + p.n_win_chunks) {
-      start = p.win_start + (ci - p.n_sink_chunks) * kTile;
-      len = min(kTile, p.T - start);
-    } else {
-      if (!waited) {  // the selection is written by the preceding select kernel
-        pdl_wait_primary();
-        waited = true;
-      }
-      const int s = ci - p.n_sink_chunks - p.n_win_chunks;
-      const int slot = s / p.chunks_per_block, piece = s % p.chunks_per_block;
-      is_sel = 1;
-      const int j = slot < p.k_eff ? __ldcg(p.sel + (int64_t)unit * p.top_k + slot) : -1;
-      if (j >= 0 && j < p.nb) {
-        const int bs = p.S + j * p.Bk;
-        const int be = min(bs + p.Bk, p.ev_end);
-        start = bs + piece * kTile;
-        len = max(0, min(kTile, be - start));
-      } else if (j != -1) {
-        atomicOr(p.status, HYB_STATUS_BAD_SELECTION);
-      }
+    const int s = ci - p.n_sink_chunks - p.n_win_chunks;
+    const int slot = s / p.chunks_per_block, piece = s % p.chunks_per_block;
+    is_sel = 1;
+    const int j = slot < p.k_eff ? __ldcg(p.sel + (int64_t)unit * p.top_k + slot) : -1;
+    if (j >= 0 && j < p.nb) {
+      const int bs = p.S + j * p.Bk;
+      const int be = min(bs + p.Bk, p.ev_end);
+      start = bs + piece * kTile;
+      len = max(0, min(kTile, be - start));
+    } else if (j != -1) {
+      atomicOr(p.status, HYB_STATUS_BAD_SELECTION);
     }
-    sm.desc[stage] = make_int4(start, len, is_sel, unit);
-    if (len > 0) {
-      const int nbox = (len + kBoxRows - 1) / kBoxRows;
-      mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)(nbox * S::kBoxBytes * 2));
-      const int row = (int)((int64_t)unit * p.cap + start);
-      const uint32_t kdst = smem_u32(sm.kv[stage][0]);
-      const uint32_t vdst = smem_u32(sm.kv[stage][1]);
-      for (int bx = 0; bx < nbox; ++bx) {
-        tma_load_3d(kdst + bx * S::kBoxBytes, tmK, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
-        tma_load_3d(vdst + bx * S::kBoxBytes, tmV, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
-      }
-    } else {
-      mbar_arrive(&sm.full[stage]);
-    }
-    issued = i + 1;
   }
-  if (*(volatile int*)&sm.abort_flag) {
-    // do not leave while copies into this CTA's shared memory may be in flight
-    for (int i = issued - 1; i >= 0 && i >= issued - kStages; --i)
-      mbar_wait_bounded(&sm.full[i % kStages], (i / kStages) & 1, kWaitLimit);
+  sm.desc[stage] = make_int4(start, len, is_sel, unit);
+  if (len > 0) {
+    const int nbox = (len + kBoxRows - 1) / kBoxRows;
+    mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)(nbox * S::kBoxBytes * 2));
+    const int row = (int)((int64_t)unit * p.cap + start);
+    const uint32_t kdst = smem_u32(sm.kv[stage][0]);
+    const uint32_t vdst = smem_u32(sm.kv[stage][1]);
+    for (int bx = 0; bx < nbox; ++bx) {
+      tma_load_3d(kdst + bx * S::kBoxBytes, tmK, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
+      tma_load_3d(vdst + bx * S::kBoxBytes, tmV, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
+    }
+  } else {
+    mbar_arrive(&sm.full[stage]);
   }
 }
 
 template <int D>
-__global__ void __maxnreg__(224)
+__global__ void __launch_bounds__(kAttendThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const AttendParams p) {
   constexpr int PF = partial_floats(D);
@@ -204,7 +190,7 @@ __global__ void __maxnreg__(224)
   const int cta = blockIdx.x;
 
   if (p.merge_only) {  // empty exact set: output = global linear term only
-    if (tid < kConsumerThreads) merge_unit<D>(p, cta, 0, -1, tid);
+    merge_unit<D>(p, cta, 0, -1, tid);
     return;
   }
 
@@ -212,24 +198,24 @@ __global__ void __maxnreg__(224)
   const int64_t c_end = (int64_t)(cta + 1) * p.total_chunks / p.grid;
   const int n_local = (int)(c_end - c_begin);
 
+  const int grp = warp / kWarpsPerGroup;
+  const int wi = warp % kWarpsPerGroup;
+  const bool leader = (wi == 0 && lane == 0);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kWarpsPerGroup);
-    }
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-
-  if (warp == kConsumerGroups * kWarpsPerGroup) {
-    if (lane == 0) producer<D>(&tmK, &tmV, p, sm, c_begin, n_local);
-    return;
+  bool waited = false;       // leader: has waited for the select kernel
+  int next_issue = grp;      // leader: next local chunk index of this group to issue
+  if (leader) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    for (; next_issue < n_local && next_issue < kStages; next_issue += kConsumerGroups)
+      issue_chunk<D>(&tmK, &tmV, p, sm, c_begin, next_issue, waited);
   }
 
-  // ---------------------------------------------------------------- consumers
-  const int grp = warp / kWarpsPerGroup;
-  const int wi = warp % kWarpsPerGroup;
   const int g = lane >> 2, tig = lane & 3;
   const bool p_lane = g < 4;           // rows 0-3: softmax part; rows 4-7: Taylor part
   const int head = g & 3;
@@ -258,8 +244,8 @@ __global__ void __maxnreg__(224)
     for (int n = 0; n < NT8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
     float m_run = -INFINITY, l_run = 0.f, dsel_run = 0.f;
 
-    for (int64_t cc = c + grp; cc < seg_end; cc += kConsumerGroups) {
-      const int i = (int)(cc - c_begin);
+    const int i_seg = (int)(c - c_begin);
+    for (int i = i_seg + ((i_seg & 1) != grp ? 1 : 0); c_begin + i < seg_end; i += kConsumerGroups) {
       const int stage = i % kStages;
       bool ok = !*(volatile int*)&sm.abort_flag;
       if (ok && !mbar_wait_bounded(&sm.full[stage], (i / kStages) & 1, kWaitLimit)) {
@@ -342,8 +328,11 @@ __global__ void __maxnreg__(224)
           mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2, b3);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[stage]);
+      group_sync(grp);  // the group is done with this stage
+      if (leader && next_issue < n_local && !*(volatile int*)&sm.abort_flag) {
+        issue_chunk<D>(&tmK, &tmV, p, sm, c_begin, next_issue, waited);
+        next_issue += kConsumerGroups;
+      }
     }
 
     // ---- this warp's partial -> shared memory
@@ -368,7 +357,7 @@ __global__ void __maxnreg__(224)
         dst[n * 8 + 2 * tig + 1] = O[n][1] + O[n][3];
       }
     }
-    consumer_sync();
+    __syncthreads();
     // ---- combine the 8 warps -> one partial record for (cta, unit)
     {
       constexpr int NW = kConsumerGroups * kWarpsPerGroup;
@@ -403,21 +392,26 @@ __global__ void __maxnreg__(224)
       }
       __threadfence();
     }
-    consumer_sync();
+    __syncthreads();
     const int64_t first = cta_of_chunk((int64_t)unit * cpu, p.total_chunks, p.grid);
     const int64_t last = cta_of_chunk((int64_t)(unit + 1) * cpu - 1, p.total_chunks, p.grid);
     if (tid == 0) {
       const uint32_t prev = atomicAdd(&p.tickets[unit], 1u);
       sm.last_flag = (prev == (uint32_t)(last - first));
     }
-    consumer_sync();
+    __syncthreads();
     if (sm.last_flag) {
       __threadfence();
       merge_unit<D>(p, unit, first, last, tid);
       if (tid == 0) p.tickets[unit] = 0u;
     }
-    consumer_sync();
+    __syncthreads();
     c = seg_end;
+  }
+  if (leader && *(volatile int*)&sm.abort_flag) {
+    // do not leave while copies into this CTA's shared memory may be in flight
+    for (int i = next_issue - kConsumerGroups; i >= 0 && i >= next_issue - kStages; i -= kConsumerGroups)
+      mbar_wait_bounded(&sm.full[i % kStages], (i / kStages) & 1, kWaitLimit);
   }
 }
 

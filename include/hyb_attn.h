@@ -220,6 +220,10 @@ int hyb_attn_set_timing_events(hyb_attn_ctx* ctx, cudaEvent_t begin, cudaEvent_t
 /* Release the host context (device buffers stay with the caller). */
 void hyb_attn_destroy(hyb_attn_ctx* ctx);
 
+/* Name and description of the last CUDA error that made a call on this thread
+ * return HYB_ECUDA ("cudaSuccess: no error" if none).  Host only. */
+const char* hyb_attn_last_cuda_error(void);
+
 /* Static description of a return code. */
 const char* hyb_attn_strerror(int code);
 
