@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's layer count (smaller instances for profiling)")
     return ap.parse_args()
 
 
@@ -124,13 +126,13 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- native arm
 
 class Bench:
-    def __init__(self, w, steps, warmup, device):
+    def __init__(self, w, n_steps, device):
         import torch
         import syngen.device as SD
         from syngen import host as SH
         from hybrid_sparse_linear_decode_b200 import HybridAttentionLayer, make_config
         self.w, self.device = w, device
-        self.n_steps = warmup + steps + 1
+        self.n_steps = n_steps
         n_app = self.n_steps
         cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window,
                           w.top_k, w.T0 + n_app)
@@ -178,9 +180,11 @@ def run_native(args, rank, world):
     from syngen import configs as C
     torch.cuda.set_device(rank % torch.cuda.device_count())
     device = torch.device("cuda", torch.cuda.current_device())
-    w = C.get_workload(args.workload)
+    w = C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {}))
     K, Wm = args.steps, args.warmup
-    b = Bench(w, K, Wm, device)
+    Kk = min(K, 20)                      # steps of the attention-kernel timing pass
+    Ke = 0 if args.no_e2e else min(K, 20)  # steps of the end-to-end pass
+    b = Bench(w, Wm + K + Kk + Ke, device)
     T_mid = w.T0 + Wm + K // 2
     dec_b, app_b, att_b = algorithmic_bytes(w, T_mid)
     units = w.layers * w.units_per_layer
@@ -236,7 +240,6 @@ def run_native(args, rank, world):
     # ---- attention-kernel timing (events around the attention launch of every layer)
     ka, kb_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kern_ms, n_kern = 0.0, 0
-    Kk = min(K, 20)
     pool = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in b.layers]
             for _ in range(Kk)]
     for i in range(Kk):
@@ -264,7 +267,6 @@ def run_native(args, rank, world):
     # ---- e2e through the host-buffer entry point (pinned host q / k / v / out)
     e2e = None
     if not args.no_e2e:
-        Ke = min(K, 20)
         qh = [[t.cpu().pin_memory() for t in qs] for qs in b.q]
         kh = [t.cpu().pin_memory() for t in b.app_k]
         vh = [t.cpu().pin_memory() for t in b.app_v]

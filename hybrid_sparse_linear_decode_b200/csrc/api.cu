@@ -99,11 +99,15 @@ Geometry geometry(const hyb_attn_config& c, int64_t T) {
   return g;
 }
 
-int attend_grid(int64_t total_chunks, int n_sm) {
-  int64_t g = total_chunks;
-  if (g > n_sm) g = n_sm;
-  if (g > kMaxAttendCtas) g = kMaxAttendCtas;
-  return (int)(g < 1 ? 1 : g);
+// CTAs per unit for the attention kernel: enough to fill kAttendCtasPerSm CTAs
+// on every SM in one wave, never more than the unit's chunks.
+int attend_splits(int units, int chunks_per_unit, int n_sm) {
+  if (chunks_per_unit <= 0) return 0;
+  int64_t s = (int64_t)n_sm * kAttendCtasPerSm / units;
+  if (s < 1) s = 1;
+  if (s > chunks_per_unit) s = chunks_per_unit;
+  if (s * units > kMaxAttendCtas + units) s = 1;
+  return (int)s;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -133,14 +137,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// KV cache viewed as [rows = B*Hkv*capacity][D/64][64] bf16; a box is 16 rows x
-// D columns, swizzled 128 B.
-bool make_kv_map(CUtensorMap* m, void* base, int64_t rows, int D) {
+// KV cache viewed as [rows = B*Hkv*capacity][D/64][64] bf16; a box is
+// `box_rows` rows x D columns, swizzled 128 B.
+bool make_kv_map(CUtensorMap* m, void* base, int64_t rows, int D, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)(D / 64), (cuuint64_t)rows};
   cuuint64_t strides[2] = {128, (cuuint64_t)D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)(D / 64), (cuuint32_t)kBoxRows};
+  cuuint32_t box[3] = {64, (cuuint32_t)(D / 64), (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -166,7 +170,7 @@ struct hyb_attn_ctx {
   int64_t T;
   int device, n_sm;
   float scale;
-  CUtensorMap tmK, tmV;
+  CUtensorMap maps[4];  // K, V with 64-row boxes; K, V with 16-row boxes
   cudaEvent_t ev_begin, ev_end;
   template <class P>
   P* w(size_t off) const {
@@ -225,7 +229,6 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   ap.status = sp.status;
   ap.out = out;
   ap.cap = c.capacity;
-  ap.total_chunks = (int64_t)k.units * g.chunks_per_unit;
   ap.T = (int32_t)g.T;
   ap.S = c.n_sink;
   ap.Bk = c.block_size;
@@ -242,11 +245,12 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   ap.units = k.units;
   ap.G = k.G;
   ap.merge_only = g.chunks_per_unit == 0 ? 1 : 0;
-  ap.grid = ap.merge_only ? k.units : attend_grid(ap.total_chunks, x->n_sm);
+  ap.splits = attend_splits(k.units, g.chunks_per_unit, x->n_sm);
+  ap.grid = ap.merge_only ? k.units : k.units * ap.splits;
   ap.scale = x->scale;
   const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
   if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
-  e = launch_attend(&x->tmK, &x->tmV, ap, k.D, /*pdl=*/!timed, stream);
+  e = launch_attend(x->maps, ap, k.D, /*pdl=*/!timed, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
   return HYB_OK;
@@ -288,9 +292,9 @@ int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_
   out->k_eff = g.k_eff;
   out->exact_tokens = g.sink_len + (T - g.win_start) + g.k_eff * cfg->block_size;
   out->chunks_per_unit = g.chunks_per_unit;
-  const int64_t total = (int64_t)k.units * g.chunks_per_unit;
-  out->attend_ctas = total == 0 ? k.units : attend_grid(total, n_sm);
-  out->partial_slots = total == 0 ? 0 : out->attend_ctas + k.units - 1;
+  const int splits = attend_splits(k.units, g.chunks_per_unit, n_sm);
+  out->attend_ctas = g.chunks_per_unit == 0 ? k.units : k.units * splits;
+  out->partial_slots = g.chunks_per_unit == 0 ? 0 : k.units * splits;
   out->score_ctas_per_unit = g.nb > 0 ? (int32_t)ceil_div(g.nb, kScoreBlocksPerCta) : 0;
   out->linear_ctas_per_unit = k.D / 32;
   return HYB_OK;
@@ -331,11 +335,16 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   x->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)k.D);
   x->ev_begin = x->ev_end = nullptr;
   const int64_t rows = (int64_t)k.units * cfg->capacity;
-  if (!make_kv_map(&x->tmK, buf->k_cache, rows, k.D) || !make_kv_map(&x->tmV, buf->v_cache, rows, k.D)) {
+  if (!make_kv_map(&x->maps[0], buf->k_cache, rows, k.D, kTile) ||
+      !make_kv_map(&x->maps[1], buf->v_cache, rows, k.D, kTile) ||
+      !make_kv_map(&x->maps[2], buf->k_cache, rows, k.D, kBoxRows) ||
+      !make_kv_map(&x->maps[3], buf->v_cache, rows, k.D, kBoxRows)) {
     delete x;
     return HYB_ECUDA;
   }
-  const cudaError_t pe = prepare_attend(k.D);
+  cudaError_t pe = prepare_attend(k.D);
+  if (pe == cudaSuccess) pe = prepare_select(k.D);
+  if (pe == cudaSuccess) pe = prepare_state(k.D);
   if (pe != cudaSuccess) {
     delete x;
     return cuda_fail(pe);

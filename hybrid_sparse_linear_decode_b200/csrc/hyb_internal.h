@@ -12,13 +12,13 @@ namespace hyb {
 
 constexpr int kTile = 64;             // tokens per attention chunk (one pipeline stage)
 constexpr int kBoxRows = 16;          // rows per TMA box
-constexpr int kStages = 4;            // attention pipeline depth
-constexpr int kConsumerGroups = 2;    // warp groups consuming alternate chunks
-constexpr int kWarpsPerGroup = 4;     // each consumer warp takes 16 tokens of a 64-token chunk
-constexpr int kAttendThreads = kConsumerGroups * kWarpsPerGroup * 32;
+constexpr int kStages = 3;            // attention pipeline depth per CTA
+constexpr int kAttendThreads = 128;   // 4 warps; warp w takes tokens [16w, 16w+16) of a chunk
+constexpr int kAttendCtasPerSm = 2;
 constexpr int kMaxAttendCtas = 1024;  // upper bound of the attention grid (sizes the workspace)
 constexpr int kScoreBlocksPerCta = 64;
 constexpr int kSelectThreads = 256;
+constexpr int kSelCache = 64;         // selection entries a warp group caches in shared memory
 constexpr int kMaxGroup = 4;          // query heads per KV head supported by the attention kernel
 constexpr uint64_t kWaitLimit = 1000000000ull;  // ns: a kernel-internal wait gives up after ~1 s
 
@@ -65,11 +65,11 @@ struct AttendParams {
   uint32_t* status;
   float* out;                 // [B][Hq][D]
   int64_t cap;                // cache rows per unit
-  int64_t total_chunks;
   int32_t T, S, Bk, top_k, nb, k_eff;
   int32_t sink_len, win_start, ev_end;
   int32_t n_sink_chunks, n_win_chunks, chunks_per_block, chunks_per_unit;
   int32_t units, G, grid;
+  int32_t splits;             // CTAs per unit; CTA x works on unit x / splits
   int32_t merge_only;         // no exact tokens at all: each CTA merges one unit
   float scale;
 };
@@ -99,11 +99,14 @@ struct InitParams {
 
 // Launchers (kernels live in the .cu files); return cudaError_t of the launch.
 cudaError_t launch_select(const SelectParams& p, int D, int grid_x, cudaStream_t s);
-cudaError_t launch_attend(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttendParams& p, int D,
-                          bool pdl, cudaStream_t s);
+// maps: K and V with 64-row boxes, then K and V with 16-row boxes
+cudaError_t launch_attend(const CUtensorMap* maps, const AttendParams& p, int D, bool pdl, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s);
 cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s);
 size_t attend_smem_bytes(int D);
-cudaError_t prepare_attend(int D);  // per device, before the first attention launch
+// per device, before the first launch: shared-memory size and carveout attributes
+cudaError_t prepare_attend(int D);
+cudaError_t prepare_select(int D);
+cudaError_t prepare_state(int D);
 
 }  // namespace hyb

@@ -4,18 +4,19 @@
 //
 // Work: each unit (batch row, KV head) owns a fixed list of <= 64-token chunks
 // of its exact set X (sink pieces, window pieces, then ceil(Bk/64) pieces per
-// selected block).  The units' lists are concatenated and cut into `grid`
-// contiguous ranges, one per CTA (split-K); every (CTA, unit) pair writes one
-// partial record, and the last CTA to finish a unit (atomic ticket, no
-// spinning) merges that unit's partials with the global linear term.
+// selected block).  A unit's chunks are dealt to `splits` CTAs, CTA part p
+// taking chunks p, p + splits, p + 2*splits, ... (split-K), so every CTA works
+// on one unit, gets a mix of window and selected chunks, and meets the
+// selection (written by the preceding select kernel) as late as possible.
+// Each CTA writes one partial record; the last CTA of a unit to finish (atomic
+// ticket, no spinning) merges the unit's partials with the global linear term.
 //
-// CTA: 2 groups of 4 warps (8 warps, so two per SM sub-partition and up to 255
-// registers a thread).  A 4-stage shared-memory ring is filled with TMA tensor
-// loads (cp.async.bulk.tensor, 128-byte swizzle, 16-row boxes, no multicast) of
-// each chunk's K and V rows; group g owns the chunks of local index i = g (mod 2)
-// and hence stages g and g + 2: after its 4 warps have consumed chunk i (group
-// barrier), the group's leader thread reuses the stage for chunk i + 4.  Warp w
-// of a group handles tokens [16w, 16w+16) of a chunk.
+// CTA: 4 warps, two CTAs per SM.  A 3-stage shared-memory ring is filled with
+// TMA tensor loads (cp.async.bulk.tensor, 128-byte swizzle, no multicast): a
+// full 64-token chunk as one 64-row box per tensor, a ragged chunk (sinks, the
+// window's tail, a partial block) as the 16-row boxes it touches.  After the 4
+// warps have consumed chunk j (CTA barrier) thread 0 refills the stage with
+// chunk j + 3.  Warp w handles tokens [16w, 16w + 16) of a chunk.
 //
 // Per warp and 16 tokens, on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
 // accumulate), with the G <= 4 query heads of the KV group packed into the
@@ -32,6 +33,11 @@
 // for Long Context Modeling", Abstract: residual = global - selected; "SLAKE",
 // Abstract: first-order Taylor exp(s) ~ 1 + s).
 //
+// Launch chaining: this kernel is launched programmatically after the select
+// kernel; it waits for it (griddepcontrol.wait) before reading the selection or
+// the linear term, and lets its own dependents (the append kernel) start once
+// the select kernel has completed -- the append touches nothing this kernel reads.
+//
 // Merge of a unit (per query head, base-2 exponent m of the exact part):
 //   o = (N_ex + 2^{-m} (N_glob - N_sel)) / (D_ex + 2^{-m} (D_glob - D_sel)),
 // evaluated as the equal form (N_ex 2^m + ...)/(D_ex 2^m + ...) when m < 0.
@@ -43,16 +49,25 @@ namespace hyb {
 namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
-constexpr int kConsumerThreads = kConsumerGroups * kWarpsPerGroup * 32;
+
+struct KVMaps {  // the same KV caches seen with 64-row and 16-row TMA boxes
+  CUtensorMap k64, v64, k16, v16;
+};
 
 template <int D>
 struct AttendSmem {
-  static constexpr int kTileBytes = kTile * D * 2;      // one of K or V for 64 tokens
+  static constexpr int kTileBytes = kTile * D * 2;  // one of K or V for 64 tokens
   static constexpr int kBoxBytes = kBoxRows * D * 2;
-  uint8_t kv[kStages][2][kTileBytes];                   // 1024-byte aligned (base aligned)
-  float wpart[kConsumerGroups * kWarpsPerGroup][partial_floats(D)];
+  uint8_t kv[kStages][2][kTileBytes];               // 1024-byte aligned (base aligned)
+  float wpart[2][partial_floats(D)];                // combine slots (contiguous after kv: the
+                                                    // merge stages partial records over both)
+  float mscr[16];                                   // merge: per-head max, D_ex, D_sel
+  float fscr[4 * 64];                               // merge: per-slot, per-head rescale factors
   uint64_t full[kStages];
-  int4 desc[kStages];                                   // start, len, is_sel, unit
+  uint64_t merge_bar;
+  int4 desc[kStages];                               // start, len, is_sel, unit
+  int32_t sel_cache[kSelCache];                     // the unit's selection row
+  int sel_loaded;
   int abort_flag;
   int last_flag;
 };
@@ -65,14 +80,6 @@ __device__ __forceinline__ uint32_t swz(int t, int C) {
   return (uint32_t)(L * 128 + (((C & 7) ^ (L & 7)) << 4));
 }
 
-__device__ __forceinline__ void group_sync(int grp) {
-  asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "n"(kWarpsPerGroup * 32) : "memory");
-}
-
-__device__ __forceinline__ int64_t cta_of_chunk(int64_t c, int64_t total, int grid) {
-  return ((c + 1) * grid - 1) / total;
-}
-
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   const float2 hf = __bfloat1622float2(h);
@@ -81,29 +88,98 @@ __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint3
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Merge the partial records of `unit` written by CTAs [first, last] (slot =
-// cta + unit) with the global linear term; consumer threads only.
+// Merge the `nslot` partial records [slot0, slot0 + nslot) of `unit` with the
+// global linear term and write the unit's output.  All threads of the CTA, after
+// its own chunks are done (the stage buffers are free).  The unit's records are
+// contiguous in the workspace: thread 0 pulls up to kMergeSlots of them into
+// shared memory with one bulk copy, then the reductions run from shared memory.
 template <int D>
-__device__ void merge_unit(const AttendParams& p, int unit, int64_t first, int64_t last, int ctid) {
+__device__ void merge_unit(const AttendParams& p, int unit, int64_t slot0, int nslot, int tid, AttendSmem<D>& sm) {
   constexpr int PF = partial_floats(D);
+  constexpr int CAP = (int)((sizeof(sm.kv) + sizeof(sm.wpart)) / (PF * sizeof(float)));
+  static_assert(CAP >= 1 && CAP <= 64, "merge staging capacity");
+  constexpr int NV = 2 * D;  // float4 columns of [acc | nsel]
+  constexpr int VPT = (NV + kAttendThreads - 1) / kAttendThreads;
+  float* rec = reinterpret_cast<float*>(&sm.kv[0][0][0]);  // staged records, then the column sums
+  float* s_M = sm.mscr;
+  float* s_Dex = sm.mscr + 4;
+  float* s_Dsel = sm.mscr + 8;
+  const int warp = tid >> 5, lane = tid & 31;
+  const float* base = p.partials + slot0 * PF;
   pdl_wait_primary();  // the linear term comes from the preceding select kernel
+  {                    // warp h: max of head h over all slots
+    float mx = -INFINITY;
+    for (int k = lane; k < nslot; k += 32) mx = fmaxf(mx, __ldcg(base + (int64_t)k * PF + warp));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    if (lane == 0) s_M[warp] = (mx == -INFINITY) ? 0.f : mx;
+  }
+  float4 vacc[VPT];
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) vacc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float dex = 0.f, dsel = 0.f;
+  for (int kb = 0, batch = 0; kb < nslot; kb += CAP, ++batch) {
+    const int nb = min(CAP, nslot - kb);
+    __syncthreads();  // previous batch consumed; s_M visible
+    if (tid == 0) {
+      // the records were written by other CTAs' generic-proxy stores (ordered by
+      // the ticket); order them before this async-proxy read
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      const uint32_t bytes = (uint32_t)(nb * PF * sizeof(float));
+      mbar_arrive_expect_tx(&sm.merge_bar, bytes);
+      bulk_load(smem_u32(rec), base + (int64_t)kb * PF, bytes, &sm.merge_bar);
+    }
+    if (!mbar_wait_bounded(&sm.merge_bar, batch & 1, kWaitLimit))
+      atomicOr(p.status, HYB_STATUS_TIMEOUT);  // keep the barrier sequence; the output is flagged
+    for (int e = tid; e < 4 * nb; e += kAttendThreads) {
+      const float m = rec[(e >> 2) * PF + (e & 3)];
+      sm.fscr[e] = (m == -INFINITY) ? 0.f : exp2f(m - s_M[e & 3]);
+    }
+    __syncthreads();
+    for (int k = lane; k < nb; k += 32) {  // warp h accumulates head h
+      dex += rec[k * PF + 4 + warp] * sm.fscr[4 * k + warp];
+      dsel += rec[k * PF + 8 + warp];
+    }
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int v = tid + u * kAttendThreads;
+      if (v < NV) {
+        const int vh = (4 * v) / D;  // head of an acc column (v < D)
+        for (int k = 0; k < nb; ++k) {
+          const float4 x = *reinterpret_cast<const float4*>(rec + k * PF + 16 + 4 * v);
+          const float f = (v < D) ? sm.fscr[4 * k + vh] : 1.f;
+          vacc[u].x += x.x * f;
+          vacc[u].y += x.y * f;
+          vacc[u].z += x.z * f;
+          vacc[u].w += x.w * f;
+        }
+      }
+    }
+  }
+  __syncthreads();  // the staging area is free again
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    dex += __shfl_xor_sync(kFull, dex, o);
+    dsel += __shfl_xor_sync(kFull, dsel, o);
+  }
+  if (lane == 0) {
+    s_Dex[warp] = dex;
+    s_Dsel[warp] = dsel;
+  }
+  float* s_vec = rec;  // [8 D] column sums
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int v = tid + u * kAttendThreads;
+    if (v < NV) *reinterpret_cast<float4*>(s_vec + 4 * v) = vacc[u];
+  }
+  __syncthreads();
   const int G = p.G;
   const float* lin = p.lin + (int64_t)unit * G * (D + 1);
-  for (int e = ctid; e < G * D; e += kConsumerThreads) {
+  for (int e = tid; e < G * D; e += kAttendThreads) {
     const int i = e / D, d = e % D;
-    float M = -INFINITY;
-    for (int64_t c = first; c <= last; ++c) M = fmaxf(M, __ldcg(p.partials + (c + unit) * PF + i));
-    const float Ms = (M == -INFINITY) ? 0.f : M;
-    float Dex = 0.f, Nex = 0.f, Dsel = 0.f, Nsel = 0.f;
-    for (int64_t c = first; c <= last; ++c) {
-      const float* gp = p.partials + (c + unit) * PF;
-      const float m = __ldcg(gp + i);
-      const float f = (m == -INFINITY) ? 0.f : exp2f(m - Ms);
-      Dex += __ldcg(gp + 4 + i) * f;
-      Dsel += __ldcg(gp + 8 + i);
-      Nex += __ldcg(gp + 16 + i * D + d) * f;
-      Nsel += __ldcg(gp + 16 + 4 * D + i * D + d);
-    }
+    const float Ms = s_M[i];
+    const float Nex = s_vec[i * D + d], Nsel = s_vec[4 * D + i * D + d];
+    const float Dex = s_Dex[i], Dsel = s_Dsel[i];
     const float Ng = __ldcg(lin + (int64_t)i * (D + 1) + d);
     const float Dg = __ldcg(lin + (int64_t)i * (D + 1) + D);
     float num, den;
@@ -123,18 +199,14 @@ __device__ void merge_unit(const AttendParams& p, int unit, int64_t first, int64
   }
 }
 
-// Hand chunk i (local index within this CTA's range) to its pipeline stage:
-// write its descriptor and start the TMA loads of its K and V rows (16-row boxes;
-// rows past the chunk end are read too and ignored).  Called by one thread.
+// Hand local chunk j (unit chunk index ci) to stage j % kStages: write its
+// descriptor and start the TMA loads of its K and V rows (rows past the chunk
+// end inside a box are read too and ignored).  Called by thread 0 only.
 template <int D>
-__device__ void issue_chunk(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttendParams& p,
-                            AttendSmem<D>& sm, int64_t c_begin, int i, bool& waited) {
+__device__ void issue_chunk(const KVMaps* tm, const AttendParams& p, AttendSmem<D>& sm, int unit, int ci, int j,
+                            bool& waited) {
   using S = AttendSmem<D>;
-  const int64_t c = c_begin + i;
-  const int cpu = p.chunks_per_unit;
-  const int unit = (int)(c / cpu);
-  const int ci = (int)(c % cpu);
-  const int stage = i % kStages;
+  const int stage = j % kStages;
   int start = 0, len = 0, is_sel = 0;
   if (ci < p.n_sink_chunks) {
     start = ci * kTile;
@@ -145,31 +217,56 @@ __device__ void issue_chunk(const CUtensorMap* tmK, const CUtensorMap* tmV, cons
   } else {
     if (!waited) {  // the selection is written by the preceding select kernel
       pdl_wait_primary();
+      pdl_allow_dependents();  // the select kernel is complete: the append may run
       waited = true;
     }
     const int s = ci - p.n_sink_chunks - p.n_win_chunks;
     const int slot = s / p.chunks_per_block, piece = s % p.chunks_per_block;
     is_sel = 1;
-    const int j = slot < p.k_eff ? __ldcg(p.sel + (int64_t)unit * p.top_k + slot) : -1;
-    if (j >= 0 && j < p.nb) {
-      const int bs = p.S + j * p.Bk;
+    int jb = -1;
+    if (slot < p.k_eff) {
+      const int32_t* row = p.sel + (int64_t)unit * p.top_k;
+      if (p.top_k <= kSelCache) {  // one round trip for the whole row, then shared memory
+        if (!sm.sel_loaded) {
+          for (int t0 = 0; t0 < p.top_k; t0 += 16) {
+            int32_t v[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) v[t] = t0 + t < p.top_k ? __ldcg(row + t0 + t) : -1;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) sm.sel_cache[(t0 + t) & (kSelCache - 1)] = v[t];
+          }
+          sm.sel_loaded = 1;
+        }
+        jb = sm.sel_cache[slot];
+      } else {
+        jb = __ldcg(row + slot);
+      }
+    }
+    if (jb >= 0 && jb < p.nb) {
+      const int bs = p.S + jb * p.Bk;
       const int be = min(bs + p.Bk, p.ev_end);
       start = bs + piece * kTile;
       len = max(0, min(kTile, be - start));
-    } else if (j != -1) {
+    } else if (jb != -1) {
       atomicOr(p.status, HYB_STATUS_BAD_SELECTION);
     }
   }
   sm.desc[stage] = make_int4(start, len, is_sel, unit);
   if (len > 0) {
-    const int nbox = (len + kBoxRows - 1) / kBoxRows;
-    mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)(nbox * S::kBoxBytes * 2));
     const int row = (int)((int64_t)unit * p.cap + start);
     const uint32_t kdst = smem_u32(sm.kv[stage][0]);
     const uint32_t vdst = smem_u32(sm.kv[stage][1]);
-    for (int bx = 0; bx < nbox; ++bx) {
-      tma_load_3d(kdst + bx * S::kBoxBytes, tmK, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
-      tma_load_3d(vdst + bx * S::kBoxBytes, tmV, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
+    if (len == kTile) {  // full chunk: one 64-row box per tensor
+      mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)(2 * S::kTileBytes));
+      tma_load_3d(kdst, &tm->k64, 0, 0, row, &sm.full[stage]);
+      tma_load_3d(vdst, &tm->v64, 0, 0, row, &sm.full[stage]);
+    } else {             // ragged chunk: only the 16-row boxes it touches
+      const int nbox = (len + kBoxRows - 1) / kBoxRows;
+      mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)(nbox * S::kBoxBytes * 2));
+      for (int bx = 0; bx < nbox; ++bx) {
+        tma_load_3d(kdst + bx * S::kBoxBytes, &tm->k16, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
+        tma_load_3d(vdst + bx * S::kBoxBytes, &tm->v16, 0, 0, row + bx * kBoxRows, &sm.full[stage]);
+      }
     }
   } else {
     mbar_arrive(&sm.full[stage]);
@@ -177,9 +274,8 @@ __device__ void issue_chunk(const CUtensorMap* tmK, const CUtensorMap* tmV, cons
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttendThreads, 1)
-    attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const AttendParams p) {
+__global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm)
+    attend_kernel(const __grid_constant__ KVMaps tm, const AttendParams p) {
   constexpr int PF = partial_floats(D);
   constexpr int NT8 = D / 8;   // 8-column tiles of the head dimension
   constexpr int KS = D / 16;   // k-steps of the QK product
@@ -189,261 +285,251 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
 
-  if (p.merge_only) {  // empty exact set: output = global linear term only
-    merge_unit<D>(p, cta, 0, -1, tid);
-    return;
-  }
-
-  const int64_t c_begin = (int64_t)cta * p.total_chunks / p.grid;
-  const int64_t c_end = (int64_t)(cta + 1) * p.total_chunks / p.grid;
-  const int n_local = (int)(c_end - c_begin);
-
-  const int grp = warp / kWarpsPerGroup;
-  const int wi = warp % kWarpsPerGroup;
-  const bool leader = (wi == 0 && lane == 0);
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
+    mbar_init(&sm.merge_bar, 1);
+    sm.sel_loaded = 0;
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  bool waited = false;       // leader: has waited for the select kernel
-  int next_issue = grp;      // leader: next local chunk index of this group to issue
-  if (leader) {
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-    for (; next_issue < n_local && next_issue < kStages; next_issue += kConsumerGroups)
-      issue_chunk<D>(&tmK, &tmV, p, sm, c_begin, next_issue, waited);
+  if (p.merge_only) {  // empty exact set: output = global linear term only
+    merge_unit<D>(p, cta, 0, 0, tid, sm);
+    if (tid == 0) pdl_allow_dependents();
+    return;
+  }
+  const int unit = cta / p.splits, part = cta % p.splits;
+  const int n_local = (p.chunks_per_unit - part + p.splits - 1) / p.splits;  // chunks part + j*splits
+
+  bool waited = false;  // thread 0: has waited for the select kernel
+  int next_issue = 0;   // thread 0: next local chunk to issue
+  if (tid == 0) {
+    tma_prefetch_desc(&tm.k64);
+    tma_prefetch_desc(&tm.v64);
+    for (; next_issue < n_local && next_issue < kStages; ++next_issue)
+      issue_chunk<D>(&tm, p, sm, unit, part + next_issue * p.splits, next_issue, waited);
   }
 
   const int g = lane >> 2, tig = lane & 3;
-  const bool p_lane = g < 4;           // rows 0-3: softmax part; rows 4-7: Taylor part
+  const bool p_lane = g < 4;  // rows 0-3: softmax part; rows 4-7: Taylor part
   const int head = g & 3;
   const bool head_ok = head < p.G;
-  const int cpu = p.chunks_per_unit;
-  const int r0 = wi * 16;
+  const int r0 = warp * 16;
   const int mi = lane >> 3, rr = lane & 7;
 
-  int64_t c = c_begin;
-  while (c < c_end) {
-    const int unit = (int)(c / cpu);
-    const int64_t seg_end = min(c_end, (int64_t)(unit + 1) * cpu);
+  uint32_t qa[KS][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (head_ok ? head : 0)) * D);
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = head_ok ? __ldg(qrow + kk * 8 + tig) : 0u;
+      qa[kk][1] = head_ok ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
+    }
+  }
+  float O[NT8][4];
+#pragma unroll
+  for (int n = 0; n < NT8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f, dsel_run = 0.f;
 
-    uint32_t qa[KS][2];
-    {
-      const uint32_t* qrow =
-          reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (head_ok ? head : 0)) * D);
+  for (int j = 0; j < n_local; ++j) {
+    const int stage = j % kStages;
+    bool ok = !*(volatile int*)&sm.abort_flag;
+    if (ok && !mbar_wait_bounded(&sm.full[stage], (j / kStages) & 1, kWaitLimit)) {
+      sm.abort_flag = 1;
+      atomicOr(p.status, HYB_STATUS_TIMEOUT);
+      ok = false;
+    }
+    const int4 dsc = sm.desc[stage];
+    const int nvalid = ok ? min(16, dsc.y - r0) : 0;
+    if (nvalid > 0) {
+      const uint32_t kb = smem_u32(sm.kv[stage][0]);
+      const uint32_t vb = smem_u32(sm.kv[stage][1]);
+      if (nvalid < 16) {
+        // rows past the chunk may hold tokens beyond T (unwritten cache rows):
+        // zero their V rows so that 0-weight * garbage cannot make a NaN
+        constexpr int CPR = D / 8;  // 16-byte chunks per row
+        for (int e = lane; e < (16 - nvalid) * CPR; e += 32) {
+          const int t = r0 + nvalid + e / CPR;
+          *reinterpret_cast<uint4*>(&sm.kv[stage][1][swz<D>(t, e % CPR)]) = make_uint4(0, 0, 0, 0);
+        }
+        // order these generic-proxy writes before the next TMA write of the stage
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
+      // ---- S^T = Qpad K^T for 16 tokens (two 8-token n-tiles)
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
-        qa[kk][0] = head_ok ? __ldg(qrow + kk * 8 + tig) : 0u;
-        qa[kk][1] = head_ok ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + swz<D>(r0 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)), b0, b1, b2, b3);
+        mma_16816(sacc[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+        mma_16816(sacc[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+      }
+      // ---- weights of this lane's 4 tokens: n-tile nt, element e -> token nt*8 + 2*tig + e
+      float s[4], x[4];
+      bool v[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int nt = q4 >> 1, e = q4 & 1;
+        v[q4] = (nt * 8 + 2 * tig + e) < nvalid;
+        s[q4] = sacc[nt][e] * p.scale;
+        x[q4] = (p_lane && v[q4]) ? s[q4] * kLog2e : -INFINITY;
+      }
+      float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
+      const float m_new = fmaxf(m_run, tmax);
+      const float alpha = (p_lane && m_new != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+      const bool sel_tok = dsc.z != 0;
+      float w[4], wsum = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        w[q4] = p_lane ? (v[q4] ? exp2f(x[q4] - m_new) : 0.f) : ((v[q4] && sel_tok) ? 1.f + s[q4] : 0.f);
+        wsum += w[q4];
+      }
+      if (p_lane) {
+        l_run = l_run * alpha + wsum;
+        m_run = m_new;
+      } else {
+        dsel_run += wsum;
+      }
+      if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+        for (int n = 0; n < NT8; ++n) {
+          O[n][0] *= alpha;
+          O[n][1] *= alpha;
+          O[n][2] *= alpha;
+          O[n][3] *= alpha;
+        }
+      }
+      uint32_t a0, a1, a2, a3;  // rows g (hi) / g+8 (lo), tokens 0-7 / 8-15 of the k=16 step
+      split_bf16(w[0], w[1], a0, a1);
+      split_bf16(w[2], w[3], a2, a3);
+      // ---- O += A V over 16 tokens
+#pragma unroll
+      for (int np = 0; np < NT8 / 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + swz<D>(r0 + (mi & 1) * 8 + rr, np * 2 + (mi >> 1)), b0, b1, b2, b3);
+        mma_16816(O[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-    float O[NT8][4];
-#pragma unroll
-    for (int n = 0; n < NT8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f, dsel_run = 0.f;
-
-    const int i_seg = (int)(c - c_begin);
-    for (int i = i_seg + ((i_seg & 1) != grp ? 1 : 0); c_begin + i < seg_end; i += kConsumerGroups) {
-      const int stage = i % kStages;
-      bool ok = !*(volatile int*)&sm.abort_flag;
-      if (ok && !mbar_wait_bounded(&sm.full[stage], (i / kStages) & 1, kWaitLimit)) {
-        sm.abort_flag = 1;
-        atomicOr(p.status, HYB_STATUS_TIMEOUT);
-        ok = false;
-      }
-      const int4 dsc = sm.desc[stage];
-      const int nvalid = ok ? min(16, dsc.y - r0) : 0;
-      if (nvalid > 0) {
-        const uint32_t kb = smem_u32(sm.kv[stage][0]);
-        const uint32_t vb = smem_u32(sm.kv[stage][1]);
-        if (nvalid < 16) {
-          // rows past the chunk may hold tokens beyond T (unwritten cache rows):
-          // zero their V rows so that 0-weight * garbage cannot make a NaN
-          constexpr int CPR = D / 8;  // 16-byte chunks per row
-          for (int e = lane; e < (16 - nvalid) * CPR; e += 32) {
-            const int t = r0 + nvalid + e / CPR;
-            *reinterpret_cast<uint4*>(&sm.kv[stage][1][swz<D>(t, e % CPR)]) = make_uint4(0, 0, 0, 0);
-          }
-          // order these generic-proxy writes before the next TMA write of the stage
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-        }
-        // ---- S^T = Qpad K^T for 16 tokens (two 8-token n-tiles)
-        float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + swz<D>(r0 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)), b0, b1, b2, b3);
-          mma_16816(sacc[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-          mma_16816(sacc[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
-        }
-        // ---- weights of this lane's 4 tokens: n-tile nt, element e -> token nt*8 + 2*tig + e
-        float s[4], x[4];
-        bool v[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int nt = q4 >> 1, e = q4 & 1;
-          v[q4] = (nt * 8 + 2 * tig + e) < nvalid;
-          s[q4] = sacc[nt][e] * p.scale;
-          x[q4] = (p_lane && v[q4]) ? s[q4] * kLog2e : -INFINITY;
-        }
-        float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
-        tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
-        const float m_new = fmaxf(m_run, tmax);
-        const float alpha = (p_lane && m_new != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
-        const bool sel_tok = dsc.z != 0;
-        float w[4], wsum = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          w[q4] = p_lane ? (v[q4] ? exp2f(x[q4] - m_new) : 0.f) : ((v[q4] && sel_tok) ? 1.f + s[q4] : 0.f);
-          wsum += w[q4];
-        }
-        if (p_lane) {
-          l_run = l_run * alpha + wsum;
-          m_run = m_new;
-        } else {
-          dsel_run += wsum;
-        }
-        if (__any_sync(kFull, alpha != 1.f)) {
-#pragma unroll
-          for (int n = 0; n < NT8; ++n) {
-            O[n][0] *= alpha;
-            O[n][1] *= alpha;
-            O[n][2] *= alpha;
-            O[n][3] *= alpha;
-          }
-        }
-        uint32_t a0, a1, a2, a3;  // rows g (hi) / g+8 (lo), tokens 0-7 / 8-15 of the k=16 step
-        split_bf16(w[0], w[1], a0, a1);
-        split_bf16(w[2], w[3], a2, a3);
-        // ---- O += A V over 16 tokens
-#pragma unroll
-        for (int np = 0; np < NT8 / 2; ++np) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vb + swz<D>(r0 + (mi & 1) * 8 + rr, np * 2 + (mi >> 1)), b0, b1, b2, b3);
-          mma_16816(O[2 * np], a0, a1, a2, a3, b0, b1);
-          mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-      group_sync(grp);  // the group is done with this stage
-      if (leader && next_issue < n_local && !*(volatile int*)&sm.abort_flag) {
-        issue_chunk<D>(&tmK, &tmV, p, sm, c_begin, next_issue, waited);
-        next_issue += kConsumerGroups;
-      }
+    __syncthreads();  // every warp is done with this stage
+    if (tid == 0 && next_issue < n_local && !*(volatile int*)&sm.abort_flag) {
+      issue_chunk<D>(&tm, p, sm, unit, part + next_issue * p.splits, next_issue, waited);
+      ++next_issue;
     }
-
-    // ---- this warp's partial -> shared memory
-    {
-      float l = l_run + __shfl_xor_sync(kFull, l_run, 1);
-      l += __shfl_xor_sync(kFull, l, 2);
-      float ds = dsel_run + __shfl_xor_sync(kFull, dsel_run, 1);
-      ds += __shfl_xor_sync(kFull, ds, 2);
-      float* wp = sm.wpart[warp];
-      if (tig == 0) {
-        if (p_lane) {
-          wp[head] = m_run;
-          wp[4 + head] = l;
-        } else {
-          wp[8 + head] = ds;
-        }
-      }
-      float* dst = wp + 16 + (p_lane ? 0 : 4 * D) + head * D;
-#pragma unroll
-      for (int n = 0; n < NT8; ++n) {
-        dst[n * 8 + 2 * tig] = O[n][0] + O[n][2];
-        dst[n * 8 + 2 * tig + 1] = O[n][1] + O[n][3];
-      }
-    }
-    __syncthreads();
-    // ---- combine the 8 warps -> one partial record for (cta, unit)
-    {
-      constexpr int NW = kConsumerGroups * kWarpsPerGroup;
-      float* gp = p.partials + (int64_t)(cta + unit) * PF;
-      if (tid < 4) {
-        float M = -INFINITY;
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, sm.wpart[w][tid]);
-        float l = 0.f, ds = 0.f;
-        for (int w = 0; w < NW; ++w) {
-          const float m = sm.wpart[w][tid];
-          l += (m == -INFINITY) ? 0.f : sm.wpart[w][4 + tid] * exp2f(m - M);
-          ds += sm.wpart[w][8 + tid];
-        }
-        gp[tid] = M;
-        gp[4 + tid] = l;
-        gp[8 + tid] = ds;
-      }
-      for (int e = tid; e < 8 * D; e += kConsumerThreads) {
-        float acc = 0.f;
-        if (e < 4 * D) {
-          const int hh = e / D;
-          float M = -INFINITY;
-          for (int w = 0; w < NW; ++w) M = fmaxf(M, sm.wpart[w][hh]);
-          for (int w = 0; w < NW; ++w) {
-            const float m = sm.wpart[w][hh];
-            if (m != -INFINITY) acc += sm.wpart[w][16 + e] * exp2f(m - M);
-          }
-        } else {
-          for (int w = 0; w < NW; ++w) acc += sm.wpart[w][16 + e];
-        }
-        gp[16 + e] = acc;
-      }
-      __threadfence();
-    }
-    __syncthreads();
-    const int64_t first = cta_of_chunk((int64_t)unit * cpu, p.total_chunks, p.grid);
-    const int64_t last = cta_of_chunk((int64_t)(unit + 1) * cpu - 1, p.total_chunks, p.grid);
-    if (tid == 0) {
-      const uint32_t prev = atomicAdd(&p.tickets[unit], 1u);
-      sm.last_flag = (prev == (uint32_t)(last - first));
-    }
-    __syncthreads();
-    if (sm.last_flag) {
-      __threadfence();
-      merge_unit<D>(p, unit, first, last, tid);
-      if (tid == 0) p.tickets[unit] = 0u;
-    }
-    __syncthreads();
-    c = seg_end;
   }
-  if (leader && *(volatile int*)&sm.abort_flag) {
+
+  if (tid == 0 && !waited) {  // a CTA with no selected chunk
+    pdl_wait_primary();
+    pdl_allow_dependents();
+    waited = true;
+  }
+
+  // ---- combine the 4 warps' partials in registers (a tree through two shared
+  //      slots: warps 2, 3 -> 0, 1, then warp 1 -> 0); warp 0 writes the record
+  float l = l_run + __shfl_xor_sync(kFull, l_run, 1);
+  l += __shfl_xor_sync(kFull, l, 2);
+  float ds = dsel_run + __shfl_xor_sync(kFull, dsel_run, 1);
+  ds += __shfl_xor_sync(kFull, ds, 2);
+  const int voff = (p_lane ? 0 : 4 * D) + head * D;
+  auto emit = [&](float* wp) {  // write this warp's partial (hi + lo rows summed)
+    if (tig == 0) {
+      if (p_lane) {
+        wp[head] = m_run;
+        wp[4 + head] = l;
+      } else {
+        wp[8 + head] = ds;
+      }
+    }
+    float* dst = wp + 16 + voff;
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+      *reinterpret_cast<float2*>(dst + n * 8 + 2 * tig) = make_float2(O[n][0] + O[n][2], O[n][1] + O[n][3]);
+  };
+  auto absorb = [&](const float* wp) {  // fold another warp's partial into this one
+    const float mp = wp[head], lp = wp[4 + head], dsp = wp[8 + head];
+    float fa = 1.f, fb = 1.f;
+    if (p_lane) {
+      const float M = fmaxf(m_run, mp);
+      fa = (m_run == -INFINITY) ? 0.f : exp2f(m_run - M);
+      fb = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
+      l = l * fa + lp * fb;
+      m_run = M;
+    } else {
+      ds += dsp;
+    }
+    const float* src = wp + 16 + voff;
+#pragma unroll
+    for (int n = 0; n < NT8; ++n) {
+      const float2 y = *reinterpret_cast<const float2*>(src + n * 8 + 2 * tig);
+      O[n][0] = (O[n][0] + O[n][2]) * fa + y.x * fb;
+      O[n][1] = (O[n][1] + O[n][3]) * fa + y.y * fb;
+      O[n][2] = O[n][3] = 0.f;
+    }
+  };
+  if (warp >= 2) emit(sm.wpart[warp - 2]);
+  __syncthreads();
+  if (warp < 2) absorb(sm.wpart[warp]);
+  __syncthreads();
+  if (warp == 1) emit(sm.wpart[0]);
+  __syncthreads();
+  if (warp == 0) {
+    absorb(sm.wpart[0]);
+    emit(p.partials + (int64_t)cta * PF);
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();  // release the partial record before the ticket
+      const uint32_t prev = atomicAdd(&p.tickets[unit], 1u);
+      sm.last_flag = (prev == (uint32_t)p.splits - 1u);
+      __threadfence();
+    }
+  }
+  __syncthreads();
+  if (sm.last_flag) {
+    merge_unit<D>(p, unit, (int64_t)unit * p.splits, p.splits, tid, sm);
+    if (tid == 0) p.tickets[unit] = 0u;  // ready for the next decode
+  }
+  if (tid == 0 && *(volatile int*)&sm.abort_flag) {
     // do not leave while copies into this CTA's shared memory may be in flight
-    for (int i = next_issue - kConsumerGroups; i >= 0 && i >= next_issue - kStages; i -= kConsumerGroups)
-      mbar_wait_bounded(&sm.full[i % kStages], (i / kStages) & 1, kWaitLimit);
+    for (int j = next_issue - 1; j >= 0 && j >= next_issue - kStages; --j)
+      mbar_wait_bounded(&sm.full[j % kStages], (j / kStages) & 1, kWaitLimit);
   }
 }
 
 }  // namespace
 
-size_t attend_smem_bytes(int D);
-
-cudaError_t prepare_attend(int D) {
-  const int smem = (int)attend_smem_bytes(D);
-  if (D == 128) return cudaFuncSetAttribute(attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  return cudaFuncSetAttribute(attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-}
-
 size_t attend_smem_bytes(int D) {
   return (D == 128 ? sizeof(AttendSmem<128>) : sizeof(AttendSmem<64>)) + 1024;
 }
 
-cudaError_t launch_attend(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttendParams& p, int D, bool pdl,
-                          cudaStream_t s) {
-  const size_t smem = attend_smem_bytes(D);
+cudaError_t prepare_attend(int D) {
+  const int smem = (int)attend_smem_bytes(D);
+  const void* f = D == 128 ? (const void*)attend_kernel<128> : (const void*)attend_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
+cudaError_t launch_attend(const CUtensorMap* maps, const AttendParams& p, int D, bool pdl, cudaStream_t s) {
+  KVMaps tm;
+  tm.k64 = maps[0];
+  tm.v64 = maps[1];
+  tm.k16 = maps[2];
+  tm.v16 = maps[3];
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.merge_only ? p.units : p.grid);
+  cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3(kAttendThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = attend_smem_bytes(D);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  if (D == 128) return cudaLaunchKernelEx(&cfg, attend_kernel<128>, *tmK, *tmV, p);
-  return cudaLaunchKernelEx(&cfg, attend_kernel<64>, *tmK, *tmV, p);
+  if (D == 128) return cudaLaunchKernelEx(&cfg, attend_kernel<128>, tm, p);
+  return cudaLaunchKernelEx(&cfg, attend_kernel<64>, tm, p);
 }
 
 }  // namespace hyb

@@ -36,9 +36,14 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+constexpr int kKeysInSmem = 4096;  // blocks whose keys fit the staging buffer (16 KB)
+
 // Top-k of scores[0, nb) with ties to the lower index; writes sel[0, top_k)
-// ascending, -1 padded.  Runs on one CTA of kSelectThreads threads.
+// ascending, -1 padded.  Runs on one CTA of kSelectThreads threads.  The score
+// keys are staged once in shared memory (when nb <= kKeysInSmem), so the radix
+// passes and the compaction run at shared-memory latency.
 __device__ void select_top_k(const SelectParams& p, int unit) {
+  __shared__ uint32_t s_keys[kKeysInSmem];
   __shared__ uint32_t s_hist[256];
   __shared__ uint32_t s_wcnt[2][kSelectThreads / 32];
   __shared__ uint32_t s_digit, s_above;
@@ -49,19 +54,27 @@ __device__ void select_top_k(const SelectParams& p, int unit) {
   const int nb = p.nb;
   const int k = p.k_eff;
 
+  const bool staged = nb <= kKeysInSmem;
+  auto key = [&](int j) -> uint32_t { return staged ? s_keys[j] : float_key(__ldcg(sc + j)); };
   if (k >= nb) {
     for (int j = tid; j < p.top_k; j += kSelectThreads) sel[j] = j < nb ? j : -1;
   } else {
-    uint32_t prefix = 0, pmask = 0, need = (uint32_t)k;
     bool nan_seen = false;
+    if (staged) {
+      for (int j = tid; j < nb; j += kSelectThreads) {
+        const float f = __ldcg(sc + j);
+        nan_seen |= (f != f);
+        s_keys[j] = float_key(f);
+      }
+    }
+    uint32_t prefix = 0, pmask = 0, need = (uint32_t)k;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       for (int i = tid; i < 256; i += kSelectThreads) s_hist[i] = 0;
       __syncthreads();
       for (int j = tid; j < nb; j += kSelectThreads) {
-        const float f = __ldcg(sc + j);
-        if (pass == 0 && f != f) nan_seen = true;
-        const uint32_t u = float_key(f);
+        const uint32_t u = key(j);
+        if (!staged && pass == 0 && u == 0u) nan_seen |= (__ldcg(sc + j) != __ldcg(sc + j));
         if ((u & pmask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255u], 1u);
       }
       __syncthreads();
@@ -105,7 +118,7 @@ __device__ void select_top_k(const SelectParams& p, int unit) {
     uint32_t taken_base = 0, eq_base = 0;
     for (int base = 0; base < nb; base += kSelectThreads) {
       const int j = base + tid;
-      const uint32_t u = j < nb ? float_key(__ldcg(sc + j)) : 0u;
+      const uint32_t u = j < nb ? key(j) : 0u;
       const bool gt = j < nb && u > tau;
       const bool eq = j < nb && u == tau;
       const uint32_t beq = __ballot_sync(kFull, eq);
@@ -198,16 +211,16 @@ __device__ void score_blocks(const SelectParams& p, int unit, const float (*s_q)
   }
 
   if (!p.do_select) return;
-  __threadfence();
   __syncthreads();
   __shared__ int s_last;
   if (tid == 0) {
+    __threadfence();  // release this CTA's scores (ordered after the barrier)
     const uint32_t prev = atomicAdd(&p.tickets[unit], 1u);
     s_last = (prev == (uint32_t)p.score_ctas - 1u);
+    __threadfence();
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   select_top_k(p, unit);
   if (tid == 0) p.tickets[unit] = 0u;  // ready for the next decode
 }
@@ -276,6 +289,13 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
 }
 
 }  // namespace
+
+cudaError_t prepare_select(int D) {
+  // the same shared-memory carveout as the attention kernel, so the SMs need no
+  // reconfiguration between the two launches of a decode
+  const void* f = D == 128 ? (const void*)select_kernel<128> : (const void*)select_kernel<64>;
+  return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
 
 cudaError_t launch_select(const SelectParams& p, int D, int grid_x, cudaStream_t s) {
   const dim3 grid(grid_x, p.units);

@@ -73,6 +73,12 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     p.k_cache[(ub + p.T) * D + tid] = p.k_new[(int64_t)unit * D + tid];
     p.v_cache[(ub + p.T) * D + tid] = p.v_new[(int64_t)unit * D + tid];
   }
+  // Launched programmatically after a decode's attention kernel, this kernel may
+  // run beside it (it writes nothing that kernel reads; the attention kernel lets
+  // it start only after the select kernel, which reads the state, has finished).
+  // Waiting for the attention kernel before exiting keeps "this kernel complete"
+  // meaning "the decode before it complete" for whatever the stream runs next.
+  pdl_wait_primary();
 }
 
 // ---------------------------------------------------------------- init
@@ -192,13 +198,31 @@ __global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) 
 
 }  // namespace
 
+cudaError_t prepare_state(int D) {
+  const void* fs[] = {D == 128 ? (const void*)append_kernel<128> : (const void*)append_kernel<64>,
+                      D == 128 ? (const void*)init_linear_kernel<128> : (const void*)init_linear_kernel<64>,
+                      D == 128 ? (const void*)init_stats_kernel<128> : (const void*)init_stats_kernel<64>,
+                      D == 128 ? (const void*)init_finalize_kernel<128> : (const void*)init_finalize_kernel<64>};
+  for (const void* f : fs) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {
-  const dim3 grid(D * D / 1024, p.units);
-  if (D == 128)
-    append_kernel<128><<<grid, 256, 0, s>>>(p);
-  else
-    append_kernel<64><<<grid, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(D * D / 1024, p.units);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) return cudaLaunchKernelEx(&cfg, append_kernel<128>, p);
+  return cudaLaunchKernelEx(&cfg, append_kernel<64>, p);
 }
 
 cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s) {

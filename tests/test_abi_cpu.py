@@ -104,7 +104,8 @@ def test_init_rejects_bad_arguments_without_touching_a_gpu(lib):
 @pytest.mark.parametrize("T", [0, 1, 3, 4, 5, 1027, 1028, 1029, 1092, 1093, 32768, 32768 + 64])
 def test_plan_partition(lib, T):
     """Chunk counts of the exact set follow the partition: sinks, window, and
-    ceil(Bk/64) chunks per selected block; the grid never exceeds the SM count."""
+    ceil(Bk/64) chunks per selected block; each unit's chunks go to at most two
+    CTAs per SM in one wave."""
     import hybrid_sparse_linear_decode_b200 as H
     c = _cfg()
     p = H.hyb_attn_plan(c, T, 148)
@@ -115,8 +116,9 @@ def test_plan_partition(lib, T):
     sink = min(S, T)
     win = T - max(S, T - W) if T > S else 0
     assert p.chunks_per_unit == -(-sink // 64) + -(-win // 64) + p.k_eff
-    total = 8 * p.chunks_per_unit
-    if total:
-        assert p.attend_ctas == min(total, 148)
-        assert p.partial_slots == p.attend_ctas + 8 - 1
+    if p.chunks_per_unit:
+        splits = min(max(1, 148 * 2 // 8), p.chunks_per_unit)   # two CTAs per SM, one unit per CTA
+        assert p.attend_ctas == 8 * splits and p.partial_slots == 8 * splits
+    else:
+        assert p.attend_ctas == 8 and p.partial_slots == 0
     assert p.score_ctas_per_unit == -(-nb // 64)
