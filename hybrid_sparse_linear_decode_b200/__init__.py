@@ -20,6 +20,7 @@ from ._abi import (  # noqa: F401
     hyb_attn_decode,
     hyb_attn_decode_with_selection,
     hyb_attn_step_host,
+    hyb_attn_decode_noalloc,
     hyb_attn_length,
     hyb_attn_status,
     hyb_attn_set_timing_events,

@@ -21,6 +21,7 @@ HYB_ECAPACITY = -2
 HYB_ECUDA = -3
 HYB_ESTATE = -4
 HYB_ENOMEM = -5
+HYB_ESCRATCH = -6
 
 HYB_STATUS_NONFINITE = 0x1
 HYB_STATUS_DENOMINATOR = 0x2
@@ -65,6 +66,7 @@ SIGNATURES = [
     ("hyb_attn_decode", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_with_selection", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_step_host", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_decode_noalloc", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_length", c_i64, [c_vp]),
     ("hyb_attn_status", ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, c_vp]),
     ("hyb_attn_set_timing_events", ctypes.c_int, [c_vp, c_vp, c_vp]),
@@ -156,6 +158,12 @@ def hyb_attn_decode_with_selection(ctx: int, q: int, sel: int, out: int, stream:
 
 def hyb_attn_step_host(ctx: int, q_host: int, k_host, v_host, out_host: int, stream: int) -> None:
     _check("hyb_attn_step_host", load_library().hyb_attn_step_host(ctx, q_host, k_host, v_host, out_host, stream))
+
+
+def hyb_attn_decode_noalloc(ctx: int, q: int, out: int, sel_out, stream: int) -> None:
+    """Decode using the library's fixed device scratch instead of the context's
+    workspace (for callers that cannot allocate device memory)."""
+    _check("hyb_attn_decode_noalloc", load_library().hyb_attn_decode_noalloc(ctx, q, out, sel_out, stream))
 
 
 def hyb_attn_length(ctx: int) -> int:

@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "../../include/hyb_attn.h"
@@ -160,6 +161,30 @@ bool is_device_ptr(const void* p, int device) {
   return a.type == cudaMemoryTypeDevice && a.device == device;
 }
 
+}  // namespace
+
+// Fixed scratch of hyb_attn_decode_noalloc: a file-scope device array, one per
+// GPU that loads this library.  Host code only ever uses its device address,
+// looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HYB_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+int noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return HYB_EINVAL;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[device] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_addr[device] = p;
+  }
+  *out = g_noalloc_addr[device];
+  return HYB_OK;
+}
 }  // namespace
 
 struct hyb_attn_ctx {
@@ -453,6 +478,25 @@ int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, 
   return HYB_OK;
 }
 
+int hyb_attn_decode_noalloc(hyb_attn_ctx* x, const void* q, float* out, int32_t* sel_out, cudaStream_t stream) {
+  if (x == nullptr) return HYB_EINVAL;
+  int device = -1;
+  if (cudaGetDevice(&device) != cudaSuccess) return HYB_ECUDA;
+  if (device != x->device) return HYB_EINVAL;
+  // the decode uses the workspace regions that precede the init accumulators
+  if (x->ws.H64 > HYB_NOALLOC_SCRATCH_BYTES) return HYB_ESCRATCH;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch(device, &scratch);
+  if (rc != HYB_OK) return rc;
+  // status and tickets must start at zero; the array keeps the previous call's contents
+  const cudaError_t e = cudaMemsetAsync(scratch, 0, x->ws.scores, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  hyb_attn_ctx view = *x;  // the same context with its scratch rebased onto the fixed array
+  view.buf.workspace = scratch;
+  view.buf.workspace_bytes = HYB_NOALLOC_SCRATCH_BYTES;
+  return decode_impl(&view, q, out, nullptr, sel_out, nullptr, stream);
+}
+
 int64_t hyb_attn_length(const hyb_attn_ctx* x) { return x ? x->T : -1; }
 
 int hyb_attn_status(hyb_attn_ctx* x, uint32_t* flags, int clear, cudaStream_t stream) {
@@ -487,6 +531,7 @@ const char* hyb_attn_strerror(int code) {
     case HYB_ECUDA: return "CUDA call or kernel launch failed";
     case HYB_ESTATE: return "call not valid in the current state";
     case HYB_ENOMEM: return "host allocation failed";
+    case HYB_ESCRATCH: return "decode scratch exceeds the fixed device area of the no-allocation entry point";
     default: return "unknown error code";
   }
 }

@@ -63,6 +63,7 @@ extern "C" {
 #define HYB_ECUDA      (-3)  /* a CUDA call or kernel launch failed */
 #define HYB_ESTATE     (-4)  /* call not valid in the current state (e.g. decode at T = 0) */
 #define HYB_ENOMEM     (-5)  /* host allocation of the context failed */
+#define HYB_ESCRATCH   (-6)  /* the call needs more scratch than the library's fixed device area */
 
 /* ---- device status bits (hyb_attn_status) -------------------------------- */
 #define HYB_STATUS_NONFINITE     0x1u  /* an output element was NaN or Inf */
@@ -204,6 +205,33 @@ int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32
  * is valid once `stream` has been synchronised. */
 int hyb_attn_step_host(hyb_attn_ctx* ctx, const void* q_host, const void* k_host,
                        const void* v_host, float* out_host, cudaStream_t stream);
+
+/* Decode without any allocation, for callers that cannot allocate device
+ * memory themselves: code that runs under an allocator it does not own (a
+ * framework's caching pool, a plugin host, an embedded runtime) or that must
+ * not call cudaMalloc/cudaFree on its hot path, where those calls synchronise
+ * the device.  The pages have no counterpart for this call; it exists for the
+ * library's users.
+ *
+ * Same arguments and result as hyb_attn_decode without scores_out, but the
+ * per-call scratch (block scores, selection, split-K partial records, tickets,
+ * status) comes from a fixed device array inside the library, of
+ * HYB_NOALLOC_SCRATCH_BYTES (16 MiB) per GPU, that every GPU which loads the
+ * library holds until the process exits.  A configuration whose decode scratch
+ * exceeds it is rejected with HYB_ESCRATCH (the context's own workspace is not
+ * used by this call).  The call allocates nothing: no cudaMalloc, no cudaFree,
+ * no allocating library routine.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  The current device must be the context's device.  All calls share
+ * the one array and it keeps the last call's contents: the call clears what
+ * must start at zero itself, but calls whose work overlaps on the GPU (two
+ * streams, two threads) race on the array and must be serialised by the caller.
+ * Device status bits raised by this call stay in the array and are not reported
+ * by hyb_attn_status.  Errors: HYB_EINVAL, HYB_ESTATE, HYB_ESCRATCH, HYB_ECUDA. */
+#define HYB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int hyb_attn_decode_noalloc(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out, cudaStream_t stream);
 
 /* Current length T (host mirror; no device access). */
 int64_t hyb_attn_length(const hyb_attn_ctx* ctx);
