@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 
 L2_FLUSH_BYTES = 512 << 20
 METRIC = "hybrid decode-attn steps/s and achieved HBM GB/s (% of peak) at 32K-256K ctx"
-DEFAULT_WORKLOAD = "llama8b_32k_layer"
+DEFAULT_WORKLOAD = "llama8b_32layers_b8_32k"
 
 
 def parse():
@@ -48,6 +48,32 @@ def parse():
     return ap.parse_args()
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_workload(w, rank: int):
+    """Each rank runs its own replica of the workload's units (weak scaling): the
+    same shapes, its own seeded data, no collective on the data path."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + rank) if rank else w
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks take this step, in the same order)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_steps_per_s(ms_per_step_max: float, world: int) -> float:
+    """Whole-job throughput: every rank completes one step of its own units per
+    ms_per_step_max."""
+    return world * 1e3 / ms_per_step_max
+
+
 # ----------------------------------------------------------------------------- bytes model
 
 def algorithmic_bytes(w, T):
@@ -60,6 +86,26 @@ def algorithmic_bytes(w, T):
     append = (2 * d * 2) + (2 * d * 2) + 2 * d * d * 4 + 2 * 2 * d * 4 + 2 * 2 * d * 4 + 2 * 4
     attend = per["exact_kv"] + per["q_out"]
     return decode, append, attend
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per attention-kernel launch from the committed ncu summary of this
+    workload, if the kernel's sources are unchanged since that capture (else None)."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", f"attend_kernel_{workload}.md")
+    if not os.path.exists(prof):
+        return None
+    text = open(prof).read()
+    mh = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]{16})", text)
+    mt = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    if not (mh and mt):
+        return None
+    csrc = os.path.join(ROOT, "hybrid_sparse_linear_decode_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("k_attend.cu", "hyb_device.cuh", "hyb_internal.h"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return int(mt.group(1)) if h.hexdigest()[:16] == mh.group(1) else None
 
 
 def peaks():
@@ -180,7 +226,7 @@ def run_native(args, rank, world):
     from syngen import configs as C
     torch.cuda.set_device(rank % torch.cuda.device_count())
     device = torch.device("cuda", torch.cuda.current_device())
-    w = C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {}))
+    w = rank_workload(C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {})), rank)
     K, Wm = args.steps, args.warmup
     Kk = min(K, 20)                      # steps of the attention-kernel timing pass
     Ke = 0 if args.no_e2e else min(K, 20)  # steps of the end-to-end pass
@@ -229,11 +275,7 @@ def run_native(args, rank, world):
         total_ms = e0.elapsed_time(e1)
     barrier()
     clocks = clk.stop()
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, device)
     ms_per_step = total_ms / K
     steps_s = 1e3 / ms_per_step
 
@@ -284,15 +326,10 @@ def run_native(args, rank, world):
             if flush:
                 scratch.zero_()
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(c) for a, c in evs) / Ke
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs) / Ke, world, device)
         h2d = w.layers * (w.batch * w.n_q_heads * w.head_dim * 2 + 2 * w.batch * w.n_kv_heads * w.head_dim * 2)
         d2h = w.layers * w.batch * w.n_q_heads * w.head_dim * 4
-        e2e = {"value": round(world * 1e3 / e2e_ms, 3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": round(aggregate_steps_per_s(e2e_ms, world), 3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)}
 
     status = 0
@@ -300,7 +337,7 @@ def run_native(args, rank, world):
         status |= L.status()
     result = {
         "metric": METRIC,
-        "value": round(world * steps_s, 3),
+        "value": round(aggregate_steps_per_s(ms_per_step, world), 3),
         "unit": "steps/s",
         "n_gpus": world,
         "steps": K,
@@ -326,7 +363,8 @@ def run_native(args, rank, world):
         "roofline": {"bound": "hbm", "kernel": "attend_kernel (exact part + subtraction + merge)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
-                     "traffic": None, "bytes_per_launch": attend_bytes, "avg_launch_us": round(attend_ms * 1e3, 3)},
+                     "traffic": measured_traffic(w.name), "bytes_per_launch": attend_bytes,
+                     "avg_launch_us": round(attend_ms * 1e3, 3)},
         "e2e": e2e,
         "gpu_launches": b.launches_per_step() * K,
         "clocks": clocks,
