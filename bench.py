@@ -3,7 +3,10 @@
 
 One step = for every layer of the workload: one decode (block scores, top-k,
 gather, exact softmax part, Taylor linear part by subtraction, merge) and one
-append (cache write, window eviction, linear-state and block-stat update).
+append (cache write; the evicted token's fold into the linear state and block
+statistics happens in the next decode's select kernel), issued as one
+hyb_attn_decode_append call: two kernel launches chained with programmatic
+dependent launch.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
 on a bounded sample of the same workload instead.
@@ -83,29 +86,39 @@ def algorithmic_bytes(w, T):
     d, G = w.head_dim, w.group
     per = w.bytes_per_unit(T)
     decode = sum(per.values())
-    append = (2 * d * 2) + (2 * d * 2) + 2 * d * d * 4 + 2 * 2 * d * 4 + 2 * 2 * d * 4 + 2 * 4
-    attend = per["exact_kv"] + per["q_out"]
-    return decode, append, attend
+    # cache write of the new token, read of the evicted token, and the write-back
+    # of the state the decode already reads: H, zk, zv, n, and one block's mean /
+    # variance row
+    append = (2 * d * 2) + (2 * d * 2) + d * d * 4 + 2 * d * 4 + 4 + 2 * d * 4
+    return decode, append
+
+
+KERNEL_SOURCES = ("k_attend.cu", "k_select.cu", "hyb_device.cuh", "hyb_internal.h")
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+    csrc = os.path.join(ROOT, "hybrid_sparse_linear_decode_b200", "csrc")
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(workload: str):
-    """DRAM bytes per attention-kernel launch from the committed ncu summary of this
-    workload, if the kernel's sources are unchanged since that capture (else None)."""
-    import hashlib
+    """DRAM bytes of one layer's decode kernels (select + attention) from the
+    committed ncu summary of this workload, if the kernels' sources are unchanged
+    since that capture (else None)."""
     import re
-    prof = os.path.join(ROOT, "profiles", f"attend_kernel_{workload}.md")
+    prof = os.path.join(ROOT, "profiles", f"decode_kernels_{workload}.md")
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
     mh = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]{16})", text)
-    mt = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    mt = re.search(r"traffic_bytes_per_decode:\s*(\d+)", text)
     if not (mh and mt):
         return None
-    csrc = os.path.join(ROOT, "hybrid_sparse_linear_decode_b200", "csrc")
-    h = hashlib.sha256()
-    for f in ("k_attend.cu", "hyb_device.cuh", "hyb_internal.h"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
-    return int(mt.group(1)) if h.hexdigest()[:16] == mh.group(1) else None
+    return int(mt.group(1)) if kernel_sources_hash() == mh.group(1) else None
 
 
 def peaks():
@@ -213,12 +226,13 @@ class Bench:
         s = self.step_idx
         for l, L in enumerate(self.layers):
             q = self.q[l][s % len(self.q[l])]
-            L.decode(q, out=self.out)
-            L.append(self.app_k[l][s], self.app_v[l][s])
+            L.decode_append(q, self.app_k[l][s], self.app_v[l][s], out=self.out)
         self.step_idx += 1
 
     def launches_per_step(self):
-        return 3 * len(self.layers)   # select, attend, append per layer
+        """Kernels per step: the select and attention launches of every layer's
+        decode (the append's cache write rides in the attention kernel)."""
+        return 2 * len(self.layers)
 
 
 def run_native(args, rank, world):
@@ -232,7 +246,7 @@ def run_native(args, rank, world):
     Ke = 0 if args.no_e2e else min(K, 20)  # steps of the end-to-end pass
     b = Bench(w, Wm + K + Kk + Ke, device)
     T_mid = w.T0 + Wm + K // 2
-    dec_b, app_b, att_b = algorithmic_bytes(w, T_mid)
+    dec_b, app_b = algorithmic_bytes(w, T_mid)
     units = w.layers * w.units_per_layer
     step_bytes = units * (dec_b + app_b)
     flush = step_bytes < 4 * 126e6      # the step's data would otherwise stay in L2
@@ -279,7 +293,7 @@ def run_native(args, rank, world):
     ms_per_step = total_ms / K
     steps_s = 1e3 / ms_per_step
 
-    # ---- attention-kernel timing (events around the attention launch of every layer)
+    # ---- decode timing: events around each layer's decode (its two chained kernels)
     ka, kb_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kern_ms, n_kern = 0.0, 0
     pool = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in b.layers]
@@ -300,10 +314,10 @@ def run_native(args, rank, world):
         for e0, e1 in pool[i]:
             kern_ms += e0.elapsed_time(e1)
             n_kern += 1
-    attend_ms = kern_ms / n_kern
-    attend_bytes = w.units_per_layer * att_b
+    decode_ms = kern_ms / n_kern
+    decode_bytes = w.units_per_layer * dec_b
     hbm_peak, peak_kind = peaks()
-    achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
+    achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # ---- e2e through the host-buffer entry point (pinned host q / k / v / out)
@@ -360,11 +374,12 @@ def run_native(args, rank, world):
         "achieved_gbs_step": round(step_gbs, 1),
         "pct_of_hbm_peak_step": round(100 * step_gbs / hbm_peak, 2),
         "bytes_per_step": step_bytes,
-        "roofline": {"bound": "hbm", "kernel": "attend_kernel (exact part + subtraction + merge)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "one layer's decode: select + attention kernels (PDL-chained)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
-                     "traffic": measured_traffic(w.name), "bytes_per_launch": attend_bytes,
-                     "avg_launch_us": round(attend_ms * 1e3, 3)},
+                     "traffic": measured_traffic(w.name), "bytes_per_launch": decode_bytes,
+                     "avg_launch_us": round(decode_ms * 1e3, 3)},
         "e2e": e2e,
         "gpu_launches": b.launches_per_step() * K,
         "clocks": clocks,

@@ -50,8 +50,8 @@ class hyb_attn_buffers(ctypes.Structure):
 
 class hyb_attn_plan_info(ctypes.Structure):
     _fields_ = [("T", c_i64), ("n_blocks", c_i64), ("k_eff", c_i64), ("exact_tokens", c_i64),
-                ("chunks_per_unit", c_i32), ("attend_ctas", c_i32), ("partial_slots", c_i32),
-                ("score_ctas_per_unit", c_i32), ("linear_ctas_per_unit", c_i32)]
+                ("chunks_per_unit", c_i32), ("select_ctas", c_i32), ("attend_ctas", c_i32),
+                ("partial_slots", c_i32), ("score_items_per_unit", c_i32), ("linear_items_per_unit", c_i32)]
 
 
 # (name, restype, argtypes) of every entry point declared in include/hyb_attn.h
@@ -63,7 +63,9 @@ SIGNATURES = [
     ("hyb_attn_init", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
                                      ctypes.POINTER(hyb_attn_buffers), c_i64, c_vp]),
     ("hyb_attn_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_sync_state", ctypes.c_int, [c_vp, c_vp]),
     ("hyb_attn_decode", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_decode_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_with_selection", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_step_host", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_noalloc", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
@@ -147,8 +149,18 @@ def hyb_attn_append(ctx: int, k_new: int, v_new: int, stream: int) -> None:
     _check("hyb_attn_append", load_library().hyb_attn_append(ctx, k_new, v_new, stream))
 
 
+def hyb_attn_sync_state(ctx: int, stream: int) -> None:
+    _check("hyb_attn_sync_state", load_library().hyb_attn_sync_state(ctx, stream))
+
+
 def hyb_attn_decode(ctx: int, q: int, out: int, sel_out, scores_out, stream: int) -> None:
     _check("hyb_attn_decode", load_library().hyb_attn_decode(ctx, q, out, sel_out, scores_out, stream))
+
+
+def hyb_attn_decode_append(ctx: int, q: int, k_new: int, v_new: int, out: int, sel_out, scores_out,
+                           stream: int) -> None:
+    _check("hyb_attn_decode_append",
+           load_library().hyb_attn_decode_append(ctx, q, k_new, v_new, out, sel_out, scores_out, stream))
 
 
 def hyb_attn_decode_with_selection(ctx: int, q: int, sel: int, out: int, stream: int) -> None:

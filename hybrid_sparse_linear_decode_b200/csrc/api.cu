@@ -57,6 +57,12 @@ int check_config(const hyb_attn_config* c, Checked* out) {
   return HYB_OK;
 }
 
+// Upper bound of the partial records of a unit (one per attention CTA).
+size_t max_slots_per_unit(int units) {
+  const int per = kMaxAttendCtas / units;
+  return (size_t)(per > 1 ? per : 1);
+}
+
 WsLayout ws_layout(const hyb_attn_config& c, const Checked& k) {
   WsLayout w{};
   size_t off = 0;
@@ -71,8 +77,8 @@ WsLayout ws_layout(const hyb_attn_config& c, const Checked& k) {
   w.tk_att = take(U * sizeof(uint32_t));
   w.scores = take(U * (size_t)(k.max_blocks > 0 ? k.max_blocks : 1) * sizeof(float));
   w.sel = take(U * (size_t)(c.top_k > 0 ? c.top_k : 1) * sizeof(int32_t));
-  w.lin = take(U * G * (D + 1) * sizeof(float));
-  w.partials = take(((size_t)kMaxAttendCtas + U) * (size_t)partial_floats((int)D) * sizeof(float));
+  w.lin = take(U * (size_t)sel_lin_items((int)D) * G * (D + 1) * sizeof(float));
+  w.partials = take(U * (size_t)max_slots_per_unit(k.units) * (size_t)partial_floats((int)D) * sizeof(float));
   w.H64 = take(U * D * D * sizeof(double));
   w.z64 = take(U * 2 * D * sizeof(double));
   w.stage_q = take(U * G * D * 2);
@@ -100,15 +106,33 @@ Geometry geometry(const hyb_attn_config& c, int64_t T) {
   return g;
 }
 
-// CTAs per unit for the attention kernel: enough to fill kAttendCtasPerSm CTAs
-// on every SM in one wave, never more than the unit's chunks.
-int attend_splits(int units, int chunks_per_unit, int n_sm) {
-  if (chunks_per_unit <= 0) return 0;
-  int64_t s = (int64_t)n_sm * kAttendCtasPerSm / units;
+// CTAs per unit for an attention launch over `chunks` chunks per unit: enough
+// for `per_sm` CTAs on every SM in one wave, never more than the chunks, and
+// within kMaxAttendCtas CTAs (one per unit at least).
+int attend_splits(int units, int chunks, int n_sm, int per_sm) {
+  int64_t s = (int64_t)n_sm * per_sm / units;
+  const int64_t cap = kMaxAttendCtas / units;
+  if (s > cap) s = cap;
+  if (s > chunks) s = chunks;
   if (s < 1) s = 1;
-  if (s > chunks_per_unit) s = chunks_per_unit;
-  if (s * units > kMaxAttendCtas + units) s = 1;
   return (int)s;
+}
+
+struct LaunchPlan {
+  int splits;          // attention CTAs per unit (>= 1)
+  int score_items, lin_items, items_per_unit, total_items, select_grid;
+};
+
+LaunchPlan plan_launches(const Geometry& g, const Checked& k, int n_sm) {
+  LaunchPlan lp{};
+  lp.splits = attend_splits(k.units, g.chunks_per_unit, n_sm, kAttendCtasPerSm);
+  lp.score_items = (int)ceil_div(g.nb, sel_item_blocks(k.D));
+  lp.lin_items = sel_lin_items(k.D);
+  lp.items_per_unit = lp.score_items + lp.lin_items;
+  lp.total_items = lp.items_per_unit * k.units;
+  const int64_t grid = (int64_t)n_sm * kSelectCtasPerSm;
+  lp.select_grid = (int)(grid < lp.total_items ? grid : lp.total_items);
+  return lp;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -193,6 +217,7 @@ struct hyb_attn_ctx {
   Checked ck;
   WsLayout ws;
   int64_t T;
+  int64_t folded_end;   // the state holds the evicted positions [S, folded_end)
   int device, n_sm;
   float scale;
   CUtensorMap maps[4];  // K, V with 64-row boxes; K, V with 16-row boxes
@@ -205,55 +230,83 @@ struct hyb_attn_ctx {
 
 namespace {
 
-int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_given, int32_t* sel_out,
-                float* scores_out, cudaStream_t stream) {
-  if (x == nullptr || q == nullptr || out == nullptr) return HYB_EINVAL;
-  if (!aligned16(q) || !aligned16(out)) return HYB_EINVAL;
-  if (sel_given != nullptr && !aligned16(sel_given)) return HYB_EINVAL;
-  if (sel_out != nullptr && (reinterpret_cast<uintptr_t>(sel_out) & 3u)) return HYB_EINVAL;
-  if (scores_out != nullptr && (reinterpret_cast<uintptr_t>(scores_out) & 15u)) return HYB_EINVAL;
-  if (x->T == 0) return HYB_ESTATE;
+SelectParams select_params(const hyb_attn_ctx* x, const Geometry& g, const LaunchPlan& lp) {
   const hyb_attn_config& c = x->cfg;
   const Checked& k = x->ck;
-  const Geometry g = geometry(c, x->T);
-
   SelectParams sp{};
-  sp.q = static_cast<const __nv_bfloat16*>(q);
   sp.mu = x->buf.mu;
   sp.var = x->buf.var;
   sp.H = x->buf.H;
   sp.zk = x->buf.zk;
   sp.zv = x->buf.zv;
   sp.n = x->buf.n;
-  sp.scores = scores_out ? scores_out : x->w<float>(x->ws.scores);
-  sp.sel = x->w<int32_t>(x->ws.sel);
-  sp.sel_out = sel_given ? nullptr : sel_out;
+  sp.k_cache = static_cast<const __nv_bfloat16*>(x->buf.k_cache);
+  sp.v_cache = static_cast<const __nv_bfloat16*>(x->buf.v_cache);
+  sp.scores = x->w<float>(x->ws.scores);
   sp.lin = x->w<float>(x->ws.lin);
-  sp.tickets = x->w<uint32_t>(x->ws.tk_sel);
   sp.status = x->w<uint32_t>(x->ws.status);
   sp.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
+  sp.cap = c.capacity;
+  sp.fold_begin = x->folded_end;
+  sp.fold_end = g.ev_end;
   sp.units = k.units;
   sp.G = k.G;
   sp.nb = (int32_t)g.nb;
-  sp.top_k = c.top_k;
-  sp.k_eff = (int32_t)g.k_eff;
-  sp.do_select = sel_given ? 0 : 1;
-  const bool need_scores = (sel_given == nullptr) ? (g.nb > 0) : (scores_out != nullptr && g.nb > 0);
-  sp.score_ctas = need_scores ? (int32_t)ceil_div(g.nb, kScoreBlocksPerCta) : 0;
-  sp.lin_ctas = k.D / 32;
+  sp.S = c.n_sink;
+  sp.Bk = c.block_size;
+  sp.score_items = lp.score_items;
+  sp.lin_items = lp.lin_items;
+  sp.items_per_unit = lp.items_per_unit;
+  sp.total_items = lp.total_items;
   sp.scale = x->scale;
-  cudaError_t e = launch_select(sp, k.D, sp.score_ctas + sp.lin_ctas, stream);
+  return sp;
+}
+
+// One decode at the current T: the select kernel (scores, linear term, pending
+// folds), then the attention kernel (sinks + window beside it; top-k, selected
+// blocks, merge; writes the appended token when k_new is given).
+int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_given, int32_t* sel_out,
+                float* scores_out, const void* k_new, const void* v_new, cudaStream_t stream) {
+  if (x == nullptr || q == nullptr || out == nullptr) return HYB_EINVAL;
+  if (!aligned16(q) || !aligned16(out)) return HYB_EINVAL;
+  if (sel_given != nullptr && !aligned16(sel_given)) return HYB_EINVAL;
+  if (sel_out != nullptr && (reinterpret_cast<uintptr_t>(sel_out) & 3u)) return HYB_EINVAL;
+  if (scores_out != nullptr && (reinterpret_cast<uintptr_t>(scores_out) & 15u)) return HYB_EINVAL;
+  if ((k_new == nullptr) != (v_new == nullptr)) return HYB_EINVAL;
+  if (k_new != nullptr && (!aligned16(k_new) || !aligned16(v_new))) return HYB_EINVAL;
+  if (x->T == 0) return HYB_ESTATE;
+  if (k_new != nullptr && x->T >= x->cfg.capacity) return HYB_ECAPACITY;
+  const hyb_attn_config& c = x->cfg;
+  const Checked& k = x->ck;
+  const Geometry g = geometry(c, x->T);
+  const LaunchPlan lp = plan_launches(g, k, x->n_sm);
+  const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
+  if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
+
+  SelectParams sp = select_params(x, g, lp);
+  sp.q = static_cast<const __nv_bfloat16*>(q);
+  if (scores_out) sp.scores = scores_out;
+  cudaError_t e = launch_select(sp, k.D, lp.select_grid, stream);
   if (e != cudaSuccess) return cuda_fail(e);
+  x->folded_end = g.ev_end;
 
   AttendParams ap{};
-  ap.q = sp.q;
-  ap.sel = sel_given ? sel_given : sp.sel;
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.scores = sp.scores;
+  ap.sel_given = sel_given;
+  ap.sel = x->w<int32_t>(x->ws.sel);
+  ap.sel_out = sel_given ? nullptr : sel_out;
   ap.lin = sp.lin;
   ap.partials = x->w<float>(x->ws.partials);
   ap.tickets = x->w<uint32_t>(x->ws.tk_att);
   ap.status = sp.status;
   ap.out = out;
+  ap.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  ap.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  ap.k_cache = static_cast<__nv_bfloat16*>(x->buf.k_cache);
+  ap.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
   ap.cap = c.capacity;
+  ap.max_blocks = sp.max_blocks;
   ap.T = (int32_t)g.T;
   ap.S = c.n_sink;
   ap.Bk = c.block_size;
@@ -269,14 +322,13 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   ap.chunks_per_unit = g.chunks_per_unit;
   ap.units = k.units;
   ap.G = k.G;
-  ap.merge_only = g.chunks_per_unit == 0 ? 1 : 0;
-  ap.splits = attend_splits(k.units, g.chunks_per_unit, x->n_sm);
-  ap.grid = ap.merge_only ? k.units : k.units * ap.splits;
+  ap.lin_items = lp.lin_items;
+  ap.splits = lp.splits;
+  ap.grid = k.units * lp.splits;
   ap.scale = x->scale;
-  const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
-  if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
-  e = launch_attend(x->maps, ap, k.D, /*pdl=*/!timed, stream);
+  e = launch_attend(x->maps, ap, k.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (k_new != nullptr) x->T += 1;
   if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
   return HYB_OK;
 }
@@ -317,11 +369,12 @@ int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_
   out->k_eff = g.k_eff;
   out->exact_tokens = g.sink_len + (T - g.win_start) + g.k_eff * cfg->block_size;
   out->chunks_per_unit = g.chunks_per_unit;
-  const int splits = attend_splits(k.units, g.chunks_per_unit, n_sm);
-  out->attend_ctas = g.chunks_per_unit == 0 ? k.units : k.units * splits;
-  out->partial_slots = g.chunks_per_unit == 0 ? 0 : k.units * splits;
-  out->score_ctas_per_unit = g.nb > 0 ? (int32_t)ceil_div(g.nb, kScoreBlocksPerCta) : 0;
-  out->linear_ctas_per_unit = k.D / 32;
+  const LaunchPlan lp = plan_launches(g, k, n_sm);
+  out->select_ctas = lp.select_grid;
+  out->attend_ctas = k.units * lp.splits;
+  out->partial_slots = k.units * lp.splits;
+  out->score_items_per_unit = lp.score_items;
+  out->linear_items_per_unit = lp.lin_items;
   return HYB_OK;
 }
 
@@ -405,6 +458,7 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
     delete x;
     return HYB_ECUDA;
   }
+  x->folded_end = g.ev_end;
   *out = x;
   return HYB_OK;
 }
@@ -412,45 +466,49 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
 int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaStream_t stream) {
   if (x == nullptr || k_new == nullptr || v_new == nullptr) return HYB_EINVAL;
   if (!aligned16(k_new) || !aligned16(v_new)) return HYB_EINVAL;
-  const hyb_attn_config& c = x->cfg;
-  if (x->T >= c.capacity) return HYB_ECAPACITY;
+  if (x->T >= x->cfg.capacity) return HYB_ECAPACITY;
   AppendParams p{};
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
   p.k_cache = static_cast<__nv_bfloat16*>(x->buf.k_cache);
   p.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
-  p.H = x->buf.H;
-  p.zk = x->buf.zk;
-  p.zv = x->buf.zv;
-  p.n = x->buf.n;
-  p.mu = x->buf.mu;
-  p.var = x->buf.var;
-  p.cap = c.capacity;
+  p.cap = x->cfg.capacity;
   p.T = x->T;
-  p.max_blocks = x->ck.max_blocks > 0 ? x->ck.max_blocks : 1;
   p.units = x->ck.units;
-  // after the append the window is [T + 1 - W, T + 1): position T - W leaves it
-  p.p = x->T - c.window;
-  p.evict = (p.p >= c.n_sink) ? 1 : 0;
-  if (p.evict) {
-    p.blk = (int32_t)((p.p - c.n_sink) / c.block_size);
-    p.cnt = (int32_t)((p.p - c.n_sink) % c.block_size + 1);
-  }
   const cudaError_t e = launch_append(p, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->T += 1;
   return HYB_OK;
 }
 
+int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
+  if (x == nullptr) return HYB_EINVAL;
+  const Geometry g = geometry(x->cfg, x->T);
+  if (g.ev_end <= x->folded_end) return HYB_OK;  // nothing evicted since the last fold
+  const LaunchPlan lp = plan_launches(g, x->ck, x->n_sm);
+  SelectParams sp = select_params(x, g, lp);
+  sp.q = nullptr;  // fold only
+  const cudaError_t e = launch_select(sp, x->ck.D, lp.select_grid, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  x->folded_end = g.ev_end;
+  return HYB_OK;
+}
+
 int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out, float* scores_out,
                     cudaStream_t stream) {
-  return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, stream);
+  return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, nullptr, nullptr, stream);
+}
+
+int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, const void* v_new, float* out,
+                           int32_t* sel_out, float* scores_out, cudaStream_t stream) {
+  if (k_new == nullptr || v_new == nullptr) return HYB_EINVAL;
+  return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, k_new, v_new, stream);
 }
 
 int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32_t* sel, float* out,
                                    cudaStream_t stream) {
   if (sel == nullptr) return HYB_EINVAL;
-  return decode_impl(ctx, q, out, sel, nullptr, nullptr, stream);
+  return decode_impl(ctx, q, out, sel, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, const void* v_host,
@@ -467,12 +525,10 @@ int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, 
         cudaMemcpyAsync(x->w<void>(x->ws.stage_v), v_host, U * D * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess)
       return HYB_ECUDA;
   }
-  int rc = decode_impl(x, dq, dout, nullptr, nullptr, nullptr, stream);
+  const void* dk = k_host ? x->w<void>(x->ws.stage_k) : nullptr;
+  const void* dv = k_host ? x->w<void>(x->ws.stage_v) : nullptr;
+  const int rc = decode_impl(x, dq, dout, nullptr, nullptr, nullptr, dk, dv, stream);
   if (rc != HYB_OK) return rc;
-  if (k_host != nullptr) {
-    rc = hyb_attn_append(x, x->w<void>(x->ws.stage_k), x->w<void>(x->ws.stage_v), stream);
-    if (rc != HYB_OK) return rc;
-  }
   if (cudaMemcpyAsync(out_host, dout, U * G * D * sizeof(float), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return HYB_ECUDA;
   return HYB_OK;
@@ -494,7 +550,9 @@ int hyb_attn_decode_noalloc(hyb_attn_ctx* x, const void* q, float* out, int32_t*
   hyb_attn_ctx view = *x;  // the same context with its scratch rebased onto the fixed array
   view.buf.workspace = scratch;
   view.buf.workspace_bytes = HYB_NOALLOC_SCRATCH_BYTES;
-  return decode_impl(&view, q, out, nullptr, sel_out, nullptr, stream);
+  const int drc = decode_impl(&view, q, out, nullptr, sel_out, nullptr, nullptr, nullptr, stream);
+  x->folded_end = view.folded_end;  // the state buffers are the context's own
+  return drc;
 }
 
 int64_t hyb_attn_length(const hyb_attn_ctx* x) { return x ? x->T : -1; }

@@ -1,22 +1,35 @@
-// Exact attention over the gathered sinks, window and selected blocks, the
-// selected blocks' (1 + s) subtraction terms, and the merge under one shared
-// normaliser -- one launch per decode step.
+// Exact attention over the sinks, the window and the top-k selected blocks,
+// the selected blocks' (1 + s) subtraction terms, and the merge under one
+// shared normaliser -- the second launch of a decode step.
 //
 // Work: each unit (batch row, KV head) owns a fixed list of <= 64-token chunks
-// of its exact set X (sink pieces, window pieces, then ceil(Bk/64) pieces per
-// selected block).  A unit's chunks are dealt to `splits` CTAs, CTA part p
-// taking chunks p, p + splits, p + 2*splits, ... (split-K), so every CTA works
-// on one unit, gets a mix of window and selected chunks, and meets the
-// selection (written by the preceding select kernel) as late as possible.
-// Each CTA writes one partial record; the last CTA of a unit to finish (atomic
-// ticket, no spinning) merges the unit's partials with the global linear term.
+// of its exact set X: sink pieces, window pieces, then ceil(Bk/64) pieces per
+// selected block.  A unit's chunks are dealt to `splits` CTAs, CTA part p taking
+// chunks p, p + splits, p + 2*splits, ... (split-K), so every CTA meets its
+// window chunks first and its selected chunks last.  The kernel starts beside
+// the select kernel (one CTA per SM next to its two) and streams the window
+// while the block scores are computed; a CTA waits for the select grid only
+// when its next chunk to load is a selected one.  Then warp 0 selects the
+// unit's top_k blocks from the scores itself (every CTA of the unit derives the
+// same selection; no hand-off between CTAs), while the other warps work on the
+// chunks already loaded.  Each CTA writes one partial record; the last CTA of
+// a unit to finish (atomic ticket, no spinning) merges the unit's records with
+// the global linear term.
 //
-// CTA: 4 warps, two CTAs per SM.  A 3-stage shared-memory ring is filled with
-// TMA tensor loads (cp.async.bulk.tensor, 128-byte swizzle, no multicast): a
-// full 64-token chunk as one 64-row box per tensor, a ragged chunk (sinks, the
-// window's tail, a partial block) as the 16-row boxes it touches.  After the 4
-// warps have consumed chunk j (CTA barrier) thread 0 refills the stage with
-// chunk j + 3.  Warp w handles tokens [16w, 16w + 16) of a chunk.
+// Top-k (ties to the lower block index, ascending output, "SPLA: Block Sparse
+// Plus Linear Attention for Long Context Modeling", "Principled Block Selection
+// via Taylor Expansion"): over order-preserving integer keys of the scores, the
+// k-th largest key is the largest value v with count(key >= v) >= k, found bit
+// by bit below the common prefix of the smallest and largest key (one warp-wide
+// count per bit), then an index-ordered ballot compaction takes every larger
+// key and the lowest-index keys equal to it.
+//
+// CTA: 4 warps.  A 3-stage shared-memory ring is filled with TMA tensor loads
+// (cp.async.bulk.tensor, 128-byte swizzle, no multicast): a full 64-token chunk
+// as one 64-row box per tensor, a ragged chunk (sinks, the window's tail, a
+// partial block) as the 16-row boxes it touches.  After the 4 warps have
+// consumed chunk j (CTA barrier) thread 0 refills the stage with chunk j + 3.
+// Warp w handles tokens [16w, 16w + 16) of a chunk.
 //
 // Per warp and 16 tokens, on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
 // accumulate), with the G <= 4 query heads of the KV group packed into the
@@ -29,18 +42,18 @@
 //                        rows 8-15: the bf16 rounding remainders of rows 0-7
 //                        (hi/lo split), so the weights enter at ~16-bit precision.
 // So the exact part N_ex, D_ex and the subtraction terms N_sel, D_sel come out of
-// the same pass over each K/V tile ("SPLA: Block Sparse Plus Linear Attention
-// for Long Context Modeling", Abstract: residual = global - selected; "SLAKE",
-// Abstract: first-order Taylor exp(s) ~ 1 + s).
-//
-// Launch chaining: this kernel is launched programmatically after the select
-// kernel; it waits for it (griddepcontrol.wait) before reading the selection or
-// the linear term, and lets its own dependents (the append kernel) start once
-// the select kernel has completed -- the append touches nothing this kernel reads.
+// the same pass over each K/V tile ("SPLA", Abstract: residual = global -
+// selected; "SLAKE", Abstract: first-order Taylor exp(s) ~ 1 + s).
 //
 // Merge of a unit (per query head, base-2 exponent m of the exact part):
 //   o = (N_ex + 2^{-m} (N_glob - N_sel)) / (D_ex + 2^{-m} (D_glob - D_sel)),
 // evaluated as the equal form (N_ex 2^m + ...)/(D_ex 2^m + ...) when m < 0.
+// A decode that also appends writes the new token at row T (no kernel of the
+// decode reads that row).
+//
+// Launch chaining (programmatic dependent launch): the select kernel lets this
+// grid start at once; it lets the next decode's select kernel launch at its own
+// start -- that kernel waits for this grid before touching memory.
 #include "hyb_device.cuh"
 #include "hyb_internal.h"
 
@@ -66,8 +79,10 @@ struct AttendSmem {
   uint64_t full[kStages];
   uint64_t merge_bar;
   int4 desc[kStages];                               // start, len, is_sel, unit
-  int32_t sel_cache[kSelCache];                     // the unit's selection row
-  int sel_loaded;
+  int32_t sel_cache[kSelCache];                     // the unit's selection (state 1)
+  int sel_state;    // 0 unknown, 1 in sel_cache, 2 in a global row (sel_row), 3 every block
+  const int32_t* sel_row;
+  int waited;       // thread 0 has waited for the select grid
   int abort_flag;
   int last_flag;
 };
@@ -88,6 +103,192 @@ __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint3
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+// ---------------------------------------------------------------- top-k
+constexpr int kKeysPerLane = 16;  // register-resident keys of the fast path (nb <= 512)
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Index-ordered compaction: take every key above tau and the first need_eq
+// keys equal to it; dst[0, k) ascending (and the optional copy).
+template <class KeyFn>
+__device__ __forceinline__ void topk_emit(int nb, uint32_t tau, uint32_t need_eq, KeyFn key, int32_t* dst,
+                                          int32_t* copy) {
+  const int lane = threadIdx.x & 31;
+  uint32_t taken = 0u, eq_seen = 0u;
+  for (int base = 0; base < nb; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < nb ? key(j) : 0u;
+    const bool gt = j < nb && u > tau;
+    const bool eq = j < nb && u == tau;
+    const uint32_t beq = __ballot_sync(kFull, eq);
+    const uint32_t rank = eq_seen + __popc(beq & lanemask_lt());
+    const bool take = gt || (eq && rank < need_eq);
+    const uint32_t bt = __ballot_sync(kFull, take);
+    if (take) {
+      const uint32_t pos = taken + __popc(bt & lanemask_lt());
+      dst[pos] = j;
+      if (copy) copy[pos] = j;
+    }
+    taken += __popc(bt);
+    eq_seen += __popc(beq);
+  }
+}
+
+// The k < nb largest of scores[0, nb) by one warp; writes dst[0, k) ascending
+// (and copy[0, k) when given).  Keys live in registers when nb <= 32 *
+// kKeysPerLane, else in `kbuf` (kbuf_words shared words) when they fit, else
+// they are re-read from L2 for every count.  Returns whether a score was NaN.
+__device__ bool topk_warp(const float* sc, int nb, int k, int32_t* dst, int32_t* copy, uint32_t* kbuf,
+                          int kbuf_words) {
+  const int lane = threadIdx.x & 31;
+  bool nan = false;
+  if (nb <= 32 * kKeysPerLane) {
+    uint32_t kr[kKeysPerLane];
+    float f[kKeysPerLane];
+#pragma unroll
+    for (int i = 0; i < kKeysPerLane; ++i) {  // all loads in flight at once
+      const int j = lane + 32 * i;
+      f[i] = j < nb ? __ldcg(sc + j) : 0.f;
+    }
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+    for (int i = 0; i < kKeysPerLane; ++i) {
+      const bool v = lane + 32 * i < nb;
+      nan |= v && (f[i] != f[i]);
+      kr[i] = v ? float_key(f[i]) : 0u;  // 0 is below every key a count can reach
+      if (v) {
+        kmin = min(kmin, kr[i]);
+        kmax = max(kmax, kr[i]);
+      }
+    }
+    kmin = __reduce_min_sync(kFull, kmin);
+    kmax = __reduce_max_sync(kFull, kmax);
+    const int free_bits = 32 - __clz(kmin ^ kmax);  // bits below the common prefix
+    uint32_t tau = free_bits == 32 ? 0u : (kmax & ~((1u << free_bits) - 1u));
+    for (int bit = free_bits - 1; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      uint32_t c = 0u;
+#pragma unroll
+      for (int i = 0; i < kKeysPerLane; ++i) c += (kr[i] >= cand) ? 1u : 0u;
+      if (__reduce_add_sync(kFull, c) >= (uint32_t)k) tau = cand;
+    }
+    uint32_t gt = 0u;
+#pragma unroll
+    for (int i = 0; i < kKeysPerLane; ++i) gt += (kr[i] > tau) ? 1u : 0u;
+    gt = __reduce_add_sync(kFull, gt);
+    // the keys of row i are blocks 32i .. 32i+31: index order is row order
+    uint32_t taken = 0u, eq_seen = 0u;
+    const uint32_t need_eq = (uint32_t)k - gt;
+#pragma unroll
+    for (int i = 0; i < kKeysPerLane; ++i) {
+      if (32 * i < nb) {
+        const int j = 32 * i + lane;
+        const bool gtb = j < nb && kr[i] > tau;
+        const bool eqb = j < nb && kr[i] == tau;
+        const uint32_t beq = __ballot_sync(kFull, eqb);
+        const uint32_t rank = eq_seen + __popc(beq & lanemask_lt());
+        const bool take = gtb || (eqb && rank < need_eq);
+        const uint32_t bt = __ballot_sync(kFull, take);
+        if (take) {
+          const uint32_t pos = taken + __popc(bt & lanemask_lt());
+          dst[pos] = j;
+          if (copy) copy[pos] = j;
+        }
+        taken += __popc(bt);
+        eq_seen += __popc(beq);
+      }
+    }
+  } else {
+    const bool staged = nb <= kbuf_words;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j0 = 0; j0 < nb; j0 += 32 * kKeysPerLane) {  // batches of loads in flight
+      float f[kKeysPerLane];
+#pragma unroll
+      for (int i = 0; i < kKeysPerLane; ++i) {
+        const int j = j0 + lane + 32 * i;
+        f[i] = j < nb ? __ldcg(sc + j) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kKeysPerLane; ++i) {
+        const int j = j0 + lane + 32 * i;
+        if (j < nb) {
+          nan |= (f[i] != f[i]);
+          const uint32_t u = float_key(f[i]);
+          if (staged) kbuf[j] = u;
+          kmin = min(kmin, u);
+          kmax = max(kmax, u);
+        }
+      }
+    }
+    __syncwarp();
+    kmin = __reduce_min_sync(kFull, kmin);
+    kmax = __reduce_max_sync(kFull, kmax);
+    auto key = [&](int j) -> uint32_t { return staged ? kbuf[j] : float_key(__ldcg(sc + j)); };
+    const int free_bits = 32 - __clz(kmin ^ kmax);
+    uint32_t tau = free_bits == 32 ? 0u : (kmax & ~((1u << free_bits) - 1u));
+    for (int bit = free_bits - 1; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      uint32_t c = 0u;
+      for (int j = lane; j < nb; j += 32) c += (key(j) >= cand) ? 1u : 0u;
+      if (__reduce_add_sync(kFull, c) >= (uint32_t)k) tau = cand;
+    }
+    uint32_t gt = 0u;
+    for (int j = lane; j < nb; j += 32) gt += (key(j) > tau) ? 1u : 0u;
+    gt = __reduce_add_sync(kFull, gt);
+    topk_emit(nb, tau, (uint32_t)k - gt, key, dst, copy);
+  }
+  return __any_sync(kFull, nan);
+}
+
+// Make the unit's selection known to this CTA (warp 0, all lanes): the
+// caller's row, every block (k >= nb) or none (k == 0), or the top-k of the
+// select kernel's scores.  The writer CTA also fills the caller's copy.
+template <int D>
+__device__ void resolve_selection(const AttendParams& p, AttendSmem<D>& sm, int unit, bool writer) {
+  const int lane = threadIdx.x & 31;
+  int32_t* copy = (p.sel_out != nullptr && writer) ? p.sel_out + (int64_t)unit * p.top_k : nullptr;
+  if (p.sel_given != nullptr) {
+    const int32_t* row = p.sel_given + (int64_t)unit * p.top_k;
+    if (p.top_k <= kSelCache) {
+      for (int j = lane; j < p.top_k; j += 32) sm.sel_cache[j] = __ldg(row + j);
+      if (lane == 0) sm.sel_state = 1;
+    } else if (lane == 0) {
+      sm.sel_row = row;
+      sm.sel_state = 2;
+    }
+  } else if (p.k_eff == 0 || p.k_eff >= p.nb) {  // no block, or every block: no scores needed
+    if (copy)
+      for (int j = lane; j < p.top_k; j += 32) copy[j] = (p.k_eff > 0 && j < p.nb) ? j : -1;
+    if (lane == 0) sm.sel_state = 3;
+  } else {
+    if (lane == 0 && !sm.waited) {  // the scores come from the select grid
+      pdl_wait_primary();
+      sm.waited = 1;
+    }
+    __syncwarp();
+    {
+      int32_t* dst = p.k_eff <= kSelCache ? sm.sel_cache : p.sel + (int64_t)unit * p.top_k;
+      // the combine slots are idle until the main loop ends: they hold the keys
+      uint32_t* kbuf = reinterpret_cast<uint32_t*>(&sm.wpart[0][0]);
+      const int kbuf_words = (int)(sizeof(sm.wpart) / sizeof(uint32_t));
+      const bool nan = topk_warp(p.scores + (int64_t)unit * p.max_blocks, p.nb, p.k_eff, dst, copy, kbuf,
+                                 kbuf_words);
+      if (copy)
+        for (int j = p.k_eff + lane; j < p.top_k; j += 32) copy[j] = -1;
+      if (lane == 0) {
+        if (nan) atomicOr(p.status, HYB_STATUS_NAN_SCORE);
+        sm.sel_row = dst;
+        sm.sel_state = p.k_eff <= kSelCache ? 1 : 2;
+      }
+    }
+  }
+  __syncwarp();
+}
+
 // Merge the `nslot` partial records [slot0, slot0 + nslot) of `unit` with the
 // global linear term and write the unit's output.  All threads of the CTA, after
 // its own chunks are done (the stage buffers are free).  The unit's records are
@@ -106,7 +307,11 @@ __device__ void merge_unit(const AttendParams& p, int unit, int64_t slot0, int n
   float* s_Dsel = sm.mscr + 8;
   const int warp = tid >> 5, lane = tid & 31;
   const float* base = p.partials + slot0 * PF;
-  pdl_wait_primary();  // the linear term comes from the preceding select kernel
+  if (tid == 0 && !sm.waited) {  // the linear term comes from the select grid
+    pdl_wait_primary();
+    sm.waited = 1;
+  }
+  __syncthreads();
   {                    // warp h: max of head h over all slots
     float mx = -INFINITY;
     for (int k = lane; k < nslot; k += 32) mx = fmaxf(mx, __ldcg(base + (int64_t)k * PF + warp));
@@ -174,37 +379,55 @@ __device__ void merge_unit(const AttendParams& p, int unit, int64_t slot0, int n
   }
   __syncthreads();
   const int G = p.G;
-  const float* lin = p.lin + (int64_t)unit * G * (D + 1);
-  for (int e = tid; e < G * D; e += kAttendThreads) {
-    const int i = e / D, d = e % D;
-    const float Ms = s_M[i];
-    const float Nex = s_vec[i * D + d], Nsel = s_vec[4 * D + i * D + d];
-    const float Dex = s_Dex[i], Dsel = s_Dsel[i];
-    const float Ng = __ldcg(lin + (int64_t)i * (D + 1) + d);
-    const float Dg = __ldcg(lin + (int64_t)i * (D + 1) + D);
-    float num, den;
-    if (Ms >= 0.f) {
-      const float f = exp2f(-Ms);
-      num = Nex + f * (Ng - Nsel);
-      den = Dex + f * (Dg - Dsel);
-    } else {
-      const float f = exp2f(Ms);
-      num = Nex * f + (Ng - Nsel);
-      den = Dex * f + (Dg - Dsel);
+  const float* lin = p.lin + (int64_t)unit * p.lin_items * G * (D + 1);  // [lin_items][G][D + 1]
+  // every load of the linear term first (independent, in flight together), then
+  // the arithmetic and the stores
+  constexpr int EPT = kMaxGroup * D / kAttendThreads;  // output elements per thread
+  float Ng[EPT], Dg[EPT];
+#pragma unroll
+  for (int r = 0; r < EPT; ++r) {
+    const int e = tid + r * kAttendThreads;
+    Ng[r] = 0.f;
+    Dg[r] = 0.f;
+    if (e < G * D) {
+      const int i = e / D, d = e % D;
+      for (int g = 0; g < p.lin_items; ++g) Ng[r] += __ldcg(lin + ((int64_t)g * G + i) * (D + 1) + d);
+      Dg[r] = __ldcg(lin + (int64_t)i * (D + 1) + D);
     }
-    const float o = num / den;
-    p.out[((int64_t)unit * G + i) * D + d] = o;
-    if (!(den > 0.f)) atomicOr(p.status, HYB_STATUS_DENOMINATOR);
-    if (!isfinite(o)) atomicOr(p.status, HYB_STATUS_NONFINITE);
   }
+  uint32_t flags = 0u;
+#pragma unroll
+  for (int r = 0; r < EPT; ++r) {
+    const int e = tid + r * kAttendThreads;
+    if (e < G * D) {
+      const int i = e / D, d = e % D;
+      const float Ms = s_M[i];
+      const float Nex = s_vec[i * D + d], Nsel = s_vec[4 * D + i * D + d];
+      const float Dex = s_Dex[i], Dsel = s_Dsel[i];
+      float num, den;
+      if (Ms >= 0.f) {
+        const float f = exp2f(-Ms);
+        num = Nex + f * (Ng[r] - Nsel);
+        den = Dex + f * (Dg[r] - Dsel);
+      } else {
+        const float f = exp2f(Ms);
+        num = Nex * f + (Ng[r] - Nsel);
+        den = Dex * f + (Dg[r] - Dsel);
+      }
+      const float o = num / den;
+      p.out[((int64_t)unit * G + i) * D + d] = o;
+      if (!(den > 0.f)) flags |= HYB_STATUS_DENOMINATOR;
+      if (!isfinite(o)) flags |= HYB_STATUS_NONFINITE;
+    }
+  }
+  if (flags) atomicOr(p.status, flags);
 }
 
 // Hand local chunk j (unit chunk index ci) to stage j % kStages: write its
 // descriptor and start the TMA loads of its K and V rows (rows past the chunk
-// end inside a box are read too and ignored).  Called by thread 0 only.
+// end inside a box are read too and ignored).  Thread 0.
 template <int D>
-__device__ void issue_chunk(const KVMaps* tm, const AttendParams& p, AttendSmem<D>& sm, int unit, int ci, int j,
-                            bool& waited) {
+__device__ void issue_chunk(const KVMaps* tm, const AttendParams& p, AttendSmem<D>& sm, int unit, int ci, int j) {
   using S = AttendSmem<D>;
   const int stage = j % kStages;
   int start = 0, len = 0, is_sel = 0;
@@ -214,33 +437,14 @@ __device__ void issue_chunk(const KVMaps* tm, const AttendParams& p, AttendSmem<
   } else if (ci < p.n_sink_chunks + p.n_win_chunks) {
     start = p.win_start + (ci - p.n_sink_chunks) * kTile;
     len = min(kTile, p.T - start);
-  } else {
-    if (!waited) {  // the selection is written by the preceding select kernel
-      pdl_wait_primary();
-      pdl_allow_dependents();  // the select kernel is complete: the append may run
-      waited = true;
-    }
+  } else {  // the selection is resolved before a selected chunk is issued
     const int s = ci - p.n_sink_chunks - p.n_win_chunks;
     const int slot = s / p.chunks_per_block, piece = s % p.chunks_per_block;
     is_sel = 1;
     int jb = -1;
     if (slot < p.k_eff) {
-      const int32_t* row = p.sel + (int64_t)unit * p.top_k;
-      if (p.top_k <= kSelCache) {  // one round trip for the whole row, then shared memory
-        if (!sm.sel_loaded) {
-          for (int t0 = 0; t0 < p.top_k; t0 += 16) {
-            int32_t v[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t) v[t] = t0 + t < p.top_k ? __ldcg(row + t0 + t) : -1;
-#pragma unroll
-            for (int t = 0; t < 16; ++t) sm.sel_cache[(t0 + t) & (kSelCache - 1)] = v[t];
-          }
-          sm.sel_loaded = 1;
-        }
-        jb = sm.sel_cache[slot];
-      } else {
-        jb = __ldcg(row + slot);
-      }
+      const int st = sm.sel_state;
+      jb = st == 3 ? slot : st == 1 ? sm.sel_cache[slot] : __ldcg(sm.sel_row + slot);
     }
     if (jb >= 0 && jb < p.nb) {
       const int bs = p.S + jb * p.Bk;
@@ -274,40 +478,52 @@ __device__ void issue_chunk(const KVMaps* tm, const AttendParams& p, AttendSmem<
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm)
+__global__ void __maxnreg__(kAttendMaxRegs)
     attend_kernel(const __grid_constant__ KVMaps tm, const AttendParams p) {
   constexpr int PF = partial_floats(D);
   constexpr int NT8 = D / 8;   // 8-column tiles of the head dimension
   constexpr int KS = D / 16;   // k-steps of the QK product
   extern __shared__ uint8_t smem_raw[];
-  AttendSmem<D>& sm = *reinterpret_cast<AttendSmem<D>*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned (the 128-byte swizzle repeats every 1024 bytes); offsetting
+  // the shared array keeps every access through `sm` in the shared space
+  AttendSmem<D>& sm = *reinterpret_cast<AttendSmem<D>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
 
   if (tid == 0) {
+    tma_prefetch_desc(&tm.k64);
+    tma_prefetch_desc(&tm.v64);
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
     mbar_init(&sm.merge_bar, 1);
-    sm.sel_loaded = 0;
+    sm.sel_state = 0;
+    sm.waited = 0;
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  if (p.merge_only) {  // empty exact set: output = global linear term only
-    merge_unit<D>(p, cta, 0, 0, tid, sm);
-    if (tid == 0) pdl_allow_dependents();
-    return;
-  }
+  // the next decode's select kernel may be scheduled; it waits for this grid
+  pdl_allow_dependents();
   const int unit = cta / p.splits, part = cta % p.splits;
   const int n_local = (p.chunks_per_unit - part + p.splits - 1) / p.splits;  // chunks part + j*splits
+  const int n_pre = p.n_sink_chunks + p.n_win_chunks;                       // selection-free chunks
+  const int j_sel = part < n_pre ? (n_pre - part + p.splits - 1) / p.splits : 0;  // first selected local chunk
+  // the CTA that owns the unit's first selected chunk fills the caller's copy
+  // of the selection (part 0 when there is none)
+  const bool writer = part == (p.chunks_per_unit > n_pre ? n_pre % p.splits : 0);
 
-  bool waited = false;  // thread 0: has waited for the select kernel
-  int next_issue = 0;   // thread 0: next local chunk to issue
-  if (tid == 0) {
-    tma_prefetch_desc(&tm.k64);
-    tma_prefetch_desc(&tm.v64);
-    for (; next_issue < n_local && next_issue < kStages; ++next_issue)
-      issue_chunk<D>(&tm, p, sm, unit, part + next_issue * p.splits, next_issue, waited);
+  if (warp == 0 && ((j_sel == 0 && n_local > 0) || (writer && p.chunks_per_unit == n_pre)))
+    resolve_selection<D>(p, sm, unit, writer);
+  int next_issue = 0;  // thread 0: next local chunk to issue
+  if (tid == 0)
+    for (; next_issue < n_local && next_issue < kStages && (next_issue < j_sel || sm.sel_state != 0); ++next_issue)
+      issue_chunk<D>(&tm, p, sm, unit, part + next_issue * p.splits, next_issue);
+  if (p.k_new != nullptr && part == 0 && tid < D / 4) {
+    // the decode's appended token: row T of the caches (16 bytes per thread)
+    const bool is_v = tid >= D / 8;
+    const int e = (tid % (D / 8)) * 8;
+    const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + (int64_t)unit * D + e;
+    __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e;
+    *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
   }
 
   const int g = lane >> 2, tig = lane & 3;
@@ -415,16 +631,15 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm)
       }
     }
     __syncthreads();  // every warp is done with this stage
-    if (tid == 0 && next_issue < n_local && !*(volatile int*)&sm.abort_flag) {
-      issue_chunk<D>(&tm, p, sm, unit, part + next_issue * p.splits, next_issue, waited);
-      ++next_issue;
+    if (warp == 0) {
+      // the next chunk to load may be the first selected one: warp 0 resolves
+      // the selection now, while warps 1-3 go on with the chunks already loaded
+      const int ni = __shfl_sync(kFull, next_issue, 0);
+      if (ni < n_local && ni >= j_sel && sm.sel_state == 0) resolve_selection<D>(p, sm, unit, writer);
+      if (lane == 0)
+        for (; next_issue < n_local && next_issue <= j + kStages && !*(volatile int*)&sm.abort_flag; ++next_issue)
+          issue_chunk<D>(&tm, p, sm, unit, part + next_issue * p.splits, next_issue);
     }
-  }
-
-  if (tid == 0 && !waited) {  // a CTA with no selected chunk
-    pdl_wait_primary();
-    pdl_allow_dependents();
-    waited = true;
   }
 
   // ---- combine the 4 warps' partials in registers (a tree through two shared
@@ -496,6 +711,9 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm)
     for (int j = next_issue - 1; j >= 0 && j >= next_issue - kStages; --j)
       mbar_wait_bounded(&sm.full[j % kStages], (j / kStages) & 1, kWaitLimit);
   }
+  // this grid completes only after the select grid (its scores and linear term
+  // are read above; a CTA that needed neither still waits, in one thread)
+  if (tid == 0 && !sm.waited) pdl_wait_primary();
 }
 
 }  // namespace
@@ -512,7 +730,7 @@ cudaError_t prepare_attend(int D) {
   return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
 }
 
-cudaError_t launch_attend(const CUtensorMap* maps, const AttendParams& p, int D, bool pdl, cudaStream_t s) {
+cudaError_t launch_attend(const CUtensorMap* maps, const AttendParams& p, int D, cudaStream_t s) {
   KVMaps tm;
   tm.k64 = maps[0];
   tm.v64 = maps[1];
@@ -527,7 +745,7 @@ cudaError_t launch_attend(const CUtensorMap* maps, const AttendParams& p, int D,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = 1;
   if (D == 128) return cudaLaunchKernelEx(&cfg, attend_kernel<128>, tm, p);
   return cudaLaunchKernelEx(&cfg, attend_kernel<64>, tm, p);
 }

@@ -1,26 +1,38 @@
-// Block scoring, top-k block selection and the global linear term of one
-// decode step (one launch).
+// Block scoring and the global linear term of one decode step, plus the fold
+// of the evictions since the previous decode into the state (one launch).
 //
-// Grid (score_ctas + lin_ctas, units).  A unit is one (batch row, KV head).
+// Persistent grid of kSelectCtasPerSm CTAs per SM.  The work of a decode is a
+// list of equal-sized items, unit-major (a unit is one (batch row, KV head)):
+// per unit, ceil(nb / R) score items of R consecutive blocks, then
+// sel_lin_items(D) linear items of sel_item_rows(D) rows of H each.  CTA c
+// takes the contiguous item range [c*N/grid, (c+1)*N/grid), so its data is
+// one near-sequential stream; thread 0 pulls each item (the rows, and the
+// unit's query heads) into a kSelStages-deep shared-memory ring with untiled
+// bulk copies (cp.async.bulk, no multicast) and the CTA works from there.
 //
-// * Score CTAs: each scores up to kScoreBlocksPerCta candidate blocks with the
-//   second-order Taylor block score of "SPLA: Block Sparse Plus Linear Attention
-//   for Long Context Modeling" (Abstract; "Principled Block Selection via Taylor
-//   Expansion"), summed over the query heads of the KV group ("Grouped
-//   Sparsity"):
-//       score_j = sum_i q'_i . mu_j + 1/2 sum_i sum_c q'_ic^2 var_jc
-//               = Q1 . mu_j + Q2 . var_j,   Q1 = sum_i q'_i,  Q2 = 1/2 sum_i q'_i^2,
-//   i.e. two fp32 dot products per block, read with 16-byte vector loads: the
-//   kernel is a single streaming pass over the block statistics.
-//   The last score CTA of a unit (atomic ticket, no spinning) selects the top_k
-//   blocks: a 4-pass 8-bit radix select finds the k-th largest score key, then
-//   an order-preserving block-wide compaction emits every larger block plus the
-//   lowest-index blocks equal to it -- ties go to the lower index and the output
-//   is ascending.
-// * Linear CTAs: phi(q)^T state for the global linear term of SLAKE's
-//   first-order Taylor kernel (exp(s) ~ 1 + s): per query head i,
-//       N_glob_i = zv + H^T q'_i,   D_glob_i = n + q'_i . zk,
-//   each CTA owning 32 columns of H (coalesced row reads, fp32 accumulation).
+// * Score items: the second-order Taylor block score of "SPLA: Block Sparse
+//   Plus Linear Attention for Long Context Modeling" (Abstract; "Principled
+//   Block Selection via Taylor Expansion"), summed over the query heads of the
+//   KV group ("Grouped Sparsity"):
+//       score_j = sum_i ( q'_i . mu_j + 1/2 sum_c q'_ic^2 var_jc ).
+//   The top-k over these scores runs in the attention kernel, which reads them.
+// * Linear items: phi(q)^T state of the global linear term of SLAKE's
+//   first-order Taylor kernel (exp(s) ~ 1 + s), per query head i and row group g:
+//       N_i += sum_{r in g} q'_ir H[r][:]  (+ zv in group 0),
+//       D_i  = n + q'_i . zk               (group 0),
+//   written as one partial per row group; the attention merge adds the groups.
+// * Evictions since the previous decode (positions [fold_begin, fold_end) of
+//   the evicted stream, usually one token) are folded into the rows each item
+//   holds before it uses them: H += k v^T, zk += k, zv += v, n += 1 (the
+//   recurrence of SPLA's residual linear attention) and Welford's running mean
+//   / population variance of the token's block (B. P. Welford, Technometrics
+//   4(3), 1962).  With q == null the kernel only folds (items with nothing to
+//   fold load nothing).
+//
+// Launch chaining (programmatic dependent launch): the first kernel of a
+// decode; it waits for its predecessor grid before touching memory, then lets
+// the attention kernel start at once, which streams the window beside it and
+// waits for this grid only before it needs the scores.
 #include "hyb_device.cuh"
 #include "hyb_internal.h"
 
@@ -30,280 +42,315 @@ namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
 
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = bf16_lo(w[e]);
+    f[2 * e + 1] = bf16_hi(w[e]);
+  }
 }
 
-constexpr int kKeysInSmem = 4096;  // blocks whose keys fit the staging buffer (16 KB)
+template <int D>
+struct SelectSmem {
+  struct Stage {
+    float data[kSelItemBytes / 4];         // mean rows then variance rows, or rows of H
+    __nv_bfloat16 q[kMaxGroup * D];        // the item's query heads
+  };
+  Stage st[kSelStages];
+  uint64_t full[kSelStages];
+  int abort;
+};
 
-// Top-k of scores[0, nb) with ties to the lower index; writes sel[0, top_k)
-// ascending, -1 padded.  Runs on one CTA of kSelectThreads threads.  The score
-// keys are staged once in shared memory (when nb <= kKeysInSmem), so the radix
-// passes and the compaction run at shared-memory latency.
-__device__ void select_top_k(const SelectParams& p, int unit) {
-  __shared__ uint32_t s_keys[kKeysInSmem];
-  __shared__ uint32_t s_hist[256];
-  __shared__ uint32_t s_wcnt[2][kSelectThreads / 32];
-  __shared__ uint32_t s_digit, s_above;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int nwarps = kSelectThreads / 32;
-  const float* sc = p.scores + (int64_t)unit * p.max_blocks;
-  int32_t* sel = p.sel + (int64_t)unit * p.top_k;
-  const int nb = p.nb;
-  const int k = p.k_eff;
+// ---------------------------------------------------------------- items
+__device__ __forceinline__ bool item_has_fold(const SelectParams& p, int local, int R) {
+  if (p.fold_end <= p.fold_begin) return false;
+  if (local >= p.score_items) return true;  // every linear item folds into its rows
+  const int64_t j0 = (int64_t)local * R;
+  const int64_t jb0 = (p.fold_begin - p.S) / p.Bk, jb1 = (p.fold_end - 1 - p.S) / p.Bk;
+  return jb1 >= j0 && jb0 < j0 + R;
+}
 
-  const bool staged = nb <= kKeysInSmem;
-  auto key = [&](int j) -> uint32_t { return staged ? s_keys[j] : float_key(__ldcg(sc + j)); };
-  if (k >= nb) {
-    for (int j = tid; j < p.top_k; j += kSelectThreads) sel[j] = j < nb ? j : -1;
+// Start the copies of item `it` into stage `stage` (thread 0).
+template <int D>
+__device__ void issue_item(const SelectParams& p, SelectSmem<D>& sm, int it, int stage) {
+  constexpr int R = sel_item_blocks(D), RL = sel_item_rows(D);
+  const int unit = it / p.items_per_unit, local = it % p.items_per_unit;
+  auto& st = sm.st[stage];
+  if (p.q == nullptr && !item_has_fold(p, local, R)) {
+    mbar_arrive(&sm.full[stage]);
+    return;
+  }
+  const uint32_t qbytes = p.q ? (uint32_t)(p.G * D * 2) : 0u;
+  uint32_t bytes;
+  const float* src0;
+  const float* src1 = nullptr;
+  if (local < p.score_items) {
+    const int j0 = local * R;
+    const int nblk = min(R, p.nb - j0);
+    bytes = (uint32_t)(nblk * D * 4);
+    src0 = p.mu + ((int64_t)unit * p.max_blocks + j0) * D;
+    src1 = p.var + ((int64_t)unit * p.max_blocks + j0) * D;
   } else {
-    bool nan_seen = false;
-    if (staged) {
-      for (int j = tid; j < nb; j += kSelectThreads) {
-        const float f = __ldcg(sc + j);
-        nan_seen |= (f != f);
-        s_keys[j] = float_key(f);
-      }
-    }
-    uint32_t prefix = 0, pmask = 0, need = (uint32_t)k;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int i = tid; i < 256; i += kSelectThreads) s_hist[i] = 0;
-      __syncthreads();
-      for (int j = tid; j < nb; j += kSelectThreads) {
-        const uint32_t u = key(j);
-        if (!staged && pass == 0 && u == 0u) nan_seen |= (__ldcg(sc + j) != __ldcg(sc + j));
-        if ((u & pmask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane l owns digits 255-8l .. 248-8l, highest first
-        uint32_t cnt[8], local = 0;
+    const int r0 = (local - p.score_items) * RL;
+    bytes = (uint32_t)(RL * D * 4);
+    src0 = p.H + ((int64_t)unit * D + r0) * D;
+  }
+  mbar_arrive_expect_tx(&sm.full[stage], qbytes + (src1 ? 2u : 1u) * bytes);
+  if (qbytes) bulk_load(smem_u32(st.q), p.q + (int64_t)unit * p.G * D, qbytes, &sm.full[stage]);
+  bulk_load(smem_u32(st.data), src0, bytes, &sm.full[stage]);
+  if (src1) bulk_load(smem_u32(st.data + R * D), src1, bytes, &sm.full[stage]);
+}
+
+// Score item: R blocks, D/8 lanes per block, 8 channels per lane.
+template <int D>
+__device__ void score_item(const SelectParams& p, typename SelectSmem<D>::Stage& st, int unit, int local) {
+  constexpr int R = sel_item_blocks(D), LPB = D / 8;
+  static_assert(R * LPB == kSelectThreads, "one thread per 8 channels of a block");
+  const int tid = threadIdx.x, b = tid / LPB, li = tid % LPB;
+  const int j = local * R + b;
+  const bool valid = j < p.nb;
+  float m[8], v[8];
+  {
+    const float4* pm = reinterpret_cast<const float4*>(st.data + b * D + li * 8);
+    const float4* pv = reinterpret_cast<const float4*>(st.data + R * D + b * D + li * 8);
+    const float4 m0 = pm[0], m1 = pm[1], v0 = pv[0], v1 = pv[1];
+    m[0] = m0.x; m[1] = m0.y; m[2] = m0.z; m[3] = m0.w; m[4] = m1.x; m[5] = m1.y; m[6] = m1.z; m[7] = m1.w;
+    v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+  }
+  if (valid && p.fold_end > p.fold_begin) {
+    const int64_t bs = p.S + (int64_t)j * p.Bk;
+    const int64_t a = max(bs, p.fold_begin), e = min(bs + p.Bk, p.fold_end);
+    if (a < e) {
+      for (int64_t t = a; t < e; ++t) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.k_cache + ((int64_t)unit * p.cap + t) * D + li * 8));
+        float x[8];
+        bf16x8_to_f32(raw, x);
+        if (t == bs) {  // the block's first token: the stored row is not read
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          cnt[e] = s_hist[255 - 8 * lane - e];
-          local += cnt[e];
-        }
-        uint32_t incl = local;
+          for (int c = 0; c < 8; ++c) {
+            m[c] = x[c];
+            v[c] = 0.f;
+          }
+        } else {
+          const float cnt = (float)(t - bs + 1);
+          const float inv = 1.f / cnt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t v = __shfl_up_sync(kFull, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const uint32_t excl = incl - local;
-        if (excl < need && incl >= need) {
-          uint32_t c = excl;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (c + cnt[e] >= need) {
-              s_digit = 255u - 8u * lane - e;
-              s_above = c;
-              break;
-            }
-            c += cnt[e];
+          for (int c = 0; c < 8; ++c) {
+            const float delta = x[c] - m[c];
+            const float m1 = m[c] + delta * inv;
+            v[c] = (v[c] * (cnt - 1.f) + delta * (x[c] - m1)) * inv;
+            m[c] = m1;
           }
         }
       }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      pmask |= 0xffu << shift;
-      need -= s_above;
-      __syncthreads();
+      float4* gm = reinterpret_cast<float4*>(p.mu + ((int64_t)unit * p.max_blocks + j) * D + li * 8);
+      float4* gv = reinterpret_cast<float4*>(p.var + ((int64_t)unit * p.max_blocks + j) * D + li * 8);
+      gm[0] = make_float4(m[0], m[1], m[2], m[3]);
+      gm[1] = make_float4(m[4], m[5], m[6], m[7]);
+      gv[0] = make_float4(v[0], v[1], v[2], v[3]);
+      gv[1] = make_float4(v[4], v[5], v[6], v[7]);
     }
-    if (nan_seen) atomicOr(p.status, HYB_STATUS_NAN_SCORE);
-    const uint32_t tau = prefix;  // key of the k-th largest score
-    // `need` blocks equal to tau are taken, lowest index first
-    uint32_t taken_base = 0, eq_base = 0;
-    for (int base = 0; base < nb; base += kSelectThreads) {
-      const int j = base + tid;
-      const uint32_t u = j < nb ? key(j) : 0u;
-      const bool gt = j < nb && u > tau;
-      const bool eq = j < nb && u == tau;
-      const uint32_t beq = __ballot_sync(kFull, eq);
-      if (lane == 0) s_wcnt[0][warp] = __popc(beq);
-      __syncthreads();
-      uint32_t eq_rank = eq_base + __popc(beq & lanemask_lt());
-      for (int w = 0; w < warp; ++w) eq_rank += s_wcnt[0][w];
-      const bool take = gt || (eq && eq_rank < need);
-      const uint32_t bt = __ballot_sync(kFull, take);
-      if (lane == 0) s_wcnt[1][warp] = __popc(bt);
-      __syncthreads();
-      uint32_t pos = taken_base + __popc(bt & lanemask_lt());
-      for (int w = 0; w < warp; ++w) pos += s_wcnt[1][w];
-      if (take) sel[pos] = j;
-      uint32_t tt = 0, te = 0;
-      for (int w = 0; w < nwarps; ++w) {
-        tt += s_wcnt[1][w];
-        te += s_wcnt[0][w];
+  }
+  if (p.q == nullptr) return;
+  float acc = 0.f;  // sum over the group's heads of q'_i . mu + 1/2 q'_i^2 . var (8 channels)
+  for (int i = 0; i < p.G; ++i) {
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(st.q + i * D + li * 8), f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float qs = f[c] * p.scale;
+      acc += qs * (m[c] + 0.5f * qs * v[c]);
+    }
+  }
+#pragma unroll
+  for (int o = LPB / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+  if (li == 0 && valid) p.scores[(int64_t)unit * p.max_blocks + j] = acc;
+}
+
+// Linear item `rg`: rows [rg*RL, (rg+1)*RL) of H; thread (h, c) holds column c
+// of RPT consecutive rows.
+template <int D>
+__device__ void lin_item(const SelectParams& p, typename SelectSmem<D>::Stage& st, int unit, int rg) {
+  constexpr int RL = sel_item_rows(D), NH = kSelectThreads / D, RPT = RL / NH;
+  static_assert(RPT % 8 == 0, "rows per thread come in 16-byte key loads");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid % D, h = tid / D;
+  const int rl = h * RPT;          // first row of this thread inside the item
+  const int r0 = rg * RL + rl;     // ... and inside H
+  const bool fold = p.fold_end > p.fold_begin;
+  if (p.q == nullptr && !fold) return;
+  float hv[RPT];
+#pragma unroll
+  for (int rr = 0; rr < RPT; ++rr) hv[rr] = st.data[(rl + rr) * D + c];
+  const bool zrow = (rg == 0 && h == 0);                     // owner of zk[c], zv[c]
+  const bool nown = (rg == 0 && tid == kSelectThreads - 32);  // owner of n (writes D_glob too)
+  float zkc = 0.f, zvc = 0.f, n_new = 0.f;
+  if (zrow) {
+    zkc = p.zk[(int64_t)unit * D + c];
+    zvc = p.zv[(int64_t)unit * D + c];
+  }
+  if (nown) n_new = p.n[unit];
+  if (fold) {
+    const int64_t ub = (int64_t)unit * p.cap;
+    for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
+      const __nv_bfloat16* kt = p.k_cache + (ub + t) * D;
+      const float vt = __bfloat162float(p.v_cache[(ub + t) * D + c]);
+#pragma unroll
+      for (int r8 = 0; r8 < RPT; r8 += 8) {
+        float kf[8];
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kt + r0 + r8)), kf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) hv[r8 + e] += kf[e] * vt;
       }
-      taken_base += tt;
-      eq_base += te;
-      __syncthreads();
+      if (zrow) {
+        zkc += __bfloat162float(kt[c]);
+        zvc += vt;
+      }
     }
-    for (int j = k + tid; j < p.top_k; j += kSelectThreads) sel[j] = -1;
-  }
-  if (p.sel_out != nullptr) {
-    __syncthreads();
-    __threadfence_block();
-    for (int j = tid; j < p.top_k; j += kSelectThreads)
-      p.sel_out[(int64_t)unit * p.top_k + j] = sel[j];
-  }
-}
-
-template <int D>
-__device__ void score_blocks(const SelectParams& p, int unit, const float (*s_q)[D]) {
-  __shared__ __align__(16) float s_q1[D];
-  __shared__ __align__(16) float s_q2[D];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int c = tid; c < D; c += kSelectThreads) {
-    float a = 0.f, b = 0.f;
-    for (int i = 0; i < p.G; ++i) {
-      a += s_q[i][c];
-      b += s_q[i][c] * s_q[i][c];
-    }
-    s_q1[c] = a;
-    s_q2[c] = 0.5f * b;
-  }
-  __syncthreads();
-
-  constexpr int LPB = D / 8;                  // lanes per block, 8 channels each
-  constexpr int BPW = 32 / LPB;               // blocks per warp per pass
-  constexpr int BPP = (kSelectThreads / 32) * BPW;  // blocks per CTA pass
-  constexpr int PASSES = kScoreBlocksPerCta / BPP;
-  static_assert(kScoreBlocksPerCta % BPP == 0, "blocks per CTA must be a multiple of the pass width");
-  const int sub = lane / LPB, li = lane % LPB;
-  const float4 qa0 = *reinterpret_cast<const float4*>(&s_q1[li * 8]);
-  const float4 qa1 = *reinterpret_cast<const float4*>(&s_q1[li * 8 + 4]);
-  const float4 qb0 = *reinterpret_cast<const float4*>(&s_q2[li * 8]);
-  const float4 qb1 = *reinterpret_cast<const float4*>(&s_q2[li * 8 + 4]);
-  const int j0 = blockIdx.x * kScoreBlocksPerCta;
-  const int64_t ubase = (int64_t)unit * p.max_blocks;
-  const float* mu = p.mu + ubase * D;
-  const float* var = p.var + ubase * D;
-
-  float4 m0[PASSES], m1[PASSES], v0[PASSES], v1[PASSES];
+    float* Hg = p.H + ((int64_t)unit * D + r0) * D + c;
 #pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {           // issue every load first
-    const int j = j0 + ps * BPP + warp * BPW + sub;
-    if (j < p.nb) {
-      const float4* pm = reinterpret_cast<const float4*>(mu + (int64_t)j * D + li * 8);
-      const float4* pv = reinterpret_cast<const float4*>(var + (int64_t)j * D + li * 8);
-      m0[ps] = __ldg(pm);
-      m1[ps] = __ldg(pm + 1);
-      v0[ps] = __ldg(pv);
-      v1[ps] = __ldg(pv + 1);
-    } else {
-      m0[ps] = m1[ps] = v0[ps] = v1[ps] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int rr = 0; rr < RPT; ++rr) Hg[(int64_t)rr * D] = hv[rr];
+    if (zrow) {
+      p.zk[(int64_t)unit * D + c] = zkc;
+      p.zv[(int64_t)unit * D + c] = zvc;
+    }
+    if (nown) {
+      n_new += (float)(p.fold_end - p.fold_begin);
+      p.n[unit] = n_new;
     }
   }
-#pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    float acc = qa0.x * m0[ps].x + qa0.y * m0[ps].y + qa0.z * m0[ps].z + qa0.w * m0[ps].w;
-    acc += qa1.x * m1[ps].x + qa1.y * m1[ps].y + qa1.z * m1[ps].z + qa1.w * m1[ps].w;
-    acc += qb0.x * v0[ps].x + qb0.y * v0[ps].y + qb0.z * v0[ps].z + qb0.w * v0[ps].w;
-    acc += qb1.x * v1[ps].x + qb1.y * v1[ps].y + qb1.z * v1[ps].z + qb1.w * v1[ps].w;
-#pragma unroll
-    for (int o = LPB / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-    const int j = j0 + ps * BPP + warp * BPW + sub;
-    if (li == 0 && j < p.nb) p.scores[ubase + j] = acc;
-  }
+  if (p.q == nullptr) return;
 
-  if (!p.do_select) return;
-  __syncthreads();
-  __shared__ int s_last;
-  if (tid == 0) {
-    __threadfence();  // release this CTA's scores (ordered after the barrier)
-    const uint32_t prev = atomicAdd(&p.tickets[unit], 1u);
-    s_last = (prev == (uint32_t)p.score_ctas - 1u);
-    __threadfence();
-  }
-  __syncthreads();
-  if (!s_last) return;
-  select_top_k(p, unit);
-  if (tid == 0) p.tickets[unit] = 0u;  // ready for the next decode
-}
-
-template <int D>
-__device__ void linear_term(const SelectParams& p, int unit, const float (*s_q)[D]) {
-  __shared__ float s_red[kSelectThreads / 32][kMaxGroup][32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = kSelectThreads / 32;
-  constexpr int RPW = D / NW;  // rows of H per warp
-  const int cb = blockIdx.x - p.score_ctas;
-  const int c = cb * 32 + lane;
-  const float* H = p.H + (int64_t)unit * D * D;
+  const int G = p.G;
   float acc[kMaxGroup] = {0.f, 0.f, 0.f, 0.f};
-  float h[RPW];
+  float zdot[kMaxGroup] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) h[rr] = __ldg(H + (int64_t)(warp * RPW + rr) * D + c);
+  for (int i = 0; i < kMaxGroup; ++i) {
+    if (i < G) {
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int r = warp * RPW + rr;
+      for (int r8 = 0; r8 < RPT; r8 += 8) {
+        float qf[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(st.q + i * D + r0 + r8), qf);
 #pragma unroll
-    for (int i = 0; i < kMaxGroup; ++i)
-      if (i < p.G) acc[i] += s_q[i][r] * h[rr];
-  }
-#pragma unroll
-  for (int i = 0; i < kMaxGroup; ++i) s_red[warp][i][lane] = acc[i];
-  __syncthreads();
-  const int64_t lbase = (int64_t)unit * p.G * (D + 1);
-  if (warp == 0) {
-    const float zv = __ldg(p.zv + (int64_t)unit * D + c);
-    for (int i = 0; i < p.G; ++i) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) s += s_red[w][i][lane];
-      p.lin[lbase + (int64_t)i * (D + 1) + c] = zv + s;
+        for (int e = 0; e < 8; ++e) acc[i] += qf[e] * hv[r8 + e];
+      }
+      acc[i] *= p.scale;
+      if (zrow) zdot[i] = __bfloat162float(st.q[i * D + c]) * p.scale * zkc;
     }
-  } else if (warp == 1 && cb == 0) {
-    const float* zk = p.zk + (int64_t)unit * D;
-    for (int i = 0; i < p.G; ++i) {
+  }
+  __syncthreads();  // every thread has its rows: the stage data becomes the reduction buffer
+  float* red = st.data;             // [NH][G][D]
+  float* zred = st.data + NH * kMaxGroup * D;  // [G][D]
+#pragma unroll
+  for (int i = 0; i < kMaxGroup; ++i) {
+    if (i < G) {
+      red[(h * kMaxGroup + i) * D + c] = acc[i];
+      if (zrow) zred[i * D + c] = zdot[i];
+    }
+  }
+  __syncthreads();
+  float* lin = p.lin + ((int64_t)unit * p.lin_items + rg) * G * (D + 1);
+  if (h == 0) {
+    for (int i = 0; i < G; ++i) {
+      float s = (rg == 0) ? zvc : 0.f;
+#pragma unroll
+      for (int hh = 0; hh < NH; ++hh) s += red[(hh * kMaxGroup + i) * D + c];
+      lin[i * (D + 1) + c] = s;
+    }
+  }
+  if (rg == 0 && warp == kSelectThreads / 32 - 1) {
+    for (int i = 0; i < G; ++i) {
       float s = 0.f;
-      for (int r = lane; r < D; r += 32) s += s_q[i][r] * __ldg(zk + r);
+      for (int cc = lane; cc < D; cc += 32) s += zred[i * D + cc];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
-      if (lane == 0) p.lin[lbase + (int64_t)i * (D + 1) + D] = __ldg(p.n + unit) + s;
+      if (lane == 0) lin[i * (D + 1) + D] = n_new + s;
     }
-  } else if (warp == 2 && cb == 0 && p.nb == 0 && p.sel_out != nullptr) {
-    for (int j = lane; j < p.top_k; j += 32) p.sel_out[(int64_t)unit * p.top_k + j] = -1;
   }
+  // the stage was written through the generic proxy: order that before the
+  // next bulk copy into it
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectParams p) {
-  // the attention kernel may be scheduled now; it waits for this grid before
-  // reading the selection and the linear term
-  pdl_allow_dependents();
-  __shared__ __align__(16) float s_q[kMaxGroup][D];
-  const int unit = blockIdx.y;
-  const __nv_bfloat16* q = p.q + (int64_t)unit * p.G * D;
-  for (int e = threadIdx.x; e < p.G * D; e += kSelectThreads)
-    s_q[e / D][e % D] = __bfloat162float(q[e]) * p.scale;
+__global__ void __maxnreg__(kSelectMaxRegs) select_kernel(const SelectParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte aligned; offsetting the shared array keeps accesses in the shared space
+  SelectSmem<D>& sm = *reinterpret_cast<SelectSmem<D>*>(smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u));
+  const int tid = threadIdx.x;
+  // one thread waits for the predecessor grid (the barrier below holds the rest)
+  if (tid == 0) pdl_wait_primary();
+
+  const int it0 = (int)((int64_t)p.total_items * blockIdx.x / gridDim.x);
+  const int it1 = (int)((int64_t)p.total_items * (blockIdx.x + 1) / gridDim.x);
+  const int n_mine = it1 - it0;
+  if (tid == 0) {
+    for (int s = 0; s < kSelStages; ++s) mbar_init(&sm.full[s], 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
   __syncthreads();
-  if ((int)blockIdx.x < p.score_ctas)
-    score_blocks<D>(p, unit, s_q);
-  else
-    linear_term<D>(p, unit, s_q);
+  pdl_allow_dependents();  // the attention kernel starts now and streams beside this grid
+  int issued = 0;  // thread 0: items whose copies have been started
+  if (tid == 0)
+    for (; issued < n_mine && issued < kSelStages; ++issued) issue_item<D>(p, sm, it0 + issued, issued);
+
+  for (int i = 0; i < n_mine; ++i) {
+    const int it = it0 + i, stage = i % kSelStages;
+    const int unit = it / p.items_per_unit, local = it % p.items_per_unit;
+    if (tid == 0 && !mbar_wait_bounded(&sm.full[stage], (i / kSelStages) & 1, kWaitLimit)) {
+      atomicOr(p.status, HYB_STATUS_TIMEOUT);
+      sm.abort = 1;
+    }
+    __syncthreads();  // the stage's data (or the abort flag) is visible to all
+    if (sm.abort) break;
+    if (local < p.score_items)
+      score_item<D>(p, sm.st[stage], unit, local);
+    else
+      lin_item<D>(p, sm.st[stage], unit, local - p.score_items);
+    __syncthreads();  // the stage is consumed
+    if (tid == 0 && issued < n_mine) {
+      issue_item<D>(p, sm, it0 + issued, issued % kSelStages);
+      ++issued;
+    }
+  }
+  if (sm.abort && tid == 0) {
+    // do not leave while copies into this CTA's ring may be in flight
+    for (int j = issued - 1; j >= 0 && j >= issued - kSelStages; --j)
+      mbar_wait_bounded(&sm.full[j % kSelStages], (j / kSelStages) & 1, kWaitLimit);
+  }
 }
 
 }  // namespace
 
+size_t select_smem_bytes(int D) {
+  return (D == 128 ? sizeof(SelectSmem<128>) : sizeof(SelectSmem<64>)) + 128;
+}
+
 cudaError_t prepare_select(int D) {
-  // the same shared-memory carveout as the attention kernel, so the SMs need no
-  // reconfiguration between the two launches of a decode
+  const int smem = (int)select_smem_bytes(D);
   const void* f = D == 128 ? (const void*)select_kernel<128> : (const void*)select_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // the same carveout as the attention kernels, so that SMs need no
+  // reconfiguration between the launches of a decode
   return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
 }
 
-cudaError_t launch_select(const SelectParams& p, int D, int grid_x, cudaStream_t s) {
-  const dim3 grid(grid_x, p.units);
-  if (D == 128)
-    select_kernel<128><<<grid, kSelectThreads, 0, s>>>(p);
-  else
-    select_kernel<64><<<grid, kSelectThreads, 0, s>>>(p);
-  return cudaGetLastError();
+cudaError_t launch_select(const SelectParams& p, int D, int grid, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSelectThreads);
+  cfg.dynamicSmemBytes = select_smem_bytes(D);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) return cudaLaunchKernelEx(&cfg, select_kernel<128>, p);
+  return cudaLaunchKernelEx(&cfg, select_kernel<64>, p);
 }
 
 }  // namespace hyb

@@ -1,5 +1,6 @@
-// State kernels: the per-token append and the build of the state of a
-// prefilled history.
+// State kernels: the per-token append (a cache write) and the build of the
+// state of a prefilled history.  Between decodes the state lags the history by
+// the tokens evicted since the last decode; the select kernel folds those in.
 //
 // The state of a unit (batch row, KV head) covers the evicted tokens
 // L = [S, T - W) -- past the sinks and out of the sliding window ("SALSA:
@@ -19,66 +20,20 @@ namespace hyb {
 namespace {
 
 // ---------------------------------------------------------------- append
-// Grid (D / RPC, units), 256 threads; CTA x owns rows [x*RPC, (x+1)*RPC) of H.
-// CTA 0 also writes the new token into the caches, folds the evicted token into
-// zk, zv, n and updates its block's mean / population variance with Welford's
-// online recurrence (B. P. Welford, Technometrics 4(3), 1962).
+// Writes one token per unit at row T of the caches: grid (units), D/4 threads
+// of 16 bytes.  The token's later eviction from the window is folded into the
+// state by the next decode's select kernel, which reads the caches.
 template <int D>
-__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
-  constexpr int RPC = 1024 / D;  // 256 threads x 4 floats
-  __shared__ float kp[D], vp[D];
-  const int unit = blockIdx.y, rg = blockIdx.x, tid = threadIdx.x;
-  const int64_t ub = (int64_t)unit * p.cap;
-  if (p.evict) {
-    if (tid < D) {
-      // W == 0 evicts the token being appended; read it from the input then
-      const bool self = (p.p == p.T);
-      const __nv_bfloat16* ks = self ? p.k_new + (int64_t)unit * D : p.k_cache + (ub + p.p) * D;
-      const __nv_bfloat16* vs = self ? p.v_new + (int64_t)unit * D : p.v_cache + (ub + p.p) * D;
-      kp[tid] = __bfloat162float(ks[tid]);
-      vp[tid] = __bfloat162float(vs[tid]);
-    }
-    __syncthreads();
-    const int r = rg * RPC + tid / (D / 4);
-    const int c = (tid % (D / 4)) * 4;
-    float4* hp = reinterpret_cast<float4*>(p.H + ((int64_t)unit * D + r) * D + c);
-    float4 h = *hp;
-    const float k = kp[r];
-    h.x += k * vp[c];
-    h.y += k * vp[c + 1];
-    h.z += k * vp[c + 2];
-    h.w += k * vp[c + 3];
-    *hp = h;
-    if (rg == 0 && tid < D) {
-      const int64_t zi = (int64_t)unit * D + tid;
-      p.zk[zi] += kp[tid];
-      p.zv[zi] += vp[tid];
-      const int64_t si = ((int64_t)unit * p.max_blocks + p.blk) * D + tid;
-      const float x = kp[tid];
-      if (p.cnt == 1) {
-        p.mu[si] = x;
-        p.var[si] = 0.f;
-      } else {
-        const float cnt = (float)p.cnt;
-        const float mu0 = p.mu[si];
-        const float delta = x - mu0;
-        const float mu1 = mu0 + delta / cnt;
-        p.mu[si] = mu1;
-        p.var[si] = (p.var[si] * (cnt - 1.f) + delta * (x - mu1)) / cnt;
-      }
-      if (tid == 0) p.n[unit] += 1.f;
-    }
-  }
-  if (rg == 0 && tid < D) {
-    p.k_cache[(ub + p.T) * D + tid] = p.k_new[(int64_t)unit * D + tid];
-    p.v_cache[(ub + p.T) * D + tid] = p.v_new[(int64_t)unit * D + tid];
-  }
-  // Launched programmatically after a decode's attention kernel, this kernel may
-  // run beside it (it writes nothing that kernel reads; the attention kernel lets
-  // it start only after the select kernel, which reads the state, has finished).
-  // Waiting for the attention kernel before exiting keeps "this kernel complete"
-  // meaning "the decode before it complete" for whatever the stream runs next.
-  pdl_wait_primary();
+__global__ void __launch_bounds__(D / 4) append_kernel(const AppendParams p) {
+  const int unit = blockIdx.x, tid = threadIdx.x;
+  if (tid == 0) pdl_wait_primary();  // the previous decode may still read these caches' rows
+  __syncthreads();
+  pdl_allow_dependents();
+  const bool is_v = tid >= D / 8;
+  const int e = (tid % (D / 8)) * 8;
+  const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + (int64_t)unit * D + e;
+  __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e;
+  *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
 }
 
 // ---------------------------------------------------------------- init
@@ -213,8 +168,8 @@ cudaError_t prepare_state(int D) {
 
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(D * D / 1024, p.units);
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3(p.units);
+  cfg.blockDim = dim3(D / 4);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

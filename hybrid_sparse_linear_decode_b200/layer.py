@@ -96,6 +96,24 @@ class HybridAttentionLayer:
         A.hyb_attn_decode(self.ctx, q.data_ptr(), out.data_ptr(), _ptr(sel_out), _ptr(scores_out), _stream(stream))
         return out
 
+    def decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                      out: torch.Tensor | None = None, sel_out: torch.Tensor | None = None,
+                      scores_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Decode at the current T, then append (k_new, v_new): one generation step."""
+        c = self.cfg
+        assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.shape == (c.batch, c.n_q_heads, c.head_dim)
+        for t in (k_new, v_new):
+            assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == (c.batch, c.n_kv_heads, c.head_dim)
+        if out is None:
+            out = torch.empty((c.batch, c.n_q_heads, c.head_dim), dtype=torch.float32, device=q.device)
+        if sel_out is not None:
+            assert sel_out.dtype == torch.int32 and sel_out.shape == (c.batch, c.n_kv_heads, c.top_k)
+        if scores_out is not None:
+            assert scores_out.dtype == torch.float32 and scores_out.shape[-1] == max(1, self.sizes.max_blocks)
+        A.hyb_attn_decode_append(self.ctx, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), out.data_ptr(),
+                                 _ptr(sel_out), _ptr(scores_out), _stream(stream))
+        return out
+
     def decode_with_selection(self, q: torch.Tensor, sel: torch.Tensor, out: torch.Tensor | None = None,
                               stream=None) -> torch.Tensor:
         c = self.cfg
@@ -110,6 +128,10 @@ class HybridAttentionLayer:
         for t in (k_new, v_new):
             assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == (c.batch, c.n_kv_heads, c.head_dim)
         A.hyb_attn_append(self.ctx, k_new.data_ptr(), v_new.data_ptr(), _stream(stream))
+
+    def sync_state(self, stream=None) -> None:
+        """Fold the evictions since the last decode into H, zk, zv, n, mu, var."""
+        A.hyb_attn_sync_state(self.ctx, _stream(stream))
 
     def step_host(self, q_host: torch.Tensor, k_host, v_host, out_host: torch.Tensor, stream=None) -> None:
         A.hyb_attn_step_host(self.ctx, q_host.data_ptr(), _ptr(k_host), _ptr(v_host), out_host.data_ptr(),

@@ -109,9 +109,11 @@ typedef struct hyb_attn_sizes {
  *   workspace         hyb_attn_sizes.workspace_bytes bytes, 256-byte aligned; contents are
  *                     private to the library.  Contexts whose calls are serialised on one
  *                     stream may share one workspace.
- * The state arrays (H, zk, zv, n, mu, var) are written by hyb_attn_init and kept
- * up to date by hyb_attn_append; copying them together with the caches and T is a
- * complete checkpoint of the layer. */
+ * The state arrays (H, zk, zv, n, mu, var) are written by hyb_attn_init and hold
+ * the evicted tokens up to the last decode: a token that leaves the window is
+ * folded in by the next decode (which reads the state anyway), or by
+ * hyb_attn_sync_state.  After hyb_attn_sync_state, copying them together with
+ * the caches and T is a complete checkpoint of the layer. */
 typedef struct hyb_attn_buffers {
   void*  k_cache;
   void*  v_cache;
@@ -135,10 +137,11 @@ typedef struct hyb_attn_plan_info {
   int64_t k_eff;             /* min(top_k, nb) */
   int64_t exact_tokens;      /* |sinks| + |window| + tokens of k_eff full blocks (upper bound) */
   int32_t chunks_per_unit;   /* 64-token pieces of the exact set per unit (fixed for a given T) */
-  int32_t attend_ctas;       /* grid of the attention kernel */
+  int32_t select_ctas;       /* grid of the select kernel (persistent) */
+  int32_t attend_ctas;       /* grid of the attention kernel (split-K CTAs of every unit) */
   int32_t partial_slots;     /* split-K partial records the attention kernel writes */
-  int32_t score_ctas_per_unit;
-  int32_t linear_ctas_per_unit;
+  int32_t score_items_per_unit;   /* select work items over the block statistics */
+  int32_t linear_items_per_unit;  /* select work items over rows of H */
 } hyb_attn_plan_info;
 
 /* Fill `out` with the buffer sizes of `cfg`.  Host only; never touches a GPU.
@@ -165,13 +168,19 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
                   int64_t T0, cudaStream_t stream);
 
 /* Append one token per unit: k_new, v_new bf16 [B][Hkv][d].  The token is
- * written at position T; then T += 1, and if the token at position T - W - 1
- * (after the increment) lies at or past S it leaves the window: it is folded
- * into H, zk, zv, n (a rank-1 update, SPLA "Recurrence") and into the running
- * mean / population variance of its block (Welford's update), which opens a new
- * block when the previous one is full.  Errors: HYB_EINVAL (null or misaligned
- * pointers), HYB_ECAPACITY (T == capacity), HYB_ECUDA. */
+ * written at position T; then T += 1.  If the token at position T - W - 1
+ * (after the increment) lies at or past S it has left the window: the next
+ * decode (or hyb_attn_sync_state) folds it into H, zk, zv, n (a rank-1 update,
+ * SPLA "Recurrence") and into the running mean / population variance of its
+ * block (Welford's update), which opens a new block when the previous one is
+ * full.  Any number of appends may come between decodes.  Errors: HYB_EINVAL
+ * (null or misaligned pointers), HYB_ECAPACITY (T == capacity), HYB_ECUDA. */
 int hyb_attn_append(hyb_attn_ctx* ctx, const void* k_new, const void* v_new, cudaStream_t stream);
+
+/* Fold every token evicted since the last decode into the state arrays, so that
+ * they describe L = [S, T - W) exactly (for a checkpoint, or to read them).  A
+ * no-op when nothing is pending.  Errors: HYB_EINVAL, HYB_ECUDA. */
+int hyb_attn_sync_state(hyb_attn_ctx* ctx, cudaStream_t stream);
 
 /* One decode step at the current length T for every unit:
  *   q           bf16 [B][Hq][d]  (input)
@@ -180,13 +189,22 @@ int hyb_attn_append(hyb_attn_ctx* ctx, const void* k_new, const void* v_new, cud
  *               ascending, -1 padded when nb < top_k
  *   scores_out  fp32 [B][Hkv][max_blocks] or NULL: the block scores (entries
  *               [0, nb) of each unit are written)
- * Kernels: block scoring + top-k + the global linear term phi(q)^T state, then
- * split-K exact attention over sinks, window and selected blocks with the
- * selected blocks' (1 + s) subtraction and the shared-normaliser merge.
+ * Kernels (chained with programmatic dependent launch): block scoring + the
+ * global linear term phi(q)^T state (folding in the tokens evicted since the
+ * previous decode); beside it, split-K exact attention over the sinks and the
+ * window, which then takes the top-k of the scores, attends the selected blocks
+ * with their (1 + s) subtraction, and merges under the shared normaliser.
  * Errors: HYB_EINVAL (null or misaligned pointers), HYB_ESTATE (T == 0),
  * HYB_ECUDA. */
 int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out,
                     float* scores_out, cudaStream_t stream);
+
+/* hyb_attn_decode followed by hyb_attn_append(k_new, v_new) in the same
+ * launches: the attention kernel also writes the new token at row T, then
+ * T += 1 -- one decode step of a generation loop.  The decode attends to
+ * [0, T) as stored before the call.  Errors: those of both calls. */
+int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, const void* v_new,
+                           float* out, int32_t* sel_out, float* scores_out, cudaStream_t stream);
 
 /* As hyb_attn_decode, with the block selection given by the caller instead of
  * the top-k: sel int32 [B][Hkv][top_k], each row ascending and distinct, -1
@@ -198,7 +216,7 @@ int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32
 /* One decode + append step from host memory, for callers whose inputs and
  * outputs live on the host: copies q_host (bf16 [B][Hq][d]) and k_host, v_host
  * (bf16 [B][Hkv][d]) to device staging space in the workspace, runs
- * hyb_attn_decode then hyb_attn_append, and copies the fp32 output back to
+ * hyb_attn_decode_append (hyb_attn_decode without k_host), and copies the fp32 output back to
  * out_host ([B][Hq][d]).  All copies are cudaMemcpyAsync on `stream`; host
  * buffers should be pinned for the copies to be asynchronous.  k_host / v_host
  * may be NULL to skip the append.  The call returns after enqueueing; the output
@@ -241,8 +259,9 @@ int64_t hyb_attn_length(const hyb_attn_ctx* ctx);
 int hyb_attn_status(hyb_attn_ctx* ctx, uint32_t* flags, int clear, cudaStream_t stream);
 
 /* Profiling hook: when both events are non-NULL, every later decode records
- * `begin` just before and `end` just after the attention kernel on the decode's
- * stream, so the caller can time that kernel alone.  Pass NULL, NULL to stop. */
+ * `begin` just before its first and `end` just after its last kernel on the
+ * decode's stream, so the caller can time one decode's kernels (chained as in
+ * normal use) without the rest of its stream.  Pass NULL, NULL to stop. */
 int hyb_attn_set_timing_events(hyb_attn_ctx* ctx, cudaEvent_t begin, cudaEvent_t end);
 
 /* Release the host context (device buffers stay with the caller). */

@@ -123,7 +123,10 @@ class Case:
         return out, osel, scores
 
     def state_gpu(self):
+        import torch
         L = self.layer
+        L.sync_state()  # fold the evictions since the last decode
+        torch.cuda.synchronize()
         return {n: getattr(L, n).cpu().numpy().astype(np.float64) for n in ("H", "zk", "zv", "n", "mu", "var")}
 
 

@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
     for n in ["hyb_attn_init", "hyb_attn_append", "hyb_attn_decode", "hyb_attn_decode_with_selection",
               "hyb_attn_workspace_size", "hyb_attn_length", "hyb_attn_status", "hyb_attn_destroy",
               "hyb_attn_strerror", "hyb_attn_query_sizes", "hyb_attn_plan", "hyb_attn_step_host",
-              "hyb_attn_set_timing_events"]:
+              "hyb_attn_set_timing_events", "hyb_attn_decode_append", "hyb_attn_sync_state"]:
         assert n in names, n
 
 
@@ -103,22 +103,35 @@ def test_init_rejects_bad_arguments_without_touching_a_gpu(lib):
 
 @pytest.mark.parametrize("T", [0, 1, 3, 4, 5, 1027, 1028, 1029, 1092, 1093, 32768, 32768 + 64])
 def test_plan_partition(lib, T):
-    """Chunk counts of the exact set follow the partition: sinks, window, and
-    ceil(Bk/64) chunks per selected block; each unit's chunks go to at most two
-    CTAs per SM in one wave."""
+    """Chunk counts of the exact set follow the partition (sinks, window, and
+    ceil(Bk/64) chunks per selected block); the attention kernel runs one CTA per
+    SM beside the select kernel's two; the select work items tile the blocks and
+    the rows of H."""
     import hybrid_sparse_linear_decode_b200 as H
     c = _cfg()
-    p = H.hyb_attn_plan(c, T, 148)
-    S, W, Bk = 4, 1024, 64
+    n_sm = 148
+    p = H.hyb_attn_plan(c, T, n_sm)
+    S, W, Bk, units = 4, 1024, 64, 8
     ev = max(0, T - S - W)
     nb = -(-ev // Bk)
     assert p.n_blocks == nb and p.k_eff == min(16, nb)
     sink = min(S, T)
     win = T - max(S, T - W) if T > S else 0
     assert p.chunks_per_unit == -(-sink // 64) + -(-win // 64) + p.k_eff
-    if p.chunks_per_unit:
-        splits = min(max(1, 148 * 2 // 8), p.chunks_per_unit)   # two CTAs per SM, one unit per CTA
-        assert p.attend_ctas == 8 * splits and p.partial_slots == 8 * splits
-    else:
-        assert p.attend_ctas == 8 and p.partial_slots == 0
-    assert p.score_ctas_per_unit == -(-nb // 64)
+    splits = max(1, min(n_sm // units, p.chunks_per_unit))
+    assert p.attend_ctas == units * splits and p.partial_slots == units * splits
+    R, RL = 16384 // (8 * 128), 16384 // (4 * 128)
+    assert p.score_items_per_unit == -(-nb // R)
+    assert p.linear_items_per_unit == 128 // RL
+    total = units * (p.score_items_per_unit + p.linear_items_per_unit)
+    assert p.select_ctas == min(total, 2 * n_sm)
+
+
+def test_plan_caps_grids_for_many_units(lib):
+    """With more units than CTA slots the attention kernel uses one CTA per
+    unit, and the select grid stays persistent (two CTAs per SM)."""
+    import hybrid_sparse_linear_decode_b200 as H
+    c = _cfg(batch=512, capacity=4096)
+    p = H.hyb_attn_plan(c, 4096, 148)
+    assert p.attend_ctas == 512 * 8
+    assert p.select_ctas == 296

@@ -159,3 +159,50 @@ def test_capacity_error():
     with pytest.raises(HybAttnError) as e:
         c.layer.append(k, k)
     assert e.value.code == -2
+
+
+@pytest.mark.parametrize("kw,n", [
+    (dict(T0=600, Bk=32, W=64), 70),                          # crosses block boundaries
+    (dict(T0=200, W=0, Bk=8, k=3), 20),                       # W = 0: the appended token is evicted at once
+    (dict(B=2, Hq=16, Hkv=4, T0=1500, Bk=64, W=100, k=5), 9),
+])
+def test_decode_append_equals_decode_then_append(kw, n):
+    """The fused step (decode, then the token written by the selected-block
+    kernel) gives the same outputs and selections as decode + append, and the
+    final state and decode still match the oracle."""
+    import torch
+    c1 = _case(n_append=n, seed=11, **kw)
+    c2 = _case(n_append=n, seed=11, **kw)
+    dev = c1.layer.device
+    from harness import to_device_bf16
+    for i in range(n):
+        q = c1.random_q()
+        c2.rng.standard_normal((c2.B, c2.Hq, c2.d))      # keep the rngs in step
+        out1, sel1, sc1 = c1.decode(q)
+        c1.append()
+        qd = to_device_bf16(q, dev)
+        kd = to_device_bf16(np.ascontiguousarray(c2.Kb[:, :, c2.T]), dev)
+        vd = to_device_bf16(np.ascontiguousarray(c2.Vb[:, :, c2.T]), dev)
+        sel2 = torch.full((c2.B, c2.Hkv, c2.k), -7, dtype=torch.int32, device=dev)
+        out2 = c2.layer.decode_append(qd, kd, vd, sel_out=sel2)
+        torch.cuda.synchronize()
+        c2.T += 1
+        np.testing.assert_array_equal(out2.cpu().numpy(), out1.astype(np.float32))
+        np.testing.assert_array_equal(sel2.cpu().numpy(), sel1)
+    assert c1.layer.T == c2.layer.T == c2.T
+    check_state(c2)
+    full_check(c2, c2.random_q())
+    assert c2.layer.status() == 0
+
+
+def test_state_sync_is_idempotent_and_decode_folds():
+    """After a decode nothing is pending (sync is a no-op); appends without a
+    decode leave the state behind until a sync or the next decode folds them."""
+    c = _case(T0=600, Bk=32, W=64, n_append=50)
+    c.append(50)                         # 50 evictions pending
+    full_check(c, c.random_q())          # the decode folds all of them
+    s1 = c.state_gpu()
+    s2 = c.state_gpu()
+    for k in s1:
+        np.testing.assert_array_equal(s1[k], s2[k])
+    check_state(c)

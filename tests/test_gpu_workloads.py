@@ -81,6 +81,7 @@ class WorkloadLayer:
         w = self.w
         part = O.partition(self.T, w.n_sink, w.window, w.block_size)
         L = self.layer
+        L.sync_state()  # fold the evictions since the last decode
         for (b, h) in units:
             K, V = self.host_unit(b, h)
             K, V = K[:self.T], V[:self.T]
