@@ -93,7 +93,7 @@ def algorithmic_bytes(w, T):
     return decode, append
 
 
-KERNEL_SOURCES = ("k_attend.cu", "k_select.cu", "hyb_device.cuh", "hyb_internal.h")
+KERNEL_SOURCES = ("k_fused.cu", "hyb_device.cuh", "hyb_internal.h")
 
 
 def kernel_sources_hash() -> str:
@@ -106,11 +106,11 @@ def kernel_sources_hash() -> str:
 
 
 def measured_traffic(workload: str):
-    """DRAM bytes of one layer's decode kernels (select + attention) from the
-    committed ncu summary of this workload, if the kernels' sources are unchanged
-    since that capture (else None)."""
+    """DRAM bytes of one layer's decode kernel from the committed ncu summary of
+    this workload, if the kernel's sources are unchanged since that capture
+    (else None)."""
     import re
-    prof = os.path.join(ROOT, "profiles", f"decode_kernels_{workload}.md")
+    prof = os.path.join(ROOT, "profiles", f"fused_decode_{workload}.md")
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
@@ -230,9 +230,9 @@ class Bench:
         self.step_idx += 1
 
     def launches_per_step(self):
-        """Kernels per step: the select and attention launches of every layer's
-        decode (the append's cache write rides in the attention kernel)."""
-        return 2 * len(self.layers)
+        """Kernels per step: one fused decode launch per layer (the append's
+        cache write and the fold of the previous evictions ride in it)."""
+        return len(self.layers)
 
 
 def run_native(args, rank, world):
@@ -375,7 +375,7 @@ def run_native(args, rank, world):
         "pct_of_hbm_peak_step": round(100 * step_gbs / hbm_peak, 2),
         "bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm",
-                     "kernel": "one layer's decode: select + attention kernels (PDL-chained)",
+                     "kernel": "one layer's decode: the fused decode kernel (one launch)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
                      "traffic": measured_traffic(w.name), "bytes_per_launch": decode_bytes,

@@ -50,8 +50,7 @@ class hyb_attn_buffers(ctypes.Structure):
 
 class hyb_attn_plan_info(ctypes.Structure):
     _fields_ = [("T", c_i64), ("n_blocks", c_i64), ("k_eff", c_i64), ("exact_tokens", c_i64),
-                ("chunks_per_unit", c_i32), ("select_ctas", c_i32), ("attend_ctas", c_i32),
-                ("partial_slots", c_i32), ("score_items_per_unit", c_i32), ("linear_items_per_unit", c_i32)]
+                ("chunks_per_unit", c_i32), ("cluster_ctas", c_i32), ("grid_ctas", c_i32)]
 
 
 # (name, restype, argtypes) of every entry point declared in include/hyb_attn.h

@@ -23,7 +23,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct WsLayout {
-  size_t status, tk_sel, tk_att, scores, sel, lin, partials, H64, z64, stage_q, stage_k, stage_v, stage_out, total;
+  size_t status, tk_sel, tk_att, scores, sel, H64, z64, stage_q, stage_k, stage_v, stage_out, total;
 };
 
 struct Checked {
@@ -57,12 +57,6 @@ int check_config(const hyb_attn_config* c, Checked* out) {
   return HYB_OK;
 }
 
-// Upper bound of the partial records of a unit (one per attention CTA).
-size_t max_slots_per_unit(int units) {
-  const int per = kMaxAttendCtas / units;
-  return (size_t)(per > 1 ? per : 1);
-}
-
 WsLayout ws_layout(const hyb_attn_config& c, const Checked& k) {
   WsLayout w{};
   size_t off = 0;
@@ -77,8 +71,6 @@ WsLayout ws_layout(const hyb_attn_config& c, const Checked& k) {
   w.tk_att = take(U * sizeof(uint32_t));
   w.scores = take(U * (size_t)(k.max_blocks > 0 ? k.max_blocks : 1) * sizeof(float));
   w.sel = take(U * (size_t)(c.top_k > 0 ? c.top_k : 1) * sizeof(int32_t));
-  w.lin = take(U * (size_t)sel_lin_items((int)D) * G * (D + 1) * sizeof(float));
-  w.partials = take(U * (size_t)max_slots_per_unit(k.units) * (size_t)partial_floats((int)D) * sizeof(float));
   w.H64 = take(U * D * D * sizeof(double));
   w.z64 = take(U * 2 * D * sizeof(double));
   w.stage_q = take(U * G * D * 2);
@@ -106,33 +98,14 @@ Geometry geometry(const hyb_attn_config& c, int64_t T) {
   return g;
 }
 
-// CTAs per unit for an attention launch over `chunks` chunks per unit: enough
-// for `per_sm` CTAs on every SM in one wave, never more than the chunks, and
-// within kMaxAttendCtas CTAs (one per unit at least).
-int attend_splits(int units, int chunks, int n_sm, int per_sm) {
-  int64_t s = (int64_t)n_sm * per_sm / units;
-  const int64_t cap = kMaxAttendCtas / units;
-  if (s > cap) s = cap;
-  if (s > chunks) s = chunks;
-  if (s < 1) s = 1;
-  return (int)s;
-}
-
-struct LaunchPlan {
-  int splits;          // attention CTAs per unit (>= 1)
-  int score_items, lin_items, items_per_unit, total_items, select_grid;
-};
-
-LaunchPlan plan_launches(const Geometry& g, const Checked& k, int n_sm) {
-  LaunchPlan lp{};
-  lp.splits = attend_splits(k.units, g.chunks_per_unit, n_sm, kAttendCtasPerSm);
-  lp.score_items = (int)ceil_div(g.nb, sel_item_blocks(k.D));
-  lp.lin_items = sel_lin_items(k.D);
-  lp.items_per_unit = lp.score_items + lp.lin_items;
-  lp.total_items = lp.items_per_unit * k.units;
-  const int64_t grid = (int64_t)n_sm * kSelectCtasPerSm;
-  lp.select_grid = (int)(grid < lp.total_items ? grid : lp.total_items);
-  return lp;
+// CTAs (one thread-block cluster) per unit: the largest C <= kMaxCluster with
+// one CTA per SM for every unit (units * C <= n_sm) and, when the device's
+// limits are known (fits[C] = clusters of C CTAs it can hold at once), every
+// unit's cluster resident at the same time.
+int cluster_ctas(int units, int n_sm, const int* fits) {
+  for (int c = kMaxCluster; c > 1; --c)
+    if ((int64_t)units * c <= n_sm && (fits == nullptr || fits[c] >= units)) return c;
+  return 1;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -219,6 +192,7 @@ struct hyb_attn_ctx {
   int64_t T;
   int64_t folded_end;   // the state holds the evicted positions [S, folded_end)
   int device, n_sm;
+  int fits[kMaxCluster + 1];  // clusters of C CTAs of the decode kernel the device holds at once
   float scale;
   CUtensorMap maps[4];  // K, V with 64-row boxes; K, V with 16-row boxes
   cudaEvent_t ev_begin, ev_end;
@@ -230,41 +204,47 @@ struct hyb_attn_ctx {
 
 namespace {
 
-SelectParams select_params(const hyb_attn_ctx* x, const Geometry& g, const LaunchPlan& lp) {
+FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   const hyb_attn_config& c = x->cfg;
   const Checked& k = x->ck;
-  SelectParams sp{};
-  sp.mu = x->buf.mu;
-  sp.var = x->buf.var;
-  sp.H = x->buf.H;
-  sp.zk = x->buf.zk;
-  sp.zv = x->buf.zv;
-  sp.n = x->buf.n;
-  sp.k_cache = static_cast<const __nv_bfloat16*>(x->buf.k_cache);
-  sp.v_cache = static_cast<const __nv_bfloat16*>(x->buf.v_cache);
-  sp.scores = x->w<float>(x->ws.scores);
-  sp.lin = x->w<float>(x->ws.lin);
-  sp.status = x->w<uint32_t>(x->ws.status);
-  sp.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
-  sp.cap = c.capacity;
-  sp.fold_begin = x->folded_end;
-  sp.fold_end = g.ev_end;
-  sp.units = k.units;
-  sp.G = k.G;
-  sp.nb = (int32_t)g.nb;
-  sp.S = c.n_sink;
-  sp.Bk = c.block_size;
-  sp.score_items = lp.score_items;
-  sp.lin_items = lp.lin_items;
-  sp.items_per_unit = lp.items_per_unit;
-  sp.total_items = lp.total_items;
-  sp.scale = x->scale;
-  return sp;
+  FusedParams fp{};
+  fp.mu = x->buf.mu;
+  fp.var = x->buf.var;
+  fp.H = x->buf.H;
+  fp.zk = x->buf.zk;
+  fp.zv = x->buf.zv;
+  fp.n = x->buf.n;
+  fp.k_cache = static_cast<__nv_bfloat16*>(x->buf.k_cache);
+  fp.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
+  fp.scores = x->w<float>(x->ws.scores);
+  fp.sel = x->w<int32_t>(x->ws.sel);
+  fp.status = x->w<uint32_t>(x->ws.status);
+  fp.cap = c.capacity;
+  fp.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
+  fp.fold_begin = x->folded_end;
+  fp.fold_end = g.ev_end;
+  fp.T = (int32_t)g.T;
+  fp.S = c.n_sink;
+  fp.Bk = c.block_size;
+  fp.top_k = c.top_k;
+  fp.nb = (int32_t)g.nb;
+  fp.k_eff = (int32_t)g.k_eff;
+  fp.sink_len = (int32_t)g.sink_len;
+  fp.win_start = (int32_t)g.win_start;
+  fp.ev_end = (int32_t)g.ev_end;
+  fp.n_sink_chunks = g.n_sink_chunks;
+  fp.n_win_chunks = g.n_win_chunks;
+  fp.chunks_per_block = g.chunks_per_block;
+  fp.n_sel_chunks = g.n_sel_chunks;
+  fp.units = k.units;
+  fp.G = k.G;
+  fp.C = cluster_ctas(k.units, x->n_sm, x->fits);
+  fp.scale = x->scale;
+  return fp;
 }
 
-// One decode at the current T: the select kernel (scores, linear term, pending
-// folds), then the attention kernel (sinks + window beside it; top-k, selected
-// blocks, merge; writes the appended token when k_new is given).
+// One decode at the current T: one launch of the fused kernel (writes the
+// appended token when k_new is given).
 int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_given, int32_t* sel_out,
                 float* scores_out, const void* k_new, const void* v_new, cudaStream_t stream) {
   if (x == nullptr || q == nullptr || out == nullptr) return HYB_EINVAL;
@@ -276,58 +256,20 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   if (k_new != nullptr && (!aligned16(k_new) || !aligned16(v_new))) return HYB_EINVAL;
   if (x->T == 0) return HYB_ESTATE;
   if (k_new != nullptr && x->T >= x->cfg.capacity) return HYB_ECAPACITY;
-  const hyb_attn_config& c = x->cfg;
-  const Checked& k = x->ck;
-  const Geometry g = geometry(c, x->T);
-  const LaunchPlan lp = plan_launches(g, k, x->n_sm);
+  const Geometry g = geometry(x->cfg, x->T);
+  FusedParams fp = fused_params(x, g);
+  fp.q = static_cast<const __nv_bfloat16*>(q);
+  if (scores_out) fp.scores = scores_out;
+  fp.sel_given = sel_given;
+  fp.sel_out = sel_given ? nullptr : sel_out;
+  fp.out = out;
+  fp.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  fp.v_new = static_cast<const __nv_bfloat16*>(v_new);
   const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
   if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
-
-  SelectParams sp = select_params(x, g, lp);
-  sp.q = static_cast<const __nv_bfloat16*>(q);
-  if (scores_out) sp.scores = scores_out;
-  cudaError_t e = launch_select(sp, k.D, lp.select_grid, stream);
+  const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->folded_end = g.ev_end;
-
-  AttendParams ap{};
-  ap.q = static_cast<const __nv_bfloat16*>(q);
-  ap.scores = sp.scores;
-  ap.sel_given = sel_given;
-  ap.sel = x->w<int32_t>(x->ws.sel);
-  ap.sel_out = sel_given ? nullptr : sel_out;
-  ap.lin = sp.lin;
-  ap.partials = x->w<float>(x->ws.partials);
-  ap.tickets = x->w<uint32_t>(x->ws.tk_att);
-  ap.status = sp.status;
-  ap.out = out;
-  ap.k_new = static_cast<const __nv_bfloat16*>(k_new);
-  ap.v_new = static_cast<const __nv_bfloat16*>(v_new);
-  ap.k_cache = static_cast<__nv_bfloat16*>(x->buf.k_cache);
-  ap.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
-  ap.cap = c.capacity;
-  ap.max_blocks = sp.max_blocks;
-  ap.T = (int32_t)g.T;
-  ap.S = c.n_sink;
-  ap.Bk = c.block_size;
-  ap.top_k = c.top_k;
-  ap.nb = (int32_t)g.nb;
-  ap.k_eff = (int32_t)g.k_eff;
-  ap.sink_len = (int32_t)g.sink_len;
-  ap.win_start = (int32_t)g.win_start;
-  ap.ev_end = (int32_t)g.ev_end;
-  ap.n_sink_chunks = g.n_sink_chunks;
-  ap.n_win_chunks = g.n_win_chunks;
-  ap.chunks_per_block = g.chunks_per_block;
-  ap.chunks_per_unit = g.chunks_per_unit;
-  ap.units = k.units;
-  ap.G = k.G;
-  ap.lin_items = lp.lin_items;
-  ap.splits = lp.splits;
-  ap.grid = k.units * lp.splits;
-  ap.scale = x->scale;
-  e = launch_attend(x->maps, ap, k.D, stream);
-  if (e != cudaSuccess) return cuda_fail(e);
   if (k_new != nullptr) x->T += 1;
   if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
   return HYB_OK;
@@ -369,12 +311,8 @@ int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_
   out->k_eff = g.k_eff;
   out->exact_tokens = g.sink_len + (T - g.win_start) + g.k_eff * cfg->block_size;
   out->chunks_per_unit = g.chunks_per_unit;
-  const LaunchPlan lp = plan_launches(g, k, n_sm);
-  out->select_ctas = lp.select_grid;
-  out->attend_ctas = k.units * lp.splits;
-  out->partial_slots = k.units * lp.splits;
-  out->score_items_per_unit = lp.score_items;
-  out->linear_items_per_unit = lp.lin_items;
+  out->cluster_ctas = cluster_ctas(k.units, n_sm, nullptr);
+  out->grid_ctas = k.units * out->cluster_ctas;
   return HYB_OK;
 }
 
@@ -410,6 +348,7 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   x->T = T0;
   x->device = device;
   x->n_sm = n_sm;
+  for (int c = 0; c <= kMaxCluster; ++c) x->fits[c] = 0;
   x->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)k.D);
   x->ev_begin = x->ev_end = nullptr;
   const int64_t rows = (int64_t)k.units * cfg->capacity;
@@ -420,13 +359,13 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
     delete x;
     return HYB_ECUDA;
   }
-  cudaError_t pe = prepare_attend(k.D);
-  if (pe == cudaSuccess) pe = prepare_select(k.D);
+  cudaError_t pe = prepare_fused(k.D);
   if (pe == cudaSuccess) pe = prepare_state(k.D);
   if (pe != cudaSuccess) {
     delete x;
     return cuda_fail(pe);
   }
+  for (int c = 2; c <= kMaxCluster; ++c) x->fits[c] = fused_max_clusters(k.D, c);
 
   const Geometry g = geometry(*cfg, T0);
   InitParams ip{};
@@ -485,10 +424,8 @@ int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
   if (x == nullptr) return HYB_EINVAL;
   const Geometry g = geometry(x->cfg, x->T);
   if (g.ev_end <= x->folded_end) return HYB_OK;  // nothing evicted since the last fold
-  const LaunchPlan lp = plan_launches(g, x->ck, x->n_sm);
-  SelectParams sp = select_params(x, g, lp);
-  sp.q = nullptr;  // fold only
-  const cudaError_t e = launch_select(sp, x->ck.D, lp.select_grid, stream);
+  FusedParams fp = fused_params(x, g);           // q == null: fold only
+  const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->folded_end = g.ev_end;
   return HYB_OK;

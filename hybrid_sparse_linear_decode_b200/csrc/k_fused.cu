@@ -1,0 +1,1564 @@
+// One decode step of one layer in one launch: block scores, the global linear
+// term, the top-k block selection, exact attention over sinks + window +
+// selected blocks with the selected blocks' (1 + s) subtraction, and the merge
+// under one shared normaliser; plus the fold of the tokens evicted since the
+// previous decode into the state, and the appended token's cache write.
+//
+// Grid: one thread-block cluster of C CTAs per unit (batch row, KV head), one
+// CTA per SM.  Rank r of a unit's cluster owns
+//   * its share of the blocks (equal shares rounded up to 4 blocks; score items
+//     of 32 blocks each) and rows [r D / C, (r+1) D / C) of H (H items),
+//   * window chunks r, r + C, ... and selected chunks r, r + C, ... (64-token
+//     pieces of the exact set, split-K).
+// Its items stream through a kFStages-deep shared-memory ring in the order H
+// items, score items, window chunks, selected chunks: a producer warp issues
+// the copies (TMA tensor loads for K/V chunks, untiled bulk copies for the
+// statistics and H, no multicast); the other warps consume them.
+//
+// Warp roles (8 warps; role r runs on hardware warp given by role_tid):
+//   0-3  attention: chunk c to warp c % 4, all 64 tokens, on the tensor cores
+//        (mma.sync m16n8k16, bf16 in, fp32 accumulate), G <= 4 query heads
+//        packed into the 16-row M dimension (rows 0-3 softmax, rows 4-7 the
+//        Taylor weights 1 + s of selected-block tokens, rows 8-15 the bf16
+//        rounding remainders of rows 0-7);
+//   4-6  statistics: H rows, block scores (score item i to warp i % 3), the
+//        Welford fold, the top-k (one warp), the linear term;
+//   7    producer: lane 0 issues every copy in ring order.
+//
+// Block score ("SPLA: Block Sparse Plus Linear Attention for Long Context
+// Modeling", Abstract; "Principled Block Selection via Taylor Expansion";
+// "Grouped Sparsity"): score_j = sum_i ( q'_i . mu_j + 1/2 sum_c q'_ic^2 var_jc ).
+// Each rank keeps the scores of its blocks in shared memory and bulk-copies
+// them into every other rank's scores array over distributed shared memory
+// (completing bytes on that rank's "scores" barrier); every rank then selects
+// the same top_k blocks itself (ties to the lower index), while the ring
+// streams its window chunks.
+//
+// Linear term (SLAKE, first-order Taylor exp(s) ~ 1 + s; SPLA residual
+// attention): N_glob_i = zv + H^T q'_i, D_glob_i = n + q'_i . zk, each rank
+// summing its rows of H.  Merge, by rank 0 over distributed shared memory
+// after a cluster barrier (per query head, base-2 exponent m of the exact part):
+//   o = (N_ex + 2^{-m} (N_glob - N_sel)) / (D_ex + 2^{-m} (D_glob - D_sel)),
+// as the equal form (N_ex 2^m + ...)/(D_ex 2^m + ...) when m < 0.
+//
+// Evictions since the previous decode (positions [fold_begin, fold_end), usually
+// one token) are folded into the rows an item holds before it is used:
+// H += k v^T, zk += k, zv += v, n += 1 (SPLA "Recurrence") and Welford's running
+// mean / population variance of the token's block (B. P. Welford,
+// Technometrics 4(3), 1962).  With q == null the kernel only folds.
+//
+// Every wait inside the kernel is bounded (a timeout sets a status bit and the
+// CTA skips the rest of its work); all CTAs of a cluster always reach both
+// cluster barriers.  Launch chaining: programmatic dependent launch -- the CTA
+// waits for the predecessor grid before touching memory.
+#include "hyb_device.cuh"
+#include "hyb_internal.h"
+
+namespace hyb {
+
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr int kFThreads = 256;
+constexpr int kFStages = 6;
+constexpr int kFScoresMax = 2048;   // scores a CTA keeps for its unit (else they go through global memory)
+constexpr int kAuxWarps = 3;        // statistics warps: roles 4-6
+constexpr int kAuxThreads = 32 * kAuxWarps;
+constexpr int kConsumerThreads = 128 + kAuxThreads;  // attention + statistics (roles 0-6)
+// every item's empty-barrier phase takes kEmptyCount arrivals: kEmptyPerAuxWarp
+// from each statistics warp, or kEmptyPerAttnWarp from each attention warp
+constexpr int kEmptyCount = 12, kEmptyPerAuxWarp = 4, kEmptyPerAttnWarp = 3;
+constexpr int kBarAttn = 1, kBarAux = 2, kBarConsumers = 3;   // named barriers
+
+// ---------------------------------------------------------------- cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t local_smem, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void remote_arrive(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait on a barrier that other CTAs of the cluster arrive on
+__device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+#pragma unroll 1
+  for (int i = 0; i < 32; ++i)
+    if (try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) {
+      __nanosleep(64);
+      if (try_wait_cluster(bar, parity)) return true;
+    }
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Copy `bytes` (a multiple of 16) of this CTA's shared memory at src to the
+// cluster shared address dst, completing that many transactions on the barrier
+// at cluster shared address bar (in the destination CTA).
+__device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// This thread's index in role order.  Warp w runs on sub-partition w % 4: the
+// attention roles (0-3) sit on hardware warps 0, 1, 4, 5 (sub-partitions 0, 1),
+// the statistics roles (4-6) on warps 2, 3, 6 and the producer (role 7) on
+// warp 7 (sub-partitions 2, 3), so that each sub-partition's instruction cache
+// serves the attention loop or the statistics and copy code, not both.
+__device__ __forceinline__ int role_tid() {
+  const uint32_t w = threadIdx.x >> 5;
+  return (int)((((0x76325410u >> (4u * w)) & 15u) << 5) | (threadIdx.x & 31u));
+}
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+struct KVMaps {  // the same KV caches seen with 64-row and 16-row TMA boxes
+  CUtensorMap k64, v64, k16, v16;
+};
+
+template <int D>
+struct FusedSmem {
+  static constexpr int kHalf = kTile * D * 2;        // K (or V) of one 64-token chunk, bytes
+  static constexpr int kStageBytes = 2 * kHalf;      // 32 KB at D = 128
+  static constexpr int kBoxBytes = kBoxRows * D * 2;
+  static constexpr int kPF = partial_floats(D);
+  // scores gathered in shared memory (the combine slots hold them); else via L2
+  static constexpr int kGather = 2 * kPF < kFScoresMax ? 2 * kPF : kFScoresMax;
+  uint8_t ring[kFStages][kStageBytes];               // 1024-byte aligned
+  float scores[kFScoresMax];                         // this rank's share of the unit's block scores
+  float qs[kMaxGroup][D];                            // q' = q * scale
+  float qsT[D][kMaxGroup];                           // q' transposed (H rows: one vector load per row)
+  float qsum[2][D];                                  // sum_i q'_i, 1/2 sum_i q'_i^2 (block scores)
+  float ktok[D];                                     // K and V rows of the pending token (H fold)
+  float vtok[D];
+  alignas(16) float wpart[2][kPF];                   // attention combine slots; [0] ends as the record
+  float linp[kMaxGroup][D + 1];                      // this rank's linear partial (D_glob in rank 0)
+  float hred[kAuxWarps][kMaxGroup][D];               // H rows: per-warp partials
+  float zks[D];                                      // rank 0: zk after the fold
+  int32_t sel_cache[kSelCache];
+  uint32_t hist[256];                                // top-k: radix histogram
+  uint32_t tk[8];                                    // top-k: shared scalars
+  uint32_t tks[2][4];                                // top-k: per-warp partials / scan scratch
+  uint32_t tkw[2];                                   // one-warp top-k: done, NaN seen
+  int4 desc[kFStages];                               // chunk items: start, len, is_sel
+  // A stage's items belong to one of two consumer groups.  Each group has its
+  // own "full" barrier per stage and waits only for its own items, in order,
+  // so it is never more than one phase ahead of a barrier it waits on (a
+  // parity wait cannot tell phase k from phase k - 2).
+  uint64_t full_attn[kFStages];                      // window / selected chunks
+  uint64_t full_aux[kFStages];                       // score / H items
+  uint64_t empty[kFStages];                          // one release per item
+  uint64_t scores_bar;                               // C arrivals: every rank's scores are in place
+  uint64_t sel_bar;                                  // 1 arrival: the selection is known
+  int sel_state;                                     // 1 sel_cache, 2 global row (sel_row), 3 every block
+  const int32_t* sel_row;
+  int abort;
+};
+
+}  // namespace
+}  // namespace hyb
+
+namespace hyb {
+namespace {
+
+// Byte offset of (row t, 16-byte chunk C) in a tile written by TMA with the
+// 128-byte swizzle: 128-byte line L = t*(D/64) + C/8, chunk slot (C%8) ^ (L%8).
+template <int D>
+__device__ __forceinline__ uint32_t swz(int t, int C) {
+  const int L = t * (D / 64) + (C >> 3);
+  return (uint32_t)(L * 128 + (((C & 7) ^ (L & 7)) << 4));
+}
+
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// ---------------------------------------------------------------- item sequence
+// Items of rank r, in ring order: nH H items, nS score items, nW window (and
+// sink) chunks, nX selected chunks.  The H rows come first (the statistics
+// warps fold and sum them while the first score items are in flight), the
+// scores next, so that the top-k runs while the window chunks stream in.  Every
+// thread derives the same sequence.
+struct Seq {
+  int b0, b1, nS;   // blocks [b0, b1), kFBlocks per score item
+  int h0, h1, nH;   // rows of H [h0, h1), kFRows per H item
+  int nW, nX, n;
+};
+
+template <int D>
+struct Geo {
+  static constexpr int kStageBytes = 2 * kTile * D * 2;
+  static constexpr int kBlocks = kStageBytes / (8 * D);  // mean + variance rows per score item
+  static constexpr int kRows = kStageBytes / (4 * D);    // rows of H per H item
+};
+
+// Blocks [b0, b1) of rank r: equal shares rounded up to 4 blocks, so that every
+// share's scores start on a 16-byte boundary (they travel by bulk copy).
+__device__ __forceinline__ void block_share(int nb, int C, int r, int& b0, int& b1) {
+  const int per = ((nb + C - 1) / C + 3) & ~3;
+  b0 = min(nb, r * per);
+  b1 = min(nb, b0 + per);
+}
+// Does this launch select the top-k from the scores (else: the caller's row,
+// every block, or none)?
+__device__ __forceinline__ bool runs_topk(const FusedParams& p) {
+  return p.q != nullptr && p.sel_given == nullptr && p.k_eff > 0 && p.k_eff < p.nb;
+}
+
+template <int D>
+__device__ __forceinline__ Seq make_seq(const FusedParams& p, int r) {
+  Seq q;
+  const int C = p.C;
+  block_share(p.nb, C, r, q.b0, q.b1);
+  q.nS = (q.b1 - q.b0 + Geo<D>::kBlocks - 1) / Geo<D>::kBlocks;
+  q.h0 = r * D / C;
+  q.h1 = (r + 1) * D / C;
+  q.nH = (q.h1 - q.h0 + Geo<D>::kRows - 1) / Geo<D>::kRows;
+  const int n_pre = p.n_sink_chunks + p.n_win_chunks;
+  if (p.q != nullptr) {
+    q.nW = r < n_pre ? (n_pre - r + C - 1) / C : 0;
+    q.nX = r < p.n_sel_chunks ? (p.n_sel_chunks - r + C - 1) / C : 0;
+  } else {
+    q.nW = q.nX = 0;
+  }
+  q.n = q.nS + q.nW + q.nH + q.nX;
+  return q;
+}
+
+// position in the ring order of H item i / score item i / the first chunk item
+__device__ __forceinline__ int seq_of_h(const Seq&, int i) { return i; }
+__device__ __forceinline__ int seq_of_s(const Seq& s, int i) { return s.nH + i; }
+__device__ __forceinline__ int first_chunk_item(const Seq& s) { return s.nS + s.nH; }
+
+// score item idx: does it hold a block with pending evictions?
+template <int D>
+__device__ __forceinline__ bool score_item_folds(const FusedParams& p, const Seq& s, int idx) {
+  if (p.fold_end <= p.fold_begin) return false;
+  const int64_t j0 = s.b0 + (int64_t)idx * Geo<D>::kBlocks;
+  const int64_t j1 = min((int64_t)s.b1, j0 + Geo<D>::kBlocks);
+  const int64_t jb0 = (p.fold_begin - p.S) / p.Bk, jb1 = (p.fold_end - 1 - p.S) / p.Bk;
+  return jb1 >= j0 && jb0 < j1;
+}
+
+// Producer: the copies of one K/V chunk (rows [start, start + len) of the
+// unit's caches) into ring stage `stage`; its descriptor tells the attention
+// warps what the stage holds.
+template <int D>
+__device__ __forceinline__ void issue_chunk(const KVMaps* tm, FusedSmem<D>& sm, int stage, int64_t ubase, int start,
+                                            int len, int is_sel) {
+  using Sm = FusedSmem<D>;
+  uint64_t* bar = &sm.full_attn[stage];
+  const uint32_t dst = smem_u32(sm.ring[stage]);
+  sm.desc[stage] = make_int4(start, len, is_sel, 0);
+  if (len <= 0) {
+    mbar_arrive(bar);
+    return;
+  }
+  const int row = (int)(ubase + start);
+  if (len == kTile) {  // full chunk: one 64-row box per tensor
+    mbar_arrive_expect_tx(bar, (uint32_t)(2 * Sm::kHalf));
+    tma_load_3d(dst, &tm->k64, 0, 0, row, bar);
+    tma_load_3d(dst + Sm::kHalf, &tm->v64, 0, 0, row, bar);
+  } else {             // ragged chunk: only the 16-row boxes it touches
+    const int nbox = (len + kBoxRows - 1) / kBoxRows;
+    mbar_arrive_expect_tx(bar, (uint32_t)(nbox * Sm::kBoxBytes * 2));
+    for (int bx = 0; bx < nbox; ++bx) {
+      tma_load_3d(dst + bx * Sm::kBoxBytes, &tm->k16, 0, 0, row + bx * kBoxRows, bar);
+      tma_load_3d(dst + Sm::kHalf + bx * Sm::kBoxBytes, &tm->v16, 0, 0, row + bx * kBoxRows, bar);
+    }
+  }
+}
+
+}  // namespace
+}  // namespace hyb
+
+namespace hyb {
+namespace {
+
+template <int CPL>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* src, float (&f)[CPL]) {
+  if constexpr (CPL == 4) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
+    f[0] = bf16_lo(raw.x); f[1] = bf16_hi(raw.x); f[2] = bf16_lo(raw.y); f[3] = bf16_hi(raw.y);
+  } else {
+    const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(src));
+    f[0] = bf16_lo(raw); f[1] = bf16_hi(raw);
+  }
+}
+
+// ---------------------------------------------------------------- statistics role
+template <int CPL>
+__device__ __forceinline__ void lds_vec(const float* src, float (&f)[CPL]) {
+  if constexpr (CPL == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(src);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  } else {
+    const float2 v = *reinterpret_cast<const float2*>(src);
+    f[0] = v.x; f[1] = v.y;
+  }
+}
+
+template <int CPL>
+__device__ __forceinline__ void sts_vec(float* dst, const float (&f)[CPL]) {
+  if constexpr (CPL == 4) {
+    *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+  } else {
+    *reinterpret_cast<float2*>(dst) = make_float2(f[0], f[1]);
+  }
+}
+
+// Fold the pending evictions into the statistics rows of score item `idx`, in
+// place in its ring stage, and write them back: Welford's running mean and
+// population variance, one token at a time.  One warp, lane l holding channels
+// [l*CPL, l*CPL + CPL) of each block that has pending tokens (usually one).
+template <int D>
+__device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx,
+                                                int stage) {
+  constexpr int CPL = D / 32;
+  constexpr int RB = Geo<D>::kBlocks;
+  const int lane = role_tid() & 31;
+  const int j0 = s.b0 + idx * RB;
+  const int nblk = min(RB, s.b1 - j0);
+  float* mrows = reinterpret_cast<float*>(sm.ring[stage]);
+  float* vrows = mrows + RB * D;
+  const int64_t jb0 = (p.fold_begin - p.S) / p.Bk, jb1 = (p.fold_end - 1 - p.S) / p.Bk;
+  const int bl0 = (int)max((int64_t)0, jb0 - j0), bl1 = (int)min((int64_t)nblk - 1, jb1 - j0);
+#pragma unroll 1
+  for (int bl = bl0; bl <= bl1; ++bl) {
+    const int j = j0 + bl;
+    const int64_t bs = p.S + (int64_t)j * p.Bk;
+    const int64_t t0 = max(bs, p.fold_begin), t1 = min(bs + p.Bk, p.fold_end);
+    float m[CPL], v[CPL];
+    lds_vec<CPL>(mrows + bl * D + lane * CPL, m);
+    lds_vec<CPL>(vrows + bl * D + lane * CPL, v);
+#pragma unroll 1
+    for (int64_t t = t0; t < t1; ++t) {
+      float x[CPL];
+      load_bf16<CPL>(p.k_cache + ((int64_t)unit * p.cap + t) * D + lane * CPL, x);
+      const float cnt = (float)(t - bs + 1);
+      const float inv = 1.f / cnt;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        if (t == bs) {  // the block's first token: the stored row is not read
+          m[c] = x[c];
+          v[c] = 0.f;
+        } else {
+          const float delta = x[c] - m[c];
+          const float m1 = m[c] + delta * inv;
+          v[c] = (v[c] * (cnt - 1.f) + delta * (x[c] - m1)) * inv;
+          m[c] = m1;
+        }
+      }
+    }
+    sts_vec<CPL>(mrows + bl * D + lane * CPL, m);
+    sts_vec<CPL>(vrows + bl * D + lane * CPL, v);
+    sts_vec<CPL>(p.mu + ((int64_t)unit * p.max_blocks + j) * D + lane * CPL, m);
+    sts_vec<CPL>(p.var + ((int64_t)unit * p.max_blocks + j) * D + lane * CPL, v);
+  }
+  // the stage is rewritten by bulk copies (the async proxy) later
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+}
+
+// Score item `idx` by one warp, score_j = sum_c qsum[0][c] mu_jc +
+// qsum[1][c] var_jc (qsum = sum_i q'_i and 1/2 sum_i q'_i^2): lane l forms the
+// partial sums of its channels [l*CPL, l*CPL + CPL) for all 32 blocks (each
+// row read once, conflict-free), then a transposing butterfly (31 shuffles in 5
+// rounds: in the round of width h a lane keeps the half of its values whose
+// block index has bit h equal to its own) leaves block l's score in lane l.
+template <int D>
+__device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx,
+                                                int stage) {
+  constexpr int CPL = D / 32;
+  constexpr int RB = Geo<D>::kBlocks;
+  static_assert(RB == 32, "one block per lane");
+  const int lane = role_tid() & 31;
+  const int j0 = s.b0 + idx * RB;
+  const int nblk = min(RB, s.b1 - j0);
+  const float* mrows = reinterpret_cast<const float*>(sm.ring[stage]);
+  const float* vrows = mrows + RB * D;
+  float q1[CPL], q2[CPL];
+  lds_vec<CPL>(&sm.qsum[0][lane * CPL], q1);
+  lds_vec<CPL>(&sm.qsum[1][lane * CPL], q2);
+  float part[RB];
+#pragma unroll
+  for (int b = 0; b < RB; ++b) {
+    float m[CPL], v[CPL];
+    const int bl = min(b, nblk - 1);  // rows past the item: a copy of its last row (never stored)
+    lds_vec<CPL>(mrows + bl * D + lane * CPL, m);
+    lds_vec<CPL>(vrows + bl * D + lane * CPL, v);
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc += q1[c] * m[c] + q2[c] * v[c];
+    part[b] = acc;
+  }
+#pragma unroll
+  for (int h = RB / 2; h >= 1; h >>= 1) {
+    const bool up = (lane & h) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = up ? part[i] : part[i + h];
+      const float keep = up ? part[i + h] : part[i];
+      part[i] = keep + __shfl_xor_sync(kFull, send, h);
+    }
+  }
+  if (lane < nblk) {
+    p.scores[(int64_t)unit * p.max_blocks + j0 + lane] = part[0];
+    if (p.nb <= FusedSmem<D>::kGather) sm.scores[j0 + lane] = part[0];  // this rank's share; pushed to the other ranks
+  }
+}
+
+// H item `idx`: warp aw takes rows aw, aw + 3, ... of the item; lane l columns
+// [l*CPL, l*CPL + CPL).  Folds pending evictions into the rows (written back)
+// and accumulates q'_i[r] H[r][c] into hacc (qsT[r] holds q'_0..3[r]).  With
+// one pending token (the usual case) its K and V rows come from shared memory.
+template <int D, int kFold>  // kFold: 0 none, 1 one token (ktok, vtok), 2 several (global memory)
+__device__ __forceinline__ void h_rows(const FusedParams& p, FusedSmem<D>& sm, int unit, int r0, int nrows,
+                                       const float* hrows, float (&hacc)[kMaxGroup][D / 32]) {
+  constexpr int CPL = D / 32;
+  static_assert(kMaxGroup == 4, "qsT rows are one float4");
+  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  const int64_t ub = (int64_t)unit * p.cap;
+  float v1[CPL];
+  if (kFold == 1) lds_vec<CPL>(&sm.vtok[lane * CPL], v1);
+  const bool acc = p.q != nullptr;
+#pragma unroll 2
+  for (int rl = aw; rl < nrows; rl += kAuxWarps) {
+    const int row = r0 + rl;
+    float h[CPL];
+    lds_vec<CPL>(hrows + rl * D + lane * CPL, h);
+    if (kFold == 1) {
+      const float kr = sm.ktok[row];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) h[c] += kr * v1[c];
+    } else if (kFold == 2) {
+      for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
+        const float kr = __bfloat162float(p.k_cache[(ub + t) * D + row]);
+        float vv[CPL];
+        load_bf16<CPL>(p.v_cache + (ub + t) * D + lane * CPL, vv);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) h[c] += kr * vv[c];
+      }
+    }
+    if (kFold != 0) sts_vec<CPL>(p.H + ((int64_t)unit * D + row) * D + lane * CPL, h);
+    if (acc) {
+      const float4 qr = *reinterpret_cast<const float4*>(&sm.qsT[row][0]);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        hacc[0][c] += qr.x * h[c];
+        hacc[1][c] += qr.y * h[c];
+        hacc[2][c] += qr.z * h[c];
+        hacc[3][c] += qr.w * h[c];
+      }
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void aux_h_item(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx, int stage,
+                                           float (&hacc)[kMaxGroup][D / 32]) {
+  constexpr int RH = Geo<D>::kRows;
+  const int r0 = s.h0 + idx * RH;
+  const int nrows = min(RH, s.h1 - r0);
+  const float* hrows = reinterpret_cast<const float*>(sm.ring[stage]);
+  const int64_t nf = p.fold_end - p.fold_begin;
+  if (nf == 0) h_rows<D, 0>(p, sm, unit, r0, nrows, hrows, hacc);
+  else if (nf == 1) h_rows<D, 1>(p, sm, unit, r0, nrows, hrows, hacc);
+  else h_rows<D, 2>(p, sm, unit, r0, nrows, hrows, hacc);
+}
+
+// After every H item (aux threads): sum the three warps' partials into linp;
+// rank 0 also folds the pending evictions into zk, zv, n and forms
+// N_glob += zv, D_glob = n + q'_i . zk.
+template <int D>
+__device__ void aux_finish_linear(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank,
+                                  const float (&hacc)[kMaxGroup][D / 32]) {
+  constexpr int CPL = D / 32;
+  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  if (p.q != nullptr) {
+#pragma unroll
+    for (int i = 0; i < kMaxGroup; ++i)
+      if (i < p.G)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) sm.hred[aw][i][lane * CPL + c] = hacc[i][c];
+  }
+  float nval = 0.f;
+  if (rank == 0) {
+    const bool fold = p.fold_end > p.fold_begin;
+    const int64_t ub = (int64_t)unit * p.cap;
+    for (int c = a; c < D; c += kAuxThreads) {
+      float zk = p.zk[(int64_t)unit * D + c], zv = p.zv[(int64_t)unit * D + c];
+      if (fold) {
+        for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
+          zk += __bfloat162float(p.k_cache[(ub + t) * D + c]);
+          zv += __bfloat162float(p.v_cache[(ub + t) * D + c]);
+        }
+        p.zk[(int64_t)unit * D + c] = zk;
+        p.zv[(int64_t)unit * D + c] = zv;
+      }
+      sm.zks[c] = zk;
+      sm.linp[0][c] = zv;  // scratch until the sum below
+    }
+    if (a == 0) {
+      nval = p.n[unit];
+      if (fold) {
+        nval += (float)(p.fold_end - p.fold_begin);
+        p.n[unit] = nval;
+      }
+      sm.linp[0][D] = nval;
+    }
+  }
+  named_sync(kBarAux, kAuxThreads);
+  if (p.q == nullptr) return;
+  constexpr int NZ = (D + kAuxThreads - 1) / kAuxThreads;
+  float zvs[NZ];
+#pragma unroll
+  for (int k = 0; k < NZ; ++k) {
+    const int c = a + k * kAuxThreads;
+    zvs[k] = (rank == 0 && c < D) ? sm.linp[0][c] : 0.f;
+  }
+  if (rank == 0) nval = sm.linp[0][D];
+  named_sync(kBarAux, kAuxThreads);
+  for (int i = 0; i < p.G; ++i) {
+#pragma unroll
+    for (int k = 0; k < NZ; ++k) {
+      const int c = a + k * kAuxThreads;
+      if (c < D) {
+        float v = zvs[k];
+#pragma unroll
+        for (int w = 0; w < kAuxWarps; ++w) v += sm.hred[w][i][c];
+        sm.linp[i][c] = v;
+      }
+    }
+  }
+  if (rank == 0 && aw == 0) {
+    for (int i = 0; i < p.G; ++i) {
+      float d = 0.f;
+      for (int c = lane; c < D; c += 32) d += sm.qs[i][c] * sm.zks[c];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(kFull, d, o);
+      if (lane == 0) sm.linp[i][D] = nval + d;
+    }
+  }
+}
+
+}  // namespace
+}  // namespace hyb
+
+namespace hyb {
+namespace {
+
+// ---------------------------------------------------------------- top-k
+// Exclusive prefix sum of v over the statistics threads (named barrier 2);
+// returns the sum over threads before this one, and the total in *total.
+__device__ __forceinline__ uint32_t aux_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
+  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scratch[aw] = incl;
+  named_sync(kBarAux, kAuxThreads);
+  uint32_t before = 0;
+  for (int w = 0; w < aw; ++w) before += scratch[w];
+  uint32_t tot = 0;
+  for (int w = 0; w < kAuxWarps; ++w) tot += scratch[w];
+  *total = tot;
+  named_sync(kBarAux, kAuxThreads);
+  return before + incl - v;
+}
+
+struct TopkSmem {  // the top-k's shared scratch
+  uint32_t* hist;     // [256]
+  uint32_t* tk;       // [8]
+  uint32_t* tks;      // [2][4]
+};
+
+// Order-preserving integer key of score j (from shared memory, or from global
+// memory through L2 when the unit's scores do not fit in shared memory).
+__device__ __forceinline__ uint32_t score_key(const float* src, bool glob, int j) {
+  return float_key(glob ? __ldcg(src + j) : src[j]);
+}
+
+// The k < nb largest of the nb scores at src by the statistics threads: an
+// 8-bit radix refinement over the keys' value range (at most four histogram
+// passes, usually two or three) finds the k-th largest key tau; then every key
+// above tau and the lowest-index keys equal to it are taken, in block order,
+// through prefix sums over contiguous ranges of blocks.  dst[0, k) ascending
+// (and copy[0, k)).  Returns (in every thread) whether a score was NaN.
+__device__ __forceinline__ bool aux_topk(const TopkSmem t, const float* src, bool glob, int nb, int k, int32_t* dst,
+                                      int32_t* copy) {
+  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  uint32_t kmin = 0xffffffffu, kmax = 0u, nan = 0u;
+#pragma unroll 1
+  for (int j = a; j < nb; j += kAuxThreads) {
+    const float f = glob ? __ldcg(src + j) : src[j];
+    nan |= f != f ? 1u : 0u;
+    const uint32_t u = float_key(f);
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  }
+  kmin = __reduce_min_sync(kFull, kmin);
+  kmax = __reduce_max_sync(kFull, kmax);
+  nan = __reduce_or_sync(kFull, nan);
+  if (lane == 0) {
+    t.tks[aw] = kmin;
+    t.tks[4 + aw] = kmax;
+    t.tk[4 + aw] = nan;
+  }
+  named_sync(kBarAux, kAuxThreads);
+  uint32_t lo = t.tks[0], hi = t.tks[4];
+  bool any_nan = t.tk[4] != 0u;
+  for (int w = 1; w < kAuxWarps; ++w) {
+    lo = min(lo, t.tks[w]);
+    hi = max(hi, t.tks[4 + w]);
+    any_nan |= t.tk[4 + w] != 0u;
+  }
+  uint32_t span = hi - lo;
+  uint32_t need = (uint32_t)k;
+  uint32_t tau = lo, need_eq = need;  // take u > tau, and the first need_eq keys u == tau
+#pragma unroll 1
+  for (int pass = 0; pass < 5; ++pass) {
+    if (span == 0u) {
+      tau = lo;
+      need_eq = need;
+      break;
+    }
+    const int bits = 32 - __clz(span);
+    const int shift = bits > 8 ? bits - 8 : 0;  // (span >> shift) < 256
+    for (int b = a; b < 256; b += kAuxThreads) t.hist[b] = 0u;
+    named_sync(kBarAux, kAuxThreads);
+#pragma unroll 1
+    for (int j = a; j < nb; j += kAuxThreads) {
+      const uint32_t d = score_key(src, glob, j) - lo;  // keys below lo wrap past span
+      if (d <= span) atomicAdd(&t.hist[d >> shift], 1u);
+    }
+    named_sync(kBarAux, kAuxThreads);
+    if (aw == 0) {  // lane l holds bins 255-8l .. 248-8l, highest first
+      uint32_t cnt[8], local = 0u;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt[e] = t.hist[255 - 8 * lane - e];
+        local += cnt[e];
+      }
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - local;
+      if (excl < need && incl >= need) {
+        uint32_t c = excl;
+        bool found = false;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (!found && c + cnt[e] >= need) {
+            t.tk[0] = 255u - 8u * lane - e;  // bin
+            t.tk[1] = c;                     // keys above the bin
+            t.tk[2] = cnt[e];                // keys in the bin
+            found = true;
+          }
+          c += cnt[e];
+        }
+      }
+    }
+    named_sync(kBarAux, kAuxThreads);
+    const uint32_t bin = t.tk[0], above = t.tk[1], in_bin = t.tk[2];
+    named_sync(kBarAux, kAuxThreads);  // tk is rewritten next pass
+    need -= above;
+    const uint32_t blo = lo + (bin << shift);
+    if (in_bin == need) {  // the whole bin is taken: exactly the keys >= blo
+      tau = blo;
+      need_eq = 0xffffffffu;
+      break;
+    }
+    lo = blo;
+    span = shift == 0 ? 0u : min(span - (bin << shift), (1u << shift) - 1u);
+    tau = lo;
+    need_eq = need;
+  }
+  // compaction: thread a owns blocks [a nb / kAuxThreads, (a+1) nb / kAuxThreads)
+  const int j0 = (int)((int64_t)a * nb / kAuxThreads), j1 = (int)((int64_t)(a + 1) * nb / kAuxThreads);
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll 1
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t u = score_key(src, glob, j);
+    n_gt += u > tau ? 1u : 0u;
+    n_eq += u == tau ? 1u : 0u;
+  }
+  uint32_t tot;
+  const uint32_t eq_before = aux_scan(n_eq, t.tks, &tot);
+  const uint32_t eq_take = eq_before >= need_eq ? 0u : min(n_eq, need_eq - eq_before);
+  uint32_t pos = aux_scan(n_gt + eq_take, t.tks + 4, &tot);
+  uint32_t eq_seen = eq_before;
+#pragma unroll 1
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t u = score_key(src, glob, j);
+    bool take = u > tau;
+    if (u == tau) {
+      take = eq_seen < need_eq;
+      ++eq_seen;
+    }
+    if (take && pos < (uint32_t)k) {
+      dst[pos] = j;
+      if (copy) copy[pos] = j;
+      ++pos;
+    }
+  }
+  return any_nan;
+}
+
+// The k <= 32 largest of the nb scores in shared memory (sc) by one warp, ties
+// to the lower index.  Lane l's keys are those of blocks l, l + 32, ...; at
+// least k lanes hold a key (nb > k), so the k-th largest of the 32 lane maxima,
+// tau, is at most the k-th largest key: every key of the top k is >= tau.  The
+// keys >= tau (usually a few dozen) are gathered in block order (one ballot per
+// row of 32 blocks), packed as key << 32 | ~index so that one comparison
+// orders by key and then by lower index, and ranked among themselves; the
+// ranks < k are written to dst[0, k) (and copy) in block order.  Returns false,
+// writing nothing, when more than cap keys are >= tau.
+__device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_t* dst, int32_t* copy,
+                                          unsigned long long* cand, int cap, bool& nan_out) {
+  constexpr int kRows = 16;  // rows of 32 blocks per pass
+  const int lane = role_tid() & 31;
+  const uint32_t lt = lanemask_lt();
+  uint32_t lmax = 0u;
+  bool nan = false;
+#pragma unroll 1
+  for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const int j = r0 + lane + 32 * i;
+      const float f = j < nb ? sc[j] : 0.f;
+      nan |= f != f;
+      if (j < nb) lmax = max(lmax, float_key(f));
+    }
+  }
+  nan_out = __any_sync(kFull, nan);
+  int r = 0;  // rank of this lane's maximum among the 32 (ties to the lower lane)
+#pragma unroll
+  for (int l = 0; l < 32; ++l) {
+    const uint32_t o = __shfl_sync(kFull, lmax, l);
+    r += (o > lmax || (o == lmax && l < lane)) ? 1 : 0;
+  }
+  const uint32_t tau = __shfl_sync(kFull, lmax, __ffs(__ballot_sync(kFull, r == k - 1)) - 1);
+  int m = 0;  // candidates so far (block order)
+#pragma unroll 1
+  for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
+    uint32_t kr[kRows], bal[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const int j = r0 + lane + 32 * i;
+      kr[i] = j < nb ? float_key(sc[j]) : 0u;
+      bal[i] = __ballot_sync(kFull, j < nb && kr[i] >= tau);
+    }
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const int pos = m + __popc(bal[i] & lt);
+      if (((bal[i] >> lane) & 1u) && pos < cap)
+        cand[pos] = ((unsigned long long)kr[i] << 32) | (uint32_t)~(r0 + lane + 32 * i);
+      m += __popc(bal[i]);
+    }
+  }
+  if (m > cap) return false;
+  __syncwarp();
+  int base = 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < m; c0 += 32) {
+    const int c = c0 + lane;
+    bool sel = false;
+    unsigned long long me = 0ull;
+    if (c < m) {
+      me = cand[c];
+      int rank = 0, o = 0;  // candidates above this one (all packed values differ)
+#pragma unroll 2
+      for (; o + 4 <= m; o += 4) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(&cand[o]);
+        const ulonglong2 y = *reinterpret_cast<const ulonglong2*>(&cand[o + 2]);
+        rank += (x.x > me ? 1 : 0) + (x.y > me ? 1 : 0) + (y.x > me ? 1 : 0) + (y.y > me ? 1 : 0);
+      }
+      for (; o < m; ++o) rank += cand[o] > me ? 1 : 0;
+      sel = rank < k;
+    }
+    const uint32_t b = __ballot_sync(kFull, sel);
+    if (sel) {
+      const int q = base + __popc(b & lt);
+      const int j = (int)~(uint32_t)me;
+      dst[q] = j;
+      if (copy) copy[q] = j;
+    }
+    base += __popc(b);
+  }
+  return true;
+}
+
+// Statistics threads (all of them): make the unit's selection known to the
+// producer (sel_state, then an arrival on sel_bar): the caller's row, every
+// block (k >= nb), none (k == 0), or the top-k of the unit's scores once every
+// rank's share is in place.  Rank 0 fills the caller's copy.
+template <int D>
+__device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
+  const int a = role_tid() - 128;
+  int32_t* copy = (p.sel_out != nullptr && rank == 0) ? p.sel_out + (int64_t)unit * p.top_k : nullptr;
+  int state = 3;
+  const int32_t* row = nullptr;
+  if (p.sel_given != nullptr) {
+    row = p.sel_given + (int64_t)unit * p.top_k;
+    if (p.top_k <= kSelCache) {
+      for (int j = a; j < p.top_k; j += kAuxThreads) sm.sel_cache[j] = __ldg(row + j);
+      state = 1;
+    } else {
+      state = 2;
+    }
+  } else if (!runs_topk(p)) {  // no block, or every block
+    if (copy)
+      for (int j = a; j < p.top_k; j += kAuxThreads) copy[j] = (p.k_eff > 0 && j < p.nb) ? j : -1;
+  } else {
+    if (a == 0) {  // one decision for all statistics threads (their barrier counts must match)
+      const bool ok = wait_cluster_bounded(&sm.scores_bar, 0, kWaitLimit);
+      if (!ok) {
+        atomicOr(p.status, HYB_STATUS_TIMEOUT);
+        sm.abort = 1;
+      }
+      sm.tk[7] = ok ? 1u : 0u;
+    }
+    named_sync(kBarAux, kAuxThreads);
+    if (sm.tk[7] != 0u) {
+      const bool glob = p.nb > FusedSmem<D>::kGather;
+      const float* src = glob ? p.scores + (int64_t)unit * p.max_blocks : sm.scores;
+      int32_t* dst = p.k_eff <= kSelCache ? sm.sel_cache : p.sel + (int64_t)unit * p.top_k;
+      bool nan = false, done = false;
+      if (p.k_eff <= 32 && !glob) {
+        if (a < 32) {  // one warp; the candidates go to the attention combine slots, idle until the selection is made
+          bool wn;
+          const bool ok = topk_warp(sm.scores, p.nb, p.k_eff, dst, copy,
+                                    reinterpret_cast<unsigned long long*>(&sm.wpart[0][0]), FusedSmem<D>::kPF, wn);
+          if (a == 0) {
+            sm.tkw[0] = ok ? 1u : 0u;
+            sm.tkw[1] = wn ? 1u : 0u;
+          }
+        }
+        named_sync(kBarAux, kAuxThreads);
+        done = sm.tkw[0] != 0u;
+        nan = sm.tkw[1] != 0u;
+      }
+      if (!done) {  // more than 32 blocks, or too many candidates: the radix selection
+        const TopkSmem t{sm.hist, sm.tk, &sm.tks[0][0]};
+        nan = aux_topk(t, src, glob, p.nb, p.k_eff, dst, copy);
+      }
+      if (nan && a == 0) atomicOr(p.status, HYB_STATUS_NAN_SCORE);
+      if (copy)
+        for (int j = p.k_eff + a; j < p.top_k; j += kAuxThreads) copy[j] = -1;
+      state = p.k_eff <= kSelCache ? 1 : 2;
+      row = dst;
+    }
+  }
+  named_sync(kBarAux, kAuxThreads);
+  if (a == 0) {
+    sm.sel_row = row;
+    sm.sel_state = state;
+    mbar_arrive(&sm.sel_bar);  // release: the selection is visible to the producer
+  }
+}
+
+}  // namespace
+}  // namespace hyb
+
+namespace hyb {
+namespace {
+
+// ---------------------------------------------------------------- attention role
+// Warps 0-3: every window and selected chunk of the rank, in ring order; then
+// the 4 warps' partials are combined into sm.wpart[0] (the rank's record:
+// m[4], l[4], dsel[4], pad[4], acc[4][D], nsel[4][D]).
+template <int D>
+__device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit) {
+  constexpr int NT8 = D / 8;  // 8-column tiles of the head dimension
+  constexpr int KS = D / 16;  // k-steps of the QK product
+  const int tid = role_tid(), warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const bool p_lane = g < 4;  // rows 0-3: softmax part; rows 4-7: Taylor part
+  const int head = g & 3;
+  const bool head_ok = head < p.G;
+  const int mi = lane >> 3, rr = lane & 7;
+
+  uint32_t qa[KS][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (head_ok ? head : 0)) * D);
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = head_ok ? __ldg(qrow + kk * 8 + tig) : 0u;
+      qa[kk][1] = head_ok ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
+    }
+  }
+  float O[NT8][4];
+#pragma unroll
+  for (int n = 0; n < NT8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f, dsel_run = 0.f;
+
+  // Chunk items go to the attention warps in turn (chunk c to warp c % 4), each
+  // warp taking all 64 tokens of its chunks.  Every attention warp waits for
+  // every chunk item in ring order and arrives on its stage's empty barrier
+  // (the owner after its work), so that no warp falls two phases behind a
+  // stage; a timed-out wait only stops this warp's work.
+  bool dead = false;
+  uint32_t par = 0u;  // bit s: parity of this group's next item in stage s
+  const int c0 = first_chunk_item(s);
+#pragma unroll 1
+  for (int it = c0; it < s.n; ++it) {
+    const int stage = it % kFStages;
+    const uint32_t ph = (par >> stage) & 1u;
+    par ^= 1u << stage;
+    bool have = false;
+    if (!dead) {
+      have = __all_sync(kFull, mbar_wait_bounded(&sm.full_attn[stage], ph, kWaitLimit));
+      if (!have) {
+        dead = true;
+        if (lane == 0) {
+          sm.abort = 1;
+          atomicOr(p.status, HYB_STATUS_TIMEOUT);
+        }
+      }
+    }
+    if (((it - c0) & 3) != warp) {
+      if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
+      continue;
+    }
+    const int4 dsc = sm.desc[stage];
+    const int nvalid = have ? dsc.y : 0;
+    if (nvalid > 0) {
+      const uint32_t kb = smem_u32(sm.ring[stage]);
+      const uint32_t vb = kb + FusedSmem<D>::kHalf;
+      if (nvalid < kTile) {
+        // rows past the chunk may hold tokens beyond T (unwritten cache rows):
+        // zero their V rows so that 0-weight * garbage cannot make a NaN
+        constexpr int CPR = D / 8;  // 16-byte chunks per row
+        uint8_t* vt = sm.ring[stage] + FusedSmem<D>::kHalf;
+        for (int e = lane; e < (kTile - nvalid) * CPR; e += 32) {
+          const int t = nvalid + e / CPR;
+          *reinterpret_cast<uint4*>(vt + swz<D>(t, e % CPR)) = make_uint4(0, 0, 0, 0);
+        }
+        // order these generic-proxy writes before the next copy into the stage
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
+      // ---- S^T = Qpad K^T for the 64 tokens: n-tile nt holds tokens 8nt .. 8nt+7
+      float sacc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+        for (int tg = 0; tg < 4; ++tg) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kb + swz<D>(tg * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)), b0, b1, b2, b3);
+          mma_16816(sacc[2 * tg], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+          mma_16816(sacc[2 * tg + 1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+        }
+      }
+      // ---- weights of this lane's 16 tokens: n-tile nt, element e -> token 8nt + 2tig + e
+      float sv[16], x[16];
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int nt = q >> 1, e = q & 1;
+        const bool v = (nt * 8 + 2 * tig + e) < nvalid;
+        sv[q] = v ? sacc[nt][e] * p.scale : 0.f;
+        x[q] = (p_lane && v) ? sv[q] * kLog2e : -INFINITY;
+        tmax = fmaxf(tmax, x[q]);
+      }
+      tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
+      const float m_new = fmaxf(m_run, tmax);
+      const float alpha = (p_lane && m_new != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+      const bool sel_tok = dsc.z != 0;
+      float w[16], wsum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int nt = q >> 1, e = q & 1;
+        const bool v = (nt * 8 + 2 * tig + e) < nvalid;
+        w[q] = p_lane ? (v ? exp2f(x[q] - m_new) : 0.f) : ((v && sel_tok) ? 1.f + sv[q] : 0.f);
+        wsum += w[q];
+      }
+      if (p_lane) {
+        l_run = l_run * alpha + wsum;
+        m_run = m_new;
+      } else {
+        dsel_run += wsum;
+      }
+      if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+        for (int n = 0; n < NT8; ++n) {
+          O[n][0] *= alpha;
+          O[n][1] *= alpha;
+          O[n][2] *= alpha;
+          O[n][3] *= alpha;
+        }
+      }
+      // ---- O += A V, k-step kt over tokens 16kt .. 16kt+15 (rows g: bf16 hi, g+8: lo)
+#pragma unroll
+      for (int kt = 0; kt < 4; ++kt) {
+        uint32_t a0, a1, a2, a3;
+        split_bf16(w[4 * kt + 0], w[4 * kt + 1], a0, a1);
+        split_bf16(w[4 * kt + 2], w[4 * kt + 3], a2, a3);
+#pragma unroll
+        for (int np = 0; np < NT8 / 2; ++np) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, np * 2 + (mi >> 1)), b0, b1, b2, b3);
+          mma_16816(O[2 * np], a0, a1, a2, a3, b0, b1);
+          mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
+  }
+
+  // the combine slots hold the top-k candidates until the selection is made
+  // (a rank without selected chunks gets here first)
+  if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit);
+  // ---- combine the 4 warps' partials (a tree through two shared slots: warps
+  //      2, 3 -> 0, 1, then warp 1 -> 0); warp 0 leaves the record in wpart[0]
+  float l = l_run + __shfl_xor_sync(kFull, l_run, 1);
+  l += __shfl_xor_sync(kFull, l, 2);
+  float ds = dsel_run + __shfl_xor_sync(kFull, dsel_run, 1);
+  ds += __shfl_xor_sync(kFull, ds, 2);
+  const int voff = (p_lane ? 0 : 4 * D) + head * D;
+  auto emit = [&](float* wp) {  // write this warp's partial (hi + lo rows summed)
+    if (tig == 0) {
+      if (p_lane) {
+        wp[head] = m_run;
+        wp[4 + head] = l;
+      } else {
+        wp[8 + head] = ds;
+      }
+    }
+    float* dst = wp + 16 + voff;
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+      *reinterpret_cast<float2*>(dst + n * 8 + 2 * tig) = make_float2(O[n][0] + O[n][2], O[n][1] + O[n][3]);
+  };
+  auto absorb = [&](const float* wp) {  // fold another warp's partial into this one
+    const float mp = wp[head], lp = wp[4 + head], dsp = wp[8 + head];
+    float fa = 1.f, fb = 1.f;
+    if (p_lane) {
+      const float M = fmaxf(m_run, mp);
+      fa = (m_run == -INFINITY) ? 0.f : exp2f(m_run - M);
+      fb = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
+      l = l * fa + lp * fb;
+      m_run = M;
+    } else {
+      ds += dsp;
+    }
+    const float* src = wp + 16 + voff;
+#pragma unroll
+    for (int n = 0; n < NT8; ++n) {
+      const float2 y = *reinterpret_cast<const float2*>(src + n * 8 + 2 * tig);
+      O[n][0] = (O[n][0] + O[n][2]) * fa + y.x * fb;
+      O[n][1] = (O[n][1] + O[n][3]) * fa + y.y * fb;
+      O[n][2] = O[n][3] = 0.f;
+    }
+  };
+  if (warp >= 2) emit(sm.wpart[warp - 2]);
+  named_sync(kBarAttn, 128);
+  if (warp < 2) absorb(sm.wpart[warp]);
+  named_sync(kBarAttn, 128);
+  if (warp == 1) emit(sm.wpart[0]);
+  named_sync(kBarAttn, 128);
+  if (warp == 0) {
+    absorb(sm.wpart[0]);
+    __syncwarp();
+    emit(sm.wpart[0]);
+  }
+}
+
+}  // namespace
+}  // namespace hyb
+
+namespace hyb {
+namespace {
+
+// Statistics warps (roles 4-6): H items (rows split between the warps); score
+// items, one warp per item (item i to warp i % 3); hand the scores to every
+// rank; the selection; the rank's linear partial.  Every statistics warp waits for every
+// statistics item in ring order and arrives once on its stage's empty barrier
+// (the owner after its work), so that no warp falls two phases behind a stage.
+template <int D>
+__device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int rank) {
+  constexpr int CPL = D / 32;
+  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  // a timed-out wait only stops this warp's work; it keeps visiting every item
+  // and barrier
+  bool dead = false;
+  uint32_t par = 0u;  // bit s: parity of this group's next item in stage s (items come in order)
+  auto wait_item = [&](int it) -> bool {
+    const int stage = it % kFStages;
+    const uint32_t ph = (par >> stage) & 1u;
+    par ^= 1u << stage;
+    if (dead) return false;
+    const bool have = __all_sync(kFull, mbar_wait_bounded(&sm.full_aux[stage], ph, kWaitLimit));
+    if (!have) {
+      dead = true;
+      if (lane == 0) {
+        sm.abort = 1;
+        atomicOr(p.status, HYB_STATUS_TIMEOUT);
+      }
+    }
+    return have;
+  };
+  const int64_t nf = p.fold_end - p.fold_begin;
+  if (p.q != nullptr)
+    for (int c = a; c < D; c += kAuxThreads) {
+      float q1 = 0.f, q2 = 0.f;
+      for (int i = 0; i < p.G; ++i) {
+        const float qv = sm.qs[i][c];
+        q1 += qv;
+        q2 += 0.5f * qv * qv;
+      }
+      sm.qsum[0][c] = q1;
+      sm.qsum[1][c] = q2;
+    }
+  if (nf == 1)  // the pending token's rows, for the H items
+    for (int c = a; c < D; c += kAuxThreads) {
+      const int64_t row = ((int64_t)unit * p.cap + p.fold_begin) * D + c;
+      sm.ktok[c] = __bfloat162float(p.k_cache[row]);
+      sm.vtok[c] = __bfloat162float(p.v_cache[row]);
+    }
+  named_sync(kBarAux, kAuxThreads);
+  float hacc[kMaxGroup][CPL];
+#pragma unroll
+  for (int i = 0; i < kMaxGroup; ++i)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) hacc[i][c] = 0.f;
+#pragma unroll 1
+  for (int idx = 0; idx < s.nH; ++idx) {
+    const int it = seq_of_h(s, idx), stage = it % kFStages;
+    const bool have = wait_item(it);
+    if (have && (p.q != nullptr || nf > 0)) aux_h_item<D>(p, sm, s, unit, idx, stage, hacc);
+    __syncwarp();
+    if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
+  }
+#pragma unroll 1
+  for (int idx = 0; idx < s.nS; ++idx) {
+    const int it = seq_of_s(s, idx), stage = it % kFStages;
+    const bool have = wait_item(it);
+    if (have && idx % kAuxWarps == aw) {
+      if (score_item_folds<D>(p, s, idx)) fold_score_item<D>(p, sm, s, unit, idx, stage);
+      if (p.q != nullptr) score_item_warp<D>(p, sm, s, unit, idx, stage);
+      __syncwarp();
+    }
+    if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
+  }
+  named_sync(kBarAux, kAuxThreads);  // every score of this rank is in place
+  if (runs_topk(p)) {  // hand this rank's scores to every rank
+    if (p.nb <= FusedSmem<D>::kGather) {
+      // bulk copies of the share into every other rank's scores array
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      named_sync(kBarAux, kAuxThreads);
+      if (a == 0 && s.b1 > s.b0) {
+        const uint32_t bytes = (uint32_t)(((s.b1 - s.b0) * 4 + 15) & ~15);
+        const uint32_t src = smem_u32(&sm.scores[s.b0]), bar = smem_u32(&sm.scores_bar);
+        for (int rr = 0; rr < p.C; ++rr)
+          if (rr != rank) bulk_push(map_rank(src, (uint32_t)rr), src, bytes, map_rank(bar, (uint32_t)rr));
+      }
+    } else {
+      // the scores went to global memory: release them at cluster scope
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      named_sync(kBarAux, kAuxThreads);
+      if (a == 0) {
+        const uint32_t la = smem_u32(&sm.scores_bar);
+        for (int rr = 0; rr < p.C; ++rr) remote_arrive(map_rank(la, (uint32_t)rr));
+      }
+    }
+  }
+
+  if (p.q != nullptr) aux_select<D>(p, sm, unit, rank);
+  aux_finish_linear<D>(p, sm, unit, rank, hacc);
+}
+
+// Producer (role warp 7, lane 0): every copy of the rank, in ring order, one
+// short loop per kind of item with running addresses.  Before an item goes into
+// a stage that held an earlier item, the stage's empty barrier must have
+// completed for that earlier item.
+template <int D>
+__device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit,
+                              int rank) {
+  if ((threadIdx.x & 31) != 0) return;
+  constexpr int RB = Geo<D>::kBlocks, RH = Geo<D>::kRows;
+  int stage = 0, issued = 0;
+  uint32_t epar = 0u;                  // per stage: parity of the next empty-barrier phase to wait for
+  uint32_t fpar_aux = 0u, fpar_at = 0u;  // per stage: parity of the next full-barrier phase of each group
+  uint32_t last_aux = 0u;              // per stage: the last item issued into it was a statistics item
+  bool ok = true;
+  auto acquire = [&]() -> bool {
+    if (issued >= kFStages) {
+      const uint32_t ph = (epar >> stage) & 1u;
+      epar ^= 1u << stage;
+      if (!mbar_wait_bounded(&sm.empty[stage], ph, kWaitLimit)) {
+        atomicOr(p.status, HYB_STATUS_TIMEOUT);
+        sm.abort = 1;
+        return false;
+      }
+    }
+    return *(volatile int*)&sm.abort == 0;
+  };
+  auto advance = [&](bool aux) {
+    if (aux) {
+      fpar_aux ^= 1u << stage;
+      last_aux |= 1u << stage;
+    } else {
+      fpar_at ^= 1u << stage;
+      last_aux &= ~(1u << stage);
+    }
+    ++issued;
+    stage = stage + 1 == kFStages ? 0 : stage + 1;
+  };
+  // H items: RH rows of H
+  const bool h_load = p.q != nullptr || p.fold_end > p.fold_begin;
+  for (int i = 0; i < s.nH && ok; ++i) {
+    if (!(ok = acquire())) break;
+    uint64_t* bar = &sm.full_aux[stage];
+    if (h_load) {
+      const int r0 = s.h0 + i * RH;
+      const uint32_t bytes = (uint32_t)(min(RH, s.h1 - r0) * D * 4);
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_load(smem_u32(sm.ring[stage]), p.H + ((int64_t)unit * D + r0) * D, bytes, bar);
+    } else {
+      mbar_arrive(bar);
+    }
+    advance(true);
+  }
+  // score items: the mean and variance rows of RB blocks
+  const int64_t brow = (int64_t)unit * p.max_blocks + s.b0;
+  for (int i = 0; i < s.nS && ok; ++i) {
+    if (!(ok = acquire())) break;
+    uint64_t* bar = &sm.full_aux[stage];
+    if (p.q != nullptr || score_item_folds<D>(p, s, i)) {
+      const uint32_t dst = smem_u32(sm.ring[stage]);
+      const uint32_t bytes = (uint32_t)(min(RB, s.b1 - s.b0 - i * RB) * D * 4);
+      const int64_t off = (brow + (int64_t)i * RB) * D;
+      mbar_arrive_expect_tx(bar, 2 * bytes);
+      bulk_load(dst, p.mu + off, bytes, bar);
+      bulk_load(dst + RB * D * 4, p.var + off, bytes, bar);
+    } else {
+      mbar_arrive(bar);
+    }
+    advance(true);
+  }
+  // window (and sink) chunks: chunk ci = rank + i C of the exact prefix
+  const int64_t ubase = (int64_t)unit * p.cap;
+  for (int i = 0, ci = rank; i < s.nW && ok; ++i, ci += p.C) {
+    if (!(ok = acquire())) break;
+    int start, len;
+    if (ci < p.n_sink_chunks) {
+      start = ci * kTile;
+      len = min(kTile, p.sink_len - start);
+    } else {
+      start = p.win_start + (ci - p.n_sink_chunks) * kTile;
+      len = min(kTile, p.T - start);
+    }
+    issue_chunk<D>(tm, sm, stage, ubase, start, len, 0);
+    advance(false);
+  }
+  // selected chunks: chunk sc = rank + i C is piece sc % cpb of selection slot sc / cpb
+  if (ok && s.nX > 0 && !mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit)) {
+    atomicOr(p.status, HYB_STATUS_TIMEOUT);
+    sm.abort = 1;
+    ok = false;
+  }
+  const int cpb = p.chunks_per_block;
+  int slot = rank / cpb, piece = rank - (rank / cpb) * cpb;
+  const int st = sm.sel_state;
+  for (int i = 0; i < s.nX && ok; ++i) {
+    if (!(ok = acquire())) break;
+    int jb = -1;
+    if (slot < p.k_eff) jb = st == 3 ? slot : st == 1 ? sm.sel_cache[slot] : __ldcg(sm.sel_row + slot);
+    int start = 0, len = 0;
+    if (jb >= 0 && jb < p.nb) {
+      const int bs = p.S + jb * p.Bk;
+      start = bs + piece * kTile;
+      len = max(0, min(kTile, min(bs + p.Bk, p.ev_end) - start));
+    } else if (jb != -1) {
+      atomicOr(p.status, HYB_STATUS_BAD_SELECTION);
+    }
+    issue_chunk<D>(tm, sm, stage, ubase, start, len, 1);
+    advance(false);
+    if (cpb == 1) {
+      slot += p.C;
+    } else {
+      piece += p.C;
+      slot += piece / cpb;
+      piece -= (piece / cpb) * cpb;
+    }
+  }
+  if (*(volatile int*)&sm.abort) {
+    // do not leave while copies into this CTA's ring may be in flight: wait for
+    // the last item issued into each stage (its group's full barrier, its phase)
+    for (int j = 0; j < kFStages && j < issued; ++j) {
+      const bool aux = (last_aux >> j) & 1u;
+      const uint32_t ph = (((aux ? fpar_aux : fpar_at) >> j) & 1u) ^ 1u;  // parity of the last item's phase
+      mbar_wait_bounded(aux ? &sm.full_aux[j] : &sm.full_attn[j], ph, kWaitLimit);
+    }
+  }
+}
+
+// Rank 0, all threads, after the first cluster barrier: merge the C records and
+// linear partials (read over distributed shared memory) and write the output.
+template <int D>
+__device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit) {
+  constexpr int PF = FusedSmem<D>::kPF;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = p.G, C = p.C;
+  // per rank and head: rescale factor of the exact part; per head: max, D_ex, D_sel
+  float* fac = reinterpret_cast<float*>(sm.ring[0]);  // [16][4] (the ring is idle now)
+  float* hm = fac + 16 * 4;                           // M[4], Dex[4], Dsel[4]
+  const uint32_t rec0 = smem_u32(&sm.wpart[0][0]);
+  const uint32_t lin0 = smem_u32(&sm.linp[0][0]);
+  if (warp < G) {  // warp i: head i
+    const int i = warp;
+    float m = -INFINITY, l = 0.f, ds = 0.f;
+    if (lane < C) {
+      const uint32_t rb = map_rank(rec0, lane);
+      m = ld_cluster_f32(rb + 4 * i);
+      l = ld_cluster_f32(rb + 4 * (4 + i));
+      ds = ld_cluster_f32(rb + 4 * (8 + i));
+    }
+    float M = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    if (M == -INFINITY) M = 0.f;
+    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    if (lane < C) fac[lane * 4 + i] = f;
+    float dex = l * f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      dex += __shfl_xor_sync(kFull, dex, o);
+      ds += __shfl_xor_sync(kFull, ds, o);
+    }
+    if (lane == 0) {
+      hm[i] = M;
+      hm[4 + i] = dex;
+      hm[8 + i] = ds;
+    }
+  }
+  __syncthreads();
+  uint32_t flags = 0u;
+  for (int e = tid; e < G * D; e += kFThreads) {
+    const int i = e / D, d = e % D;
+    float xa[kMaxCluster], xs[kMaxCluster], xl[kMaxCluster];  // every remote load in flight first
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      if (r < C) {
+        const uint32_t rb = map_rank(rec0, r), lb = map_rank(lin0, r);
+        xa[r] = ld_cluster_f32(rb + 4 * (16 + i * D + d));
+        xs[r] = ld_cluster_f32(rb + 4 * (16 + 4 * D + i * D + d));
+        xl[r] = ld_cluster_f32(lb + 4 * (i * (D + 1) + d));
+      }
+    }
+    float nex = 0.f, nsel = 0.f, ng = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      if (r < C) {
+        nex += xa[r] * fac[r * 4 + i];
+        nsel += xs[r];
+        ng += xl[r];
+      }
+    }
+    const float Ms = hm[i], Dex = hm[4 + i], Dsel = hm[8 + i];
+    const float Dg = sm.linp[i][D];  // rank 0 holds D_glob
+    float num, den;
+    if (Ms >= 0.f) {
+      const float f = exp2f(-Ms);
+      num = nex + f * (ng - nsel);
+      den = Dex + f * (Dg - Dsel);
+    } else {
+      const float f = exp2f(Ms);
+      num = nex * f + (ng - nsel);
+      den = Dex * f + (Dg - Dsel);
+    }
+    const float o = num / den;
+    p.out[((int64_t)unit * G + i) * D + d] = o;
+    if (!(den > 0.f)) flags |= HYB_STATUS_DENOMINATOR;
+    if (!isfinite(o)) flags |= HYB_STATUS_NONFINITE;
+  }
+  if (flags) atomicOr(p.status, flags);
+  (void)PF;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_constant__ KVMaps tm, const FusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned (the 128-byte swizzle repeats every 1024 bytes); offsetting
+  // the shared array keeps every access through `sm` in the shared space
+  FusedSmem<D>& sm = *reinterpret_cast<FusedSmem<D>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = role_tid() >> 5;
+  const int rank = (int)cluster_rank();
+  const int unit = blockIdx.x / p.C;
+  const Seq s = make_seq<D>(p, rank);
+  if (tid == 0) {
+    tma_prefetch_desc(&tm.k64);
+    tma_prefetch_desc(&tm.v64);
+    for (int i = 0; i < kFStages; ++i) {
+      mbar_init(&sm.full_attn[i], 1);
+      mbar_init(&sm.full_aux[i], 1);
+      mbar_init(&sm.empty[i], kEmptyCount);
+    }
+    // scores_bar: the other ranks' shares arriving by bulk copy (one local
+    // arrival expecting their bytes), or C arrivals when the scores go
+    // through global memory
+    const bool push = runs_topk(p) && p.nb <= FusedSmem<D>::kGather;
+    mbar_init(&sm.scores_bar, push ? 1 : p.C);
+    mbar_init(&sm.sel_bar, 1);
+    sm.sel_state = 3;
+    sm.sel_row = nullptr;
+    sm.abort = 0;
+    fence_mbar_init();
+    if (push) {
+      uint32_t bytes = 0;
+      for (int rr = 0; rr < p.C; ++rr) {
+        int b0, b1;
+        block_share(p.nb, p.C, rr, b0, b1);
+        if (rr != rank) bytes += (uint32_t)(((b1 - b0) * 4 + 15) & ~15);
+      }
+      mbar_arrive_expect_tx(&sm.scores_bar, bytes);
+    }
+    pdl_wait_primary();  // everything below reads what earlier grids wrote
+  }
+  // the barriers of every rank are initialised before any remote arrival
+  cluster_sync_all();
+  pdl_allow_dependents();
+  if (warp == 7) {
+    // the producer starts at once: it needs nothing from the lines below
+    producer_role<D>(&tm, p, sm, s, unit, rank);
+  } else {
+    const int t = role_tid();  // 0 .. kConsumerThreads - 1
+    if (p.q != nullptr)
+      for (int e = t; e < kMaxGroup * D; e += kConsumerThreads) {
+        const float qv = e < p.G * D ? __bfloat162float(p.q[(int64_t)unit * p.G * D + e]) * p.scale : 0.f;
+        sm.qs[e / D][e % D] = sm.qsT[e % D][e / D] = qv;
+      }
+    if (p.k_new != nullptr && rank == 0 && t < D / 4) {
+      // the decode's appended token: row T of the caches (16 bytes per thread)
+      const bool is_v = t >= D / 8;
+      const int e = (t % (D / 8)) * 8;
+      const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + (int64_t)unit * D + e;
+      __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e;
+      *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+    }
+    named_sync(kBarConsumers, kConsumerThreads);
+    if (warp < 4) {
+      if (p.q != nullptr) attn_role<D>(p, sm, s, unit);
+    } else {
+      aux_role<D>(p, sm, s, unit, rank);
+    }
+  }
+  cluster_sync_all();  // every rank's record and linear partial are final
+  if (rank == 0 && p.q != nullptr) merge_cluster<D>(p, sm, unit);
+  cluster_sync_all();  // the records stay readable until rank 0 is done
+}
+
+}  // namespace
+
+static_assert(sizeof(FusedSmem<128>) + 1024 <= 232448, "shared memory per CTA");
+static_assert(sizeof(FusedSmem<64>) + 1024 <= 232448, "shared memory per CTA");
+
+size_t fused_smem_bytes(int D) {
+  return (D == 128 ? sizeof(FusedSmem<128>) : sizeof(FusedSmem<64>)) + 1024;
+}
+
+cudaError_t prepare_fused(int D) {
+  const int smem = (int)fused_smem_bytes(D);
+  const void* f = D == 128 ? (const void*)fused_kernel<128> : (const void*)fused_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  return e;
+}
+
+int fused_max_clusters(int D, int c) {
+  const void* f = D == 128 ? (const void*)fused_kernel<128> : (const void*)fused_kernel<64>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = fused_smem_bytes(D);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = c;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, f, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+cudaError_t launch_fused(const CUtensorMap* maps, const FusedParams& p, int D, cudaStream_t s) {
+  KVMaps tm;
+  tm.k64 = maps[0];
+  tm.v64 = maps[1];
+  tm.k16 = maps[2];
+  tm.v16 = maps[3];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.units * p.C));
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = fused_smem_bytes(D);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (D == 128) return cudaLaunchKernelEx(&cfg, fused_kernel<128>, tm, p);
+  return cudaLaunchKernelEx(&cfg, fused_kernel<64>, tm, p);
+}
+
+}  // namespace hyb

@@ -137,11 +137,8 @@ typedef struct hyb_attn_plan_info {
   int64_t k_eff;             /* min(top_k, nb) */
   int64_t exact_tokens;      /* |sinks| + |window| + tokens of k_eff full blocks (upper bound) */
   int32_t chunks_per_unit;   /* 64-token pieces of the exact set per unit (fixed for a given T) */
-  int32_t select_ctas;       /* grid of the select kernel (persistent) */
-  int32_t attend_ctas;       /* grid of the attention kernel (split-K CTAs of every unit) */
-  int32_t partial_slots;     /* split-K partial records the attention kernel writes */
-  int32_t score_items_per_unit;   /* select work items over the block statistics */
-  int32_t linear_items_per_unit;  /* select work items over rows of H */
+  int32_t cluster_ctas;      /* CTAs per unit (one thread-block cluster); the device may use fewer */
+  int32_t grid_ctas;         /* grid of the decode kernel: units * cluster_ctas */
 } hyb_attn_plan_info;
 
 /* Fill `out` with the buffer sizes of `cfg`.  Host only; never touches a GPU.
@@ -189,18 +186,18 @@ int hyb_attn_sync_state(hyb_attn_ctx* ctx, cudaStream_t stream);
  *               ascending, -1 padded when nb < top_k
  *   scores_out  fp32 [B][Hkv][max_blocks] or NULL: the block scores (entries
  *               [0, nb) of each unit are written)
- * Kernels (chained with programmatic dependent launch): block scoring + the
- * global linear term phi(q)^T state (folding in the tokens evicted since the
- * previous decode); beside it, split-K exact attention over the sinks and the
- * window, which then takes the top-k of the scores, attends the selected blocks
- * with their (1 + s) subtraction, and merges under the shared normaliser.
+ * One kernel launch: per unit a thread-block cluster scores the blocks, folds in
+ * the tokens evicted since the previous decode, forms the global linear term
+ * phi(q)^T state, selects the top-k, attends sinks, window and selected blocks
+ * exactly (split-K over the cluster, with the selected blocks' (1 + s)
+ * subtraction) and merges under the shared normaliser.
  * Errors: HYB_EINVAL (null or misaligned pointers), HYB_ESTATE (T == 0),
  * HYB_ECUDA. */
 int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out,
                     float* scores_out, cudaStream_t stream);
 
 /* hyb_attn_decode followed by hyb_attn_append(k_new, v_new) in the same
- * launches: the attention kernel also writes the new token at row T, then
+ * launch: the decode kernel also writes the new token at row T, then
  * T += 1 -- one decode step of a generation loop.  The decode attends to
  * [0, T) as stored before the call.  Errors: those of both calls. */
 int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, const void* v_new,
@@ -259,9 +256,8 @@ int64_t hyb_attn_length(const hyb_attn_ctx* ctx);
 int hyb_attn_status(hyb_attn_ctx* ctx, uint32_t* flags, int clear, cudaStream_t stream);
 
 /* Profiling hook: when both events are non-NULL, every later decode records
- * `begin` just before its first and `end` just after its last kernel on the
- * decode's stream, so the caller can time one decode's kernels (chained as in
- * normal use) without the rest of its stream.  Pass NULL, NULL to stop. */
+ * `begin` just before and `end` just after its kernel on the decode's stream,
+ * so the caller can time one decode alone.  Pass NULL, NULL to stop. */
 int hyb_attn_set_timing_events(hyb_attn_ctx* ctx, cudaEvent_t begin, cudaEvent_t end);
 
 /* Release the host context (device buffers stay with the caller). */

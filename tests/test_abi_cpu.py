@@ -104,9 +104,8 @@ def test_init_rejects_bad_arguments_without_touching_a_gpu(lib):
 @pytest.mark.parametrize("T", [0, 1, 3, 4, 5, 1027, 1028, 1029, 1092, 1093, 32768, 32768 + 64])
 def test_plan_partition(lib, T):
     """Chunk counts of the exact set follow the partition (sinks, window, and
-    ceil(Bk/64) chunks per selected block); the attention kernel runs one CTA per
-    SM beside the select kernel's two; the select work items tile the blocks and
-    the rows of H."""
+    ceil(Bk/64) chunks per selected block); each unit gets one cluster of at
+    most 16 CTAs, as many as keep the grid within one CTA per SM."""
     import hybrid_sparse_linear_decode_b200 as H
     c = _cfg()
     n_sm = 148
@@ -118,20 +117,13 @@ def test_plan_partition(lib, T):
     sink = min(S, T)
     win = T - max(S, T - W) if T > S else 0
     assert p.chunks_per_unit == -(-sink // 64) + -(-win // 64) + p.k_eff
-    splits = max(1, min(n_sm // units, p.chunks_per_unit))
-    assert p.attend_ctas == units * splits and p.partial_slots == units * splits
-    R, RL = 16384 // (8 * 128), 16384 // (4 * 128)
-    assert p.score_items_per_unit == -(-nb // R)
-    assert p.linear_items_per_unit == 128 // RL
-    total = units * (p.score_items_per_unit + p.linear_items_per_unit)
-    assert p.select_ctas == min(total, 2 * n_sm)
+    assert p.cluster_ctas == 16 and p.grid_ctas == units * 16
 
 
-def test_plan_caps_grids_for_many_units(lib):
-    """With more units than CTA slots the attention kernel uses one CTA per
-    unit, and the select grid stays persistent (two CTAs per SM)."""
+@pytest.mark.parametrize("batch,want", [(1, 16), (2, 9), (4, 4), (8, 2), (16, 1), (512, 1)])
+def test_plan_cluster_size(lib, batch, want):
+    """8 KV heads per row on 148 SMs: min(16, floor(148 / units)) CTAs per unit."""
     import hybrid_sparse_linear_decode_b200 as H
-    c = _cfg(batch=512, capacity=4096)
+    c = _cfg(batch=batch, capacity=4096)
     p = H.hyb_attn_plan(c, 4096, 148)
-    assert p.attend_ctas == 512 * 8
-    assert p.select_ctas == 296
+    assert p.cluster_ctas == want and p.grid_ctas == batch * 8 * want
