@@ -65,21 +65,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 // Bounded wait: gives up (returns false) once about `limit_ns` nanoseconds have
-// passed without the phase completing.  After a short burst of polls the
-// thread sleeps between polls, leaving the issue slots of its SM sub-partition
-// to warps that have work.
+// passed without the phase completing.  try_wait itself suspends the thread
+// for a while when the phase is not complete (and resumes it when the phase
+// completes), so the loop polls without sleeping; a sleep between polls would
+// add its wake-up delay to every wait.  The timer is read every 256 polls.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  // (loops kept rolled: this is inlined at every wait site)
-#pragma unroll 1
-  for (int i = 0; i < 32; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
-    for (int i = 0; i < 16; ++i) {
-      __nanosleep(64);
+    for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    }
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }

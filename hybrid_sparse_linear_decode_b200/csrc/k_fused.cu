@@ -10,8 +10,8 @@
 //     of 32 blocks each) and rows [r D / C, (r+1) D / C) of H (H items),
 //   * window chunks r, r + C, ... and selected chunks r, r + C, ... (64-token
 //     pieces of the exact set, split-K).
-// Its items stream through a kFStages-deep shared-memory ring in the order H
-// items, score items, window chunks, selected chunks: a producer warp issues
+// Its items stream through a kFStages-deep shared-memory ring in the order score
+// items, window chunks, H items, selected chunks: a producer warp issues
 // the copies (TMA tensor loads for K/V chunks, untiled bulk copies for the
 // statistics and H, no multicast); the other warps consume them.
 //
@@ -21,8 +21,8 @@
 //        packed into the 16-row M dimension (rows 0-3 softmax, rows 4-7 the
 //        Taylor weights 1 + s of selected-block tokens, rows 8-15 the bf16
 //        rounding remainders of rows 0-7);
-//   4-6  statistics: H rows, block scores (score item i to warp i % 3), the
-//        Welford fold, the top-k (one warp), the linear term;
+//   4-6  statistics: block scores (score item i to warp i % 3), the Welford
+//        fold, the top-k (one warp), H rows, the linear term;
 //   7    producer: lane 0 issues every copy in ring order.
 //
 // Block score ("SPLA: Block Sparse Plus Linear Attention for Long Context
@@ -62,6 +62,7 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kFThreads = 256;
 constexpr int kFStages = 6;
 constexpr int kFScoresMax = 2048;   // scores a CTA keeps for its unit (else they go through global memory)
+static_assert(kFScoresMax >= 512, "the one-warp top-k reads 512 entries unconditionally");
 constexpr int kAuxWarps = 3;        // statistics warps: roles 4-6
 constexpr int kAuxThreads = 32 * kAuxWarps;
 constexpr int kConsumerThreads = 128 + kAuxThreads;  // attention + statistics (roles 0-6)
@@ -100,18 +101,15 @@ __device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity)
       : "memory");
   return ok != 0;
 }
-// bounded wait on a barrier that other CTAs of the cluster arrive on
+// bounded wait on a barrier that other CTAs of the cluster arrive on (polled
+// like mbar_wait_bounded)
 __device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-#pragma unroll 1
-  for (int i = 0; i < 32; ++i)
-    if (try_wait_cluster(bar, parity)) return true;
+  if (try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
-    for (int i = 0; i < 16; ++i) {
-      __nanosleep(64);
+    for (int i = 0; i < 256; ++i)
       if (try_wait_cluster(bar, parity)) return true;
-    }
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
@@ -130,15 +128,11 @@ __device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t b
                "r"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
-// This thread's index in role order.  Warp w runs on sub-partition w % 4: the
-// attention roles (0-3) sit on hardware warps 0, 1, 4, 5 (sub-partitions 0, 1),
-// the statistics roles (4-6) on warps 2, 3, 6 and the producer (role 7) on
-// warp 7 (sub-partitions 2, 3), so that each sub-partition's instruction cache
-// serves the attention loop or the statistics and copy code, not both.
-__device__ __forceinline__ int role_tid() {
-  const uint32_t w = threadIdx.x >> 5;
-  return (int)((((0x76325410u >> (4u * w)) & 15u) << 5) | (threadIdx.x & 31u));
-}
+// This thread's index in role order: role r is hardware warp r.  Warp w runs on
+// sub-partition w % 4, so each statistics warp (4-6) and the producer (7) shares
+// a sub-partition with one attention warp (0-3); the attention warps idle while
+// the score items stream, which is when the statistics warps are busiest.
+__device__ __forceinline__ int role_tid() { return (int)threadIdx.x; }
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -211,10 +205,10 @@ __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint3
 }
 
 // ---------------------------------------------------------------- item sequence
-// Items of rank r, in ring order: nH H items, nS score items, nW window (and
-// sink) chunks, nX selected chunks.  The H rows come first (the statistics
-// warps fold and sum them while the first score items are in flight), the
-// scores next, so that the top-k runs while the window chunks stream in.  Every
+// Items of rank r, in ring order: nS score items, nW window (and sink) chunks,
+// nH H items, nX selected chunks.  The scores come first, so that the top-k
+// runs while the window chunks and H rows stream in; the statistics warps take
+// the H rows after the selection, while the selected chunks stream.  Every
 // thread derives the same sequence.
 struct Seq {
   int b0, b1, nS;   // blocks [b0, b1), kFBlocks per score item
@@ -262,19 +256,31 @@ __device__ __forceinline__ Seq make_seq(const FusedParams& p, int r) {
   return q;
 }
 
-// position in the ring order of H item i / score item i / the first chunk item
-__device__ __forceinline__ int seq_of_h(const Seq&, int i) { return i; }
-__device__ __forceinline__ int seq_of_s(const Seq& s, int i) { return s.nH + i; }
-__device__ __forceinline__ int first_chunk_item(const Seq& s) { return s.nS + s.nH; }
+// position in the ring order of score item i / H item i / chunk item c (window
+// chunks first, then selected chunks)
+__device__ __forceinline__ int seq_of_s(const Seq&, int i) { return i; }
+__device__ __forceinline__ int seq_of_h(const Seq& s, int i) { return s.nS + s.nW + i; }
+__device__ __forceinline__ int seq_of_chunk(const Seq& s, int c) { return c < s.nW ? s.nS + c : s.nS + s.nH + c; }
 
+// Score items [*i0, *i1) of the rank hold the blocks with pending evictions
+// (empty when nothing is pending).  Computed once per launch.
+template <int D>
+__device__ __forceinline__ void fold_items(const FusedParams& p, const Seq& s, int* i0, int* i1) {
+  *i0 = *i1 = 0;
+  if (p.fold_end <= p.fold_begin || s.b1 <= s.b0) return;
+  // positions fit in 32 bits (units x capacity < 2^31)
+  const int jb0 = (int)(p.fold_begin - p.S) / p.Bk, jb1 = (int)(p.fold_end - 1 - p.S) / p.Bk;
+  const int lo = max(jb0, s.b0), hi = min(jb1, s.b1 - 1);
+  if (lo > hi) return;
+  *i0 = (lo - s.b0) / Geo<D>::kBlocks;
+  *i1 = (hi - s.b0) / Geo<D>::kBlocks + 1;
+}
 // score item idx: does it hold a block with pending evictions?
 template <int D>
 __device__ __forceinline__ bool score_item_folds(const FusedParams& p, const Seq& s, int idx) {
-  if (p.fold_end <= p.fold_begin) return false;
-  const int64_t j0 = s.b0 + (int64_t)idx * Geo<D>::kBlocks;
-  const int64_t j1 = min((int64_t)s.b1, j0 + Geo<D>::kBlocks);
-  const int64_t jb0 = (p.fold_begin - p.S) / p.Bk, jb1 = (p.fold_end - 1 - p.S) / p.Bk;
-  return jb1 >= j0 && jb0 < j1;
+  int i0, i1;
+  fold_items<D>(p, s, &i0, &i1);
+  return idx >= i0 && idx < i1;
 }
 
 // Producer: the copies of one K/V chunk (rows [start, start + len) of the
@@ -400,9 +406,11 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
 // Score item `idx` by one warp, score_j = sum_c qsum[0][c] mu_jc +
 // qsum[1][c] var_jc (qsum = sum_i q'_i and 1/2 sum_i q'_i^2): lane l forms the
 // partial sums of its channels [l*CPL, l*CPL + CPL) for all 32 blocks (each
-// row read once, conflict-free), then a transposing butterfly (31 shuffles in 5
-// rounds: in the round of width h a lane keeps the half of its values whose
-// block index has bit h equal to its own) leaves block l's score in lane l.
+// row read once, conflict-free, at fixed offsets from one base), then a
+// transposing butterfly (31 shuffles in 5 rounds: in the round of width h a
+// lane keeps the half of its values whose block index has bit h equal to its
+// own) leaves block l's score in lane l.  Rows past the item's last block hold
+// stale stage data: their sums stay in their own lanes and are not stored.
 template <int D>
 __device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx,
                                                 int stage) {
@@ -412,7 +420,7 @@ __device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<
   const int lane = role_tid() & 31;
   const int j0 = s.b0 + idx * RB;
   const int nblk = min(RB, s.b1 - j0);
-  const float* mrows = reinterpret_cast<const float*>(sm.ring[stage]);
+  const float* mrows = reinterpret_cast<const float*>(sm.ring[stage]) + lane * CPL;
   const float* vrows = mrows + RB * D;
   float q1[CPL], q2[CPL];
   lds_vec<CPL>(&sm.qsum[0][lane * CPL], q1);
@@ -421,9 +429,8 @@ __device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<
 #pragma unroll
   for (int b = 0; b < RB; ++b) {
     float m[CPL], v[CPL];
-    const int bl = min(b, nblk - 1);  // rows past the item: a copy of its last row (never stored)
-    lds_vec<CPL>(mrows + bl * D + lane * CPL, m);
-    lds_vec<CPL>(vrows + bl * D + lane * CPL, v);
+    lds_vec<CPL>(mrows + b * D, m);
+    lds_vec<CPL>(vrows + b * D, v);
     float acc = 0.f;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc += q1[c] * m[c] + q2[c] * v[c];
@@ -748,6 +755,17 @@ __device__ __forceinline__ bool aux_topk(const TopkSmem t, const float* src, boo
   return any_nan;
 }
 
+// The k-th largest (k <= 32) of the 32 lanes' values v, ties to the lower lane.
+__device__ __forceinline__ uint32_t kth_lane_max(uint32_t v, int lane, int k) {
+  int r = 0;
+#pragma unroll
+  for (int l = 0; l < 32; ++l) {
+    const uint32_t o = __shfl_sync(kFull, v, l);
+    r += (o > v || (o == v && l < lane)) ? 1 : 0;
+  }
+  return __shfl_sync(kFull, v, __ffs(__ballot_sync(kFull, r == k - 1)) - 1);
+}
+
 // The k <= 32 largest of the nb scores in shared memory (sc) by one warp, ties
 // to the lower index.  Lane l's keys are those of blocks l, l + 32, ...; at
 // least k lanes hold a key (nb > k), so the k-th largest of the 32 lane maxima,
@@ -764,40 +782,59 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
   const uint32_t lt = lanemask_lt();
   uint32_t lmax = 0u;
   bool nan = false;
-#pragma unroll 1
-  for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
-#pragma unroll
-    for (int i = 0; i < kRows; ++i) {
-      const int j = r0 + lane + 32 * i;
-      const float f = j < nb ? sc[j] : 0.f;
-      nan |= f != f;
-      if (j < nb) lmax = max(lmax, float_key(f));
-    }
-  }
-  nan_out = __any_sync(kFull, nan);
-  int r = 0;  // rank of this lane's maximum among the 32 (ties to the lower lane)
-#pragma unroll
-  for (int l = 0; l < 32; ++l) {
-    const uint32_t o = __shfl_sync(kFull, lmax, l);
-    r += (o > lmax || (o == lmax && l < lane)) ? 1 : 0;
-  }
-  const uint32_t tau = __shfl_sync(kFull, lmax, __ffs(__ballot_sync(kFull, r == k - 1)) - 1);
   int m = 0;  // candidates so far (block order)
-#pragma unroll 1
-  for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
-    uint32_t kr[kRows], bal[kRows];
+  if (nb <= 32 * kRows) {
+    // one pass, keys in registers, loads at fixed offsets (sc holds at least
+    // 32 kRows entries; entries past nb are read but not used)
+    uint32_t kr[kRows];
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
-      const int j = r0 + lane + 32 * i;
-      kr[i] = j < nb ? float_key(sc[j]) : 0u;
-      bal[i] = __ballot_sync(kFull, j < nb && kr[i] >= tau);
+      const float f = sc[lane + 32 * i];
+      const bool v = lane + 32 * i < nb;
+      nan |= v && f != f;
+      kr[i] = v ? float_key(f) : 0u;
+      lmax = max(lmax, kr[i]);
     }
+    nan_out = __any_sync(kFull, nan);
+    const uint32_t tau = kth_lane_max(lmax, lane, k);
+    uint32_t bal[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) bal[i] = __ballot_sync(kFull, lane + 32 * i < nb && kr[i] >= tau);
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
       const int pos = m + __popc(bal[i] & lt);
-      if (((bal[i] >> lane) & 1u) && pos < cap)
-        cand[pos] = ((unsigned long long)kr[i] << 32) | (uint32_t)~(r0 + lane + 32 * i);
+      if (((bal[i] >> lane) & 1u) && pos < cap) cand[pos] = ((unsigned long long)kr[i] << 32) | (uint32_t)~(lane + 32 * i);
       m += __popc(bal[i]);
+    }
+  } else {
+#pragma unroll 1
+    for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int j = r0 + lane + 32 * i;
+        const float f = j < nb ? sc[j] : 0.f;
+        nan |= f != f;
+        if (j < nb) lmax = max(lmax, float_key(f));
+      }
+    }
+    nan_out = __any_sync(kFull, nan);
+    const uint32_t tau = kth_lane_max(lmax, lane, k);
+#pragma unroll 1
+    for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
+      uint32_t kr[kRows], bal[kRows];
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int j = r0 + lane + 32 * i;
+        kr[i] = j < nb ? float_key(sc[j]) : 0u;
+        bal[i] = __ballot_sync(kFull, j < nb && kr[i] >= tau);
+      }
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int pos = m + __popc(bal[i] & lt);
+        if (((bal[i] >> lane) & 1u) && pos < cap)
+          cand[pos] = ((unsigned long long)kr[i] << 32) | (uint32_t)~(r0 + lane + 32 * i);
+        m += __popc(bal[i]);
+      }
     }
   }
   if (m > cap) return false;
@@ -943,9 +980,9 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
   // stage; a timed-out wait only stops this warp's work.
   bool dead = false;
   uint32_t par = 0u;  // bit s: parity of this group's next item in stage s
-  const int c0 = first_chunk_item(s);
 #pragma unroll 1
-  for (int it = c0; it < s.n; ++it) {
+  for (int c = 0; c < s.nW + s.nX; ++c) {
+    const int it = seq_of_chunk(s, c);
     const int stage = it % kFStages;
     const uint32_t ph = (par >> stage) & 1u;
     par ^= 1u << stage;
@@ -960,7 +997,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
         }
       }
     }
-    if (((it - c0) & 3) != warp) {
+    if ((c & 3) != warp) {
       if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
       continue;
     }
@@ -1118,9 +1155,9 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
 namespace hyb {
 namespace {
 
-// Statistics warps (roles 4-6): H items (rows split between the warps); score
-// items, one warp per item (item i to warp i % 3); hand the scores to every
-// rank; the selection; the rank's linear partial.  Every statistics warp waits for every
+// Statistics warps (roles 4-6): score items, one warp per item (item i to warp
+// i % 3); hand the scores to every rank; the selection; H items (rows split
+// between the warps); the rank's linear partial.  Every statistics warp waits for every
 // statistics item in ring order and arrives once on its stage's empty barrier
 // (the owner after its work), so that no warp falls two phases behind a stage.
 template <int D>
@@ -1165,25 +1202,14 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
       sm.vtok[c] = __bfloat162float(p.v_cache[row]);
     }
   named_sync(kBarAux, kAuxThreads);
-  float hacc[kMaxGroup][CPL];
-#pragma unroll
-  for (int i = 0; i < kMaxGroup; ++i)
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) hacc[i][c] = 0.f;
-#pragma unroll 1
-  for (int idx = 0; idx < s.nH; ++idx) {
-    const int it = seq_of_h(s, idx), stage = it % kFStages;
-    const bool have = wait_item(it);
-    if (have && (p.q != nullptr || nf > 0)) aux_h_item<D>(p, sm, s, unit, idx, stage, hacc);
-    __syncwarp();
-    if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
-  }
+  int fold_i0, fold_i1;
+  fold_items<D>(p, s, &fold_i0, &fold_i1);
 #pragma unroll 1
   for (int idx = 0; idx < s.nS; ++idx) {
     const int it = seq_of_s(s, idx), stage = it % kFStages;
     const bool have = wait_item(it);
     if (have && idx % kAuxWarps == aw) {
-      if (score_item_folds<D>(p, s, idx)) fold_score_item<D>(p, sm, s, unit, idx, stage);
+      if (idx >= fold_i0 && idx < fold_i1) fold_score_item<D>(p, sm, s, unit, idx, stage);
       if (p.q != nullptr) score_item_warp<D>(p, sm, s, unit, idx, stage);
       __syncwarp();
     }
@@ -1213,6 +1239,19 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
   }
 
   if (p.q != nullptr) aux_select<D>(p, sm, unit, rank);
+  float hacc[kMaxGroup][CPL];
+#pragma unroll
+  for (int i = 0; i < kMaxGroup; ++i)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) hacc[i][c] = 0.f;
+#pragma unroll 1
+  for (int idx = 0; idx < s.nH; ++idx) {
+    const int it = seq_of_h(s, idx), stage = it % kFStages;
+    const bool have = wait_item(it);
+    if (have && (p.q != nullptr || nf > 0)) aux_h_item<D>(p, sm, s, unit, idx, stage, hacc);
+    __syncwarp();
+    if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
+  }
   aux_finish_linear<D>(p, sm, unit, rank, hacc);
 }
 
@@ -1253,21 +1292,6 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
     ++issued;
     stage = stage + 1 == kFStages ? 0 : stage + 1;
   };
-  // H items: RH rows of H
-  const bool h_load = p.q != nullptr || p.fold_end > p.fold_begin;
-  for (int i = 0; i < s.nH && ok; ++i) {
-    if (!(ok = acquire())) break;
-    uint64_t* bar = &sm.full_aux[stage];
-    if (h_load) {
-      const int r0 = s.h0 + i * RH;
-      const uint32_t bytes = (uint32_t)(min(RH, s.h1 - r0) * D * 4);
-      mbar_arrive_expect_tx(bar, bytes);
-      bulk_load(smem_u32(sm.ring[stage]), p.H + ((int64_t)unit * D + r0) * D, bytes, bar);
-    } else {
-      mbar_arrive(bar);
-    }
-    advance(true);
-  }
   // score items: the mean and variance rows of RB blocks
   const int64_t brow = (int64_t)unit * p.max_blocks + s.b0;
   for (int i = 0; i < s.nS && ok; ++i) {
@@ -1299,6 +1323,21 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
     }
     issue_chunk<D>(tm, sm, stage, ubase, start, len, 0);
     advance(false);
+  }
+  // H items: RH rows of H
+  const bool h_load = p.q != nullptr || p.fold_end > p.fold_begin;
+  for (int i = 0; i < s.nH && ok; ++i) {
+    if (!(ok = acquire())) break;
+    uint64_t* bar = &sm.full_aux[stage];
+    if (h_load) {
+      const int r0 = s.h0 + i * RH;
+      const uint32_t bytes = (uint32_t)(min(RH, s.h1 - r0) * D * 4);
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_load(smem_u32(sm.ring[stage]), p.H + ((int64_t)unit * D + r0) * D, bytes, bar);
+    } else {
+      mbar_arrive(bar);
+    }
+    advance(true);
   }
   // selected chunks: chunk sc = rank + i C is piece sc % cpb of selection slot sc / cpb
   if (ok && s.nX > 0 && !mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit)) {
