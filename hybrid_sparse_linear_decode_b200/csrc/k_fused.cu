@@ -196,6 +196,13 @@ __device__ __forceinline__ uint32_t swz(int t, int C) {
   return (uint32_t)(L * 128 + (((C & 7) ^ (L & 7)) << 4));
 }
 
+// Transpose of an 8x8 matrix of 16-bit elements held in the warp (thread (g,
+// tig) holds row g, columns 2tig and 2tig+1).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   const float2 hf = __bfloat1622float2(h);
@@ -956,22 +963,27 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
   const int g = lane >> 2, tig = lane & 3;
   const bool p_lane = g < 4;  // rows 0-3: softmax part; rows 4-7: Taylor part
   const int head = g & 3;
-  const bool head_ok = head < p.G;
   const int mi = lane >> 3, rr = lane & 7;
 
-  uint32_t qa[KS][2];
+  // B fragments of Q^T for the S^T = K Q^T product: column n = lane group g is
+  // query head g (zero for g >= G)
+  uint32_t qb[KS][2];
   {
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (head_ok ? head : 0)) * D);
+    const bool real = g < p.G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (real ? g : 0)) * D);
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
-      qa[kk][0] = head_ok ? __ldg(qrow + kk * 8 + tig) : 0u;
-      qa[kk][1] = head_ok ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
+      qb[kk][0] = real ? __ldg(qrow + kk * 8 + tig) : 0u;
+      qb[kk][1] = real ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
     }
   }
   float O[NT8][4];
 #pragma unroll
   for (int n = 0; n < NT8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f, dsel_run = 0.f;
+  // lanes tig < 2: running max (log2 units) and weight sums of heads 2tig, 2tig+1;
+  // lanes tig >= 2: Taylor weight sums of heads 2tig-4, 2tig-3
+  const bool soft_lane = tig < 2;
+  float mr0 = -INFINITY, mr1 = -INFINITY, acc0 = 0.f, acc1 = 0.f;
 
   // Chunk items go to the attention warps in turn (chunk c to warp c % 4), each
   // warp taking all 64 tokens of its chunks.  Every attention warp waits for
@@ -1019,50 +1031,71 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
       }
-      // ---- S^T = Qpad K^T for the 64 tokens: n-tile nt holds tokens 8nt .. 8nt+7
-      float sacc[8][4];
+      // ---- S^T = K Q^T: m-tile mt holds tokens 16mt .. 16mt+15, columns = heads (4-7 zero)
+      float sacc[4][4];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      for (int mt = 0; mt < 4; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
 #pragma unroll
-        for (int tg = 0; tg < 4; ++tg) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + swz<D>(tg * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)), b0, b1, b2, b3);
-          mma_16816(sacc[2 * tg], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-          mma_16816(sacc[2 * tg + 1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+        for (int mt = 0; mt < 4; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kb + swz<D>(mt * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)), a0, a1, a2, a3);
+          mma_16816(sacc[mt], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
         }
       }
-      // ---- weights of this lane's 16 tokens: n-tile nt, element e -> token 8nt + 2tig + e
-      float sv[16], x[16];
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int nt = q >> 1, e = q & 1;
-        const bool v = (nt * 8 + 2 * tig + e) < nvalid;
-        sv[q] = v ? sacc[nt][e] * p.scale : 0.f;
-        x[q] = (p_lane && v) ? sv[q] * kLog2e : -INFINITY;
-        tmax = fmaxf(tmax, x[q]);
-      }
-      tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
-      tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
-      const float m_new = fmaxf(m_run, tmax);
-      const float alpha = (p_lane && m_new != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+      // lane (g, tig): tokens 16mt + g + 8j, columns 2tig, 2tig+1.  Lanes tig < 2 hold
+      // heads 2tig, 2tig+1 (softmax); lanes tig >= 2 take heads 2tig-4, 2tig-3 from
+      // lane ^ 2 (Taylor weights 1 + s on selected tokens).
       const bool sel_tok = dsc.z != 0;
-      float w[16], wsum = 0.f;
+      float w[4][4];
+      float t0m = -INFINITY, t1m = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int nt = q >> 1, e = q & 1;
-        const bool v = (nt * 8 + 2 * tig + e) < nvalid;
-        w[q] = p_lane ? (v ? exp2f(x[q] - m_new) : 0.f) : ((v && sel_tok) ? 1.f + sv[q] : 0.f);
-        wsum += w[q];
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = mt * 16 + g + 8 * (q >> 1);
+          const float sv = t < nvalid ? sacc[mt][q] * p.scale : 0.f;
+          const float spart = __shfl_xor_sync(kFull, sv, 2);
+          if (soft_lane) {
+            const float x = t < nvalid ? sv * kLog2e : -INFINITY;
+            w[mt][q] = x;
+            if (q & 1) t1m = fmaxf(t1m, x); else t0m = fmaxf(t0m, x);
+          } else {
+            w[mt][q] = (t < nvalid && sel_tok) ? 1.f + spart : 0.f;
+          }
+        }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        t0m = fmaxf(t0m, __shfl_xor_sync(kFull, t0m, o));
+        t1m = fmaxf(t1m, __shfl_xor_sync(kFull, t1m, o));
       }
-      if (p_lane) {
-        l_run = l_run * alpha + wsum;
-        m_run = m_new;
+      const float mn0 = fmaxf(mr0, t0m), mn1 = fmaxf(mr1, t1m);
+      const float al0 = (soft_lane && mn0 != -INFINITY) ? exp2f(mr0 - mn0) : 1.f;
+      const float al1 = (soft_lane && mn1 != -INFINITY) ? exp2f(mr1 - mn1) : 1.f;
+      float ws0 = 0.f, ws1 = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (soft_lane) {
+            const float mn = (q & 1) ? mn1 : mn0;
+            w[mt][q] = w[mt][q] == -INFINITY ? 0.f : exp2f(w[mt][q] - mn);
+          }
+          if (q & 1) ws1 += w[mt][q]; else ws0 += w[mt][q];
+        }
+      if (soft_lane) {
+        acc0 = acc0 * al0 + ws0;
+        acc1 = acc1 * al1 + ws1;
+        mr0 = mn0;
+        mr1 = mn1;
       } else {
-        dsel_run += wsum;
+        acc0 += ws0;
+        acc1 += ws1;
       }
+      // rescale the softmax rows (g < 4) of O by their head's factor
+      const float b0 = __shfl_sync(kFull, al0, g >> 1), b1 = __shfl_sync(kFull, al1, g >> 1);
+      const float alpha = p_lane ? ((g & 1) ? b1 : b0) : 1.f;
       if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
         for (int n = 0; n < NT8; ++n) {
@@ -1072,18 +1105,19 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
           O[n][3] *= alpha;
         }
       }
-      // ---- O += A V, k-step kt over tokens 16kt .. 16kt+15 (rows g: bf16 hi, g+8: lo)
+      // ---- O += A V: A rows = weight columns (transposed 8x8 blocks), hi then lo
 #pragma unroll
       for (int kt = 0; kt < 4; ++kt) {
-        uint32_t a0, a1, a2, a3;
-        split_bf16(w[4 * kt + 0], w[4 * kt + 1], a0, a1);
-        split_bf16(w[4 * kt + 2], w[4 * kt + 3], a2, a3);
+        uint32_t h0, l0, h1, l1;
+        split_bf16(w[kt][0], w[kt][1], h0, l0);
+        split_bf16(w[kt][2], w[kt][3], h1, l1);
+        const uint32_t a0 = movmatrix_t(h0), a1 = movmatrix_t(l0), a2 = movmatrix_t(h1), a3 = movmatrix_t(l1);
 #pragma unroll
         for (int np = 0; np < NT8 / 2; ++np) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, np * 2 + (mi >> 1)), b0, b1, b2, b3);
-          mma_16816(O[2 * np], a0, a1, a2, a3, b0, b1);
-          mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2, b3);
+          uint32_t b0v, b1v, b2v, b3v;
+          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, np * 2 + (mi >> 1)), b0v, b1v, b2v, b3v);
+          mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
+          mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
         }
       }
     }
@@ -1096,10 +1130,23 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
   if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit);
   // ---- combine the 4 warps' partials (a tree through two shared slots: warps
   //      2, 3 -> 0, 1, then warp 1 -> 0); warp 0 leaves the record in wpart[0]
-  float l = l_run + __shfl_xor_sync(kFull, l_run, 1);
-  l += __shfl_xor_sync(kFull, l, 2);
-  float ds = dsel_run + __shfl_xor_sync(kFull, dsel_run, 1);
-  ds += __shfl_xor_sync(kFull, ds, 2);
+  // per-head totals over the tokens (the lanes of one tig), then each lane takes
+  // the statistics of its O rows' head (rows g < 4 softmax, g >= 4 Taylor)
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    acc0 += __shfl_xor_sync(kFull, acc0, o);
+    acc1 += __shfl_xor_sync(kFull, acc1, o);
+  }
+  float m_run, l, ds;
+  {
+    const int src = p_lane ? (head >> 1) : 2 + (head >> 1);
+    const float v0 = __shfl_sync(kFull, acc0, src), v1 = __shfl_sync(kFull, acc1, src);
+    const float m0 = __shfl_sync(kFull, mr0, head >> 1), m1 = __shfl_sync(kFull, mr1, head >> 1);
+    const float v = (head & 1) ? v1 : v0;
+    m_run = (head & 1) ? m1 : m0;
+    l = p_lane ? v : 0.f;
+    ds = p_lane ? 0.f : v;
+  }
   const int voff = (p_lane ? 0 : 4 * D) + head * D;
   auto emit = [&](float* wp) {  // write this warp's partial (hi + lo rows summed)
     if (tig == 0) {
