@@ -36,8 +36,9 @@
 //
 // Linear term (SLAKE, first-order Taylor exp(s) ~ 1 + s; SPLA residual
 // attention): N_glob_i = zv + H^T q'_i, D_glob_i = n + q'_i . zk, each rank
-// summing its rows of H.  Merge, by rank 0 over distributed shared memory
-// after a cluster barrier (per query head, base-2 exponent m of the exact part):
+// summing its rows of H.  Merge, each rank a slice of the outputs, over
+// distributed shared memory after a cluster barrier (per query head, base-2
+// exponent m of the exact part):
 //   o = (N_ex + 2^{-m} (N_glob - N_sel)) / (D_ex + 2^{-m} (D_glob - D_sel)),
 // as the equal form (N_ex 2^m + ...)/(D_ex 2^m + ...) when m < 0.
 //
@@ -384,7 +385,11 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
 #pragma unroll 1
     for (int64_t t = t0; t < t1; ++t) {
       float x[CPL];
-      load_bf16<CPL>(p.k_cache + ((int64_t)unit * p.cap + t) * D + lane * CPL, x);
+      if (p.fold_end - p.fold_begin == 1) {
+        lds_vec<CPL>(&sm.ktok[lane * CPL], x);  // staged at the start of the statistics role
+      } else {
+        load_bf16<CPL>(p.k_cache + ((int64_t)unit * p.cap + t) * D + lane * CPL, x);
+      }
       const float cnt = (float)(t - bs + 1);
       const float inv = 1.f / cnt;
 #pragma unroll
@@ -402,11 +407,12 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
     }
     sts_vec<CPL>(mrows + bl * D + lane * CPL, m);
     sts_vec<CPL>(vrows + bl * D + lane * CPL, v);
+    // the stage is rewritten by bulk copies (the async proxy) later; fenced
+    // before the global stores below so that the fence does not wait for them
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     sts_vec<CPL>(p.mu + ((int64_t)unit * p.max_blocks + j) * D + lane * CPL, m);
     sts_vec<CPL>(p.var + ((int64_t)unit * p.max_blocks + j) * D + lane * CPL, v);
   }
-  // the stage is rewritten by bulk copies (the async proxy) later
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
 }
 
@@ -965,12 +971,13 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
   const int head = g & 3;
   const int mi = lane >> 3, rr = lane & 7;
 
-  // B fragments of Q^T for the S^T = K Q^T product: column n = lane group g is
-  // query head g (zero for g >= G)
+  // B fragments of Q^T for the S^T = K Q^T product: columns n and n + 4 (lane
+  // groups g and g + 4) are query head n (zero for n >= G), so that the lanes
+  // building the Taylor weights hold their heads' scores themselves
   uint32_t qb[KS][2];
   {
-    const bool real = g < p.G;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (real ? g : 0)) * D);
+    const bool real = (g & 3) < p.G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + ((int64_t)unit * p.G + (real ? (g & 3) : 0)) * D);
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       qb[kk][0] = real ? __ldg(qrow + kk * 8 + tig) : 0u;
@@ -1044,9 +1051,9 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
           mma_16816(sacc[mt], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
         }
       }
-      // lane (g, tig): tokens 16mt + g + 8j, columns 2tig, 2tig+1.  Lanes tig < 2 hold
-      // heads 2tig, 2tig+1 (softmax); lanes tig >= 2 take heads 2tig-4, 2tig-3 from
-      // lane ^ 2 (Taylor weights 1 + s on selected tokens).
+      // lane (g, tig): tokens 16mt + g + 8j, columns 2tig, 2tig+1, i.e. heads
+      // (2tig, 2tig+1) & 3: softmax weights in lanes tig < 2, Taylor weights
+      // 1 + s on selected tokens in lanes tig >= 2.
       const bool sel_tok = dsc.z != 0;
       float w[4][4];
       float t0m = -INFINITY, t1m = -INFINITY;
@@ -1056,13 +1063,12 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
         for (int q = 0; q < 4; ++q) {
           const int t = mt * 16 + g + 8 * (q >> 1);
           const float sv = t < nvalid ? sacc[mt][q] * p.scale : 0.f;
-          const float spart = __shfl_xor_sync(kFull, sv, 2);
           if (soft_lane) {
             const float x = t < nvalid ? sv * kLog2e : -INFINITY;
             w[mt][q] = x;
             if (q & 1) t1m = fmaxf(t1m, x); else t0m = fmaxf(t0m, x);
           } else {
-            w[mt][q] = (t < nvalid && sel_tok) ? 1.f + spart : 0.f;
+            w[mt][q] = (t < nvalid && sel_tok) ? 1.f + sv : 0.f;
           }
         }
 #pragma unroll
@@ -1428,10 +1434,11 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
   }
 }
 
-// Rank 0, all threads, after the first cluster barrier: merge the C records and
-// linear partials (read over distributed shared memory) and write the output.
+// Every rank, all threads, after the first cluster barrier: merge the C records
+// and linear partials (read over distributed shared memory) for this rank's
+// slice of the unit's G x D outputs and write them.
 template <int D>
-__device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit) {
+__device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
   constexpr int PF = FusedSmem<D>::kPF;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G, C = p.C;
@@ -1469,7 +1476,8 @@ __device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit) 
   }
   __syncthreads();
   uint32_t flags = 0u;
-  for (int e = tid; e < G * D; e += kFThreads) {
+  const int e0 = (int)((int64_t)rank * G * D / C), e1 = (int)((int64_t)(rank + 1) * G * D / C);
+  for (int e = e0 + tid; e < e1; e += kFThreads) {
     const int i = e / D, d = e % D;
     float xa[kMaxCluster], xs[kMaxCluster], xl[kMaxCluster];  // every remote load in flight first
 #pragma unroll
@@ -1491,7 +1499,7 @@ __device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit) 
       }
     }
     const float Ms = hm[i], Dex = hm[4 + i], Dsel = hm[8 + i];
-    const float Dg = sm.linp[i][D];  // rank 0 holds D_glob
+    const float Dg = ld_cluster_f32(map_rank(smem_u32(&sm.linp[i][D]), 0u));  // rank 0 holds D_glob
     float num, den;
     if (Ms >= 0.f) {
       const float f = exp2f(-Ms);
@@ -1579,8 +1587,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     }
   }
   cluster_sync_all();  // every rank's record and linear partial are final
-  if (rank == 0 && p.q != nullptr) merge_cluster<D>(p, sm, unit);
-  cluster_sync_all();  // the records stay readable until rank 0 is done
+  if (p.q != nullptr) merge_cluster<D>(p, sm, unit, rank);
+  cluster_sync_all();  // the records stay readable until every rank is done
 }
 
 }  // namespace
