@@ -358,10 +358,13 @@ __device__ __forceinline__ void sts_vec(float* dst, const float (&f)[CPL]) {
   }
 }
 
-// Fold the pending evictions into the statistics rows of score item `idx`, in
-// place in its ring stage, and write them back: Welford's running mean and
-// population variance, one token at a time.  One warp, lane l holding channels
-// [l*CPL, l*CPL + CPL) of each block that has pending tokens (usually one).
+// Fold the pending evictions into the statistics rows of score item `idx` and
+// write the rows back: Welford's running mean and population variance, one
+// token at a time.  One warp, lane l holding channels [l*CPL, l*CPL + CPL) of
+// each block that has pending tokens (usually one).  The ring stage keeps the
+// old rows (writing it would need a proxy fence against the copies in flight):
+// the block's score is recomputed here from the folded rows and replaces the
+// one score_item_warp stored from the old rows.
 template <int D>
 __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx,
                                                 int stage) {
@@ -370,10 +373,13 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
   const int lane = role_tid() & 31;
   const int j0 = s.b0 + idx * RB;
   const int nblk = min(RB, s.b1 - j0);
-  float* mrows = reinterpret_cast<float*>(sm.ring[stage]);
-  float* vrows = mrows + RB * D;
-  const int64_t jb0 = (p.fold_begin - p.S) / p.Bk, jb1 = (p.fold_end - 1 - p.S) / p.Bk;
-  const int bl0 = (int)max((int64_t)0, jb0 - j0), bl1 = (int)min((int64_t)nblk - 1, jb1 - j0);
+  const float* mrows = reinterpret_cast<const float*>(sm.ring[stage]);
+  const float* vrows = mrows + RB * D;
+  const int jb0 = (int)(p.fold_begin - p.S) / p.Bk, jb1 = (int)(p.fold_end - 1 - p.S) / p.Bk;
+  const int bl0 = max(0, jb0 - j0), bl1 = min(nblk - 1, jb1 - j0);
+  float q1[CPL], q2[CPL];
+  lds_vec<CPL>(&sm.qsum[0][lane * CPL], q1);
+  lds_vec<CPL>(&sm.qsum[1][lane * CPL], q2);
 #pragma unroll 1
   for (int bl = bl0; bl <= bl1; ++bl) {
     const int j = j0 + bl;
@@ -405,13 +411,20 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
         }
       }
     }
-    sts_vec<CPL>(mrows + bl * D + lane * CPL, m);
-    sts_vec<CPL>(vrows + bl * D + lane * CPL, v);
-    // the stage is rewritten by bulk copies (the async proxy) later; fenced
-    // before the global stores below so that the fence does not wait for them
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     sts_vec<CPL>(p.mu + ((int64_t)unit * p.max_blocks + j) * D + lane * CPL, m);
     sts_vec<CPL>(p.var + ((int64_t)unit * p.max_blocks + j) * D + lane * CPL, v);
+    if (p.q != nullptr) {
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc += q1[c] * m[c] + q2[c] * v[c];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+      __syncwarp();  // after score_item_warp's stores of the old score
+      if (lane == 0) {
+        p.scores[(int64_t)unit * p.max_blocks + j] = acc;
+        if (p.nb <= FusedSmem<D>::kGather) sm.scores[j] = acc;
+      }
+    }
   }
   __syncwarp();
 }
@@ -1027,7 +1040,8 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
       const uint32_t vb = kb + FusedSmem<D>::kHalf;
       if (nvalid < kTile) {
         // rows past the chunk may hold tokens beyond T (unwritten cache rows):
-        // zero their V rows so that 0-weight * garbage cannot make a NaN
+        // zero their V rows so that 0-weight * garbage cannot make a NaN (only
+        // the few ragged chunks of a launch pay for the proxy fence)
         constexpr int CPR = D / 8;  // 16-byte chunks per row
         uint8_t* vt = sm.ring[stage] + FusedSmem<D>::kHalf;
         for (int e = lane; e < (kTile - nvalid) * CPR; e += 32) {
@@ -1038,7 +1052,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
       }
-      // ---- S^T = K Q^T: m-tile mt holds tokens 16mt .. 16mt+15, columns = heads (4-7 zero)
+      // ---- S^T = K Q^T: m-tile mt holds tokens 16mt .. 16mt+15, columns = heads
       float sacc[4][4];
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
@@ -1262,8 +1276,8 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
     const int it = seq_of_s(s, idx), stage = it % kFStages;
     const bool have = wait_item(it);
     if (have && idx % kAuxWarps == aw) {
-      if (idx >= fold_i0 && idx < fold_i1) fold_score_item<D>(p, sm, s, unit, idx, stage);
       if (p.q != nullptr) score_item_warp<D>(p, sm, s, unit, idx, stage);
+      if (idx >= fold_i0 && idx < fold_i1) fold_score_item<D>(p, sm, s, unit, idx, stage);
       __syncwarp();
     }
     if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
