@@ -15,15 +15,16 @@
 // the copies (TMA tensor loads for K/V chunks, untiled bulk copies for the
 // statistics and H, no multicast); the other warps consume them.
 //
-// Warp roles (8 warps; role r runs on hardware warp given by role_tid):
-//   0-3  attention: chunk c to warp c % 4, all 64 tokens, on the tensor cores
+// Warp roles (12 warps; role r runs on hardware warp given by role_tid):
+//   0-7  attention, in pairs: chunk c to pair c % 4, all 64 tokens for the scores,
+//        one half of the head dimension per warp for PV, on the tensor cores
 //        (mma.sync m16n8k16, bf16 in, fp32 accumulate), G <= 4 query heads
 //        packed into the 16-row M dimension (rows 0-3 softmax, rows 4-7 the
 //        Taylor weights 1 + s of selected-block tokens, rows 8-15 the bf16
 //        rounding remainders of rows 0-7);
-//   4-6  statistics: block scores (score item i to warp i % 3), the Welford
+//   8-10 statistics: block scores (score item i to warp i % 3), the Welford
 //        fold, the top-k (one warp), H rows, the linear term;
-//   7    producer: lane 0 issues every copy in ring order.
+//   11   producer: lane 0 issues every copy in ring order.
 //
 // Block score ("SPLA: Block Sparse Plus Linear Attention for Long Context
 // Modeling", Abstract; "Principled Block Selection via Taylor Expansion";
@@ -60,17 +61,20 @@ namespace hyb {
 namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
-constexpr int kFThreads = 256;
+constexpr int kFThreads = 384;
 constexpr int kFStages = 6;
 constexpr int kFScoresMax = 2048;   // scores a CTA keeps for its unit (else they go through global memory)
 static_assert(kFScoresMax >= 512, "the one-warp top-k reads 512 entries unconditionally");
-constexpr int kAuxWarps = 3;        // statistics warps: roles 4-6
+constexpr int kAttnWarps = 8;       // attention warps: roles 0-7 (4 pairs)
+constexpr int kAttnThreads = 32 * kAttnWarps;
+constexpr int kAuxWarps = 3;        // statistics warps: roles 8-10
 constexpr int kAuxThreads = 32 * kAuxWarps;
-constexpr int kConsumerThreads = 128 + kAuxThreads;  // attention + statistics (roles 0-6)
+constexpr int kConsumerThreads = kAttnThreads + kAuxThreads;  // roles 0-10
+constexpr int kProducerWarp = kAttnWarps + kAuxWarps;         // role 11
 // every item's empty-barrier phase takes kEmptyCount arrivals: kEmptyPerAuxWarp
 // from each statistics warp, or kEmptyPerAttnWarp from each attention warp
-constexpr int kEmptyCount = 12, kEmptyPerAuxWarp = 4, kEmptyPerAttnWarp = 3;
-constexpr int kBarAttn = 1, kBarAux = 2, kBarConsumers = 3;   // named barriers
+constexpr int kEmptyCount = 24, kEmptyPerAuxWarp = 8, kEmptyPerAttnWarp = 3;
+constexpr int kBarAttn = 1, kBarAux = 2, kBarConsumers = 3, kBarPair0 = 4;   // named barriers
 
 // ---------------------------------------------------------------- cluster helpers
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -130,9 +134,10 @@ __device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t b
                : "memory");
 }
 // This thread's index in role order: role r is hardware warp r.  Warp w runs on
-// sub-partition w % 4, so each statistics warp (4-6) and the producer (7) shares
-// a sub-partition with one attention warp (0-3); the attention warps idle while
-// the score items stream, which is when the statistics warps are busiest.
+// sub-partition w % 4: each sub-partition runs two attention warps (0-7; the two
+// warps of a pair on different sub-partitions) and one statistics warp (8-10)
+// or the producer (11); the attention warps idle while the score items stream,
+// which is when the statistics warps are busiest.
 __device__ __forceinline__ int role_tid() { return (int)threadIdx.x; }
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -487,7 +492,7 @@ __device__ __forceinline__ void h_rows(const FusedParams& p, FusedSmem<D>& sm, i
                                        const float* hrows, float (&hacc)[kMaxGroup][D / 32]) {
   constexpr int CPL = D / 32;
   static_assert(kMaxGroup == 4, "qsT rows are one float4");
-  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
   const int64_t ub = (int64_t)unit * p.cap;
   float v1[CPL];
   if (kFold == 1) lds_vec<CPL>(&sm.vtok[lane * CPL], v1);
@@ -544,7 +549,7 @@ template <int D>
 __device__ void aux_finish_linear(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank,
                                   const float (&hacc)[kMaxGroup][D / 32]) {
   constexpr int CPL = D / 32;
-  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
   if (p.q != nullptr) {
 #pragma unroll
     for (int i = 0; i < kMaxGroup; ++i)
@@ -622,7 +627,7 @@ namespace {
 // Exclusive prefix sum of v over the statistics threads (named barrier 2);
 // returns the sum over threads before this one, and the total in *total.
 __device__ __forceinline__ uint32_t aux_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
-  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
   uint32_t incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -660,7 +665,7 @@ __device__ __forceinline__ uint32_t score_key(const float* src, bool glob, int j
 // (and copy[0, k)).  Returns (in every thread) whether a score was NaN.
 __device__ __forceinline__ bool aux_topk(const TopkSmem t, const float* src, bool glob, int nb, int k, int32_t* dst,
                                       int32_t* copy) {
-  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
   uint32_t kmin = 0xffffffffu, kmax = 0u, nan = 0u;
 #pragma unroll 1
   for (int j = a; j < nb; j += kAuxThreads) {
@@ -901,7 +906,7 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
 // rank's share is in place.  Rank 0 fills the caller's copy.
 template <int D>
 __device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
-  const int a = role_tid() - 128;
+  const int a = role_tid() - kAttnThreads;
   int32_t* copy = (p.sel_out != nullptr && rank == 0) ? p.sel_out + (int64_t)unit * p.top_k : nullptr;
   int state = 3;
   const int32_t* row = nullptr;
@@ -977,8 +982,10 @@ namespace {
 template <int D>
 __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit) {
   constexpr int NT8 = D / 8;  // 8-column tiles of the head dimension
+  constexpr int NH = NT8 / 2;  // the tiles of this warp's half of the columns
   constexpr int KS = D / 16;  // k-steps of the QK product
   const int tid = role_tid(), warp = tid >> 5, lane = tid & 31;
+  const int pair = warp >> 1, half = warp & 1;  // chunk c to pair c % 4; PV columns [half D/2, half D/2 + D/2)
   const int g = lane >> 2, tig = lane & 3;
   const bool p_lane = g < 4;  // rows 0-3: softmax part; rows 4-7: Taylor part
   const int head = g & 3;
@@ -997,16 +1004,17 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
       qb[kk][1] = real ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
     }
   }
-  float O[NT8][4];
+  float O[NH][4];
 #pragma unroll
-  for (int n = 0; n < NT8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+  for (int n = 0; n < NH; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
   // lanes tig < 2: running max (log2 units) and weight sums of heads 2tig, 2tig+1;
   // lanes tig >= 2: Taylor weight sums of heads 2tig-4, 2tig-3
   const bool soft_lane = tig < 2;
   float mr0 = -INFINITY, mr1 = -INFINITY, acc0 = 0.f, acc1 = 0.f;
 
-  // Chunk items go to the attention warps in turn (chunk c to warp c % 4), each
-  // warp taking all 64 tokens of its chunks.  Every attention warp waits for
+  // Chunk items go to the attention warp pairs in turn (chunk c to pair c % 4):
+  // both warps of the pair compute the chunk's scores and weights, each the
+  // PV product for half of the head dimension.  Every attention warp waits for
   // every chunk item in ring order and arrives on its stage's empty barrier
   // (the owner after its work), so that no warp falls two phases behind a
   // stage; a timed-out wait only stops this warp's work.
@@ -1029,7 +1037,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
         }
       }
     }
-    if ((c & 3) != warp) {
+    if ((c & 3) != pair) {
       if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
       continue;
     }
@@ -1076,14 +1084,14 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int t = mt * 16 + g + 8 * (q >> 1);
+          // both kinds of lanes take the same instructions (selects, no
+          // divergent branch: half the warp takes each kind)
           const float sv = t < nvalid ? sacc[mt][q] * p.scale : 0.f;
-          if (soft_lane) {
-            const float x = t < nvalid ? sv * kLog2e : -INFINITY;
-            w[mt][q] = x;
-            if (q & 1) t1m = fmaxf(t1m, x); else t0m = fmaxf(t0m, x);
-          } else {
-            w[mt][q] = (t < nvalid && sel_tok) ? 1.f + sv : 0.f;
-          }
+          const float xs = t < nvalid ? sv * kLog2e : -INFINITY;
+          const float wt = (t < nvalid && sel_tok) ? 1.f + sv : 0.f;
+          w[mt][q] = soft_lane ? xs : wt;
+          const float xm = soft_lane ? xs : -INFINITY;
+          if (q & 1) t1m = fmaxf(t1m, xm); else t0m = fmaxf(t0m, xm);
         }
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
@@ -1098,27 +1106,20 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
       for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          if (soft_lane) {
-            const float mn = (q & 1) ? mn1 : mn0;
-            w[mt][q] = w[mt][q] == -INFINITY ? 0.f : exp2f(w[mt][q] - mn);
-          }
+          const float ev = exp2f(w[mt][q] - ((q & 1) ? mn1 : mn0));  // used in the softmax lanes only
+          w[mt][q] = soft_lane ? (w[mt][q] == -INFINITY ? 0.f : ev) : w[mt][q];
           if (q & 1) ws1 += w[mt][q]; else ws0 += w[mt][q];
         }
-      if (soft_lane) {
-        acc0 = acc0 * al0 + ws0;
-        acc1 = acc1 * al1 + ws1;
-        mr0 = mn0;
-        mr1 = mn1;
-      } else {
-        acc0 += ws0;
-        acc1 += ws1;
-      }
+      acc0 = acc0 * al0 + ws0;  // al = 1 in the Taylor lanes
+      acc1 = acc1 * al1 + ws1;
+      mr0 = soft_lane ? mn0 : mr0;
+      mr1 = soft_lane ? mn1 : mr1;
       // rescale the softmax rows (g < 4) of O by their head's factor
       const float b0 = __shfl_sync(kFull, al0, g >> 1), b1 = __shfl_sync(kFull, al1, g >> 1);
       const float alpha = p_lane ? ((g & 1) ? b1 : b0) : 1.f;
       if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
-        for (int n = 0; n < NT8; ++n) {
+        for (int n = 0; n < NH; ++n) {
           O[n][0] *= alpha;
           O[n][1] *= alpha;
           O[n][2] *= alpha;
@@ -1133,9 +1134,10 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
         split_bf16(w[kt][2], w[kt][3], h1, l1);
         const uint32_t a0 = movmatrix_t(h0), a1 = movmatrix_t(l0), a2 = movmatrix_t(h1), a3 = movmatrix_t(l1);
 #pragma unroll
-        for (int np = 0; np < NT8 / 2; ++np) {
+        for (int np = 0; np < NH / 2; ++np) {
           uint32_t b0v, b1v, b2v, b3v;
-          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, np * 2 + (mi >> 1)), b0v, b1v, b2v, b3v);
+          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, (half * NH / 2 + np) * 2 + (mi >> 1)), b0v, b1v, b2v,
+                    b3v);
           mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
           mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
         }
@@ -1148,8 +1150,9 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
   // the combine slots hold the top-k candidates until the selection is made
   // (a rank without selected chunks gets here first)
   if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit);
-  // ---- combine the 4 warps' partials (a tree through two shared slots: warps
-  //      2, 3 -> 0, 1, then warp 1 -> 0); warp 0 leaves the record in wpart[0]
+  // ---- combine the 4 pairs' partials (a tree through two shared slots: pairs
+  //      2, 3 -> 0, 1, then pair 1 -> 0); pair 0 leaves the record in wpart[0].
+  //      The two warps of a pair hold the same statistics and disjoint columns.
   // per-head totals over the tokens (the lanes of one tig), then each lane takes
   // the statistics of its O rows' head (rows g < 4 softmax, g >= 4 Taylor)
 #pragma unroll
@@ -1167,9 +1170,9 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
     l = p_lane ? v : 0.f;
     ds = p_lane ? 0.f : v;
   }
-  const int voff = (p_lane ? 0 : 4 * D) + head * D;
+  const int voff = (p_lane ? 0 : 4 * D) + head * D + half * (D / 2);
   auto emit = [&](float* wp) {  // write this warp's partial (hi + lo rows summed)
-    if (tig == 0) {
+    if (tig == 0 && half == 0) {
       if (p_lane) {
         wp[head] = m_run;
         wp[4 + head] = l;
@@ -1179,7 +1182,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
     }
     float* dst = wp + 16 + voff;
 #pragma unroll
-    for (int n = 0; n < NT8; ++n)
+    for (int n = 0; n < NH; ++n)
       *reinterpret_cast<float2*>(dst + n * 8 + 2 * tig) = make_float2(O[n][0] + O[n][2], O[n][1] + O[n][3]);
   };
   auto absorb = [&](const float* wp) {  // fold another warp's partial into this one
@@ -1196,22 +1199,22 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
     }
     const float* src = wp + 16 + voff;
 #pragma unroll
-    for (int n = 0; n < NT8; ++n) {
+    for (int n = 0; n < NH; ++n) {
       const float2 y = *reinterpret_cast<const float2*>(src + n * 8 + 2 * tig);
       O[n][0] = (O[n][0] + O[n][2]) * fa + y.x * fb;
       O[n][1] = (O[n][1] + O[n][3]) * fa + y.y * fb;
       O[n][2] = O[n][3] = 0.f;
     }
   };
-  if (warp >= 2) emit(sm.wpart[warp - 2]);
-  named_sync(kBarAttn, 128);
-  if (warp < 2) absorb(sm.wpart[warp]);
-  named_sync(kBarAttn, 128);
-  if (warp == 1) emit(sm.wpart[0]);
-  named_sync(kBarAttn, 128);
-  if (warp == 0) {
+  if (pair >= 2) emit(sm.wpart[pair - 2]);
+  named_sync(kBarAttn, kAttnThreads);
+  if (pair < 2) absorb(sm.wpart[pair]);
+  named_sync(kBarAttn, kAttnThreads);
+  if (pair == 1) emit(sm.wpart[0]);
+  named_sync(kBarAttn, kAttnThreads);
+  if (pair == 0) {
     absorb(sm.wpart[0]);
-    __syncwarp();
+    named_sync(kBarPair0, 64);  // both warps have read the statistics before half 0 rewrites them
     emit(sm.wpart[0]);
   }
 }
@@ -1222,7 +1225,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
 namespace hyb {
 namespace {
 
-// Statistics warps (roles 4-6): score items, one warp per item (item i to warp
+// Statistics warps (roles 8-10): score items, one warp per item (item i to warp
 // i % 3); hand the scores to every rank; the selection; H items (rows split
 // between the warps); the rank's linear partial.  Every statistics warp waits for every
 // statistics item in ring order and arrives once on its stage's empty barrier
@@ -1230,7 +1233,7 @@ namespace {
 template <int D>
 __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int rank) {
   constexpr int CPL = D / 32;
-  const int a = role_tid() - 128, aw = a >> 5, lane = a & 31;
+  const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
   // a timed-out wait only stops this warp's work; it keeps visiting every item
   // and barrier
   bool dead = false;
@@ -1322,7 +1325,7 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
   aux_finish_linear<D>(p, sm, unit, rank, hacc);
 }
 
-// Producer (role warp 7, lane 0): every copy of the rank, in ring order, one
+// Producer (role warp 11, lane 0): every copy of the rank, in ring order, one
 // short loop per kind of item with running addresses.  Before an item goes into
 // a stage that held an earlier item, the stage's empty barrier must have
 // completed for that earlier item.
@@ -1575,7 +1578,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
   // the barriers of every rank are initialised before any remote arrival
   cluster_sync_all();
   pdl_allow_dependents();
-  if (warp == 7) {
+  if (warp == kProducerWarp) {
     // the producer starts at once: it needs nothing from the lines below
     producer_role<D>(&tm, p, sm, s, unit, rank);
   } else {
@@ -1594,7 +1597,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
       *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
     }
     named_sync(kBarConsumers, kConsumerThreads);
-    if (warp < 4) {
+    if (warp < kAttnWarps) {
       if (p.q != nullptr) attn_role<D>(p, sm, s, unit);
     } else {
       aux_role<D>(p, sm, s, unit, rank);
