@@ -239,6 +239,8 @@ FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   fp.units = k.units;
   fp.G = k.G;
   fp.C = cluster_ctas(k.units, x->n_sm, x->fits);
+  fp.mstride = merge_stride(k.G * k.D, fp.C);
+  for (int r = 0; r <= fp.C; ++r) fp.mslice[r] = merge_slice_begin(k.G * k.D, fp.C, r);
   fp.scale = x->scale;
   return fp;
 }

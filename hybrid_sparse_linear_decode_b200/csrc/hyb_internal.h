@@ -20,6 +20,21 @@ constexpr uint64_t kWaitLimit = 1000000000ull;  // ns: a kernel-internal wait gi
 // Per-slot layout of a split-K partial: m[4], l[4], dsel[4], pad[4], acc[4][D], nsel[4][D].
 __host__ __device__ constexpr int partial_floats(int D) { return 16 + 8 * D; }
 
+// Merge of a unit's outputs across its C CTAs: rank r merges outputs
+// [e0(r), e1(r)) of the unit's G x D (e0(r) = r G D / C, rounded down).  Its
+// receiving buffer holds one slot per sending rank: a header of 12 floats (per
+// head: the exact part's running max and weight sum, and D_glob - D_sel;
+// padded to 16) and a (exact part, N_glob - N_sel) pair per output of the slice.
+__host__ __device__ constexpr int merge_slice_begin(int GD, int C, int r) { return r * GD / C; }
+__host__ __device__ constexpr int merge_stride(int GD, int C) { return 16 + ((2 * ((GD + C - 1) / C) + 3) & ~3); }
+__host__ __device__ constexpr int merge_floats_for(int D, int C) { return C * merge_stride(kMaxGroup * D, C); }
+// the largest buffer over every cluster size
+__host__ __device__ constexpr int merge_floats(int D, int C = 1) {
+  return C > kMaxCluster ? 0
+                         : (merge_floats_for(D, C) > merge_floats(D, C + 1) ? merge_floats_for(D, C)
+                                                                               : merge_floats(D, C + 1));
+}
+
 struct Geometry {        // everything a decode at length T needs, computed on the host
   int64_t T;
   int64_t nb;            // candidate blocks
@@ -54,6 +69,8 @@ struct FusedParams {           // one decode (or, with q == null, the fold only)
   int32_t sink_len, win_start, ev_end;
   int32_t n_sink_chunks, n_win_chunks, chunks_per_block, n_sel_chunks;
   int32_t units, G, C;          // C: CTAs (cluster size) per unit
+  int32_t mstride;              // merge: floats per sending rank's slot (merge_stride)
+  int32_t mslice[kMaxCluster + 1];  // merge: rank r merges outputs [mslice[r], mslice[r + 1])
   float scale;
 };
 

@@ -70,9 +70,12 @@ constexpr int kAttnThreads = 32 * kAttnWarps;
 constexpr int kAuxWarps = 3;        // statistics warps: roles 8-10
 constexpr int kAuxThreads = 32 * kAuxWarps;
 constexpr int kConsumerThreads = kAttnThreads + kAuxThreads;  // roles 0-10
+static_assert(kConsumerThreads >= 2 * 128, "one thread per channel of the pending K and V rows");
 constexpr int kProducerWarp = kAttnWarps + kAuxWarps;         // role 11
 // every item's empty-barrier phase takes kEmptyCount arrivals: kEmptyPerAuxWarp
 // from each statistics warp, or kEmptyPerAttnWarp from each attention warp
+template <int D>
+constexpr int kAuxCols = (D + kAuxThreads - 1) / kAuxThreads;  // columns per statistics thread
 constexpr int kEmptyCount = 24, kEmptyPerAuxWarp = 8, kEmptyPerAttnWarp = 3;
 constexpr int kBarAttn = 1, kBarAux = 2, kBarConsumers = 3, kBarPair0 = 4;   // named barriers
 
@@ -122,6 +125,24 @@ __device__ __forceinline__ void cluster_sync_all() {
   __syncwarp();
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
+// the two halves of a cluster barrier that orders no memory, for work between them
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
+// Stores into another CTA's shared memory (cluster shared addresses) that
+// complete their bytes on the barrier at cluster shared address bar in that CTA.
+__device__ __forceinline__ void st_async_v2(uint32_t dst, float x, float y, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(dst), "f"(x),
+               "f"(y), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_v4(uint32_t dst, float x, float y, float z, float w, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(dst),
+               "f"(x), "f"(y), "f"(z), "f"(w), "r"(bar)
+               : "memory");
+}
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -166,7 +187,7 @@ struct FusedSmem {
   float vtok[D];
   alignas(16) float wpart[2][kPF];                   // attention combine slots; [0] ends as the record
   float linp[kMaxGroup][D + 1];                      // this rank's linear partial (D_glob in rank 0)
-  float hred[kAuxWarps][kMaxGroup][D];               // H rows: per-warp partials
+  alignas(16) float mrecv[merge_floats(D)];          // merge: what every rank sends this rank
   float zks[D];                                      // rank 0: zk after the fold
   int32_t sel_cache[kSelCache];
   uint32_t hist[256];                                // top-k: radix histogram
@@ -183,6 +204,7 @@ struct FusedSmem {
   uint64_t empty[kFStages];                          // one release per item
   uint64_t scores_bar;                               // C arrivals: every rank's scores are in place
   uint64_t sel_bar;                                  // 1 arrival: the selection is known
+  uint64_t merge_bar;                                // 1 arrival + the other ranks' merge bytes
   int sel_state;                                     // 1 sel_cache, 2 global row (sel_row), 3 every block
   const int32_t* sel_row;
   int abort;
@@ -301,7 +323,7 @@ __device__ __forceinline__ bool score_item_folds(const FusedParams& p, const Seq
 // warps what the stage holds.
 template <int D>
 __device__ __forceinline__ void issue_chunk(const KVMaps* tm, FusedSmem<D>& sm, int stage, int64_t ubase, int start,
-                                            int len, int is_sel) {
+                                            int len, int is_sel, uint64_t pol) {
   using Sm = FusedSmem<D>;
   uint64_t* bar = &sm.full_attn[stage];
   const uint32_t dst = smem_u32(sm.ring[stage]);
@@ -313,14 +335,14 @@ __device__ __forceinline__ void issue_chunk(const KVMaps* tm, FusedSmem<D>& sm, 
   const int row = (int)(ubase + start);
   if (len == kTile) {  // full chunk: one 64-row box per tensor
     mbar_arrive_expect_tx(bar, (uint32_t)(2 * Sm::kHalf));
-    tma_load_3d(dst, &tm->k64, 0, 0, row, bar);
-    tma_load_3d(dst + Sm::kHalf, &tm->v64, 0, 0, row, bar);
+    tma_load_3d_stream(dst, &tm->k64, 0, 0, row, bar, pol);
+    tma_load_3d_stream(dst + Sm::kHalf, &tm->v64, 0, 0, row, bar, pol);
   } else {             // ragged chunk: only the 16-row boxes it touches
     const int nbox = (len + kBoxRows - 1) / kBoxRows;
     mbar_arrive_expect_tx(bar, (uint32_t)(nbox * Sm::kBoxBytes * 2));
     for (int bx = 0; bx < nbox; ++bx) {
-      tma_load_3d(dst + bx * Sm::kBoxBytes, &tm->k16, 0, 0, row + bx * kBoxRows, bar);
-      tma_load_3d(dst + Sm::kHalf + bx * Sm::kBoxBytes, &tm->v16, 0, 0, row + bx * kBoxRows, bar);
+      tma_load_3d_stream(dst + bx * Sm::kBoxBytes, &tm->k16, 0, 0, row + bx * kBoxRows, bar, pol);
+      tma_load_3d_stream(dst + Sm::kHalf + bx * Sm::kBoxBytes, &tm->v16, 0, 0, row + bx * kBoxRows, bar, pol);
     }
   }
 }
@@ -542,78 +564,78 @@ __device__ __forceinline__ void aux_h_item(const FusedParams& p, FusedSmem<D>& s
   else h_rows<D, 2>(p, sm, unit, r0, nrows, hrows, hacc);
 }
 
-// After every H item (aux threads): sum the three warps' partials into linp;
-// rank 0 also folds the pending evictions into zk, zv, n and forms
-// N_glob += zv, D_glob = n + q'_i . zk.
+// After every H item (aux threads): the linear partial of this rank's H rows,
+// sum_r q'_i[r] H[r][:], summed over the three warps into linp one warp at a
+// time; rank 0 also folds the pending evictions into zk, zv and n (their old
+// values were loaded at the start of the role), adds zv (N_glob's count term)
+// and forms D_glob = n + q'_i . zk in linp[i][D].
 template <int D>
 __device__ void aux_finish_linear(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank,
-                                  const float (&hacc)[kMaxGroup][D / 32]) {
-  constexpr int CPL = D / 32;
+                                  const float (&hacc)[kMaxGroup][D / 32], const float (&zk0)[kAuxCols<D>],
+                                  const float (&zv0)[kAuxCols<D>], float n0) {
+  constexpr int CPL = D / 32, NZ = kAuxCols<D>;
   const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
-  if (p.q != nullptr) {
-#pragma unroll
-    for (int i = 0; i < kMaxGroup; ++i)
-      if (i < p.G)
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) sm.hred[aw][i][lane * CPL + c] = hacc[i][c];
-  }
-  float nval = 0.f;
+  float zv[NZ];
+  float nval = n0;
   if (rank == 0) {
-    const bool fold = p.fold_end > p.fold_begin;
+    const int64_t nf = p.fold_end - p.fold_begin;
     const int64_t ub = (int64_t)unit * p.cap;
-    for (int c = a; c < D; c += kAuxThreads) {
-      float zk = p.zk[(int64_t)unit * D + c], zv = p.zv[(int64_t)unit * D + c];
-      if (fold) {
-        for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
-          zk += __bfloat162float(p.k_cache[(ub + t) * D + c]);
-          zv += __bfloat162float(p.v_cache[(ub + t) * D + c]);
-        }
-        p.zk[(int64_t)unit * D + c] = zk;
-        p.zv[(int64_t)unit * D + c] = zv;
-      }
-      sm.zks[c] = zk;
-      sm.linp[0][c] = zv;  // scratch until the sum below
-    }
-    if (a == 0) {
-      nval = p.n[unit];
-      if (fold) {
-        nval += (float)(p.fold_end - p.fold_begin);
-        p.n[unit] = nval;
-      }
-      sm.linp[0][D] = nval;
-    }
-  }
-  named_sync(kBarAux, kAuxThreads);
-  if (p.q == nullptr) return;
-  constexpr int NZ = (D + kAuxThreads - 1) / kAuxThreads;
-  float zvs[NZ];
-#pragma unroll
-  for (int k = 0; k < NZ; ++k) {
-    const int c = a + k * kAuxThreads;
-    zvs[k] = (rank == 0 && c < D) ? sm.linp[0][c] : 0.f;
-  }
-  if (rank == 0) nval = sm.linp[0][D];
-  named_sync(kBarAux, kAuxThreads);
-  for (int i = 0; i < p.G; ++i) {
 #pragma unroll
     for (int k = 0; k < NZ; ++k) {
       const int c = a + k * kAuxThreads;
+      zv[k] = zv0[k];
       if (c < D) {
-        float v = zvs[k];
-#pragma unroll
-        for (int w = 0; w < kAuxWarps; ++w) v += sm.hred[w][i][c];
-        sm.linp[i][c] = v;
+        float zk = zk0[k];
+        if (nf == 1) {
+          zk += sm.ktok[c];
+          zv[k] += sm.vtok[c];
+        } else if (nf > 1) {
+          for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
+            zk += __bfloat162float(p.k_cache[(ub + t) * D + c]);
+            zv[k] += __bfloat162float(p.v_cache[(ub + t) * D + c]);
+          }
+        }
+        if (nf > 0) {
+          p.zk[(int64_t)unit * D + c] = zk;
+          p.zv[(int64_t)unit * D + c] = zv[k];
+        }
+        sm.zks[c] = zk;
       }
     }
-  }
-  if (rank == 0 && aw == 0) {
-    for (int i = 0; i < p.G; ++i) {
-      float d = 0.f;
-      for (int c = lane; c < D; c += 32) d += sm.qs[i][c] * sm.zks[c];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(kFull, d, o);
-      if (lane == 0) sm.linp[i][D] = nval + d;
+    if (nf > 0) {
+      nval += (float)nf;
+      if (a == 0) p.n[unit] = nval;
     }
+  }
+  if (p.q == nullptr) return;
+#pragma unroll 1
+  for (int w = 0; w < kAuxWarps; ++w) {
+    if (aw == w)
+#pragma unroll
+      for (int i = 0; i < kMaxGroup; ++i)
+        if (i < p.G)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            float* dst = &sm.linp[i][lane * CPL + c];
+            *dst = (w == 0 ? 0.f : *dst) + hacc[i][c];
+          }
+    named_sync(kBarAux, kAuxThreads);  // also: zks is complete
+  }
+  if (rank == 0) {
+    for (int i = 0; i < p.G; ++i)
+#pragma unroll
+      for (int k = 0; k < NZ; ++k) {
+        const int c = a + k * kAuxThreads;
+        if (c < D) sm.linp[i][c] += zv[k];
+      }
+    if (aw == 0)
+      for (int i = 0; i < p.G; ++i) {
+        float d = 0.f;
+        for (int c = lane; c < D; c += 32) d += sm.qs[i][c] * sm.zks[c];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(kFull, d, o);
+        if (lane == 0) sm.linp[i][D] = nval + d;
+      }
   }
 }
 
@@ -1254,6 +1276,17 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
     return have;
   };
   const int64_t nf = p.fold_end - p.fold_begin;
+  // rank 0's zk, zv and n, needed after the last H item: loaded now, so that
+  // their round trip is not on the path at the end
+  float zk0[kAuxCols<D>], zv0[kAuxCols<D>], n0 = 0.f;
+#pragma unroll
+  for (int k = 0; k < kAuxCols<D>; ++k) {
+    const int c = a + k * kAuxThreads;
+    const bool ld = rank == 0 && c < D;
+    zk0[k] = ld ? p.zk[(int64_t)unit * D + c] : 0.f;
+    zv0[k] = ld ? p.zv[(int64_t)unit * D + c] : 0.f;
+  }
+  if (rank == 0) n0 = p.n[unit];
   if (p.q != nullptr)
     for (int c = a; c < D; c += kAuxThreads) {
       float q1 = 0.f, q2 = 0.f;
@@ -1264,12 +1297,6 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
       }
       sm.qsum[0][c] = q1;
       sm.qsum[1][c] = q2;
-    }
-  if (nf == 1)  // the pending token's rows, for the H items
-    for (int c = a; c < D; c += kAuxThreads) {
-      const int64_t row = ((int64_t)unit * p.cap + p.fold_begin) * D + c;
-      sm.ktok[c] = __bfloat162float(p.k_cache[row]);
-      sm.vtok[c] = __bfloat162float(p.v_cache[row]);
     }
   named_sync(kBarAux, kAuxThreads);
   int fold_i0, fold_i1;
@@ -1322,7 +1349,7 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
     __syncwarp();
     if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
   }
-  aux_finish_linear<D>(p, sm, unit, rank, hacc);
+  aux_finish_linear<D>(p, sm, unit, rank, hacc, zk0, zv0, n0);
 }
 
 // Producer (role warp 11, lane 0): every copy of the rank, in ring order, one
@@ -1334,6 +1361,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
                               int rank) {
   if ((threadIdx.x & 31) != 0) return;
   constexpr int RB = Geo<D>::kBlocks, RH = Geo<D>::kRows;
+  const uint64_t pol = l2_evict_first();  // every copy of the ring streams data read once per launch
   int stage = 0, issued = 0;
   uint32_t epar = 0u;                  // per stage: parity of the next empty-barrier phase to wait for
   uint32_t fpar_aux = 0u, fpar_at = 0u;  // per stage: parity of the next full-barrier phase of each group
@@ -1372,8 +1400,8 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
       const uint32_t bytes = (uint32_t)(min(RB, s.b1 - s.b0 - i * RB) * D * 4);
       const int64_t off = (brow + (int64_t)i * RB) * D;
       mbar_arrive_expect_tx(bar, 2 * bytes);
-      bulk_load(dst, p.mu + off, bytes, bar);
-      bulk_load(dst + RB * D * 4, p.var + off, bytes, bar);
+      bulk_load_stream(dst, p.mu + off, bytes, bar, pol);
+      bulk_load_stream(dst + RB * D * 4, p.var + off, bytes, bar, pol);
     } else {
       mbar_arrive(bar);
     }
@@ -1391,7 +1419,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
       start = p.win_start + (ci - p.n_sink_chunks) * kTile;
       len = min(kTile, p.T - start);
     }
-    issue_chunk<D>(tm, sm, stage, ubase, start, len, 0);
+    issue_chunk<D>(tm, sm, stage, ubase, start, len, 0, pol);
     advance(false);
   }
   // H items: RH rows of H
@@ -1403,7 +1431,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
       const int r0 = s.h0 + i * RH;
       const uint32_t bytes = (uint32_t)(min(RH, s.h1 - r0) * D * 4);
       mbar_arrive_expect_tx(bar, bytes);
-      bulk_load(smem_u32(sm.ring[stage]), p.H + ((int64_t)unit * D + r0) * D, bytes, bar);
+      bulk_load_stream(smem_u32(sm.ring[stage]), p.H + ((int64_t)unit * D + r0) * D, bytes, bar, pol);
     } else {
       mbar_arrive(bar);
     }
@@ -1430,7 +1458,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
     } else if (jb != -1) {
       atomicOr(p.status, HYB_STATUS_BAD_SELECTION);
     }
-    issue_chunk<D>(tm, sm, stage, ubase, start, len, 1);
+    issue_chunk<D>(tm, sm, stage, ubase, start, len, 1, pol);
     advance(false);
     if (cpb == 1) {
       slot += p.C;
@@ -1451,27 +1479,81 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
   }
 }
 
-// Every rank, all threads, after the first cluster barrier: merge the C records
-// and linear partials (read over distributed shared memory) for this rank's
-// slice of the unit's G x D outputs and write them.
+// Every rank, all threads, once its record (the attention partials of its
+// chunks: per head the running max, the weight sums of the exact part and of
+// the selected tokens' Taylor terms, and their weighted value sums) and its
+// linear partial are final.  Rank r merges outputs [e0(r), e1(r)) of the
+// unit's G x D; every rank sends it a header (per head: max, exact weight sum,
+// and its share of D_glob - D_sel) and, per output of the slice, its exact
+// partial and its share of N_glob - N_sel (the merge needs only those sums).
+// Remote parts go by st.async into the receiver's mrecv, completing bytes on
+// its merge barrier; the rank's own part is stored locally.
 template <int D>
-__device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
-  constexpr int PF = FusedSmem<D>::kPF;
+__device__ __forceinline__ void merge_push(const FusedParams& p, FusedSmem<D>& sm, int rank) {
+  const int tid = threadIdx.x;
+  const int G = p.G, C = p.C;
+  const int stride = p.mstride;
+  const float* rec = sm.wpart[0];
+  const uint32_t recv0 = smem_u32(sm.mrecv), bar0 = smem_u32(&sm.merge_bar);
+  if (tid < C) {  // thread r: the header for rank r
+    float h[12];
+#pragma unroll
+    for (int i = 0; i < kMaxGroup; ++i) {
+      h[i] = rec[i];
+      h[4 + i] = rec[4 + i];
+      h[8 + i] = (rank == 0 && i < G ? sm.linp[i][D] : 0.f) - rec[8 + i];
+    }
+    const int off = rank * stride;
+    if (tid == rank) {
+#pragma unroll
+      for (int k = 0; k < 12; ++k) sm.mrecv[off + k] = h[k];
+    } else {
+      const uint32_t dst = map_rank(recv0 + 4u * (uint32_t)off, (uint32_t)tid), bar = map_rank(bar0, (uint32_t)tid);
+      st_async_v4(dst, h[0], h[1], h[2], h[3], bar);
+      st_async_v4(dst + 16u, h[4], h[5], h[6], h[7], bar);
+      st_async_v4(dst + 32u, h[8], h[9], h[10], h[11], bar);
+    }
+  }
+  for (int r = 0; r < C; ++r) {
+    const int e0 = p.mslice[r], e1 = p.mslice[r + 1];
+    const int off = rank * stride + 16;  // this rank's slot in rank r's buffer
+    const uint32_t dst0 = map_rank(recv0 + 4u * (uint32_t)off, (uint32_t)r), bar = map_rank(bar0, (uint32_t)r);
+    for (int e = e0 + tid; e < e1; e += kFThreads) {
+      const int i = e / D, d = e - i * D;
+      const float xa = rec[16 + e], xd = sm.linp[i][d] - rec[16 + 4 * D + e];
+      if (r == rank)
+        *reinterpret_cast<float2*>(&sm.mrecv[off + 2 * (e - e0)]) = make_float2(xa, xd);
+      else
+        st_async_v2(dst0 + 8u * (uint32_t)(e - e0), xa, xd, bar);
+    }
+  }
+}
+
+// Rank r's merge of its slice from the C slots of mrecv (after its merge
+// barrier): per head the global max M over ranks, each rank's exact part
+// rescaled by 2^(m_r - M); out = (N_ex + 2^-M (N_glob - N_sel)) /
+// (D_ex + 2^-M (D_glob - D_sel)), scaled by 2^M or 2^-M, whichever keeps it finite.
+template <int D>
+__device__ void merge_local(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G, C = p.C;
-  // per rank and head: rescale factor of the exact part; per head: max, D_ex, D_sel
+  const int stride = p.mstride;
+  // every thread waits; the outcome is made uniform so that all or none merge
+  if (!__syncthreads_and(wait_cluster_bounded(&sm.merge_bar, 0, kWaitLimit))) {
+    if (tid == 0) atomicOr(p.status, HYB_STATUS_TIMEOUT);
+    return;
+  }
+  // per rank and head: rescale factor of the exact part; per head: M, D_ex, D_glob - D_sel
   float* fac = reinterpret_cast<float*>(sm.ring[0]);  // [16][4] (the ring is idle now)
-  float* hm = fac + 16 * 4;                           // M[4], Dex[4], Dsel[4]
-  const uint32_t rec0 = smem_u32(&sm.wpart[0][0]);
-  const uint32_t lin0 = smem_u32(&sm.linp[0][0]);
+  float* hm = fac + 16 * 4;
   if (warp < G) {  // warp i: head i
     const int i = warp;
-    float m = -INFINITY, l = 0.f, ds = 0.f;
+    float m = -INFINITY, l = 0.f, dd = 0.f;
     if (lane < C) {
-      const uint32_t rb = map_rank(rec0, lane);
-      m = ld_cluster_f32(rb + 4 * i);
-      l = ld_cluster_f32(rb + 4 * (4 + i));
-      ds = ld_cluster_f32(rb + 4 * (8 + i));
+      const float* h = sm.mrecv + lane * stride;
+      m = h[i];
+      l = h[4 + i];
+      dd = h[8 + i];
     }
     float M = m;
 #pragma unroll
@@ -1483,57 +1565,45 @@ __device__ void merge_cluster(const FusedParams& p, FusedSmem<D>& sm, int unit, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       dex += __shfl_xor_sync(kFull, dex, o);
-      ds += __shfl_xor_sync(kFull, ds, o);
+      dd += __shfl_xor_sync(kFull, dd, o);
     }
     if (lane == 0) {
       hm[i] = M;
       hm[4 + i] = dex;
-      hm[8 + i] = ds;
+      hm[8 + i] = dd;
     }
   }
   __syncthreads();
   uint32_t flags = 0u;
-  const int e0 = (int)((int64_t)rank * G * D / C), e1 = (int)((int64_t)(rank + 1) * G * D / C);
+  const int e0 = p.mslice[rank], e1 = p.mslice[rank + 1];
   for (int e = e0 + tid; e < e1; e += kFThreads) {
-    const int i = e / D, d = e % D;
-    float xa[kMaxCluster], xs[kMaxCluster], xl[kMaxCluster];  // every remote load in flight first
+    const int i = e / D;
+    float nex = 0.f, nsub = 0.f;
 #pragma unroll
     for (int r = 0; r < kMaxCluster; ++r) {
       if (r < C) {
-        const uint32_t rb = map_rank(rec0, r), lb = map_rank(lin0, r);
-        xa[r] = ld_cluster_f32(rb + 4 * (16 + i * D + d));
-        xs[r] = ld_cluster_f32(rb + 4 * (16 + 4 * D + i * D + d));
-        xl[r] = ld_cluster_f32(lb + 4 * (i * (D + 1) + d));
+        const float2 v = *reinterpret_cast<const float2*>(&sm.mrecv[r * stride + 16 + 2 * (e - e0)]);
+        nex += v.x * fac[r * 4 + i];
+        nsub += v.y;
       }
     }
-    float nex = 0.f, nsel = 0.f, ng = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      if (r < C) {
-        nex += xa[r] * fac[r * 4 + i];
-        nsel += xs[r];
-        ng += xl[r];
-      }
-    }
-    const float Ms = hm[i], Dex = hm[4 + i], Dsel = hm[8 + i];
-    const float Dg = ld_cluster_f32(map_rank(smem_u32(&sm.linp[i][D]), 0u));  // rank 0 holds D_glob
+    const float Ms = hm[i], Dex = hm[4 + i], Dsub = hm[8 + i];
     float num, den;
     if (Ms >= 0.f) {
       const float f = exp2f(-Ms);
-      num = nex + f * (ng - nsel);
-      den = Dex + f * (Dg - Dsel);
+      num = nex + f * nsub;
+      den = Dex + f * Dsub;
     } else {
       const float f = exp2f(Ms);
-      num = nex * f + (ng - nsel);
-      den = Dex * f + (Dg - Dsel);
+      num = nex * f + nsub;
+      den = Dex * f + Dsub;
     }
     const float o = num / den;
-    p.out[((int64_t)unit * G + i) * D + d] = o;
+    p.out[(int64_t)unit * G * D + e] = o;
     if (!(den > 0.f)) flags |= HYB_STATUS_DENOMINATOR;
     if (!isfinite(o)) flags |= HYB_STATUS_NONFINITE;
   }
   if (flags) atomicOr(p.status, flags);
-  (void)PF;
 }
 
 template <int D>
@@ -1560,6 +1630,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     const bool push = runs_topk(p) && p.nb <= FusedSmem<D>::kGather;
     mbar_init(&sm.scores_bar, push ? 1 : p.C);
     mbar_init(&sm.sel_bar, 1);
+    mbar_init(&sm.merge_bar, 1);
     sm.sel_state = 3;
     sm.sel_row = nullptr;
     sm.abort = 0;
@@ -1573,6 +1644,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
       }
       mbar_arrive_expect_tx(&sm.scores_bar, bytes);
     }
+    if (p.q != nullptr)  // the other ranks' headers and pieces of this rank's slice
+      mbar_arrive_expect_tx(&sm.merge_bar, (uint32_t)((p.C - 1) * (48 + 8 * (p.mslice[rank + 1] - p.mslice[rank]))));
     pdl_wait_primary();  // everything below reads what earlier grids wrote
   }
   // the barriers of every rank are initialised before any remote arrival
@@ -1583,18 +1656,49 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     producer_role<D>(&tm, p, sm, s, unit, rank);
   } else {
     const int t = role_tid();  // 0 .. kConsumerThreads - 1
-    if (p.q != nullptr)
-      for (int e = t; e < kMaxGroup * D; e += kConsumerThreads) {
-        const float qv = e < p.G * D ? __bfloat162float(p.q[(int64_t)unit * p.G * D + e]) * p.scale : 0.f;
-        sm.qs[e / D][e % D] = sm.qsT[e % D][e / D] = qv;
+    // The prologue's global loads: one 16-byte load per thread, all issued
+    // before any of them is used, so that none waits behind the ring's first
+    // copies (a load issued after them waits for most of the start-up burst).
+    // Threads [0, QV): q; [QV, QV + D/4): the pending token's K and V rows;
+    // [QV + D/4, QV + D/2): the decode's appended token (rank 0).
+    constexpr int QV = kMaxGroup * D / 8;
+    static_assert(QV + D / 2 <= kConsumerThreads, "one 16-byte piece per thread");
+    const int tr = t - QV, ta = t - QV - D / 4;
+    const bool ld_q = p.q != nullptr && t < QV && t * 8 < p.G * D;
+    const bool ld_row = p.fold_end - p.fold_begin == 1 && tr >= 0 && tr < D / 4;
+    const bool ld_new = p.k_new != nullptr && rank == 0 && ta >= 0 && ta < D / 4;
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (ld_q) {
+      raw = __ldg(reinterpret_cast<const uint4*>(p.q + (int64_t)unit * p.G * D) + t);
+    } else if (ld_row) {
+      const int e = (tr % (D / 8)) * 8;
+      raw = __ldg(reinterpret_cast<const uint4*>((tr >= D / 8 ? p.v_cache : p.k_cache) +
+                                                 ((int64_t)unit * p.cap + p.fold_begin) * D + e));
+    } else if (ld_new) {
+      const int e = (ta % (D / 8)) * 8;
+      raw = __ldg(reinterpret_cast<const uint4*>((ta >= D / 8 ? p.v_new : p.k_new) + (int64_t)unit * D + e));
+    }
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    if (p.q != nullptr && t < QV) {  // heads past G stay zero
+      const int i = t * 8 / D, d0 = (t * 8) % D;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        const float q0 = f.x * p.scale, q1 = f.y * p.scale;
+        sm.qs[i][d0 + 2 * j] = sm.qsT[d0 + 2 * j][i] = q0;
+        sm.qs[i][d0 + 2 * j + 1] = sm.qsT[d0 + 2 * j + 1][i] = q1;
       }
-    if (p.k_new != nullptr && rank == 0 && t < D / 4) {
-      // the decode's appended token: row T of the caches (16 bytes per thread)
-      const bool is_v = t >= D / 8;
-      const int e = (t % (D / 8)) * 8;
-      const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + (int64_t)unit * D + e;
-      __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e;
-      *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+    } else if (ld_row) {  // the pending token's rows, for the folds
+      float* dst = (tr >= D / 8 ? sm.vtok : sm.ktok) + (tr % (D / 8)) * 8;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        dst[2 * j] = f.x;
+        dst[2 * j + 1] = f.y;
+      }
+    } else if (ld_new) {  // the decode's appended token: row T of the caches
+      const int e = (ta % (D / 8)) * 8;
+      *reinterpret_cast<uint4*>((ta >= D / 8 ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e) = raw;
     }
     named_sync(kBarConsumers, kConsumerThreads);
     if (warp < kAttnWarps) {
@@ -1603,9 +1707,11 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
       aux_role<D>(p, sm, s, unit, rank);
     }
   }
-  cluster_sync_all();  // every rank's record and linear partial are final
-  if (p.q != nullptr) merge_cluster<D>(p, sm, unit, rank);
-  cluster_sync_all();  // the records stay readable until every rank is done
+  __syncthreads();  // this rank's record and linear partial are final; its ring is idle
+  if (p.q != nullptr) merge_push<D>(p, sm, rank);
+  cluster_arrive_relaxed();  // the merge's data is ordered by the merge barriers
+  if (p.q != nullptr) merge_local<D>(p, sm, unit, rank);
+  cluster_wait();  // no CTA leaves the cluster before every rank has sent its parts
 }
 
 }  // namespace
