@@ -99,6 +99,11 @@ __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void* src, ui
                : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
+}
+
 // L2 policy for data read once per launch: its lines are the first to be
 // replaced, so that the kernel's code and small reused data stay in L2 while a
 // launch streams more than L2 holds.

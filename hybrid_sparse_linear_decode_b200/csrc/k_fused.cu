@@ -121,10 +121,6 @@ __device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t par
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
-__device__ __forceinline__ void cluster_sync_all() {
-  __syncwarp();
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
 // the two halves of a cluster barrier that orders no memory, for work between them
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   __syncwarp();
@@ -1299,6 +1295,7 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
       sm.qsum[1][c] = q2;
     }
   named_sync(kBarAux, kAuxThreads);
+  cluster_wait();  // every rank's barriers are initialised: remote operations are allowed from here on
   int fold_i0, fold_i1;
   fold_items<D>(p, s, &fold_i0, &fold_i1);
 #pragma unroll 1
@@ -1491,11 +1488,12 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
 template <int D>
 __device__ __forceinline__ void merge_push(const FusedParams& p, FusedSmem<D>& sm, int rank) {
   const int tid = threadIdx.x;
-  const int G = p.G, C = p.C;
+  const int G = p.G, C = p.C, GD = G * D;
   const int stride = p.mstride;
   const float* rec = sm.wpart[0];
   const uint32_t recv0 = smem_u32(sm.mrecv), bar0 = smem_u32(&sm.merge_bar);
-  if (tid < C) {  // thread r: the header for rank r
+  const int hr = tid - (kFThreads - C);  // the last C threads (the fewest outputs): the header for rank hr
+  if (hr >= 0) {
     float h[12];
 #pragma unroll
     for (int i = 0; i < kMaxGroup; ++i) {
@@ -1504,38 +1502,35 @@ __device__ __forceinline__ void merge_push(const FusedParams& p, FusedSmem<D>& s
       h[8 + i] = (rank == 0 && i < G ? sm.linp[i][D] : 0.f) - rec[8 + i];
     }
     const int off = rank * stride;
-    if (tid == rank) {
+    if (hr == rank) {
 #pragma unroll
       for (int k = 0; k < 12; ++k) sm.mrecv[off + k] = h[k];
     } else {
-      const uint32_t dst = map_rank(recv0 + 4u * (uint32_t)off, (uint32_t)tid), bar = map_rank(bar0, (uint32_t)tid);
+      const uint32_t dst = map_rank(recv0 + 4u * (uint32_t)off, (uint32_t)hr), bar = map_rank(bar0, (uint32_t)hr);
       st_async_v4(dst, h[0], h[1], h[2], h[3], bar);
       st_async_v4(dst + 16u, h[4], h[5], h[6], h[7], bar);
       st_async_v4(dst + 32u, h[8], h[9], h[10], h[11], bar);
     }
   }
-  for (int r = 0; r < C; ++r) {
-    const int e0 = p.mslice[r], e1 = p.mslice[r + 1];
-    const int off = rank * stride + 16;  // this rank's slot in rank r's buffer
-    const uint32_t dst0 = map_rank(recv0 + 4u * (uint32_t)off, (uint32_t)r), bar = map_rank(bar0, (uint32_t)r);
-    for (int e = e0 + tid; e < e1; e += kFThreads) {
-      const int i = e / D, d = e - i * D;
-      const float xa = rec[16 + e], xd = sm.linp[i][d] - rec[16 + 4 * D + e];
-      if (r == rank)
-        *reinterpret_cast<float2*>(&sm.mrecv[off + 2 * (e - e0)]) = make_float2(xa, xd);
-      else
-        st_async_v2(dst0 + 8u * (uint32_t)(e - e0), xa, xd, bar);
-    }
+  for (int e = tid; e < GD; e += kFThreads) {
+    const int r = ((e + 1) * C - 1) / GD;  // the rank that merges output e: mslice[r] <= e < mslice[r + 1]
+    const int i = e / D, d = e - i * D;
+    const float xa = rec[16 + e], xd = sm.linp[i][d] - rec[16 + 4 * D + e];
+    const int off = rank * stride + 16 + 2 * (e - p.mslice[r]);  // this rank's slot in rank r's buffer
+    if (r == rank)
+      *reinterpret_cast<float2*>(&sm.mrecv[off]) = make_float2(xa, xd);
+    else
+      st_async_v2(map_rank(recv0 + 4u * (uint32_t)off, (uint32_t)r), xa, xd, map_rank(bar0, (uint32_t)r));
   }
 }
 
 // Rank r's merge of its slice from the C slots of mrecv (after its merge
-// barrier): per head the global max M over ranks, each rank's exact part
-// rescaled by 2^(m_r - M); out = (N_ex + 2^-M (N_glob - N_sel)) /
-// (D_ex + 2^-M (D_glob - D_sel)), scaled by 2^M or 2^-M, whichever keeps it finite.
+// barrier), one output per thread: per head the global max M over ranks, each
+// rank's exact part rescaled by 2^(m_r - M); out = (N_ex + 2^-M (N_glob - N_sel))
+// / (D_ex + 2^-M (D_glob - D_sel)), scaled by 2^M or 2^-M, whichever keeps it finite.
 template <int D>
 __device__ void merge_local(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int G = p.G, C = p.C;
   const int stride = p.mstride;
   // every thread waits; the outcome is made uniform so that all or none merge
@@ -1543,58 +1538,36 @@ __device__ void merge_local(const FusedParams& p, FusedSmem<D>& sm, int unit, in
     if (tid == 0) atomicOr(p.status, HYB_STATUS_TIMEOUT);
     return;
   }
-  // per rank and head: rescale factor of the exact part; per head: M, D_ex, D_glob - D_sel
-  float* fac = reinterpret_cast<float*>(sm.ring[0]);  // [16][4] (the ring is idle now)
-  float* hm = fac + 16 * 4;
-  if (warp < G) {  // warp i: head i
-    const int i = warp;
-    float m = -INFINITY, l = 0.f, dd = 0.f;
-    if (lane < C) {
-      const float* h = sm.mrecv + lane * stride;
-      m = h[i];
-      l = h[4 + i];
-      dd = h[8 + i];
-    }
-    float M = m;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-    if (M == -INFINITY) M = 0.f;
-    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    if (lane < C) fac[lane * 4 + i] = f;
-    float dex = l * f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      dex += __shfl_xor_sync(kFull, dex, o);
-      dd += __shfl_xor_sync(kFull, dd, o);
-    }
-    if (lane == 0) {
-      hm[i] = M;
-      hm[4 + i] = dex;
-      hm[8 + i] = dd;
-    }
-  }
-  __syncthreads();
   uint32_t flags = 0u;
   const int e0 = p.mslice[rank], e1 = p.mslice[rank + 1];
   for (int e = e0 + tid; e < e1; e += kFThreads) {
     const int i = e / D;
-    float nex = 0.f, nsub = 0.f;
+    const float* h = sm.mrecv + i;
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r)
+      if (r < C) M = fmaxf(M, h[r * stride]);
+    if (M == -INFINITY) M = 0.f;
+    float nex = 0.f, nsub = 0.f, Dex = 0.f, Dsub = 0.f;
 #pragma unroll
     for (int r = 0; r < kMaxCluster; ++r) {
       if (r < C) {
+        const float m = h[r * stride];
+        const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
         const float2 v = *reinterpret_cast<const float2*>(&sm.mrecv[r * stride + 16 + 2 * (e - e0)]);
-        nex += v.x * fac[r * 4 + i];
+        nex += v.x * f;
         nsub += v.y;
+        Dex += h[r * stride + 4] * f;
+        Dsub += h[r * stride + 8];
       }
     }
-    const float Ms = hm[i], Dex = hm[4 + i], Dsub = hm[8 + i];
     float num, den;
-    if (Ms >= 0.f) {
-      const float f = exp2f(-Ms);
+    if (M >= 0.f) {
+      const float f = exp2f(-M);
       num = nex + f * nsub;
       den = Dex + f * Dsub;
     } else {
-      const float f = exp2f(Ms);
+      const float f = exp2f(M);
       num = nex * f + nsub;
       den = Dex * f + Dsub;
     }
@@ -1616,6 +1589,21 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
   const int rank = (int)cluster_rank();
   const int unit = blockIdx.x / p.C;
   const Seq s = make_seq<D>(p, rank);
+  if (warp == kProducerWarp && (tid & 31) == 0) {
+    // Before the wait for the previous grid (which may still be running):
+    // the rank's block statistics, its first items, are prefetched into L2.
+    // L2 is the point of coherence, so a line the previous grid still writes
+    // is updated there; nothing enters this CTA before the wait.
+    if (s.b1 > s.b0) {
+      const int64_t off = ((int64_t)unit * p.max_blocks + s.b0) * D;
+      const int64_t bytes = (int64_t)(s.b1 - s.b0) * D * 4;
+      for (int64_t o = 0; o < bytes; o += 32768) {
+        const uint32_t n = (uint32_t)(bytes - o < 32768 ? bytes - o : 32768);
+        bulk_prefetch_l2(reinterpret_cast<const char*>(p.mu + off) + o, n);
+        bulk_prefetch_l2(reinterpret_cast<const char*>(p.var + off) + o, n);
+      }
+    }
+  }
   if (tid == 0) {
     tma_prefetch_desc(&tm.k64);
     tma_prefetch_desc(&tm.v64);
@@ -1648,12 +1636,19 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
       mbar_arrive_expect_tx(&sm.merge_bar, (uint32_t)((p.C - 1) * (48 + 8 * (p.mslice[rank + 1] - p.mslice[rank]))));
     pdl_wait_primary();  // everything below reads what earlier grids wrote
   }
-  // the barriers of every rank are initialised before any remote arrival
-  cluster_sync_all();
+  // This CTA's barriers are initialised and every thread is ordered after the
+  // wait for the previous grid.  The cluster barrier is split: the arrival
+  // here (the barrier initialisations are released to the cluster by their
+  // fence), the wait before a thread's first remote operation (the
+  // statistics warps' score push) or after its role, so that the ring's
+  // first copies do not wait for the other ranks.
+  __syncthreads();
+  cluster_arrive_relaxed();
   pdl_allow_dependents();
   if (warp == kProducerWarp) {
     // the producer starts at once: it needs nothing from the lines below
     producer_role<D>(&tm, p, sm, s, unit, rank);
+    cluster_wait();
   } else {
     const int t = role_tid();  // 0 .. kConsumerThreads - 1
     // The prologue's global loads: one 16-byte load per thread, all issued
@@ -1703,8 +1698,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     named_sync(kBarConsumers, kConsumerThreads);
     if (warp < kAttnWarps) {
       if (p.q != nullptr) attn_role<D>(p, sm, s, unit);
+      cluster_wait();
     } else {
-      aux_role<D>(p, sm, s, unit, rank);
+      aux_role<D>(p, sm, s, unit, rank);  // waits on the cluster barrier before its score push
     }
   }
   __syncthreads();  // this rank's record and linear partial are final; its ring is idle
