@@ -90,11 +90,6 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t local_smem, uint32_t rank)
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
 __device__ __forceinline__ void remote_arrive(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
@@ -1064,20 +1059,6 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
     if (nvalid > 0) {
       const uint32_t kb = smem_u32(sm.ring[stage]);
       const uint32_t vb = kb + FusedSmem<D>::kHalf;
-      if (nvalid < kTile) {
-        // rows past the chunk may hold tokens beyond T (unwritten cache rows):
-        // zero their V rows so that 0-weight * garbage cannot make a NaN (only
-        // the few ragged chunks of a launch pay for the proxy fence)
-        constexpr int CPR = D / 8;  // 16-byte chunks per row
-        uint8_t* vt = sm.ring[stage] + FusedSmem<D>::kHalf;
-        for (int e = lane; e < (kTile - nvalid) * CPR; e += 32) {
-          const int t = nvalid + e / CPR;
-          *reinterpret_cast<uint4*>(vt + swz<D>(t, e % CPR)) = make_uint4(0, 0, 0, 0);
-        }
-        // order these generic-proxy writes before the next copy into the stage
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-      }
       // ---- S^T = K Q^T: m-tile mt holds tokens 16mt .. 16mt+15, columns = heads
       float sacc[4][4];
 #pragma unroll
@@ -1144,9 +1125,18 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
           O[n][3] *= alpha;
         }
       }
-      // ---- O += A V: A rows = weight columns (transposed 8x8 blocks), hi then lo
+      // ---- O += A V: A rows = weight columns (transposed 8x8 blocks), hi then lo.
+      // In a ragged chunk the rows past it have zero weights: k-steps wholly
+      // past it are skipped (rows past its 16-row boxes hold stale stage data),
+      // and in its last k-step the V fragments of rows past it, which may be
+      // unwritten cache rows, are zeroed in registers so that no 0 * NaN arises.
 #pragma unroll
       for (int kt = 0; kt < 4; ++kt) {
+        if (kt * 16 >= nvalid) break;
+        const bool tail = kt * 16 + 16 > nvalid;  // warp-uniform
+        const int tk = kt * 16 + 2 * tig;          // rows of the low halves of b0v / b2v (b1v / b3v: + 8)
+        const uint32_t m0 = (tk < nvalid ? 0x0000ffffu : 0u) | (tk + 1 < nvalid ? 0xffff0000u : 0u);
+        const uint32_t m1 = (tk + 8 < nvalid ? 0x0000ffffu : 0u) | (tk + 9 < nvalid ? 0xffff0000u : 0u);
         uint32_t h0, l0, h1, l1;
         split_bf16(w[kt][0], w[kt][1], h0, l0);
         split_bf16(w[kt][2], w[kt][3], h1, l1);
@@ -1156,6 +1146,12 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
           uint32_t b0v, b1v, b2v, b3v;
           ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, (half * NH / 2 + np) * 2 + (mi >> 1)), b0v, b1v, b2v,
                     b3v);
+          if (tail) {
+            b0v &= m0;
+            b1v &= m1;
+            b2v &= m0;
+            b3v &= m1;
+          }
           mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
           mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
         }

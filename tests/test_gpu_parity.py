@@ -206,3 +206,25 @@ def test_state_sync_is_idempotent_and_decode_folds():
     for k in s1:
         np.testing.assert_array_equal(s1[k], s2[k])
     check_state(c)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T0=601, W=64, capacity=700, n_append=5),               # ragged last window piece
+    dict(T0=4 + 64 + 32 * 5 + 7, capacity=400, n_append=3),     # newest block partial
+    dict(T0=3, S=4, W=16, capacity=64, n_append=2),             # sinks only, one 4-row piece
+    dict(B=2, Hq=16, Hkv=4, T0=1499, W=100, Bk=64, k=6, capacity=1600, n_append=4),
+])
+def test_unwritten_rows_past_T_do_not_leak(kw):
+    """Cache rows at and past T are capacity nobody has written: here NaN.  A
+    ragged chunk's last 16-row box reaches into them; with zero weights they
+    must leave the result unchanged (0 * NaN would be NaN), before and after
+    appends overwrite some of them."""
+    c = _case(**kw)
+    c.layer.k_cache[:, :, c.T:].fill_(float("nan"))
+    c.layer.v_cache[:, :, c.T:].fill_(float("nan"))
+    q = c.random_q()
+    full_check(c, q)
+    assert c.layer.status() == 0
+    c.append(kw["n_append"])
+    full_check(c, c.random_q())
+    assert c.layer.status() == 0
