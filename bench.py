@@ -3,10 +3,10 @@
 
 One step = for every layer of the workload: one decode (block scores, top-k,
 gather, exact softmax part, Taylor linear part by subtraction, merge) and one
-append (cache write; the evicted token's fold into the linear state and block
-statistics happens in the next decode's select kernel), issued as one
-hyb_attn_decode_append call: two kernel launches chained with programmatic
-dependent launch.
+append (the new token's cache row; the evicted token's fold into the linear
+state and block statistics happens in the next decode), issued as one
+hyb_attn_decode_append call: one launch of the fused decode kernel per layer,
+consecutive layers chained with programmatic dependent launch.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
 on a bounded sample of the same workload instead.
@@ -193,14 +193,18 @@ class Bench:
         self.w, self.device = w, device
         self.n_steps = n_steps
         n_app = self.n_steps
-        cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window,
-                          w.top_k, w.T0 + n_app)
-        ws_bytes = HybridAttentionLayer.workspace_bytes(cfg)
+
+        def cfg_of(l):  # the layer's own top-k and window when budgets vary by layer
+            wl = w.for_layer(l)
+            return make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, wl.window,
+                               wl.top_k, w.T0 + n_app)
+
+        ws_bytes = max(HybridAttentionLayer.workspace_bytes(cfg_of(l)) for l in range(w.layers))
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device)   # shared: one stream
         self.layers, self.app_k, self.app_v, self.q = [], [], [], []
         n_q = min(self.n_steps, 8)
         for l in range(w.layers):
-            L = HybridAttentionLayer(cfg, device, workspace=self.workspace)
+            L = HybridAttentionLayer(cfg_of(l), device, workspace=self.workspace)
             tb = SD.DeviceTables(w, l, L.device)
             SD.fill_kv(w, tb, L.k_cache, L.v_cache, 0, w.T0)
             shp = (w.batch, w.n_kv_heads, n_app, w.head_dim)
@@ -246,9 +250,11 @@ def run_native(args, rank, world):
     Ke = 0 if args.no_e2e else min(K, 20)  # steps of the end-to-end pass
     b = Bench(w, Wm + K + Kk + Ke, device)
     T_mid = w.T0 + Wm + K // 2
-    dec_b, app_b = algorithmic_bytes(w, T_mid)
-    units = w.layers * w.units_per_layer
-    step_bytes = units * (dec_b + app_b)
+    step_dec = step_bytes = 0
+    for l in range(w.layers):  # each layer with its own budget
+        dec_b, app_b = algorithmic_bytes(w.for_layer(l), T_mid)
+        step_dec += w.units_per_layer * dec_b
+        step_bytes += w.units_per_layer * (dec_b + app_b)
     flush = step_bytes < 4 * 126e6      # the step's data would otherwise stay in L2
     scratch = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if flush else None
 
@@ -293,7 +299,7 @@ def run_native(args, rank, world):
     ms_per_step = total_ms / K
     steps_s = 1e3 / ms_per_step
 
-    # ---- decode timing: events around each layer's decode (its two chained kernels)
+    # ---- the launch on its own: events around each layer's launch, chaining off
     ka, kb_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kern_ms, n_kern = 0.0, 0
     pool = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in b.layers]
@@ -314,10 +320,16 @@ def run_native(args, rank, world):
         for e0, e1 in pool[i]:
             kern_ms += e0.elapsed_time(e1)
             n_kern += 1
-    decode_ms = kern_ms / n_kern
-    decode_bytes = w.units_per_layer * dec_b
+    isolated_ms = kern_ms / n_kern
+    # In the timed region the step is exactly one launch of the fused kernel per
+    # layer, back to back: its average duration there is the step time over the
+    # launches, and its algorithmic bytes those of one layer's decode + append.
+    n_launch = b.launches_per_step()
+    launch_ms = ms_per_step / n_launch
+    launch_bytes = step_bytes // n_launch
     hbm_peak, peak_kind = peaks()
-    achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
+    achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
+    isolated = launch_bytes / (isolated_ms * 1e-3) / 1e9
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # ---- e2e through the host-buffer entry point (pinned host q / k / v / out)
@@ -366,6 +378,7 @@ def run_native(args, rank, world):
             "workload": w.name, "layers": w.layers, "batch": w.batch, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context_T0": w.T0, "block": w.block_size,
             "sinks": w.n_sink, "window": w.window, "top_k": w.top_k,
+            **({"layer_budgets_k_W": [list(x) for x in w.layer_budgets]} if w.layer_budgets else {}),
             "l2": "flushed between timed steps (512 MB write)" if flush else "step data >> L2 (no flush)",
             "parallelism": f"replicas x{world} (independent units per GPU)",
         },
@@ -375,11 +388,14 @@ def run_native(args, rank, world):
         "pct_of_hbm_peak_step": round(100 * step_gbs / hbm_peak, 2),
         "bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm",
-                     "kernel": "one layer's decode: the fused decode kernel (one launch)",
+                     "kernel": "the fused decode kernel: one layer's decode + append (one launch)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
-                     "traffic": measured_traffic(w.name), "bytes_per_launch": decode_bytes,
-                     "avg_launch_us": round(decode_ms * 1e3, 3)},
+                     "traffic": measured_traffic(w.name), "bytes_per_launch": launch_bytes,
+                     "decode_bytes_per_launch": step_dec // n_launch,
+                     "avg_launch_us": round(launch_ms * 1e3, 3),
+                     "isolated_launch_us": round(isolated_ms * 1e3, 3),
+                     "isolated_frac": round(isolated / hbm_peak, 4)},
         "e2e": e2e,
         "gpu_launches": b.launches_per_step() * K,
         "clocks": clocks,
@@ -401,13 +417,16 @@ def _oracle_units(w, n_units: int = 4, max_appends: int = 2048):
     import oracle as O
     from syngen import host as SH
     scale = 1 / math.sqrt(w.head_dim)
-    tb = SH.LayerTables(w, 0)
-    q_all = SH.bf16_bits_to_f64(SH.q_bits(w, 0, 0))
+    nl = max(1, len(w.layer_budgets))  # with per-layer budgets: units of layers with different budgets
     units = []
-    for i in range(min(n_units, w.batch * w.n_kv_heads)):
-        b, h = divmod(i, w.n_kv_heads)
-        K, V = SH.kv_f64(w, tb, b, h, 0, w.T0 + max_appends)
-        u = O.OracleUnit(K[:w.T0], V[:w.T0], w.n_sink, w.window, w.block_size, w.top_k, scale,
+    for i in range(min(n_units, w.batch * w.n_kv_heads * nl)):
+        layer, j = i % nl, i // nl
+        wl = w.for_layer(layer)
+        tb = SH.LayerTables(wl, layer)
+        q_all = SH.bf16_bits_to_f64(SH.q_bits(wl, layer, 0))
+        b, h = divmod(j, w.n_kv_heads)
+        K, V = SH.kv_f64(wl, tb, b, h, 0, w.T0 + max_appends)
+        u = O.OracleUnit(K[:w.T0], V[:w.T0], w.n_sink, wl.window, w.block_size, wl.top_k, scale,
                          capacity=w.T0 + max_appends)
         units.append([u, K[w.T0:], V[w.T0:], q_all[b, h * w.group:(h + 1) * w.group], 0])
     _ORACLE_UNITS[w.name] = units

@@ -17,9 +17,11 @@ from ._abi import (  # noqa: F401
     hyb_attn_plan,
     hyb_attn_init,
     hyb_attn_append,
+    hyb_attn_append_chunk,
     hyb_attn_sync_state,
     hyb_attn_decode,
     hyb_attn_decode_append,
+    hyb_attn_decode_chunk,
     hyb_attn_decode_with_selection,
     hyb_attn_step_host,
     hyb_attn_decode_noalloc,

@@ -62,9 +62,11 @@ SIGNATURES = [
     ("hyb_attn_init", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
                                      ctypes.POINTER(hyb_attn_buffers), c_i64, c_vp]),
     ("hyb_attn_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_append_chunk", ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_vp]),
     ("hyb_attn_sync_state", ctypes.c_int, [c_vp, c_vp]),
     ("hyb_attn_decode", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_decode_chunk", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_with_selection", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_step_host", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_noalloc", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
@@ -148,6 +150,10 @@ def hyb_attn_append(ctx: int, k_new: int, v_new: int, stream: int) -> None:
     _check("hyb_attn_append", load_library().hyb_attn_append(ctx, k_new, v_new, stream))
 
 
+def hyb_attn_append_chunk(ctx: int, k_new: int, v_new: int, n: int, stream: int) -> None:
+    _check("hyb_attn_append_chunk", load_library().hyb_attn_append_chunk(ctx, k_new, v_new, n, stream))
+
+
 def hyb_attn_sync_state(ctx: int, stream: int) -> None:
     _check("hyb_attn_sync_state", load_library().hyb_attn_sync_state(ctx, stream))
 
@@ -160,6 +166,12 @@ def hyb_attn_decode_append(ctx: int, q: int, k_new: int, v_new: int, out: int, s
                            stream: int) -> None:
     _check("hyb_attn_decode_append",
            load_library().hyb_attn_decode_append(ctx, q, k_new, v_new, out, sel_out, scores_out, stream))
+
+
+def hyb_attn_decode_chunk(ctx: int, q: int, k_new: int, v_new: int, n: int, out: int, sel_out,
+                          stream: int) -> None:
+    _check("hyb_attn_decode_chunk",
+           load_library().hyb_attn_decode_chunk(ctx, q, k_new, v_new, n, out, sel_out, stream))
 
 
 def hyb_attn_decode_with_selection(ctx: int, q: int, sel: int, out: int, stream: int) -> None:

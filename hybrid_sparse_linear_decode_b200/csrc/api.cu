@@ -404,10 +404,10 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   return HYB_OK;
 }
 
-int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaStream_t stream) {
-  if (x == nullptr || k_new == nullptr || v_new == nullptr) return HYB_EINVAL;
+int hyb_attn_append_chunk(hyb_attn_ctx* x, const void* k_new, const void* v_new, int32_t n, cudaStream_t stream) {
+  if (x == nullptr || k_new == nullptr || v_new == nullptr || n < 1 || n > 65535) return HYB_EINVAL;
   if (!aligned16(k_new) || !aligned16(v_new)) return HYB_EINVAL;
-  if (x->T >= x->cfg.capacity) return HYB_ECAPACITY;
+  if (x->T + n > x->cfg.capacity) return HYB_ECAPACITY;
   AppendParams p{};
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
@@ -416,10 +416,15 @@ int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaS
   p.cap = x->cfg.capacity;
   p.T = x->T;
   p.units = x->ck.units;
+  p.n = n;
   const cudaError_t e = launch_append(p, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  x->T += 1;
+  x->T += n;
   return HYB_OK;
+}
+
+int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaStream_t stream) {
+  return hyb_attn_append_chunk(x, k_new, v_new, 1, stream);
 }
 
 int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
@@ -442,6 +447,23 @@ int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, 
                            int32_t* sel_out, float* scores_out, cudaStream_t stream) {
   if (k_new == nullptr || v_new == nullptr) return HYB_EINVAL;
   return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, k_new, v_new, stream);
+}
+
+int hyb_attn_decode_chunk(hyb_attn_ctx* x, const void* q, const void* k_new, const void* v_new, int32_t n,
+                          float* out, int32_t* sel_out, cudaStream_t stream) {
+  if (x == nullptr || q == nullptr || k_new == nullptr || v_new == nullptr || out == nullptr || n < 1)
+    return HYB_EINVAL;
+  if (x->T == 0) return HYB_ESTATE;
+  if (x->T + n > x->cfg.capacity) return HYB_ECAPACITY;
+  const size_t U = (size_t)x->ck.units, D = (size_t)x->ck.D, G = (size_t)x->ck.G;
+  for (int32_t j = 0; j < n; ++j) {  // row j: decode at length T + j, then append token j
+    const int r = decode_impl(x, static_cast<const char*>(q) + j * U * G * D * 2, out + j * U * G * D, nullptr,
+                              sel_out == nullptr ? nullptr : sel_out + j * U * (size_t)x->cfg.top_k, nullptr,
+                              static_cast<const char*>(k_new) + j * U * D * 2,
+                              static_cast<const char*>(v_new) + j * U * D * 2, stream);
+    if (r != HYB_OK) return r;
+  }
+  return HYB_OK;
 }
 
 int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32_t* sel, float* out,

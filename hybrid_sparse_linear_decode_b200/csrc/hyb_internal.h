@@ -74,13 +74,13 @@ struct FusedParams {           // one decode (or, with q == null, the fold only)
   float scale;
 };
 
-struct AppendParams {       // write one token per unit at position T
-  const __nv_bfloat16* k_new; // [units][D]
+struct AppendParams {       // write n tokens per unit at positions [T, T + n)
+  const __nv_bfloat16* k_new; // [units][n][D]
   const __nv_bfloat16* v_new;
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   int64_t cap, T;
-  int32_t units;
+  int32_t units, n;
 };
 
 struct InitParams {

@@ -25,14 +25,14 @@ namespace {
 // state by the next decode's select kernel, which reads the caches.
 template <int D>
 __global__ void __launch_bounds__(D / 4) append_kernel(const AppendParams p) {
-  const int unit = blockIdx.x, tid = threadIdx.x;
+  const int unit = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;  // token j of the chunk
   if (tid == 0) pdl_wait_primary();  // the previous decode may still read these caches' rows
   __syncthreads();
   pdl_allow_dependents();
   const bool is_v = tid >= D / 8;
   const int e = (tid % (D / 8)) * 8;
-  const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + (int64_t)unit * D + e;
-  __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e;
+  const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + ((int64_t)unit * p.n + j) * D + e;
+  __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T + j) * D + e;
   *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
 }
 
@@ -168,7 +168,7 @@ cudaError_t prepare_state(int D) {
 
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.units);
+  cfg.gridDim = dim3(p.units, p.n);
   cfg.blockDim = dim3(D / 4);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

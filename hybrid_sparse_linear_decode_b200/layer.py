@@ -129,6 +129,33 @@ class HybridAttentionLayer:
             assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == (c.batch, c.n_kv_heads, c.head_dim)
         A.hyb_attn_append(self.ctx, k_new.data_ptr(), v_new.data_ptr(), _stream(stream))
 
+    def append_chunk(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+        """Append n tokens per unit in one launch: k_new, v_new [B][Hkv][n][d]."""
+        c = self.cfg
+        n = k_new.shape[2]
+        for t in (k_new, v_new):
+            assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == (c.batch, c.n_kv_heads, n, c.head_dim)
+        A.hyb_attn_append_chunk(self.ctx, k_new.data_ptr(), v_new.data_ptr(), n, _stream(stream))
+
+    def decode_chunk(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                     out: torch.Tensor | None = None, sel_out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+        """n consecutive decode + append steps: q [n][B][Hq][d], k_new, v_new
+        [n][B][Hkv][d]; row j attends to the history and the chunk's tokens
+        before j.  Returns out [n][B][Hq][d]."""
+        c = self.cfg
+        n = q.shape[0]
+        assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.shape == (n, c.batch, c.n_q_heads, c.head_dim)
+        for t in (k_new, v_new):
+            assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == (n, c.batch, c.n_kv_heads, c.head_dim)
+        if out is None:
+            out = torch.empty((n, c.batch, c.n_q_heads, c.head_dim), dtype=torch.float32, device=q.device)
+        if sel_out is not None:
+            assert sel_out.dtype == torch.int32 and sel_out.shape == (n, c.batch, c.n_kv_heads, c.top_k)
+        A.hyb_attn_decode_chunk(self.ctx, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), n, out.data_ptr(),
+                                _ptr(sel_out), _stream(stream))
+        return out
+
     def sync_state(self, stream=None) -> None:
         """Fold the evictions since the last decode into H, zk, zv, n, mu, var."""
         A.hyb_attn_sync_state(self.ctx, _stream(stream))

@@ -174,6 +174,17 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
  * (null or misaligned pointers), HYB_ECAPACITY (T == capacity), HYB_ECUDA. */
 int hyb_attn_append(hyb_attn_ctx* ctx, const void* k_new, const void* v_new, cudaStream_t stream);
 
+/* Append n >= 1 tokens per unit in one launch (a prefill continuation):
+ * k_new, v_new bf16 [B][Hkv][n][d], token j written at position T + j; then
+ * T += n.  Equivalent to n calls of hyb_attn_append: every token that leaves the
+ * window is folded by the next decode (or hyb_attn_sync_state) into H, zk, zv,
+ * n and its block's statistics, in position order (SPLA "Recurrence"; several
+ * evicted tokens make a small dense K^T V update of H).  Errors: HYB_EINVAL
+ * (null or misaligned pointers, n < 1 or n > 65535), HYB_ECAPACITY
+ * (T + n > capacity), HYB_ECUDA. */
+int hyb_attn_append_chunk(hyb_attn_ctx* ctx, const void* k_new, const void* v_new, int32_t n,
+                          cudaStream_t stream);
+
 /* Fold every token evicted since the last decode into the state arrays, so that
  * they describe L = [S, T - W) exactly (for a checkpoint, or to read them).  A
  * no-op when nothing is pending.  Errors: HYB_EINVAL, HYB_ECUDA. */
@@ -202,6 +213,19 @@ int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_o
  * [0, T) as stored before the call.  Errors: those of both calls. */
 int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, const void* v_new,
                            float* out, int32_t* sel_out, float* scores_out, cudaStream_t stream);
+
+/* n decode steps of n consecutive new tokens (speculative verification of a
+ * draft of n tokens): row j decodes q[j] at length T + j -- it attends to the
+ * stored history and to the chunk's tokens 0 .. j-1, with its own window, block
+ * scores and top-k -- and then appends token j; T += n in all.  Identical to n
+ * calls of hyb_attn_decode_append (one launch each, chained).
+ *   q       bf16 [n][B][Hq][d]     k_new, v_new  bf16 [n][B][Hkv][d]
+ *   out     fp32 [n][B][Hq][d]     sel_out       int32 [n][B][Hkv][top_k] or NULL
+ * Errors: HYB_EINVAL (null or misaligned pointers, n < 1), HYB_ESTATE (T == 0),
+ * HYB_ECAPACITY (T + n > capacity), HYB_ECUDA.  On an error at row j, rows
+ * before j have been decoded and appended. */
+int hyb_attn_decode_chunk(hyb_attn_ctx* ctx, const void* q, const void* k_new, const void* v_new, int32_t n,
+                          float* out, int32_t* sel_out, cudaStream_t stream);
 
 /* As hyb_attn_decode, with the block selection given by the caller instead of
  * the top-k: sel int32 [B][Hkv][top_k], each row ascending and distinct, -1

@@ -36,6 +36,18 @@ class Workload:
     block_offset_std: float = 0.0  # per-block key offset N(0, std^2), positions >= n_sink
     seed: int = 0
     appends_after_decode: int = 0  # extra appends after the decode steps (parity only)
+    # per-layer (top_k, window), cycled over the layers; empty: every layer has
+    # top_k and window above
+    layer_budgets: tuple = ()
+
+    def for_layer(self, layer: int) -> "Workload":
+        """The workload as layer `layer` sees it: its own top-k and window when
+        the budgets vary by layer (the generators draw the same values for the
+        same positions either way)."""
+        if not self.layer_budgets:
+            return self
+        k, win = self.layer_budgets[layer % len(self.layer_budgets)]
+        return dataclasses.replace(self, top_k=k, window=win, layer_budgets=())
 
     @property
     def group(self) -> int:
@@ -81,7 +93,7 @@ def _w(**kw) -> Workload:
     return Workload(**kw)
 
 
-# The five workloads.  Names describe shape and context length.
+# The workloads.  Names describe shape and context length.
 WORKLOADS = {
     "tiny": _w(name="tiny", batch=1, layers=1, n_q_heads=4, n_kv_heads=1, head_dim=64,
                T0=1024, block_size=32, n_sink=4, window=64, top_k=4, steps=1,
@@ -93,6 +105,13 @@ WORKLOADS = {
                                   n_q_heads=32, n_kv_heads=8, head_dim=128, T0=32768,
                                   block_size=64, n_sink=4, window=1024, top_k=16, steps=1,
                                   head_scale=True),
+    # per-layer budgets (k, W) varying over the layers: the knob a layer-wise
+    # budget allocation sets (the allocation itself needs calibration data)
+    "llama8b_32layers_b8_32k_budgets": _w(name="llama8b_32layers_b8_32k_budgets", batch=8, layers=32,
+                                          n_q_heads=32, n_kv_heads=8, head_dim=128, T0=32768,
+                                          block_size=64, n_sink=4, window=1024, top_k=16, steps=1,
+                                          head_scale=True,
+                                          layer_budgets=((8, 512), (16, 1024), (24, 1536), (32, 2048))),
     "llama8b_32layers_b4_128k": _w(name="llama8b_32layers_b4_128k", batch=4, layers=32,
                                    n_q_heads=32, n_kv_heads=8, head_dim=128, T0=131072,
                                    block_size=64, n_sink=4, window=2048, top_k=32, steps=1,

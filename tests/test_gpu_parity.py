@@ -228,3 +228,71 @@ def test_unwritten_rows_past_T_do_not_leak(kw):
     c.append(kw["n_append"])
     full_check(c, c.random_q())
     assert c.layer.status() == 0
+
+
+@pytest.mark.parametrize("kw,n", [
+    (dict(T0=600, n_append=64), 64),                                  # a block's worth, across a boundary
+    (dict(T0=600, n_append=300, capacity=1000), 300),                 # one chunk evicts many blocks
+    (dict(T0=40, S=4, W=64, n_append=50), 50),                        # the chunk starts the eviction
+    (dict(B=2, Hq=16, Hkv=4, T0=1500, Bk=64, W=100, k=6, n_append=129), 129),
+    (dict(d=64, T0=700, n_append=7), 7),
+])
+def test_append_chunk_matches_oracle(kw, n):
+    """n tokens appended in one launch: the cache rows are the host's bits, and
+    the next decode (which folds every token the chunk evicted) and the state
+    match the oracle's definitions at the new length."""
+    import torch
+    from harness import to_device_bf16
+    c = _case(**kw)
+    dev = c.layer.device
+    kb = to_device_bf16(np.ascontiguousarray(c.Kb[:, :, c.T:c.T + n]), dev)
+    vb = to_device_bf16(np.ascontiguousarray(c.Vb[:, :, c.T:c.T + n]), dev)
+    c.layer.append_chunk(kb, vb)
+    c.T += n
+    assert c.layer.T == c.T
+    torch.cuda.synchronize()
+    got = c.layer.k_cache[:, :, :c.T].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, c.Kb[:, :, :c.T].astype(np.uint16))
+    full_check(c, c.random_q())
+    assert c.layer.status() == 0
+    check_state(c)
+
+
+@pytest.mark.parametrize("kw,n", [
+    (dict(T0=600, n_append=8), 8),
+    (dict(T0=4 + 64 + 32 * 5 - 3, n_append=6), 6),                   # the chunk completes a block
+    (dict(B=2, Hq=16, Hkv=4, T0=1500, Bk=64, W=100, k=6, n_append=5), 5),
+    (dict(T0=70, S=4, W=64, n_append=4), 4),                          # eviction starts inside the chunk
+])
+def test_decode_chunk_rows_match_oracle(kw, n):
+    """Speculative verification of n draft tokens: row j is the decode at length
+    T + j (the chunk's tokens before j included), against the oracle at that
+    length; the state after the chunk against the oracle at T + n."""
+    import torch
+    from harness import to_device_bf16
+    c = _case(**kw)
+    dev = c.layer.device
+    qs = np.stack([c.random_q() for _ in range(n)])
+    q = to_device_bf16(qs, dev)
+    kb = to_device_bf16(np.ascontiguousarray(c.Kb[:, :, c.T:c.T + n].transpose(2, 0, 1, 3)), dev)
+    vb = to_device_bf16(np.ascontiguousarray(c.Vb[:, :, c.T:c.T + n].transpose(2, 0, 1, 3)), dev)
+    sel = torch.full((n, c.B, c.Hkv, c.k), -7, dtype=torch.int32, device=dev)
+    out = c.layer.decode_chunk(q, kb, vb, sel_out=sel)
+    torch.cuda.synchronize()
+    out, sel = out.cpu().numpy().astype(np.float64), sel.cpu().numpy()
+    T0 = c.T
+    for j in range(n):
+        c.T = T0 + j
+        refs, gots = [], []
+        for b in range(c.B):
+            for h in range(c.Hkv):
+                _, _, oscores = c.oracle_unit(qs[j], b, h)
+                check_selection(sel[j, b, h], oscores, c.k)
+                gsel = np.array([int(x) for x in sel[j, b, h] if x >= 0], dtype=np.int64)
+                ref, _, _ = c.oracle_unit(qs[j], b, h, sel=gsel)
+                refs.append(ref)
+                gots.append(out[j, b, h * c.G:(h + 1) * c.G])
+        check_outputs(np.array(gots), np.array(refs))
+    c.T = T0 + n
+    assert c.layer.T == c.T and c.layer.status() == 0
+    check_state(c)

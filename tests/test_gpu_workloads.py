@@ -22,6 +22,7 @@ class WorkloadLayer:
         import syngen.device as SD
         from hybrid_sparse_linear_decode_b200 import HybridAttentionLayer, make_config
         SD.build()
+        w = w.for_layer(layer)  # the layer's own top-k and window when budgets vary by layer
         self.w, self.l = w, layer
         self.n_app = w.capacity - w.T0 if n_app is None else n_app
         cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window,
@@ -138,6 +139,23 @@ def test_llama8b_32layers_b8_32k_sampled(layer):
     units = [(0, 0), (3, 5), (7, 7), (5, 2)]
     qb = wl.q_bits(0)
     out, sel = wl.decode(qb)
+    wl.check_units(qb, units, out, sel)
+    wl.append(0)
+    wl.check_state(units[:2])
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_llama8b_32layers_b8_32k_budgets_sampled(layer):
+    """Per-layer budgets: each layer its own top-k and window (k 8..32, W
+    512..2048), decoded, appended and checked against the oracle with that
+    layer's budget."""
+    w = C.get_workload("llama8b_32layers_b8_32k_budgets")
+    wl = WorkloadLayer(w, layer, n_app=1)
+    assert (wl.w.top_k, wl.w.window) == w.layer_budgets[layer]
+    units = [(0, 0), (4, 6), (7, 3)]
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    assert sel.shape[-1] == wl.w.top_k
     wl.check_units(qb, units, out, sel)
     wl.append(0)
     wl.check_state(units[:2])

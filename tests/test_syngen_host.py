@@ -118,3 +118,16 @@ def test_tiny_oracle_selects_planted_blocks():
     assert scores[tb.planted[0, 0]].min() > 4.5
     bg = np.delete(scores, tb.planted[0, 0])
     assert 1.0 < bg.mean() < 3.0
+
+
+def test_layer_budgets_view():
+    """A workload with per-layer budgets gives each layer its own (top_k,
+    window), cycled over the layers; one without gives every layer itself."""
+    from syngen import configs as C
+    w = C.get_workload("llama8b_32layers_b8_32k_budgets")
+    for l in range(w.layers):
+        v = w.for_layer(l)
+        assert (v.top_k, v.window) == w.layer_budgets[l % len(w.layer_budgets)]
+        assert v.layer_budgets == () and v.T0 == w.T0 and v.capacity == w.capacity
+    base = C.get_workload("llama8b_32layers_b8_32k")
+    assert base.for_layer(5) is base
