@@ -48,6 +48,11 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (smaller instances for profiling)")
+    ap.add_argument("--mode", default="decode", choices=["decode", "spec", "prefill"],
+                    help="decode: one decode + append per layer and step; spec: hyb_attn_decode_chunk of "
+                         "--chunk draft tokens per layer and step; prefill: hyb_attn_append_chunk of --chunk "
+                         "tokens, then one decode, per layer and step")
+    ap.add_argument("--chunk", type=int, default=4)
     return ap.parse_args()
 
 
@@ -185,14 +190,15 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- native arm
 
 class Bench:
-    def __init__(self, w, n_steps, device):
+    def __init__(self, w, n_steps, device, mode="decode", chunk=1):
         import torch
         import syngen.device as SD
         from syngen import host as SH
         from hybrid_sparse_linear_decode_b200 import HybridAttentionLayer, make_config
         self.w, self.device = w, device
         self.n_steps = n_steps
-        n_app = self.n_steps
+        self.mode, self.chunk = mode, (chunk if mode != "decode" else 1)
+        n_app = self.n_steps * self.chunk
 
         def cfg_of(l):  # the layer's own top-k and window when budgets vary by layer
             wl = w.for_layer(l)
@@ -211,32 +217,50 @@ class Bench:
             ak = torch.empty(shp, dtype=torch.bfloat16, device=device)
             av = torch.empty(shp, dtype=torch.bfloat16, device=device)
             SD.fill_kv(w, tb, ak, av, w.T0, w.T0 + n_app, t_out0=w.T0)
-            # per-step appended tokens, contiguous [step][B][Hkv][d]
-            self.app_k.append(ak.permute(2, 0, 1, 3).contiguous())
-            self.app_v.append(av.permute(2, 0, 1, 3).contiguous())
+            if self.mode == "prefill":  # per step a chunk, contiguous [step][B][Hkv][chunk][d]
+                shp5 = (w.batch, w.n_kv_heads, self.n_steps, self.chunk, w.head_dim)
+                self.app_k.append(ak.view(shp5).permute(2, 0, 1, 3, 4).contiguous())
+                self.app_v.append(av.view(shp5).permute(2, 0, 1, 3, 4).contiguous())
+            else:  # per appended token, contiguous [token][B][Hkv][d]
+                self.app_k.append(ak.permute(2, 0, 1, 3).contiguous())
+                self.app_v.append(av.permute(2, 0, 1, 3).contiguous())
             del ak, av
             qs = []
             for s in range(n_q):
                 qb = SH.q_bits(w, l, s)
                 qs.append(torch.from_numpy(qb.view("int16")).to(device).view(torch.bfloat16))
+            if self.mode == "spec":  # one chunk of draft queries [chunk][B][Hq][d], reused every step
+                qs = [torch.stack([qs[i % n_q] for i in range(self.chunk)]).contiguous()]
             self.q.append(qs)
             L.init(w.T0)
             self.layers.append(L)
         self.out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=device)
+        self.out_chunk = torch.empty((self.chunk, w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32,
+                                     device=device)
         torch.cuda.synchronize()
         self.step_idx = 0
 
     def step(self):
         s = self.step_idx
+        n = self.chunk
         for l, L in enumerate(self.layers):
             q = self.q[l][s % len(self.q[l])]
-            L.decode_append(q, self.app_k[l][s], self.app_v[l][s], out=self.out)
+            if self.mode == "spec":
+                L.decode_chunk(q, self.app_k[l][s * n:(s + 1) * n], self.app_v[l][s * n:(s + 1) * n],
+                               out=self.out_chunk)
+            elif self.mode == "prefill":
+                L.append_chunk(self.app_k[l][s], self.app_v[l][s])
+                L.decode(q, out=self.out)
+            else:
+                L.decode_append(q, self.app_k[l][s], self.app_v[l][s], out=self.out)
         self.step_idx += 1
 
     def launches_per_step(self):
         """Kernels per step: one fused decode launch per layer (the append's
-        cache write and the fold of the previous evictions ride in it)."""
-        return len(self.layers)
+        cache write and the fold of the previous evictions ride in it); spec:
+        one per draft token; prefill: the chunk's cache write and one decode."""
+        per = {"decode": 1, "spec": self.chunk, "prefill": 2}[self.mode]
+        return per * len(self.layers)
 
 
 def run_native(args, rank, world):
@@ -246,15 +270,20 @@ def run_native(args, rank, world):
     device = torch.device("cuda", torch.cuda.current_device())
     w = rank_workload(C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {})), rank)
     K, Wm = args.steps, args.warmup
-    Kk = min(K, 20)                      # steps of the attention-kernel timing pass
-    Ke = 0 if args.no_e2e else min(K, 20)  # steps of the end-to-end pass
-    b = Bench(w, Wm + K + Kk + Ke, device)
-    T_mid = w.T0 + Wm + K // 2
+    mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
+    Kk = min(K, 20) if mode == "decode" else 0  # steps of the pass timing each launch on its own
+    Ke = 0 if (args.no_e2e or mode != "decode") else min(K, 20)  # steps of the end-to-end pass
+    b = Bench(w, Wm + K + Kk + Ke, device, mode, chunk)
+    T_mid = w.T0 + (Wm + K // 2) * chunk
     step_dec = step_bytes = 0
     for l in range(w.layers):  # each layer with its own budget
         dec_b, app_b = algorithmic_bytes(w.for_layer(l), T_mid)
-        step_dec += w.units_per_layer * dec_b
-        step_bytes += w.units_per_layer * (dec_b + app_b)
+        if mode == "prefill":  # the chunk's rows and evicted tokens, the state written back once, one decode
+            d = w.head_dim
+            app_b = chunk * 8 * d + (d * d + 2 * d + 1) * 4 + (-(-chunk // w.block_size) + 1) * 2 * d * 4
+        per_step = chunk if mode == "spec" else 1  # decodes per layer and step
+        step_dec += w.units_per_layer * dec_b * per_step
+        step_bytes += w.units_per_layer * (dec_b + app_b) * per_step
     flush = step_bytes < 4 * 126e6      # the step's data would otherwise stay in L2
     scratch = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if flush else None
 
@@ -320,7 +349,7 @@ def run_native(args, rank, world):
         for e0, e1 in pool[i]:
             kern_ms += e0.elapsed_time(e1)
             n_kern += 1
-    isolated_ms = kern_ms / n_kern
+    isolated_ms = kern_ms / n_kern if n_kern else None
     # In the timed region the step is exactly one launch of the fused kernel per
     # layer, back to back: its average duration there is the step time over the
     # launches, and its algorithmic bytes those of one layer's decode + append.
@@ -329,12 +358,12 @@ def run_native(args, rank, world):
     launch_bytes = step_bytes // n_launch
     hbm_peak, peak_kind = peaks()
     achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
-    isolated = launch_bytes / (isolated_ms * 1e-3) / 1e9
+    isolated = launch_bytes / (isolated_ms * 1e-3) / 1e9 if isolated_ms else None
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # ---- e2e through the host-buffer entry point (pinned host q / k / v / out)
     e2e = None
-    if not args.no_e2e:
+    if Ke > 0:
         qh = [[t.cpu().pin_memory() for t in qs] for qs in b.q]
         kh = [t.cpu().pin_memory() for t in b.app_k]
         vh = [t.cpu().pin_memory() for t in b.app_v]
@@ -381,8 +410,9 @@ def run_native(args, rank, world):
             **({"layer_budgets_k_W": [list(x) for x in w.layer_budgets]} if w.layer_budgets else {}),
             "l2": "flushed between timed steps (512 MB write)" if flush else "step data >> L2 (no flush)",
             "parallelism": f"replicas x{world} (independent units per GPU)",
+            **({"mode": mode, "chunk": chunk} if mode != "decode" else {}),
         },
-        "attention_tokens_per_s": round(world * steps_s * w.batch, 3),
+        "attention_tokens_per_s": round(world * steps_s * w.batch * chunk, 3),
         "context_tokens_per_s": round(world * steps_s * w.batch * w.layers * T_mid, 1),
         "achieved_gbs_step": round(step_gbs, 1),
         "pct_of_hbm_peak_step": round(100 * step_gbs / hbm_peak, 2),
@@ -394,8 +424,8 @@ def run_native(args, rank, world):
                      "traffic": measured_traffic(w.name), "bytes_per_launch": launch_bytes,
                      "decode_bytes_per_launch": step_dec // n_launch,
                      "avg_launch_us": round(launch_ms * 1e3, 3),
-                     "isolated_launch_us": round(isolated_ms * 1e3, 3),
-                     "isolated_frac": round(isolated / hbm_peak, 4)},
+                     "isolated_launch_us": round(isolated_ms * 1e3, 3) if isolated_ms else None,
+                     "isolated_frac": round(isolated / hbm_peak, 4) if isolated else None},
         "e2e": e2e,
         "gpu_launches": b.launches_per_step() * K,
         "clocks": clocks,
@@ -508,12 +538,13 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_native(args, rank, world)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and args.mode != "prefill":
         from syngen import configs as C
         w = C.get_workload(args.workload)
         s, desc = oracle_sample(w, args.cpu_sample_seconds)
-        res["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": "steps/s", "cores": cpu_cores(),
-                               "kind": "oracle", "sample": desc}
+        n = args.chunk if args.mode == "spec" else 1  # a spec step is n decode + append steps
+        res["cpu_baseline"] = {"value": round(1.0 / (n * s), 6), "unit": "steps/s", "cores": cpu_cores(),
+                               "kind": "oracle", "sample": desc + (f"; x{n} decode + append per step" if n > 1 else "")}
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
