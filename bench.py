@@ -258,8 +258,9 @@ class Bench:
     def launches_per_step(self):
         """Kernels per step: one fused decode launch per layer (the append's
         cache write and the fold of the previous evictions ride in it); spec:
-        one per draft token; prefill: the chunk's cache write and one decode."""
-        per = {"decode": 1, "spec": self.chunk, "prefill": 2}[self.mode]
+        one per draft token; prefill: the chunk's cache write, the dense fold of
+        the tokens it evicted (4 or more) and one decode."""
+        per = {"decode": 1, "spec": self.chunk, "prefill": 2 + (self.chunk >= 4)}[self.mode]
         return per * len(self.layers)
 
 

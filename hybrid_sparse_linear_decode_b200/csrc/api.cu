@@ -245,8 +245,36 @@ FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   return fp;
 }
 
+// Several pending evictions (a chunked append, or many appends since the last
+// fold): one dense pass of fold_kernel over them, so that the decode kernel
+// folds at most a few tokens itself.
+int fold_pending(hyb_attn_ctx* x, const Geometry& g, cudaStream_t stream) {
+  if (g.ev_end - x->folded_end < kFoldKernelMin) return HYB_OK;
+  FoldParams p{};
+  p.k_cache = static_cast<const __nv_bfloat16*>(x->buf.k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(x->buf.v_cache);
+  p.H = x->buf.H;
+  p.zk = x->buf.zk;
+  p.zv = x->buf.zv;
+  p.n = x->buf.n;
+  p.mu = x->buf.mu;
+  p.var = x->buf.var;
+  p.cap = x->cfg.capacity;
+  p.max_blocks = x->ck.max_blocks > 0 ? x->ck.max_blocks : 1;
+  p.fb = x->folded_end;
+  p.fe = g.ev_end;
+  p.units = x->ck.units;
+  p.S = x->cfg.n_sink;
+  p.Bk = x->cfg.block_size;
+  const cudaError_t e = launch_fold(p, x->ck.D, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  x->folded_end = g.ev_end;
+  return HYB_OK;
+}
+
 // One decode at the current T: one launch of the fused kernel (writes the
-// appended token when k_new is given).
+// appended token when k_new is given), after fold_kernel when several
+// evictions are pending.
 int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_given, int32_t* sel_out,
                 float* scores_out, const void* k_new, const void* v_new, cudaStream_t stream) {
   if (x == nullptr || q == nullptr || out == nullptr) return HYB_EINVAL;
@@ -259,6 +287,8 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   if (x->T == 0) return HYB_ESTATE;
   if (k_new != nullptr && x->T >= x->cfg.capacity) return HYB_ECAPACITY;
   const Geometry g = geometry(x->cfg, x->T);
+  const int rf = fold_pending(x, g, stream);
+  if (rf != HYB_OK) return rf;
   FusedParams fp = fused_params(x, g);
   fp.q = static_cast<const __nv_bfloat16*>(q);
   if (scores_out) fp.scores = scores_out;
@@ -431,6 +461,7 @@ int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
   if (x == nullptr) return HYB_EINVAL;
   const Geometry g = geometry(x->cfg, x->T);
   if (g.ev_end <= x->folded_end) return HYB_OK;  // nothing evicted since the last fold
+  if (g.ev_end - x->folded_end >= kFoldKernelMin) return fold_pending(x, g, stream);
   FusedParams fp = fused_params(x, g);           // q == null: fold only
   const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -83,6 +83,18 @@ struct AppendParams {       // write n tokens per unit at positions [T, T + n)
   int32_t units, n;
 };
 
+struct FoldParams {         // fold the evicted positions [fb, fe) of every unit into the state
+  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* v_cache;
+  float* H; float* zk; float* zv; float* n; float* mu; float* var;
+  int64_t cap, max_blocks;
+  int64_t fb, fe;
+  int32_t units, S, Bk;
+};
+// pending evictions from which a decode or a state sync folds them with
+// fold_kernel (one dense pass) instead of inside the decode kernel
+constexpr int64_t kFoldKernelMin = 4;
+
 struct InitParams {
   const __nv_bfloat16* k_cache;
   const __nv_bfloat16* v_cache;
@@ -105,6 +117,7 @@ cudaError_t prepare_fused(int D);
 // clusters of c CTAs of the decode kernel the current device can hold at once (0: none)
 int fused_max_clusters(int D, int c);
 cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s);
+cudaError_t launch_fold(const FoldParams& p, int D, cudaStream_t s);
 // per device, before the first launch: shared-memory size, cluster and carveout attributes
 cudaError_t prepare_state(int D);
 

@@ -36,6 +36,104 @@ __global__ void __launch_bounds__(D / 4) append_kernel(const AppendParams p) {
   *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
 }
 
+// ---------------------------------------------------------------- chunk fold
+// The evicted positions [fb, fe) of every unit folded into the state in one
+// pass, for several pending tokens (a chunked append, or many appends between
+// decodes; SPLA "Recurrence" applied to a run of tokens is a small dense
+// update).  One CTA per unit: H += K^T V over the run (fp32 thread tiles of the
+// D x D outer-product sum, keys / values staged through shared memory 32
+// tokens at a time), zk += sum k, zv += sum v, n += count; then, per block the
+// run touches, the block's mean and population variance merged with those of
+// its new tokens by the pairwise combination of Chan, Golub and LeVeque
+// (n = na + nb, mean = ma + d nb / n, M2 = M2a + M2b + d^2 na nb / n, with
+// d = mb - ma), in fp64.  The tokens of a block folded before fb are exactly
+// those before fb, as folds go in position order.
+template <int D>
+__global__ void __launch_bounds__(256) fold_kernel(const FoldParams p) {
+  constexpr int RT = D / 16;
+  __shared__ __align__(16) float ks[32][D];
+  __shared__ __align__(16) float vs[32][D];
+  const int unit = blockIdx.x, tid = threadIdx.x;
+  if (tid == 0) pdl_wait_primary();  // the caches' rows and the state may come from the previous grid
+  __syncthreads();
+  pdl_allow_dependents();
+  const int tr = tid / 16, tc = tid % 16;
+  const int64_t ub = (int64_t)unit * p.cap;
+  float acc[RT][RT];
+#pragma unroll
+  for (int i = 0; i < RT; ++i)
+#pragma unroll
+    for (int j = 0; j < RT; ++j) acc[i][j] = 0.f;
+  float zacc = 0.f;
+  for (int64_t tt = p.fb; tt < p.fe; tt += 32) {
+    const int n = (int)min((int64_t)32, p.fe - tt);
+    for (int e = tid; e < 32 * D; e += 256) {
+      const int r = e / D, c = e % D;
+      float kv = 0.f, vv = 0.f;
+      if (r < n) {
+        kv = __bfloat162float(p.k_cache[(ub + tt + r) * D + c]);
+        vv = __bfloat162float(p.v_cache[(ub + tt + r) * D + c]);
+      }
+      ks[r][c] = kv;
+      vs[r][c] = vv;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < 32; ++r) {
+      float a[RT], b[RT];
+#pragma unroll
+      for (int i = 0; i < RT; ++i) {
+        a[i] = ks[r][tr * RT + i];
+        b[i] = vs[r][tc * RT + i];
+      }
+#pragma unroll
+      for (int i = 0; i < RT; ++i)
+#pragma unroll
+        for (int j = 0; j < RT; ++j) acc[i][j] += a[i] * b[j];
+    }
+    if (tid < D) {
+      for (int r = 0; r < n; ++r) zacc += ks[r][tid];
+    } else if (tid < 2 * D) {
+      for (int r = 0; r < n; ++r) zacc += vs[r][tid - D];
+    }
+    __syncthreads();
+  }
+  float* H = p.H + (int64_t)unit * D * D;
+#pragma unroll
+  for (int i = 0; i < RT; ++i)
+#pragma unroll
+    for (int j = 0; j < RT; ++j) H[(int64_t)(tr * RT + i) * D + tc * RT + j] += acc[i][j];
+  if (tid < D) p.zk[(int64_t)unit * D + tid] += zacc;
+  else if (tid < 2 * D) p.zv[(int64_t)unit * D + tid - D] += zacc;
+  if (tid == 0) p.n[unit] += (float)(p.fe - p.fb);
+  if (tid < D) {  // one channel per thread
+    const __nv_bfloat16* kc = p.k_cache + ub * D + tid;
+    const int64_t j0 = (p.fb - p.S) / p.Bk, j1 = (p.fe - 1 - p.S) / p.Bk;
+    for (int64_t j = j0; j <= j1; ++j) {
+      const int64_t bs = p.S + j * p.Bk;
+      const int64_t a0 = max(bs, p.fb), a1 = min(bs + (int64_t)p.Bk, p.fe);
+      const double na = (double)(a0 - bs), nb = (double)(a1 - a0);
+      double sb = 0.0, qb = 0.0;
+      for (int64_t t = a0; t < a1; ++t) sb += (double)__bfloat162float(kc[t * D]);
+      const double mb = sb / nb;
+      for (int64_t t = a0; t < a1; ++t) {
+        const double d = (double)__bfloat162float(kc[t * D]) - mb;
+        qb += d * d;
+      }
+      const int64_t so = ((int64_t)unit * p.max_blocks + j) * D + tid;
+      double mu = mb, m2 = qb, nn = nb;
+      if (na > 0.0) {
+        const double ma = (double)p.mu[so], m2a = (double)p.var[so] * na, d = mb - ma;
+        nn = na + nb;
+        mu = ma + d * nb / nn;
+        m2 = m2a + qb + d * d * na * nb / nn;
+      }
+      p.mu[so] = (float)mu;
+      p.var[so] = (float)(m2 / nn);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- init
 // (1) H, zk, zv over L: grid (ceil(|L| / tokens_per_cta), units).  Each CTA
 //     accumulates its token range in fp32 (thread tile RT x RT of the D x D
@@ -155,6 +253,7 @@ __global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) 
 
 cudaError_t prepare_state(int D) {
   const void* fs[] = {D == 128 ? (const void*)append_kernel<128> : (const void*)append_kernel<64>,
+                      D == 128 ? (const void*)fold_kernel<128> : (const void*)fold_kernel<64>,
                       D == 128 ? (const void*)init_linear_kernel<128> : (const void*)init_linear_kernel<64>,
                       D == 128 ? (const void*)init_stats_kernel<128> : (const void*)init_stats_kernel<64>,
                       D == 128 ? (const void*)init_finalize_kernel<128> : (const void*)init_finalize_kernel<64>};
@@ -164,6 +263,20 @@ cudaError_t prepare_state(int D) {
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_fold(const FoldParams& p, int D, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.units);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) return cudaLaunchKernelEx(&cfg, fold_kernel<128>, p);
+  return cudaLaunchKernelEx(&cfg, fold_kernel<64>, p);
 }
 
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {

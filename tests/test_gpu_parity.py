@@ -64,6 +64,8 @@ def test_all_selected_is_softmax_and_q0_is_mean():
 @pytest.mark.parametrize("kw,n", [
     (dict(T0=600, Bk=32, W=64), 40),
     (dict(T0=4 + 64 + 32 * 3, Bk=32, W=64), 3),               # the first append opens a new block
+    (dict(T0=601, Bk=32, W=64), 2),                           # two pending: folded inside the decode kernel
+    (dict(T0=601, Bk=32, W=64), 4),                           # four pending: the dense fold pass
     (dict(T0=10, S=4, W=16, Bk=8), 40),                       # grows from sinks-only through eviction
     (dict(T0=200, W=0, Bk=8), 20),                            # W = 0 evicts the appended token itself
     (dict(T0=300, S=0, W=5, Bk=7, d=64), 30),
