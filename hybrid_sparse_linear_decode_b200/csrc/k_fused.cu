@@ -810,6 +810,22 @@ __device__ __forceinline__ uint32_t kth_lane_max(uint32_t v, int lane, int k) {
   return __shfl_sync(kFull, v, __ffs(__ballot_sync(kFull, r == k - 1)) - 1);
 }
 
+// The k-th largest (k <= 32) of the 64 values {v0, v1} of the 32 lanes, in the
+// strict order by value, then lower lane, then v0 before v1.
+__device__ __forceinline__ uint32_t kth_of_lane_pairs(uint32_t v0, uint32_t v1, int lane, int k) {
+  int r0 = 0, r1 = 0;  // values ordered before (lane, v0) / before (lane, v1)
+#pragma unroll
+  for (int l = 0; l < 32; ++l) {
+    const uint32_t o0 = __shfl_sync(kFull, v0, l), o1 = __shfl_sync(kFull, v1, l);
+    r0 += (o0 > v0 || (o0 == v0 && l < lane)) ? 1 : 0;
+    r0 += (o1 > v0 || (o1 == v0 && l < lane)) ? 1 : 0;
+    r1 += (o0 > v1 || (o0 == v1 && l <= lane)) ? 1 : 0;
+    r1 += (o1 > v1 || (o1 == v1 && l < lane)) ? 1 : 0;
+  }
+  const uint32_t b0 = __ballot_sync(kFull, r0 == k - 1), b1 = __ballot_sync(kFull, r1 == k - 1);
+  return b0 ? __shfl_sync(kFull, v0, __ffs(b0) - 1) : __shfl_sync(kFull, v1, __ffs(b1) - 1);
+}
+
 // The k <= 32 largest of the nb scores in shared memory (sc) by one warp, ties
 // to the lower index.  Lane l's keys are those of blocks l, l + 32, ...; at
 // least k lanes hold a key (nb > k), so the k-th largest of the 32 lane maxima,
@@ -818,7 +834,10 @@ __device__ __forceinline__ uint32_t kth_lane_max(uint32_t v, int lane, int k) {
 // row of 32 blocks), packed as key << 32 | ~index so that one comparison
 // orders by key and then by lower index, and ranked among themselves; the
 // ranks < k are written to dst[0, k) (and copy) in block order.  Returns false,
-// writing nothing, when more than cap keys are >= tau.
+// writing nothing, when more than cap keys are >= tau.  Above 512 blocks the
+// bound is the k-th largest of the lanes' two largest keys (also keys, so still
+// at most the k-th largest key, and much closer to it: ~35 candidates of 2016
+// instead of ~110, whose exact ranking costs the square of their count).
 __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_t* dst, int32_t* copy,
                                           unsigned long long* cand, int cap, bool& nan_out) {
   constexpr int kRows = 16;  // rows of 32 blocks per pass
@@ -851,6 +870,7 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
       m += __popc(bal[i]);
     }
   } else {
+    uint32_t lsec = 0u;  // the lane's second largest key (0, below every key, if it has one key)
 #pragma unroll 1
     for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
 #pragma unroll
@@ -858,11 +878,13 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
         const int j = r0 + lane + 32 * i;
         const float f = j < nb ? sc[j] : 0.f;
         nan |= f != f;
-        if (j < nb) lmax = max(lmax, float_key(f));
+        const uint32_t u = j < nb ? float_key(f) : 0u;
+        lsec = max(lsec, min(lmax, u));
+        lmax = max(lmax, u);
       }
     }
     nan_out = __any_sync(kFull, nan);
-    const uint32_t tau = kth_lane_max(lmax, lane, k);
+    const uint32_t tau = kth_of_lane_pairs(lmax, lsec, lane, k);
 #pragma unroll 1
     for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
       uint32_t kr[kRows], bal[kRows];

@@ -298,3 +298,40 @@ def test_decode_chunk_rows_match_oracle(kw, n):
     c.T = T0 + n
     assert c.layer.T == c.T and c.layer.status() == 0
     check_state(c)
+
+
+@pytest.mark.parametrize("nbk,copies,k,d", [
+    (700, (3, 150, 333, 480, 690), 3, 64),    # one unit: a cluster of 16 ranks, copies in different shares
+    (1300, (10, 11, 700, 1299), 2, 128),      # the second copy in the same share, the last in the last share
+])
+def test_ties_across_rank_shares_above_512_blocks(nbk, copies, k, d):
+    """Above 512 blocks (the selection's multi-pass path, its bound from the
+    lanes' two largest keys): blocks with identical scores, in different ranks'
+    shares of the scoring, must still go to the lowest indices."""
+    B, Hkv, S, W, Bk = 1, 1, 4, 32, 8
+    T0 = S + nbk * Bk + W
+    rng = np.random.default_rng(5)
+    Kf = rng.standard_normal((B, Hkv, T0, d))
+    Vf = rng.standard_normal((B, Hkv, T0, d))
+    blk = rng.standard_normal((Bk, d))
+    for j in copies:
+        Kf[0, 0, S + j * Bk:S + (j + 1) * Bk] = blk * 0.3 + 2.0
+    from harness import bf16_bits
+    c = Case(B, 4, Hkv, d, T0, Bk, S, W, k, kv_bits=(bf16_bits(Kf), bf16_bits(Vf)))
+    q = bf16_bits(np.abs(rng.standard_normal((1, 4, d))))
+    out, sel, scores = c.decode(q)
+    assert list(sel[0, 0]) == sorted(copies)[:k]
+    s = scores[0, 0]
+    assert all(s[j] == s[copies[0]] for j in copies)
+    full_check(c, q)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T0=4 + 64 + 8 * 900, Bk=8, W=64, k=20),                       # one unit, 900 blocks
+    dict(B=2, Hq=8, Hkv=2, T0=4 + 128 + 16 * 600, Bk=16, W=128, k=32),  # 4 units, k = 32
+    dict(d=64, T0=4 + 64 + 8 * 800, Bk=8, W=64, k=12),                 # head dim 64
+])
+def test_selection_above_512_blocks(kw):
+    c = _case(**kw)
+    full_check(c, c.random_q())
+    assert c.layer.status() == 0
