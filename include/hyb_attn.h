@@ -187,7 +187,9 @@ int hyb_attn_append_chunk(hyb_attn_ctx* ctx, const void* k_new, const void* v_ne
 
 /* Fold every token evicted since the last decode into the state arrays, so that
  * they describe L = [S, T - W) exactly (for a checkpoint, or to read them).  A
- * no-op when nothing is pending.  Errors: HYB_EINVAL, HYB_ECUDA. */
+ * no-op when nothing is pending; one launch otherwise (the dense fold pass when
+ * 4 or more tokens are pending, else the decode kernel in fold-only mode).
+ * Errors: HYB_EINVAL, HYB_ECUDA. */
 int hyb_attn_sync_state(hyb_attn_ctx* ctx, cudaStream_t stream);
 
 /* One decode step at the current length T for every unit:
@@ -201,7 +203,10 @@ int hyb_attn_sync_state(hyb_attn_ctx* ctx, cudaStream_t stream);
  * the tokens evicted since the previous decode, forms the global linear term
  * phi(q)^T state, selects the top-k, attends sinks, window and selected blocks
  * exactly (split-K over the cluster, with the selected blocks' (1 + s)
- * subtraction) and merges under the shared normaliser.
+ * subtraction) and merges under the shared normaliser.  When 4 or more evicted
+ * tokens are pending (a chunked append, or many appends since the last fold),
+ * a dense fold pass over them is launched first (H += K^T V over the run, zk,
+ * zv, n, and the touched blocks' statistics merged pairwise).
  * Errors: HYB_EINVAL (null or misaligned pointers), HYB_ESTATE (T == 0),
  * HYB_ECUDA. */
 int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out,
