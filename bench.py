@@ -464,14 +464,17 @@ def _oracle_units(w, n_units: int = 4, max_appends: int = 2048):
     return units
 
 
-def oracle_sample(w, seconds: float):
-    """Time the fp64 oracle's decode + append of whole units of the workload,
-    round robin over a few prepared units, for about `seconds` of CPU work;
-    returns seconds per full step (scaled by the units in a step) and a
-    description of the sample."""
+def oracle_sample(w, seconds: float, mode: str = "decode", chunk: int = 1):
+    """Time the fp64 oracle's decodes and appends of whole units of the
+    workload, round robin over a few prepared units, for about `seconds` of CPU
+    work; returns seconds per full step (scaled by the units in a step) and a
+    description of the sample.  A step per unit: decode + append; spec: chunk x
+    (decode + append); prefill: chunk appends and one decode (the oracle appends
+    one token at a time)."""
     units = _oracle_units(w)
-    spent, n = 0.0, 0
-    while spent < seconds:
+    t_dec = t_app = 0.0
+    n = 0
+    while t_dec + t_app < seconds:
         progressed = False
         for e in units:
             u, Kt, Vt, q, pos = e
@@ -479,18 +482,24 @@ def oracle_sample(w, seconds: float):
                 continue
             t0 = time.perf_counter()
             u.decode(q)
+            t1 = time.perf_counter()
             u.append(Kt[pos], Vt[pos])
-            spent += time.perf_counter() - t0
+            t2 = time.perf_counter()
+            t_dec += t1 - t0
+            t_app += t2 - t1
             e[4] = pos + 1
             n += 1
             progressed = True
         if not progressed:
             break
-    per_unit_step = spent / max(1, n)
+    d, a = t_dec / max(1, n), t_app / max(1, n)
+    per_unit_step = {"decode": d + a, "spec": chunk * (d + a), "prefill": chunk * a + d}[mode]
     units_per_step = w.layers * w.units_per_layer
-    return per_unit_step * units_per_step, (f"{n} unit-steps (decode+append of one (layer, b, kv-head) at "
-                                            f"{w.T0}+ tokens) round robin over {len(units)} units, "
-                                            f"scaled x{units_per_step} units per step")
+    what = {"decode": "decode + append", "spec": f"{chunk} x (decode + append)",
+            "prefill": f"{chunk} appends + decode"}[mode]
+    return per_unit_step * units_per_step, (f"{n} unit decode + append pairs of one (layer, b, kv-head) at "
+                                            f"{w.T0}+ tokens, round robin over {len(units)} units, timed "
+                                            f"apart; a step = {what} per unit, x{units_per_step} units")
 
 
 def cpu_cores():
@@ -503,13 +512,14 @@ def cpu_cores():
 
 def run_reference(args, rank, world):
     from syngen import configs as C
-    w = C.get_workload(args.workload)
+    w = C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {}))
+    mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
     oracle_sample(w, 0.2)   # prepare the units, warm numpy / BLAS
     samples = []
     for _ in range(args.warmup):
         oracle_sample(w, 0.05)
     for _ in range(args.steps):
-        s, desc = oracle_sample(w, args.cpu_sample_seconds / max(1, args.steps))
+        s, desc = oracle_sample(w, args.cpu_sample_seconds / max(1, args.steps), mode, chunk)
         samples.append(s)
     ms = 1e3 * statistics.mean(samples)
     v = 1e3 / ms
@@ -517,7 +527,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name},
+        "config": {"workload": w.name, "layers": w.layers, **({"mode": mode, "chunk": chunk} if mode != "decode" else {})},
         "cpu_baseline": {"value": round(v, 6), "unit": "steps/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(v, 6), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -539,13 +549,12 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_native(args, rank, world)
-    if rank == 0 and not args.no_cpu_baseline and args.mode != "prefill":
+    if rank == 0 and not args.no_cpu_baseline:
         from syngen import configs as C
-        w = C.get_workload(args.workload)
-        s, desc = oracle_sample(w, args.cpu_sample_seconds)
-        n = args.chunk if args.mode == "spec" else 1  # a spec step is n decode + append steps
-        res["cpu_baseline"] = {"value": round(1.0 / (n * s), 6), "unit": "steps/s", "cores": cpu_cores(),
-                               "kind": "oracle", "sample": desc + (f"; x{n} decode + append per step" if n > 1 else "")}
+        w = C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {}))
+        s, desc = oracle_sample(w, args.cpu_sample_seconds, args.mode, args.chunk if args.mode != "decode" else 1)
+        res["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": "steps/s", "cores": cpu_cores(),
+                               "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
