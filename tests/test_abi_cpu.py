@@ -97,6 +97,8 @@ def test_init_rejects_bad_arguments_without_touching_a_gpu(lib):
     # null context handles
     assert lib.hyb_attn_decode(None, None, None, None, None, None) == -1
     assert lib.hyb_attn_append(None, None, None, None) == -1
+    assert lib.hyb_attn_append_chunk(None, None, None, 4, None) == -1
+    assert lib.hyb_attn_decode_chunk(None, None, None, None, 4, None, None, None) == -1
     assert lib.hyb_attn_length(None) == -1
     assert H.hyb_attn_strerror(-2).startswith("KV cache capacity")
 

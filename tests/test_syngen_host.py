@@ -131,3 +131,20 @@ def test_layer_budgets_view():
         assert v.layer_budgets == () and v.T0 == w.T0 and v.capacity == w.capacity
     base = C.get_workload("llama8b_32layers_b8_32k")
     assert base.for_layer(5) is base
+
+
+def test_algorithmic_bytes_match_the_scope_table():
+    """The benchmark's algorithmic bytes per (layer, b) at the workloads' prefill
+    length, against the per-KV-head figures of the survey's scope table: exact
+    KV 2052 x 128 x 4, statistics nb x 2 x 128 x 4, state (128^2 + 2 x 128 + 1) x 4,
+    q + out 4 x 128 x 6."""
+    import bench
+    from syngen import configs as C
+    w = C.get_workload("llama8b_32k_layer")
+    dec, _ = bench.algorithmic_bytes(w, w.T0)
+    assert w.n_blocks(w.T0) == 496 and w.exact_tokens(w.T0) == 2052
+    assert dec == 1_050_624 + 507_904 + 66_564 + 3_072
+    assert dec * w.n_kv_heads == 13_025_312
+    w4 = C.get_workload("llama8b_32layers_b4_128k")
+    dec4, _ = bench.algorithmic_bytes(w4, w4.T0)
+    assert dec4 * w4.n_kv_heads == 33_865_760
