@@ -28,6 +28,8 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -96,6 +98,24 @@ def algorithmic_bytes(w, T):
     # variance row
     append = (2 * d * 2) + (2 * d * 2) + d * d * 4 + 2 * d * 4 + 4 + 2 * d * 4
     return decode, append
+
+
+def step_bytes_model(w, mode: str, chunk: int, T: int):
+    """(decode bytes, all bytes, flush L2?) of one step at length about T: every
+    layer with its own budget; prefill: the chunk's rows and evicted tokens, the
+    state written back once, one decode; spec: one decode per draft row (the
+    bytes of per-row decodes)."""
+    step_dec = step_bytes = 0
+    for l in range(w.layers):
+        dec_b, app_b = algorithmic_bytes(w.for_layer(l), T)
+        if mode == "prefill":
+            d = w.head_dim
+            app_b = chunk * 8 * d + (d * d + 2 * d + 1) * 4 + (-(-chunk // w.block_size) + 1) * 2 * d * 4
+        per_step = chunk if mode == "spec" else 1  # decodes per layer and step
+        step_dec += w.units_per_layer * dec_b * per_step
+        step_bytes += w.units_per_layer * (dec_b + app_b) * per_step
+    flush = step_bytes < 4 * 126e6      # the step's data would otherwise stay in L2
+    return step_dec, step_bytes, flush
 
 
 KERNEL_SOURCES = ("k_fused.cu", "hyb_device.cuh", "hyb_internal.h")
@@ -276,16 +296,7 @@ def run_native(args, rank, world):
     Ke = 0 if (args.no_e2e or mode != "decode") else min(K, 20)  # steps of the end-to-end pass
     b = Bench(w, Wm + K + Kk + Ke, device, mode, chunk)
     T_mid = w.T0 + (Wm + K // 2) * chunk
-    step_dec = step_bytes = 0
-    for l in range(w.layers):  # each layer with its own budget
-        dec_b, app_b = algorithmic_bytes(w.for_layer(l), T_mid)
-        if mode == "prefill":  # the chunk's rows and evicted tokens, the state written back once, one decode
-            d = w.head_dim
-            app_b = chunk * 8 * d + (d * d + 2 * d + 1) * 4 + (-(-chunk // w.block_size) + 1) * 2 * d * 4
-        per_step = chunk if mode == "spec" else 1  # decodes per layer and step
-        step_dec += w.units_per_layer * dec_b * per_step
-        step_bytes += w.units_per_layer * (dec_b + app_b) * per_step
-    flush = step_bytes < 4 * 126e6      # the step's data would otherwise stay in L2
+    step_dec, step_bytes, flush = step_bytes_model(w, mode, chunk, T_mid)
     scratch = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if flush else None
 
     def barrier():
@@ -404,15 +415,7 @@ def run_native(args, rank, world):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator; no dataset, no weights)",
-        "config": {
-            "workload": w.name, "layers": w.layers, "batch": w.batch, "n_q_heads": w.n_q_heads,
-            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context_T0": w.T0, "block": w.block_size,
-            "sinks": w.n_sink, "window": w.window, "top_k": w.top_k,
-            **({"layer_budgets_k_W": [list(x) for x in w.layer_budgets]} if w.layer_budgets else {}),
-            "l2": "flushed between timed steps (512 MB write)" if flush else "step data >> L2 (no flush)",
-            "parallelism": f"replicas x{world} (independent units per GPU)",
-            **({"mode": mode, "chunk": chunk} if mode != "decode" else {}),
-        },
+        "config": workload_config(w, mode, chunk, world, flush),
         "attention_tokens_per_s": round(world * steps_s * w.batch * chunk, 3),
         "context_tokens_per_s": round(world * steps_s * w.batch * w.layers * T_mid, 1),
         "achieved_gbs_step": round(step_gbs, 1),
@@ -436,101 +439,236 @@ def run_native(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
+#
+# The fp64 oracle is timed on whole units of the workload in worker processes,
+# one single-threaded worker per host core (BLAS limited to one thread), so that
+# "cores" is the number of threads that actually ran.  Workers are started with
+# the spawn method (never forked from a process that has used CUDA) and import
+# neither torch nor the CUDA library.  A full step holds more units than host
+# memory does (32 layers x 64 units at 32K is ~137 GB in fp64), so the workers
+# time decode + append pairs on copies of a few units and the step time is
+# extrapolated from them.
 
-_ORACLE_UNITS = {}
-
-
-def _oracle_units(w, n_units: int = 4, max_appends: int = 2048):
-    """A few whole units of the workload prepared once for the oracle (inputs
-    generated, state built): [unit, appended K rows, appended V rows, q, next]."""
-    if w.name in _ORACLE_UNITS:
-        return _ORACLE_UNITS[w.name]
-    import oracle as O
+def _oracle_unit_inputs(w, unit_id: int, max_appends: int):
+    """Inputs of unit `unit_id` of the workload (layers cycle first, so that
+    units of different per-layer budgets and head scales are sampled): its keys
+    and values for [0, T0 + max_appends), the step-0 query of its group, and its
+    layer's (window, top_k)."""
     from syngen import host as SH
-    scale = 1 / math.sqrt(w.head_dim)
-    nl = max(1, len(w.layer_budgets))  # with per-layer budgets: units of layers with different budgets
-    units = []
-    for i in range(min(n_units, w.batch * w.n_kv_heads * nl)):
-        layer, j = i % nl, i // nl
-        wl = w.for_layer(layer)
-        tb = SH.LayerTables(wl, layer)
-        q_all = SH.bf16_bits_to_f64(SH.q_bits(wl, layer, 0))
-        b, h = divmod(j, w.n_kv_heads)
-        K, V = SH.kv_f64(wl, tb, b, h, 0, w.T0 + max_appends)
-        u = O.OracleUnit(K[:w.T0], V[:w.T0], w.n_sink, wl.window, w.block_size, wl.top_k, scale,
-                         capacity=w.T0 + max_appends)
-        units.append([u, K[w.T0:], V[w.T0:], q_all[b, h * w.group:(h + 1) * w.group], 0])
-    _ORACLE_UNITS[w.name] = units
-    return units
+    layer, j = unit_id % w.layers, unit_id // w.layers
+    wl = w.for_layer(layer)
+    b, h = divmod(j % (w.batch * w.n_kv_heads), w.n_kv_heads)
+    tb = SH.LayerTables(wl, layer)
+    q_all = SH.bf16_bits_to_f64(SH.q_bits(wl, layer, 0))
+    K, V = SH.kv_f64(wl, tb, b, h, 0, w.T0 + max_appends)
+    return K, V, np.ascontiguousarray(q_all[b, h * w.group:(h + 1) * w.group]), wl.window, wl.top_k
 
 
-def oracle_sample(w, seconds: float, mode: str = "decode", chunk: int = 1):
-    """Time the fp64 oracle's decodes and appends of whole units of the
-    workload, round robin over a few prepared units, for about `seconds` of CPU
-    work; returns seconds per full step (scaled by the units in a step) and a
-    description of the sample.  A step per unit: decode + append; spec: chunk x
-    (decode + append); prefill: chunk appends and one decode (the oracle appends
-    one token at a time)."""
-    units = _oracle_units(w)
+def _oracle_sample_unit(e, seconds: float):
+    """Decode + append pairs on one unit for about `seconds` of timed work; when
+    its prepared tokens are used up it starts again from T0 (the rebuild is not
+    timed).  Returns (pairs, decode seconds, append seconds)."""
     t_dec = t_app = 0.0
     n = 0
     while t_dec + t_app < seconds:
-        progressed = False
-        for e in units:
-            u, Kt, Vt, q, pos = e
-            if pos >= len(Kt):
-                continue
-            t0 = time.perf_counter()
-            u.decode(q)
-            t1 = time.perf_counter()
-            u.append(Kt[pos], Vt[pos])
-            t2 = time.perf_counter()
-            t_dec += t1 - t0
-            t_app += t2 - t1
-            e[4] = pos + 1
-            n += 1
-            progressed = True
-        if not progressed:
-            break
-    d, a = t_dec / max(1, n), t_app / max(1, n)
-    per_unit_step = {"decode": d + a, "spec": chunk * (d + a), "prefill": chunk * a + d}[mode]
-    units_per_step = w.layers * w.units_per_layer
-    what = {"decode": "decode + append", "spec": f"{chunk} x (decode + append)",
-            "prefill": f"{chunk} appends + decode"}[mode]
-    return per_unit_step * units_per_step, (f"{n} unit decode + append pairs of one (layer, b, kv-head) at "
-                                            f"{w.T0}+ tokens, round robin over {len(units)} units, timed "
-                                            f"apart; a step = {what} per unit, x{units_per_step} units")
+        if e["pos"] >= e["n_app"]:
+            e["u"], e["pos"] = e["fresh"](), 0
+        u, pos = e["u"], e["pos"]
+        t0 = time.perf_counter()
+        u.decode(e["q"])
+        t1 = time.perf_counter()
+        u.append(e["K"][e["T0"] + pos], e["V"][e["T0"] + pos])
+        t2 = time.perf_counter()
+        t_dec += t1 - t0
+        t_app += t2 - t1
+        e["pos"] = pos + 1
+        n += 1
+    if n == 0:
+        raise RuntimeError("oracle sample timed no unit")
+    return n, t_dec, t_app
 
 
-def cpu_cores():
+def _oracle_worker(conn, spec: dict):
+    """Worker process: one BLAS thread; its unit built once from the inputs in
+    shared memory, then one sample per request until it receives None."""
     try:
-        from threadpoolctl import threadpool_info
-        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:
+        pass
+    sys.path.insert(0, ROOT)
+    from multiprocessing import shared_memory
+    import oracle as O
+    shm = shared_memory.SharedMemory(name=spec["shm"])
+    T, d, G = spec["T"], spec["d"], spec["G"]
+    buf = np.ndarray((2 * T * d + G * d,), dtype=np.float64, buffer=shm.buf)
+    K = buf[:T * d].reshape(T, d)
+    V = buf[T * d:2 * T * d].reshape(T, d)
+    q = buf[2 * T * d:].reshape(G, d).copy()
+    T0 = spec["T0"]
+
+    def fresh():
+        return O.OracleUnit(K[:T0], V[:T0], spec["S"], spec["W"], spec["Bk"], spec["k"], spec["scale"],
+                            capacity=T)
+
+    e = {"fresh": fresh, "u": fresh(), "K": K, "V": V, "q": q, "T0": T0, "n_app": T - T0, "pos": 0}
+    conn.send("ready")
+    try:
+        while True:
+            msg = conn.recv()
+            if msg is None:
+                break
+            conn.send(_oracle_sample_unit(e, msg))
+    finally:
+        del K, V, buf, e
+        shm.close()
+        conn.close()
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
 
 
+class OraclePool:
+    """Single-threaded oracle worker processes, one per host core (bounded by
+    host memory).  The parent generates the inputs of a few distinct units once
+    into shared memory; every worker builds its own oracle unit from one of them
+    and times decode + append pairs on it (the oracle's cost does not depend on
+    the values)."""
+
+    def __init__(self, w, max_appends: int = 256):
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        try:
+            import psutil
+            avail = psutil.virtual_memory().available
+        except Exception:
+            avail = 16 << 30
+        d, G = w.head_dim, w.group
+        T = w.T0 + max_appends
+        n_units_total = w.layers * w.units_per_layer
+        n_distinct = min(n_units_total, 2 if w.T0 <= 65536 else 1)
+        per_worker = 2 * T * d * 8 + 2 * (w.n_blocks(T) + 1) * d * 8   # the oracle unit's K, V copy, block sums
+        by_mem = max(1, int((0.5 * avail - n_distinct * 2 * T * d * 8) // per_worker))
+        self.workers = max(1, min(host_cores(), by_mem))
+        self.w = w
+        self.units = n_distinct
+        self.shms, specs = [], []
+        for i in range(n_distinct):
+            K, V, q, win, k = _oracle_unit_inputs(w, i, max_appends)
+            shm = shared_memory.SharedMemory(create=True, size=(2 * T * d + G * d) * 8)
+            buf = np.ndarray((2 * T * d + G * d,), dtype=np.float64, buffer=shm.buf)
+            buf[:T * d] = K.reshape(-1)
+            buf[T * d:2 * T * d] = V.reshape(-1)
+            buf[2 * T * d:] = q.reshape(-1)
+            del buf
+            self.shms.append(shm)
+            specs.append({"shm": shm.name, "T": T, "T0": w.T0, "d": d, "G": G, "S": w.n_sink, "W": win,
+                          "Bk": w.block_size, "k": k, "scale": 1 / math.sqrt(d)})
+        ctx = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        for i in range(self.workers):
+            a, b = ctx.Pipe()
+            p = ctx.Process(target=_oracle_worker, args=(b, specs[i % n_distinct]), daemon=True)
+            p.start()
+            self.conns.append(a)
+            self.procs.append(p)
+        for c in self.conns:
+            if c.recv() != "ready":
+                raise RuntimeError("oracle worker failed to start")
+
+    def sample(self, seconds: float, mode: str = "decode", chunk: int = 1):
+        """All workers time `seconds` of decode + append pairs at once.  Returns
+        (seconds per full step, extrapolated from the timed units; pairs timed)."""
+        for c in self.conns:
+            c.send(seconds)
+        res = [c.recv() for c in self.conns]
+        rate = 0.0   # unit steps per second, all workers together
+        pairs = 0
+        for n, td, ta in res:
+            dd, aa = td / n, ta / n
+            per_unit_step = {"decode": dd + aa, "spec": chunk * (dd + aa), "prefill": chunk * aa + dd}[mode]
+            rate += 1.0 / per_unit_step
+            pairs += n
+        units_per_step = self.w.layers * self.w.units_per_layer
+        return units_per_step / rate, pairs
+
+    def describe(self, pairs: int, mode: str, chunk: int) -> str:
+        w = self.w
+        what = {"decode": "decode + append", "spec": f"{chunk} x (decode + append)",
+                "prefill": f"{chunk} appends + decode"}[mode]
+        return (f"extrapolated from {self.units} units: {pairs} timed decode + append pairs on whole "
+                f"(layer, b, kv-head) units at {w.T0}+ tokens, {self.workers} single-threaded worker processes "
+                f"at once, each with its own copy of one of the {self.units} units; a step = {what} per unit, "
+                f"x{w.layers * w.units_per_layer} units")
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send(None)
+            except Exception:
+                pass
+        for p in self.procs:
+            p.join(timeout=10)
+            if p.is_alive():
+                p.terminate()
+        for shm in self.shms:
+            shm.close()
+            shm.unlink()
+        self.shms = []
+
+
+def workload_config(w, mode: str, chunk: int, world: int, flush: bool) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    return {
+        "workload": w.name, "layers": w.layers, "batch": w.batch, "n_q_heads": w.n_q_heads,
+        "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context_T0": w.T0, "block": w.block_size,
+        "sinks": w.n_sink, "window": w.window, "top_k": w.top_k,
+        **({"layer_budgets_k_W": [list(x) for x in w.layer_budgets]} if w.layer_budgets else {}),
+        "l2": "flushed between timed steps (512 MB write)" if flush else "step data >> L2 (no flush)",
+        "parallelism": f"replicas x{world} (independent units per GPU)",
+        **({"mode": mode, "chunk": chunk} if mode != "decode" else {}),
+    }
+
+
 def run_reference(args, rank, world):
     from syngen import configs as C
-    w = C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {}))
+    overrides = {"layers": args.layers} if args.layers else {}
+    w = C.get_workload(args.workload, **overrides)
     mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
-    oracle_sample(w, 0.2)   # prepare the units, warm numpy / BLAS
-    samples = []
-    for _ in range(args.warmup):
-        oracle_sample(w, 0.05)
-    for _ in range(args.steps):
-        s, desc = oracle_sample(w, args.cpu_sample_seconds / max(1, args.steps), mode, chunk)
-        samples.append(s)
+    pool = OraclePool(w)
+    try:
+        per = args.cpu_sample_seconds / max(1, args.steps)
+        for _ in range(args.warmup):
+            pool.sample(min(0.1, per), mode, chunk)
+        samples, pairs = [], 0
+        t_wall = time.perf_counter()
+        for _ in range(args.steps):
+            s, n = pool.sample(per, mode, chunk)
+            samples.append(s)
+            pairs += n
+        t_wall = time.perf_counter() - t_wall
+    finally:
+        pool.close()
     ms = 1e3 * statistics.mean(samples)
     v = 1e3 / ms
+    _, _, flush = step_bytes_model(w, mode, chunk, w.T0)
+    desc = pool.describe(pairs, mode, chunk)
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "layers": w.layers, **({"mode": mode, "chunk": chunk} if mode != "decode" else {})},
-        "cpu_baseline": {"value": round(v, 6), "unit": "steps/s", "cores": cpu_cores(), "kind": "oracle",
-                         "sample": desc},
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator; no dataset, no weights)",
+        "config": workload_config(w, mode, chunk, world, flush),
+        "cpu_baseline": {"value": round(v, 6), "unit": "steps/s", "cores": pool.workers, "kind": "oracle",
+                         "sample": desc, "extrapolated_from_units": pool.units},
         "e2e": {"value": round(v, 6), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "extrapolated": f"each step is a {per:.3f} s sample of {pool.units} units timed on {pool.workers} host "
+                        f"cores, scaled to the workload's {w.layers * w.units_per_layer} units; wall time of the "
+                        f"timed samples {t_wall:.2f} s",
     }
 
 
@@ -549,12 +687,20 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_native(args, rank, world)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
         from syngen import configs as C
-        w = C.get_workload(args.workload, **({"layers": args.layers} if args.layers else {}))
-        s, desc = oracle_sample(w, args.cpu_sample_seconds, args.mode, args.chunk if args.mode != "decode" else 1)
-        res["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": "steps/s", "cores": cpu_cores(),
-                               "kind": "oracle", "sample": desc}
+        overrides = {"layers": args.layers} if args.layers else {}
+        w = C.get_workload(args.workload, **overrides)
+        mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
+        pool = OraclePool(w)
+        try:
+            pool.sample(0.1, mode, chunk)   # warm numpy in every worker
+            s, pairs = pool.sample(args.cpu_sample_seconds, mode, chunk)
+        finally:
+            pool.close()
+        res["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": "steps/s", "cores": pool.workers,
+                               "kind": "oracle", "sample": pool.describe(pairs, mode, chunk),
+                               "extrapolated_from_units": pool.units}
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

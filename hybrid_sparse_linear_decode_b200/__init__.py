@@ -16,6 +16,7 @@ from ._abi import (  # noqa: F401
     hyb_attn_workspace_size,
     hyb_attn_plan,
     hyb_attn_init,
+    hyb_attn_attach,
     hyb_attn_append,
     hyb_attn_append_chunk,
     hyb_attn_sync_state,
@@ -28,6 +29,8 @@ from ._abi import (  # noqa: F401
     hyb_attn_length,
     hyb_attn_status,
     hyb_attn_set_timing_events,
+    hyb_attn_set_wait_limit,
+    hyb_attn_set_test_flags,
     hyb_attn_destroy,
     hyb_attn_strerror,
     hyb_attn_last_cuda_error,
@@ -38,5 +41,6 @@ from ._abi import (  # noqa: F401
     HYB_STATUS_BAD_SELECTION,
     HYB_STATUS_TIMEOUT,
     HYB_STATUS_NAN_SCORE,
+    HYB_TEST_WITHHOLD_SCORES,
 )
 from .layer import HybridAttentionLayer, make_config  # noqa: F401

@@ -29,6 +29,8 @@ HYB_STATUS_BAD_SELECTION = 0x4
 HYB_STATUS_TIMEOUT = 0x8
 HYB_STATUS_NAN_SCORE = 0x10
 
+HYB_TEST_WITHHOLD_SCORES = 0x1
+
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
 
@@ -61,6 +63,8 @@ SIGNATURES = [
                                      ctypes.POINTER(hyb_attn_plan_info)]),
     ("hyb_attn_init", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
                                      ctypes.POINTER(hyb_attn_buffers), c_i64, c_vp]),
+    ("hyb_attn_attach", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
+                                       ctypes.POINTER(hyb_attn_buffers), c_i64, c_vp]),
     ("hyb_attn_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_append_chunk", ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_vp]),
     ("hyb_attn_sync_state", ctypes.c_int, [c_vp, c_vp]),
@@ -73,6 +77,8 @@ SIGNATURES = [
     ("hyb_attn_length", c_i64, [c_vp]),
     ("hyb_attn_status", ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, c_vp]),
     ("hyb_attn_set_timing_events", ctypes.c_int, [c_vp, c_vp, c_vp]),
+    ("hyb_attn_set_wait_limit", ctypes.c_int, [c_vp, ctypes.c_uint64]),
+    ("hyb_attn_set_test_flags", ctypes.c_int, [c_vp, ctypes.c_uint32]),
     ("hyb_attn_destroy", None, [c_vp]),
     ("hyb_attn_strerror", ctypes.c_char_p, [ctypes.c_int]),
     ("hyb_attn_last_cuda_error", ctypes.c_char_p, []),
@@ -146,6 +152,13 @@ def hyb_attn_init(cfg: hyb_attn_config, buf: hyb_attn_buffers, T0: int, stream: 
     return h.value
 
 
+def hyb_attn_attach(cfg: hyb_attn_config, buf: hyb_attn_buffers, T: int, stream: int) -> int:
+    h = c_vp()
+    _check("hyb_attn_attach", load_library().hyb_attn_attach(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(buf),
+                                                             T, stream))
+    return h.value
+
+
 def hyb_attn_append(ctx: int, k_new: int, v_new: int, stream: int) -> None:
     _check("hyb_attn_append", load_library().hyb_attn_append(ctx, k_new, v_new, stream))
 
@@ -184,8 +197,9 @@ def hyb_attn_step_host(ctx: int, q_host: int, k_host, v_host, out_host: int, str
 
 
 def hyb_attn_decode_noalloc(ctx: int, q: int, out: int, sel_out, stream: int) -> None:
-    """Decode using the library's fixed device scratch instead of the context's
-    workspace (for callers that cannot allocate device memory)."""
+    """Decode with the block scores and the selection in the library's fixed
+    device array instead of the context's workspace (for callers that cannot
+    allocate device memory)."""
     _check("hyb_attn_decode_noalloc", load_library().hyb_attn_decode_noalloc(ctx, q, out, sel_out, stream))
 
 
@@ -201,6 +215,14 @@ def hyb_attn_status(ctx: int, clear: bool, stream: int) -> int:
 
 def hyb_attn_set_timing_events(ctx: int, begin, end) -> None:
     _check("hyb_attn_set_timing_events", load_library().hyb_attn_set_timing_events(ctx, begin, end))
+
+
+def hyb_attn_set_wait_limit(ctx: int, ns: int) -> None:
+    _check("hyb_attn_set_wait_limit", load_library().hyb_attn_set_wait_limit(ctx, ns))
+
+
+def hyb_attn_set_test_flags(ctx: int, flags: int) -> None:
+    _check("hyb_attn_set_test_flags", load_library().hyb_attn_set_test_flags(ctx, flags))
 
 
 def hyb_attn_destroy(ctx: int) -> None:

@@ -11,6 +11,8 @@
 #include <mutex>
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/hyb_attn.h"
 #include "hyb_internal.h"
 
@@ -22,8 +24,10 @@ constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Workspace regions.  The decode uses status, scores and sel; init uses the
+// fp64 accumulators H64 and z64; hyb_attn_step_host the staging copies.
 struct WsLayout {
-  size_t status, tk_sel, tk_att, scores, sel, H64, z64, stage_q, stage_k, stage_v, stage_out, total;
+  size_t status, scores, sel, H64, z64, stage_q, stage_k, stage_v, stage_out, total;
 };
 
 struct Checked {
@@ -67,8 +71,6 @@ WsLayout ws_layout(const hyb_attn_config& c, const Checked& k) {
   };
   const size_t U = (size_t)k.units, D = (size_t)k.D, G = (size_t)k.G;
   w.status = take(sizeof(uint32_t));
-  w.tk_sel = take(U * sizeof(uint32_t));
-  w.tk_att = take(U * sizeof(uint32_t));
   w.scores = take(U * (size_t)(k.max_blocks > 0 ? k.max_blocks : 1) * sizeof(float));
   w.sel = take(U * (size_t)(c.top_k > 0 ? c.top_k : 1) * sizeof(int32_t));
   w.H64 = take(U * D * D * sizeof(double));
@@ -109,6 +111,14 @@ int cluster_ctas(int units, int n_sm, const int* fits) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around every entry point (visible to Nsight tools; costs a
+// call into a stub when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+#define HYB_RANGE NvtxRange hyb_range_(__func__)
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
@@ -160,9 +170,10 @@ bool is_device_ptr(const void* p, int device) {
 
 }  // namespace
 
-// Fixed scratch of hyb_attn_decode_noalloc: a file-scope device array, one per
-// GPU that loads this library.  Host code only ever uses its device address,
-// looked up once per device with that device current.
+// Fixed scratch of hyb_attn_decode_noalloc (block scores and the selection of
+// one decode): a file-scope device array, one per GPU that loads this library.
+// Host code only ever uses its device address, looked up once per device with
+// that device current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[HYB_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -194,6 +205,9 @@ struct hyb_attn_ctx {
   int device, n_sm;
   int fits[kMaxCluster + 1];  // clusters of C CTAs of the decode kernel the device holds at once
   float scale;
+  uint64_t wait_ns;     // limit of the kernels' bounded waits for progress
+  uint32_t test_flags;  // HYB_TEST_* failure injection (tests only)
+  uint32_t* status;     // the device status word (in the context's workspace)
   CUtensorMap maps[4];  // K, V with 64-row boxes; K, V with 16-row boxes
   cudaEvent_t ev_begin, ev_end;
   template <class P>
@@ -218,7 +232,7 @@ FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   fp.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
   fp.scores = x->w<float>(x->ws.scores);
   fp.sel = x->w<int32_t>(x->ws.sel);
-  fp.status = x->w<uint32_t>(x->ws.status);
+  fp.status = x->status;
   fp.cap = c.capacity;
   fp.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
   fp.fold_begin = x->folded_end;
@@ -242,6 +256,8 @@ FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   fp.mstride = merge_stride(k.G * k.D, fp.C);
   for (int r = 0; r <= fp.C; ++r) fp.mslice[r] = merge_slice_begin(k.G * k.D, fp.C, r);
   fp.scale = x->scale;
+  fp.wait_ns = x->wait_ns;
+  fp.test_flags = x->test_flags;
   return fp;
 }
 
@@ -348,13 +364,16 @@ int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_
   return HYB_OK;
 }
 
-int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T0,
-                  cudaStream_t stream) {
-  if (out == nullptr) return HYB_EINVAL;
-  *out = nullptr;
+}  // extern "C"
+
+namespace {
+
+// Validate a configuration and its buffers and build the host context of a
+// layer at length T (TMA descriptors, kernel attributes); no kernel is launched.
+int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T, hyb_attn_ctx** out) {
   Checked k;
   if (check_config(cfg, &k) != HYB_OK || buf == nullptr) return HYB_EINVAL;
-  if (T0 < 0 || T0 > cfg->capacity) return HYB_EINVAL;
+  if (T < 0 || T > cfg->capacity) return HYB_EINVAL;
   const void* ptrs[] = {buf->k_cache, buf->v_cache, buf->H, buf->zk, buf->zv, buf->n, buf->workspace};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return HYB_EINVAL;
@@ -377,11 +396,14 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   x->buf = *buf;
   x->ck = k;
   x->ws = ws;
-  x->T = T0;
+  x->T = T;
   x->device = device;
   x->n_sm = n_sm;
   for (int c = 0; c <= kMaxCluster; ++c) x->fits[c] = 0;
   x->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)k.D);
+  x->wait_ns = kWaitLimit;
+  x->test_flags = 0u;
+  x->status = x->w<uint32_t>(ws.status);
   x->ev_begin = x->ev_end = nullptr;
   const int64_t rows = (int64_t)k.units * cfg->capacity;
   if (!make_kv_map(&x->maps[0], buf->k_cache, rows, k.D, kTile) ||
@@ -398,7 +420,24 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
     return cuda_fail(pe);
   }
   for (int c = 2; c <= kMaxCluster; ++c) x->fits[c] = fused_max_clusters(k.D, c);
+  x->folded_end = geometry(*cfg, T).ev_end;
+  *out = x;
+  return HYB_OK;
+}
 
+}  // namespace
+
+extern "C" {
+
+int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T0,
+                  cudaStream_t stream) {
+  HYB_RANGE;
+  if (out == nullptr) return HYB_EINVAL;
+  *out = nullptr;
+  hyb_attn_ctx* x = nullptr;
+  const int rc = create_ctx(cfg, buf, T0, &x);
+  if (rc != HYB_OK) return rc;
+  const Checked& k = x->ck;
   const Geometry g = geometry(*cfg, T0);
   InitParams ip{};
   ip.k_cache = static_cast<const __nv_bfloat16*>(buf->k_cache);
@@ -409,11 +448,9 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   ip.n = buf->n;
   ip.mu = buf->mu;
   ip.var = buf->var;
-  ip.H64 = x->w<double>(ws.H64);
-  ip.z64 = x->w<double>(ws.z64);
-  ip.tickets_sel = x->w<uint32_t>(ws.tk_sel);
-  ip.tickets_att = x->w<uint32_t>(ws.tk_att);
-  ip.status = x->w<uint32_t>(ws.status);
+  ip.H64 = x->w<double>(x->ws.H64);
+  ip.z64 = x->w<double>(x->ws.z64);
+  ip.status = x->status;
   ip.cap = cfg->capacity;
   ip.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
   ip.ev_begin = cfg->n_sink;
@@ -423,18 +460,36 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   ip.Bk = cfg->block_size;
   ip.nb = (int32_t)g.nb;
   ip.tokens_per_cta = 2048;
-  if (cudaMemsetAsync(ip.H64, 0, (size_t)k.units * k.D * k.D * sizeof(double), stream) != cudaSuccess ||
-      cudaMemsetAsync(ip.z64, 0, (size_t)k.units * 2 * k.D * sizeof(double), stream) != cudaSuccess ||
-      launch_init(ip, k.D, stream) != cudaSuccess) {
+  cudaError_t e = cudaMemsetAsync(ip.H64, 0, (size_t)k.units * k.D * k.D * sizeof(double), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ip.z64, 0, (size_t)k.units * 2 * k.D * sizeof(double), stream);
+  if (e == cudaSuccess) e = launch_init(ip, k.D, stream);
+  if (e != cudaSuccess) {
     delete x;
-    return HYB_ECUDA;
+    return cuda_fail(e);
   }
-  x->folded_end = g.ev_end;
+  *out = x;
+  return HYB_OK;
+}
+
+int hyb_attn_attach(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T,
+                    cudaStream_t stream) {
+  HYB_RANGE;
+  if (out == nullptr) return HYB_EINVAL;
+  *out = nullptr;
+  hyb_attn_ctx* x = nullptr;
+  const int rc = create_ctx(cfg, buf, T, &x);
+  if (rc != HYB_OK) return rc;
+  const cudaError_t e = cudaMemsetAsync(x->status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) {
+    delete x;
+    return cuda_fail(e);
+  }
   *out = x;
   return HYB_OK;
 }
 
 int hyb_attn_append_chunk(hyb_attn_ctx* x, const void* k_new, const void* v_new, int32_t n, cudaStream_t stream) {
+  HYB_RANGE;
   if (x == nullptr || k_new == nullptr || v_new == nullptr || n < 1 || n > 65535) return HYB_EINVAL;
   if (!aligned16(k_new) || !aligned16(v_new)) return HYB_EINVAL;
   if (x->T + n > x->cfg.capacity) return HYB_ECAPACITY;
@@ -458,6 +513,7 @@ int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaS
 }
 
 int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
+  HYB_RANGE;
   if (x == nullptr) return HYB_EINVAL;
   const Geometry g = geometry(x->cfg, x->T);
   if (g.ev_end <= x->folded_end) return HYB_OK;  // nothing evicted since the last fold
@@ -471,17 +527,20 @@ int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
 
 int hyb_attn_decode(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out, float* scores_out,
                     cudaStream_t stream) {
+  HYB_RANGE;
   return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, nullptr, nullptr, stream);
 }
 
 int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, const void* v_new, float* out,
                            int32_t* sel_out, float* scores_out, cudaStream_t stream) {
+  HYB_RANGE;
   if (k_new == nullptr || v_new == nullptr) return HYB_EINVAL;
   return decode_impl(ctx, q, out, nullptr, sel_out, scores_out, k_new, v_new, stream);
 }
 
 int hyb_attn_decode_chunk(hyb_attn_ctx* x, const void* q, const void* k_new, const void* v_new, int32_t n,
                           float* out, int32_t* sel_out, cudaStream_t stream) {
+  HYB_RANGE;
   if (x == nullptr || q == nullptr || k_new == nullptr || v_new == nullptr || out == nullptr || n < 1)
     return HYB_EINVAL;
   if (x->T == 0) return HYB_ESTATE;
@@ -499,12 +558,14 @@ int hyb_attn_decode_chunk(hyb_attn_ctx* x, const void* q, const void* k_new, con
 
 int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32_t* sel, float* out,
                                    cudaStream_t stream) {
+  HYB_RANGE;
   if (sel == nullptr) return HYB_EINVAL;
   return decode_impl(ctx, q, out, sel, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, const void* v_host,
                        float* out_host, cudaStream_t stream) {
+  HYB_RANGE;
   if (x == nullptr || q_host == nullptr || out_host == nullptr) return HYB_EINVAL;
   if ((k_host == nullptr) != (v_host == nullptr)) return HYB_EINVAL;
   if (k_host != nullptr && x->T >= x->cfg.capacity) return HYB_ECAPACITY;
@@ -527,18 +588,20 @@ int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, 
 }
 
 int hyb_attn_decode_noalloc(hyb_attn_ctx* x, const void* q, float* out, int32_t* sel_out, cudaStream_t stream) {
+  HYB_RANGE;
   if (x == nullptr) return HYB_EINVAL;
   int device = -1;
   if (cudaGetDevice(&device) != cudaSuccess) return HYB_ECUDA;
   if (device != x->device) return HYB_EINVAL;
-  // the decode uses the workspace regions that precede the init accumulators
+  // the decode's scratch (block scores, the selection) is the workspace regions
+  // before the init accumulators; the array takes the same layout
   if (x->ws.H64 > HYB_NOALLOC_SCRATCH_BYTES) return HYB_ESCRATCH;
   void* scratch = nullptr;
   const int rc = noalloc_scratch(device, &scratch);
   if (rc != HYB_OK) return rc;
-  // status and tickets must start at zero; the array keeps the previous call's contents
-  const cudaError_t e = cudaMemsetAsync(scratch, 0, x->ws.scores, stream);
-  if (e != cudaSuccess) return cuda_fail(e);
+  // Nothing in the scratch needs to start at zero: every score and selection
+  // entry a decode reads it has written first.  The device status word stays
+  // the context's own, so that hyb_attn_status reports this call's bits.
   hyb_attn_ctx view = *x;  // the same context with its scratch rebased onto the fixed array
   view.buf.workspace = scratch;
   view.buf.workspace_bytes = HYB_NOALLOC_SCRATCH_BYTES;
@@ -550,6 +613,7 @@ int hyb_attn_decode_noalloc(hyb_attn_ctx* x, const void* q, float* out, int32_t*
 int64_t hyb_attn_length(const hyb_attn_ctx* x) { return x ? x->T : -1; }
 
 int hyb_attn_status(hyb_attn_ctx* x, uint32_t* flags, int clear, cudaStream_t stream) {
+  HYB_RANGE;
   if (x == nullptr || flags == nullptr) return HYB_EINVAL;
   uint32_t* d = x->w<uint32_t>(x->ws.status);
   if (cudaMemcpyAsync(flags, d, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return HYB_ECUDA;
@@ -562,6 +626,20 @@ int hyb_attn_set_timing_events(hyb_attn_ctx* x, cudaEvent_t begin, cudaEvent_t e
   if (x == nullptr || ((begin == nullptr) != (end == nullptr))) return HYB_EINVAL;
   x->ev_begin = begin;
   x->ev_end = end;
+  return HYB_OK;
+}
+
+int hyb_attn_set_wait_limit(hyb_attn_ctx* x, uint64_t ns) {
+  if (x == nullptr) return HYB_EINVAL;
+  if (ns == 0) ns = kWaitLimit;
+  if (ns < 100000ull || ns > 60000000000ull) return HYB_EINVAL;
+  x->wait_ns = ns;
+  return HYB_OK;
+}
+
+int hyb_attn_set_test_flags(hyb_attn_ctx* x, uint32_t flags) {
+  if (x == nullptr || (flags & ~HYB_TEST_WITHHOLD_SCORES) != 0u) return HYB_EINVAL;
+  x->test_flags = flags;
   return HYB_OK;
 }
 

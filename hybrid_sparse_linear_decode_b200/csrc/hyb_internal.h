@@ -15,7 +15,7 @@ constexpr int kBoxRows = 16;          // rows per TMA box of a ragged chunk
 constexpr int kMaxCluster = 16;       // CTAs per unit (thread-block cluster; above 8 is non-portable)
 constexpr int kSelCache = 256;        // selection entries a CTA keeps in shared memory
 constexpr int kMaxGroup = 4;          // query heads per KV head
-constexpr uint64_t kWaitLimit = 1000000000ull;  // ns: a kernel-internal wait gives up after ~1 s
+constexpr uint64_t kWaitLimit = 1000000000ull;  // ns: a kernel-internal wait gives up after ~1 s (default)
 
 // Per-slot layout of a split-K partial: m[4], l[4], dsel[4], pad[4], acc[4][D], nsel[4][D].
 __host__ __device__ constexpr int partial_floats(int D) { return 16 + 8 * D; }
@@ -72,6 +72,8 @@ struct FusedParams {           // one decode (or, with q == null, the fold only)
   int32_t mstride;              // merge: floats per sending rank's slot (merge_stride)
   int32_t mslice[kMaxCluster + 1];  // merge: rank r merges outputs [mslice[r], mslice[r + 1])
   float scale;
+  uint64_t wait_ns;             // limit of every bounded wait inside the kernel
+  uint32_t test_flags;          // HYB_TEST_* (0 in normal use)
 };
 
 struct AppendParams {       // write n tokens per unit at positions [T, T + n)
@@ -101,7 +103,7 @@ struct InitParams {
   float* H; float* zk; float* zv; float* n; float* mu; float* var;
   double* H64;                // [units][D][D] accumulators
   double* z64;                // [units][2][D]
-  uint32_t* tickets_sel; uint32_t* tickets_att; uint32_t* status;
+  uint32_t* status;
   int64_t cap, max_blocks;
   int64_t ev_begin, ev_end;   // evicted range [S, T0 - W)
   int32_t units, S, Bk, nb, tokens_per_cta;

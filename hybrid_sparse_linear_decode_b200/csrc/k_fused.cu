@@ -51,7 +51,10 @@
 //
 // Every wait inside the kernel is bounded (a timeout sets a status bit and the
 // CTA skips the rest of its work); all CTAs of a cluster always reach both
-// cluster barriers.  Launch chaining: programmatic dependent launch -- the CTA
+// cluster barriers.  The limit of the waits for progress (ring items, the
+// scores, the selection, a free stage) comes with the launch; the two waits
+// that guard the CTA's exit (copies in flight into its ring, the other ranks'
+// merge stores) keep the long default limit.  Launch chaining: programmatic dependent launch -- the CTA
 // waits for the predecessor grid before touching memory.
 #include "hyb_device.cuh"
 #include "hyb_internal.h"
@@ -958,7 +961,7 @@ __device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int
       for (int j = a; j < p.top_k; j += kAuxThreads) copy[j] = (p.k_eff > 0 && j < p.nb) ? j : -1;
   } else {
     if (a == 0) {  // one decision for all statistics threads (their barrier counts must match)
-      const bool ok = wait_cluster_bounded(&sm.scores_bar, 0, kWaitLimit);
+      const bool ok = wait_cluster_bounded(&sm.scores_bar, 0, p.wait_ns);
       if (!ok) {
         atomicOr(p.status, HYB_STATUS_TIMEOUT);
         sm.abort = 1;
@@ -1063,7 +1066,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
     par ^= 1u << stage;
     bool have = false;
     if (!dead) {
-      have = __all_sync(kFull, mbar_wait_bounded(&sm.full_attn[stage], ph, kWaitLimit));
+      have = __all_sync(kFull, mbar_wait_bounded(&sm.full_attn[stage], ph, p.wait_ns));
       if (!have) {
         dead = true;
         if (lane == 0) {
@@ -1185,7 +1188,7 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
 
   // the combine slots hold the top-k candidates until the selection is made
   // (a rank without selected chunks gets here first)
-  if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit);
+  if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, p.wait_ns);
   // ---- combine the 4 pairs' partials (a tree through two shared slots: pairs
   //      2, 3 -> 0, 1, then pair 1 -> 0); pair 0 leaves the record in wpart[0].
   //      The two warps of a pair hold the same statistics and disjoint columns.
@@ -1279,7 +1282,7 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
     const uint32_t ph = (par >> stage) & 1u;
     par ^= 1u << stage;
     if (dead) return false;
-    const bool have = __all_sync(kFull, mbar_wait_bounded(&sm.full_aux[stage], ph, kWaitLimit));
+    const bool have = __all_sync(kFull, mbar_wait_bounded(&sm.full_aux[stage], ph, p.wait_ns));
     if (!have) {
       dead = true;
       if (lane == 0) {
@@ -1333,7 +1336,10 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
       // bulk copies of the share into every other rank's scores array
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       named_sync(kBarAux, kAuxThreads);
-      if (a == 0 && s.b1 > s.b0) {
+      // test hook: rank 1 withholds its scores, so that the other ranks' bounded
+      // wait for them runs out (nothing else ever skips this push)
+      const bool withhold = (p.test_flags & HYB_TEST_WITHHOLD_SCORES) != 0u && rank == 1;
+      if (a == 0 && s.b1 > s.b0 && !withhold) {
         const uint32_t bytes = (uint32_t)(((s.b1 - s.b0) * 4 + 15) & ~15);
         const uint32_t src = smem_u32(&sm.scores[s.b0]), bar = smem_u32(&sm.scores_bar);
         for (int rr = 0; rr < p.C; ++rr)
@@ -1386,7 +1392,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
     if (issued >= kFStages) {
       const uint32_t ph = (epar >> stage) & 1u;
       epar ^= 1u << stage;
-      if (!mbar_wait_bounded(&sm.empty[stage], ph, kWaitLimit)) {
+      if (!mbar_wait_bounded(&sm.empty[stage], ph, p.wait_ns)) {
         atomicOr(p.status, HYB_STATUS_TIMEOUT);
         sm.abort = 1;
         return false;
@@ -1453,7 +1459,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
     advance(true);
   }
   // selected chunks: chunk sc = rank + i C is piece sc % cpb of selection slot sc / cpb
-  if (ok && s.nX > 0 && !mbar_wait_bounded(&sm.sel_bar, 0, kWaitLimit)) {
+  if (ok && s.nX > 0 && !mbar_wait_bounded(&sm.sel_bar, 0, p.wait_ns)) {
     atomicOr(p.status, HYB_STATUS_TIMEOUT);
     sm.abort = 1;
     ok = false;
@@ -1485,7 +1491,9 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
   }
   if (*(volatile int*)&sm.abort) {
     // do not leave while copies into this CTA's ring may be in flight: wait for
-    // the last item issued into each stage (its group's full barrier, its phase)
+    // the last item issued into each stage (its group's full barrier, its phase);
+    // every issued item completes, so this wait keeps the long default limit
+    // whatever limit the progress waits have
     for (int j = 0; j < kFStages && j < issued; ++j) {
       const bool aux = (last_aux >> j) & 1u;
       const uint32_t ph = (((aux ? fpar_aux : fpar_at) >> j) & 1u) ^ 1u;  // parity of the last item's phase
@@ -1551,7 +1559,9 @@ __device__ void merge_local(const FusedParams& p, FusedSmem<D>& sm, int unit, in
   const int tid = threadIdx.x;
   const int G = p.G, C = p.C;
   const int stride = p.mstride;
-  // every thread waits; the outcome is made uniform so that all or none merge
+  // every thread waits; the outcome is made uniform so that all or none merge.
+  // Every rank pushes its parts whatever happened before, so this wait keeps
+  // the long default limit (no rank leaves with another's stores in flight)
   if (!__syncthreads_and(wait_cluster_bounded(&sm.merge_bar, 0, kWaitLimit))) {
     if (tid == 0) atomicOr(p.status, HYB_STATUS_TIMEOUT);
     return;

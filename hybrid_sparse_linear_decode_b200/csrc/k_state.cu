@@ -1,6 +1,8 @@
-// State kernels: the per-token append (a cache write) and the build of the
-// state of a prefilled history.  Between decodes the state lags the history by
-// the tokens evicted since the last decode; the select kernel folds those in.
+// State kernels: the cache write of an append, the dense fold of a run of
+// evicted tokens, and the build of the state of a prefilled history.  Between
+// decodes the state lags the history by the tokens evicted since the last
+// decode; the next decode folds those in (the fused decode kernel itself for up
+// to three tokens, fold_kernel first for more).
 //
 // The state of a unit (batch row, KV head) covers the evicted tokens
 // L = [S, T - W) -- past the sinks and out of the sliding window ("SALSA:
@@ -20,9 +22,9 @@ namespace hyb {
 namespace {
 
 // ---------------------------------------------------------------- append
-// Writes one token per unit at row T of the caches: grid (units), D/4 threads
-// of 16 bytes.  The token's later eviction from the window is folded into the
-// state by the next decode's select kernel, which reads the caches.
+// Writes n tokens per unit at rows [T, T + n) of the caches: grid (units, n),
+// D/4 threads of 16 bytes.  A token's later eviction from the window is folded
+// into the state by the decode after it, which reads the caches.
 template <int D>
 __global__ void __launch_bounds__(D / 4) append_kernel(const AppendParams p) {
   const int unit = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;  // token j of the chunk
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(256) init_stats_kernel(const InitParams p) {
   }
 }
 
-// (3) fp64 accumulators -> fp32 state; reset the tickets and the status word.
+// (3) fp64 accumulators -> fp32 state; reset the status word.
 template <int D>
 __global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) {
   const int unit = blockIdx.x, tid = threadIdx.x;
@@ -243,8 +245,6 @@ __global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) 
   }
   if (tid == 0) {
     p.n[unit] = (float)(p.ev_end - p.ev_begin);
-    p.tickets_sel[unit] = 0u;
-    p.tickets_att[unit] = 0u;
     if (unit == 0) *p.status = 0u;
   }
 }

@@ -79,6 +79,20 @@ class HybridAttentionLayer:
         with torch.cuda.device(self.device):
             self.ctx = A.hyb_attn_init(self.cfg, self.buffers(), T0, _stream(stream))
 
+    def attach(self, T: int, stream=None) -> None:
+        """Bind a context to buffers that already hold the synced state of a
+        history of length T (a restored checkpoint), without rebuilding it."""
+        if self.ctx is not None:
+            A.hyb_attn_destroy(self.ctx)
+        with torch.cuda.device(self.device):
+            self.ctx = A.hyb_attn_attach(self.cfg, self.buffers(), T, _stream(stream))
+
+    def set_wait_limit(self, ns: int) -> None:
+        A.hyb_attn_set_wait_limit(self.ctx, ns)
+
+    def set_test_flags(self, flags: int) -> None:
+        A.hyb_attn_set_test_flags(self.ctx, flags)
+
     @property
     def T(self) -> int:
         return A.hyb_attn_length(self.ctx)

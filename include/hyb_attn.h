@@ -72,6 +72,11 @@ extern "C" {
 #define HYB_STATUS_TIMEOUT       0x8u  /* a bounded wait inside a kernel gave up */
 #define HYB_STATUS_NAN_SCORE     0x10u /* a block score was NaN (ranked last) */
 
+/* ---- failure injection for tests (hyb_attn_set_test_flags) ---------------- */
+#define HYB_TEST_WITHHOLD_SCORES 0x1u  /* rank 1 of every unit's cluster does not hand its block
+                                          scores to the other ranks, whose bounded wait for them
+                                          then runs out (HYB_STATUS_TIMEOUT; outputs invalid) */
+
 /* ---- configuration ------------------------------------------------------- */
 typedef struct hyb_attn_config {
   int32_t batch;       /* B  >= 1 */
@@ -113,7 +118,12 @@ typedef struct hyb_attn_sizes {
  * the evicted tokens up to the last decode: a token that leaves the window is
  * folded in by the next decode (which reads the state anyway), or by
  * hyb_attn_sync_state.  After hyb_attn_sync_state, copying them together with
- * the caches and T is a complete checkpoint of the layer. */
+ * the caches and T is a complete checkpoint of the layer (restored with
+ * hyb_attn_attach).
+ * There is no separate running sum and sum of squares of the newest (open)
+ * block: its mean and variance rows are updated in place, one evicted token at
+ * a time (Welford's update), so the open block is an ordinary candidate row of
+ * mu / var and a decode reads one layout for every block. */
 typedef struct hyb_attn_buffers {
   void*  k_cache;
   void*  v_cache;
@@ -163,6 +173,15 @@ int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_
  * HYB_ENOMEM, HYB_ECUDA.  On error *out is set to NULL. */
 int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
                   int64_t T0, cudaStream_t stream);
+
+/* Create a context over buffers that already hold the synced state of a
+ * history of length T -- the caches' positions [0, T) and H, zk, zv, n, mu,
+ * var exactly as hyb_attn_sync_state left them (a checkpoint copied back by the
+ * caller) -- without rebuilding the state, so that the next decode is
+ * bit-identical to the one the checkpointed context would have made.  Resets
+ * the device status word.  Errors as hyb_attn_init. */
+int hyb_attn_attach(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
+                    int64_t T, cudaStream_t stream);
 
 /* Append one token per unit: k_new, v_new bf16 [B][Hkv][d].  The token is
  * written at position T; then T += 1.  If the token at position T - W - 1
@@ -258,22 +277,22 @@ int hyb_attn_step_host(hyb_attn_ctx* ctx, const void* q_host, const void* k_host
  * library's users.
  *
  * Same arguments and result as hyb_attn_decode without scores_out, but the
- * per-call scratch (block scores, selection, split-K partial records, tickets,
- * status) comes from a fixed device array inside the library, of
- * HYB_NOALLOC_SCRATCH_BYTES (16 MiB) per GPU, that every GPU which loads the
- * library holds until the process exits.  A configuration whose decode scratch
- * exceeds it is rejected with HYB_ESCRATCH (the context's own workspace is not
- * used by this call).  The call allocates nothing: no cudaMalloc, no cudaFree,
- * no allocating library routine.
+ * per-call scratch (the block scores and the selection) comes from a fixed
+ * device array inside the library, of HYB_NOALLOC_SCRATCH_BYTES (16 MiB) per
+ * GPU, that every GPU which loads the library holds until the process exits.
+ * A configuration whose decode scratch exceeds it is rejected with
+ * HYB_ESCRATCH.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.  Its device status bits go to the context's
+ * status word, as for every other call (read with hyb_attn_status).
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  The current device must be the context's device.  All calls share
- * the one array and it keeps the last call's contents: the call clears what
- * must start at zero itself, but calls whose work overlaps on the GPU (two
- * streams, two threads) race on the array and must be serialised by the caller.
- * Device status bits raised by this call stay in the array and are not reported
- * by hyb_attn_status.  Errors: HYB_EINVAL, HYB_ESTATE, HYB_ESCRATCH, HYB_ECUDA. */
+ * the one array and it keeps the last call's contents (nothing in it needs to
+ * start at zero: a decode writes every score and selection entry before it
+ * reads it), so calls whose work overlaps on the GPU (two streams, two
+ * threads) race on the array and must be serialised by the caller.
+ * Errors: HYB_EINVAL, HYB_ESTATE, HYB_ESCRATCH, HYB_ECUDA. */
 #define HYB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int hyb_attn_decode_noalloc(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out, cudaStream_t stream);
 
@@ -281,13 +300,29 @@ int hyb_attn_decode_noalloc(hyb_attn_ctx* ctx, const void* q, float* out, int32_
 int64_t hyb_attn_length(const hyb_attn_ctx* ctx);
 
 /* Copy the device status word to *flags (synchronises `stream`); with clear != 0
- * reset it to zero afterwards.  Returns HYB_OK or HYB_ECUDA. */
+ * reset it to zero afterwards.  Returns HYB_OK or HYB_ECUDA.  The status word
+ * lives in the context's workspace, so reading it is a device-to-host copy on
+ * the caller's stream followed by a synchronisation of that stream (the word is
+ * valid only once the decodes before it have finished), and `clear` lets a
+ * caller poll and reset in one call. */
 int hyb_attn_status(hyb_attn_ctx* ctx, uint32_t* flags, int clear, cudaStream_t stream);
 
 /* Profiling hook: when both events are non-NULL, every later decode records
  * `begin` just before and `end` just after its kernel on the decode's stream,
  * so the caller can time one decode alone.  Pass NULL, NULL to stop. */
 int hyb_attn_set_timing_events(hyb_attn_ctx* ctx, cudaEvent_t begin, cudaEvent_t end);
+
+/* Limit, in nanoseconds, of the kernels' bounded waits for progress (a ring
+ * stage, the other ranks' scores, the selection); 0 restores the default of
+ * 1 s.  A wait that runs out sets HYB_STATUS_TIMEOUT and its CTA skips the
+ * rest of its work; the waits that guard a CTA's exit keep the default.
+ * Accepted: 0 or [1e5, 6e10].  Host only. */
+int hyb_attn_set_wait_limit(hyb_attn_ctx* ctx, uint64_t ns);
+
+/* Failure injection for tests: HYB_TEST_* flags applied to every later decode
+ * (0 turns them off).  No flag faults, traps or hangs the GPU; a withheld
+ * hand-off makes a bounded wait run out.  Host only. */
+int hyb_attn_set_test_flags(hyb_attn_ctx* ctx, uint32_t flags);
 
 /* Release the host context (device buffers stay with the caller). */
 void hyb_attn_destroy(hyb_attn_ctx* ctx);

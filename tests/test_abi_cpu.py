@@ -33,8 +33,24 @@ def test_header_declares_the_boundary():
     for n in ["hyb_attn_init", "hyb_attn_append", "hyb_attn_decode", "hyb_attn_decode_with_selection",
               "hyb_attn_workspace_size", "hyb_attn_length", "hyb_attn_status", "hyb_attn_destroy",
               "hyb_attn_strerror", "hyb_attn_query_sizes", "hyb_attn_plan", "hyb_attn_step_host",
-              "hyb_attn_set_timing_events", "hyb_attn_decode_append", "hyb_attn_sync_state"]:
+              "hyb_attn_set_timing_events", "hyb_attn_decode_append", "hyb_attn_sync_state",
+              "hyb_attn_attach", "hyb_attn_set_wait_limit", "hyb_attn_set_test_flags"]:
         assert n in names, n
+
+
+def test_documented_departures_from_the_scope_table_signatures():
+    """Two documented departures from the survey's sketch of the boundary: the
+    status call takes (ctx, uint32_t* flags, int clear, stream), and the
+    buffers hold no open-block running sums (the open block's mean / variance
+    rows are updated in place)."""
+    src = open(HEADER).read()
+    flat = re.sub(r"\s+", " ", re.sub(r"/\*.*?\*/", "", src, flags=re.S))
+    assert "int hyb_attn_status(hyb_attn_ctx* ctx, uint32_t* flags, int clear, cudaStream_t stream);" in flat
+    body = re.search(r"typedef struct hyb_attn_buffers \{(.*?)\} hyb_attn_buffers;", flat).group(1)
+    fields = re.findall(r"(\w+);", body)
+    assert fields == ["k_cache", "v_cache", "H", "zk", "zv", "n", "mu", "var", "workspace", "workspace_bytes"]
+    assert "open_sum" not in flat and "open_sq" not in flat
+    assert "Welford" in src and "hyb_attn_status" in src
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -100,6 +116,10 @@ def test_init_rejects_bad_arguments_without_touching_a_gpu(lib):
     assert lib.hyb_attn_append_chunk(None, None, None, 4, None) == -1
     assert lib.hyb_attn_decode_chunk(None, None, None, None, 4, None, None, None) == -1
     assert lib.hyb_attn_length(None) == -1
+    assert lib.hyb_attn_set_wait_limit(None, 0) == -1
+    assert lib.hyb_attn_set_test_flags(None, 0) == -1
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_attach(c, buf, 100, 0)
     assert H.hyb_attn_strerror(-2).startswith("KV cache capacity")
 
 

@@ -120,7 +120,7 @@ def test_llama8b_32k_layer_every_unit():
     qb = wl.q_bits(0)
     out, sel = wl.decode(qb)
     wl.check_units(qb, units, out, sel)
-    wl.check_state(units[:2])
+    wl.check_state(units)
     # every planted block is selected
     for h in range(w.n_kv_heads):
         assert set(wl.tables.host.planted[0, h].tolist()) <= set(sel[0, h].tolist())
@@ -136,7 +136,12 @@ def test_llama8b_32k_layer_every_unit():
 def test_llama8b_32layers_b8_32k_sampled(layer):
     w = C.get_workload("llama8b_32layers_b8_32k")
     wl = WorkloadLayer(w, layer, n_app=1)
-    units = [(0, 0), (3, 5), (7, 7), (5, 2)]
+    # the layer's KV heads with the smallest and the largest scale (U(0.5, 2)),
+    # at both batch ends, and two more
+    sc = SH.head_scales(w)[layer]
+    lo, hi = int(np.argmin(sc)), int(np.argmax(sc))
+    rest = [h for h in range(w.n_kv_heads) if h not in (lo, hi)]
+    units = [(0, lo), (7, hi), (3, rest[0]), (5, rest[-1])]
     qb = wl.q_bits(0)
     out, sel = wl.decode(qb)
     wl.check_units(qb, units, out, sel)
@@ -161,20 +166,29 @@ def test_llama8b_32layers_b8_32k_budgets_sampled(layer):
     wl.check_state(units[:2])
 
 
-def test_llama8b_32layers_b4_128k_sampled():
+@pytest.mark.parametrize("layer,units", [
+    (9, [(0, 0), (0, 7), (3, 0), (3, 7), (1, 4)]),     # both batch ends, both ends of the KV heads
+    (22, [(0, 3), (3, 2), (2, 6), (1, 1), (2, 0)]),
+])
+def test_llama8b_32layers_b4_128k_sampled(layer, units):
+    """Ten units over two layers of the 128K workload: every unit's keys carry
+    its own per-block offsets, so the sample spans the offset regime; selection
+    above 512 blocks (2016 candidates, k = 32)."""
     w = C.get_workload("llama8b_32layers_b4_128k")
-    wl = WorkloadLayer(w, 9, n_app=0)
-    units = [(0, 0), (2, 3), (3, 7)]
+    wl = WorkloadLayer(w, layer, n_app=0)
     qb = wl.q_bits(0)
     out, sel = wl.decode(qb)
     wl.check_units(qb, units, out, sel)
+    assert wl.layer.status() == 0
 
 
-def test_llama8b_256k_256_steps_sampled():
+def test_llama8b_256k_256_steps_every_unit():
+    """All 8 units of the 256K workload at steps 0, 97 and 255 of 256 decode +
+    append steps, and the state of every unit after the 256 appends."""
     w = C.get_workload("llama8b_256k_256steps")
     wl = WorkloadLayer(w, 0)
     assert wl.n_app == 256
-    units = [(0, 1), (0, 6)]
+    units = [(0, h) for h in range(w.n_kv_heads)]
     for step in range(w.steps):
         qb = wl.q_bits(step)
         out, sel = wl.decode(qb)

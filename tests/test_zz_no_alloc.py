@@ -32,5 +32,6 @@ def test_decode_noalloc_matches_decode_twice():
         assert torch.equal(sel, sel_ref)
         check_outputs(out.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64),
                       max_abs=OUT_MAX_ABS, rel_l2=OUT_REL_L2)
+        # the call's device status bits land in the context's status word
+        assert c.layer.status() == 0
         c.append()   # the second call sees a longer history
-    assert c.layer.status() == 0
