@@ -16,7 +16,9 @@ from ._abi import (  # noqa: F401
     hyb_attn_workspace_size,
     hyb_attn_plan,
     hyb_attn_init,
+    hyb_attn_init_rows,
     hyb_attn_attach,
+    hyb_attn_attach_rows,
     hyb_attn_append,
     hyb_attn_append_chunk,
     hyb_attn_sync_state,
@@ -25,8 +27,11 @@ from ._abi import (  # noqa: F401
     hyb_attn_decode_chunk,
     hyb_attn_decode_with_selection,
     hyb_attn_step_host,
+    hyb_attn_step_layers_staging_bytes,
+    hyb_attn_step_layers_host,
     hyb_attn_decode_noalloc,
     hyb_attn_length,
+    hyb_attn_row_length,
     hyb_attn_status,
     hyb_attn_set_timing_events,
     hyb_attn_set_wait_limit,

@@ -37,7 +37,8 @@ c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float
 class hyb_attn_config(ctypes.Structure):
     _fields_ = [("batch", c_i32), ("n_q_heads", c_i32), ("n_kv_heads", c_i32), ("head_dim", c_i32),
                 ("block_size", c_i32), ("n_sink", c_i32), ("window", c_i32), ("top_k", c_i32),
-                ("capacity", c_i64), ("scale", c_f32)]
+                ("capacity", c_i64), ("scale", c_f32),
+                ("head_window", ctypes.POINTER(c_i32)), ("head_top_k", ctypes.POINTER(c_i32))]
 
 
 class hyb_attn_sizes(ctypes.Structure):
@@ -63,8 +64,12 @@ SIGNATURES = [
                                      ctypes.POINTER(hyb_attn_plan_info)]),
     ("hyb_attn_init", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
                                      ctypes.POINTER(hyb_attn_buffers), c_i64, c_vp]),
+    ("hyb_attn_init_rows", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
+                                          ctypes.POINTER(hyb_attn_buffers), ctypes.POINTER(c_i64), c_vp]),
     ("hyb_attn_attach", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
                                        ctypes.POINTER(hyb_attn_buffers), c_i64, c_vp]),
+    ("hyb_attn_attach_rows", ctypes.c_int, [ctypes.POINTER(c_vp), ctypes.POINTER(hyb_attn_config),
+                                            ctypes.POINTER(hyb_attn_buffers), ctypes.POINTER(c_i64), c_vp]),
     ("hyb_attn_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_append_chunk", ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_vp]),
     ("hyb_attn_sync_state", ctypes.c_int, [c_vp, c_vp]),
@@ -73,8 +78,11 @@ SIGNATURES = [
     ("hyb_attn_decode_chunk", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_with_selection", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_step_host", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_step_layers_staging_bytes", c_sz, [ctypes.POINTER(c_vp), c_i32]),
+    ("hyb_attn_step_layers_host", ctypes.c_int, [ctypes.POINTER(c_vp), c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
     ("hyb_attn_decode_noalloc", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_length", c_i64, [c_vp]),
+    ("hyb_attn_row_length", c_i64, [c_vp, c_i32]),
     ("hyb_attn_status", ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, c_vp]),
     ("hyb_attn_set_timing_events", ctypes.c_int, [c_vp, c_vp, c_vp]),
     ("hyb_attn_set_wait_limit", ctypes.c_int, [c_vp, ctypes.c_uint64]),
@@ -152,6 +160,25 @@ def hyb_attn_init(cfg: hyb_attn_config, buf: hyb_attn_buffers, T0: int, stream: 
     return h.value
 
 
+def _i64_array(vals):
+    return (c_i64 * len(vals))(*[int(v) for v in vals])
+
+
+def hyb_attn_init_rows(cfg: hyb_attn_config, buf: hyb_attn_buffers, row_T0, stream: int) -> int:
+    h = c_vp()
+    _check("hyb_attn_init_rows", load_library().hyb_attn_init_rows(ctypes.byref(h), ctypes.byref(cfg),
+                                                                   ctypes.byref(buf), _i64_array(row_T0), stream))
+    return h.value
+
+
+def hyb_attn_attach_rows(cfg: hyb_attn_config, buf: hyb_attn_buffers, row_T, stream: int) -> int:
+    h = c_vp()
+    _check("hyb_attn_attach_rows", load_library().hyb_attn_attach_rows(ctypes.byref(h), ctypes.byref(cfg),
+                                                                       ctypes.byref(buf), _i64_array(row_T),
+                                                                       stream))
+    return h.value
+
+
 def hyb_attn_attach(cfg: hyb_attn_config, buf: hyb_attn_buffers, T: int, stream: int) -> int:
     h = c_vp()
     _check("hyb_attn_attach", load_library().hyb_attn_attach(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(buf),
@@ -196,6 +223,21 @@ def hyb_attn_step_host(ctx: int, q_host: int, k_host, v_host, out_host: int, str
     _check("hyb_attn_step_host", load_library().hyb_attn_step_host(ctx, q_host, k_host, v_host, out_host, stream))
 
 
+def _ctx_array(ctxs):
+    return (c_vp * len(ctxs))(*ctxs)
+
+
+def hyb_attn_step_layers_staging_bytes(ctxs) -> int:
+    return int(load_library().hyb_attn_step_layers_staging_bytes(_ctx_array(ctxs), len(ctxs)))
+
+
+def hyb_attn_step_layers_host(ctxs, in_host: int, out_host: int, staging: int, staging_bytes: int,
+                              stream: int) -> None:
+    _check("hyb_attn_step_layers_host",
+           load_library().hyb_attn_step_layers_host(_ctx_array(ctxs), len(ctxs), in_host, out_host, staging,
+                                                    staging_bytes, stream))
+
+
 def hyb_attn_decode_noalloc(ctx: int, q: int, out: int, sel_out, stream: int) -> None:
     """Decode with the block scores and the selection in the library's fixed
     device array instead of the context's workspace (for callers that cannot
@@ -205,6 +247,10 @@ def hyb_attn_decode_noalloc(ctx: int, q: int, out: int, sel_out, stream: int) ->
 
 def hyb_attn_length(ctx: int) -> int:
     return int(load_library().hyb_attn_length(ctx))
+
+
+def hyb_attn_row_length(ctx: int, b: int) -> int:
+    return int(load_library().hyb_attn_row_length(ctx, b))
 
 
 def hyb_attn_status(ctx: int, clear: bool, stream: int) -> int:

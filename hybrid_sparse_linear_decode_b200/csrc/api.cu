@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <new>
 
@@ -52,6 +53,15 @@ int check_config(const hyb_attn_config* c, Checked* out) {
   const int64_t ev_cap = c->capacity - c->n_sink - c->window;
   const int64_t mb = ev_cap > 0 ? ceil_div(ev_cap, c->block_size) : 0;
   if (mb >= ((int64_t)1 << 30)) return HYB_EINVAL;
+  // per-head budgets refine (window, top_k): windows at least `window`, top-k at most `top_k`
+  if ((c->head_window == nullptr) != (c->head_top_k == nullptr)) return HYB_EINVAL;
+  if (c->head_window != nullptr) {
+    if (c->n_kv_heads > kMaxHeadBudgets) return HYB_EINVAL;
+    for (int h = 0; h < c->n_kv_heads; ++h) {
+      if (c->head_window[h] < c->window || c->head_top_k[h] < 0 || c->head_top_k[h] > c->top_k) return HYB_EINVAL;
+      if ((int64_t)c->n_sink + c->head_window[h] >= ((int64_t)1 << 30)) return HYB_EINVAL;
+    }
+  }
   if (out) {
     out->D = c->head_dim;
     out->G = G;
@@ -200,8 +210,9 @@ struct hyb_attn_ctx {
   hyb_attn_buffers buf;
   Checked ck;
   WsLayout ws;
-  int64_t T;
-  int64_t folded_end;   // the state holds the evicted positions [S, folded_end)
+  int64_t T;            // length of the longest row (row b: T - tb.row_lag[b])
+  int64_t pending;      // appends whose evictions are not folded into the state yet
+  UnitTables tb;        // per-row lengths and per-head budgets (uniform when not given)
   int device, n_sm;
   int fits[kMaxCluster + 1];  // clusters of C CTAs of the decode kernel the device holds at once
   float scale;
@@ -218,7 +229,7 @@ struct hyb_attn_ctx {
 
 namespace {
 
-FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
+FusedParams fused_params(const hyb_attn_ctx* x) {
   const hyb_attn_config& c = x->cfg;
   const Checked& k = x->ck;
   FusedParams fp{};
@@ -235,22 +246,15 @@ FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   fp.status = x->status;
   fp.cap = c.capacity;
   fp.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
-  fp.fold_begin = x->folded_end;
-  fp.fold_end = g.ev_end;
-  fp.T = (int32_t)g.T;
+  fp.T = (int32_t)x->T;
   fp.S = c.n_sink;
+  fp.W = c.window;
   fp.Bk = c.block_size;
   fp.top_k = c.top_k;
-  fp.nb = (int32_t)g.nb;
-  fp.k_eff = (int32_t)g.k_eff;
-  fp.sink_len = (int32_t)g.sink_len;
-  fp.win_start = (int32_t)g.win_start;
-  fp.ev_end = (int32_t)g.ev_end;
-  fp.n_sink_chunks = g.n_sink_chunks;
-  fp.n_win_chunks = g.n_win_chunks;
-  fp.chunks_per_block = g.chunks_per_block;
-  fp.n_sel_chunks = g.n_sel_chunks;
+  fp.pending = (int32_t)x->pending;
+  fp.chunks_per_block = (int32_t)ceil_div(c.block_size, kTile);
   fp.units = k.units;
+  fp.Hkv = c.n_kv_heads;
   fp.G = k.G;
   fp.C = cluster_ctas(k.units, x->n_sm, x->fits);
   fp.mstride = merge_stride(k.G * k.D, fp.C);
@@ -258,14 +262,15 @@ FusedParams fused_params(const hyb_attn_ctx* x, const Geometry& g) {
   fp.scale = x->scale;
   fp.wait_ns = x->wait_ns;
   fp.test_flags = x->test_flags;
+  fp.tb = x->tb;
   return fp;
 }
 
-// Several pending evictions (a chunked append, or many appends since the last
-// fold): one dense pass of fold_kernel over them, so that the decode kernel
-// folds at most a few tokens itself.
-int fold_pending(hyb_attn_ctx* x, const Geometry& g, cudaStream_t stream) {
-  if (g.ev_end - x->folded_end < kFoldKernelMin) return HYB_OK;
+// Several pending appends (a chunked append, or many appends since the last
+// fold): one dense pass of fold_kernel over every unit's evictions, so that the
+// decode kernel folds at most a few tokens itself.
+int fold_pending(hyb_attn_ctx* x, cudaStream_t stream) {
+  if (x->pending < kFoldKernelMin) return HYB_OK;
   FoldParams p{};
   p.k_cache = static_cast<const __nv_bfloat16*>(x->buf.k_cache);
   p.v_cache = static_cast<const __nv_bfloat16*>(x->buf.v_cache);
@@ -277,14 +282,17 @@ int fold_pending(hyb_attn_ctx* x, const Geometry& g, cudaStream_t stream) {
   p.var = x->buf.var;
   p.cap = x->cfg.capacity;
   p.max_blocks = x->ck.max_blocks > 0 ? x->ck.max_blocks : 1;
-  p.fb = x->folded_end;
-  p.fe = g.ev_end;
-  p.units = x->ck.units;
+  p.T = (int32_t)x->T;
   p.S = x->cfg.n_sink;
+  p.W = x->cfg.window;
   p.Bk = x->cfg.block_size;
+  p.pending = (int32_t)x->pending;
+  p.units = x->ck.units;
+  p.Hkv = x->cfg.n_kv_heads;
+  p.tb = x->tb;
   const cudaError_t e = launch_fold(p, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  x->folded_end = g.ev_end;
+  x->pending = 0;
   return HYB_OK;
 }
 
@@ -302,10 +310,9 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   if (k_new != nullptr && (!aligned16(k_new) || !aligned16(v_new))) return HYB_EINVAL;
   if (x->T == 0) return HYB_ESTATE;
   if (k_new != nullptr && x->T >= x->cfg.capacity) return HYB_ECAPACITY;
-  const Geometry g = geometry(x->cfg, x->T);
-  const int rf = fold_pending(x, g, stream);
+  const int rf = fold_pending(x, stream);
   if (rf != HYB_OK) return rf;
-  FusedParams fp = fused_params(x, g);
+  FusedParams fp = fused_params(x);
   fp.q = static_cast<const __nv_bfloat16*>(q);
   if (scores_out) fp.scores = scores_out;
   fp.sel_given = sel_given;
@@ -317,8 +324,11 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
   const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  x->folded_end = g.ev_end;
-  if (k_new != nullptr) x->T += 1;
+  x->pending = 0;
+  if (k_new != nullptr) {  // the new token's eviction, if any, is folded by the next decode
+    x->T += 1;
+    x->pending = 1;
+  }
   if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
   return HYB_OK;
 }
@@ -370,10 +380,29 @@ namespace {
 
 // Validate a configuration and its buffers and build the host context of a
 // layer at length T (TMA descriptors, kernel attributes); no kernel is launched.
-int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T, hyb_attn_ctx** out) {
+int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T, const int64_t* row_T,
+               hyb_attn_ctx** out) {
   Checked k;
   if (check_config(cfg, &k) != HYB_OK || buf == nullptr) return HYB_EINVAL;
+  UnitTables tb{};
+  if (row_T != nullptr) {  // per-row lengths: T is the longest, row b lags it by T - row_T[b]
+    if (cfg->batch > kMaxRaggedRows) return HYB_EINVAL;
+    T = 0;
+    for (int b = 0; b < cfg->batch; ++b) {
+      if (row_T[b] < 1 || row_T[b] > cfg->capacity) return HYB_EINVAL;
+      T = row_T[b] > T ? row_T[b] : T;
+    }
+    tb.ragged = 1;
+    for (int b = 0; b < cfg->batch; ++b) tb.row_lag[b] = (int32_t)(T - row_T[b]);
+  }
   if (T < 0 || T > cfg->capacity) return HYB_EINVAL;
+  if (cfg->head_window != nullptr) {
+    tb.per_head = 1;
+    for (int h = 0; h < cfg->n_kv_heads; ++h) {
+      tb.head_W[h] = cfg->head_window[h];
+      tb.head_k[h] = cfg->head_top_k[h];
+    }
+  }
   const void* ptrs[] = {buf->k_cache, buf->v_cache, buf->H, buf->zk, buf->zv, buf->n, buf->workspace};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return HYB_EINVAL;
@@ -393,10 +422,13 @@ int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t 
   hyb_attn_ctx* x = new (std::nothrow) hyb_attn_ctx();
   if (x == nullptr) return HYB_ENOMEM;
   x->cfg = *cfg;
+  x->cfg.head_window = x->cfg.head_top_k = nullptr;  // the caller's arrays are copied into tb
   x->buf = *buf;
   x->ck = k;
   x->ws = ws;
   x->T = T;
+  x->pending = 0;
+  x->tb = tb;
   x->device = device;
   x->n_sm = n_sm;
   for (int c = 0; c <= kMaxCluster; ++c) x->fits[c] = 0;
@@ -420,7 +452,6 @@ int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t 
     return cuda_fail(pe);
   }
   for (int c = 2; c <= kMaxCluster; ++c) x->fits[c] = fused_max_clusters(k.D, c);
-  x->folded_end = geometry(*cfg, T).ev_end;
   *out = x;
   return HYB_OK;
 }
@@ -429,16 +460,18 @@ int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t 
 
 extern "C" {
 
-int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T0,
-                  cudaStream_t stream) {
-  HYB_RANGE;
+}  // extern "C"
+
+namespace {
+
+int init_impl(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T0,
+              const int64_t* row_T0, cudaStream_t stream) {
   if (out == nullptr) return HYB_EINVAL;
   *out = nullptr;
   hyb_attn_ctx* x = nullptr;
-  const int rc = create_ctx(cfg, buf, T0, &x);
+  const int rc = create_ctx(cfg, buf, T0, row_T0, &x);
   if (rc != HYB_OK) return rc;
   const Checked& k = x->ck;
-  const Geometry g = geometry(*cfg, T0);
   InitParams ip{};
   ip.k_cache = static_cast<const __nv_bfloat16*>(buf->k_cache);
   ip.v_cache = static_cast<const __nv_bfloat16*>(buf->v_cache);
@@ -453,12 +486,22 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   ip.status = x->status;
   ip.cap = cfg->capacity;
   ip.max_blocks = k.max_blocks > 0 ? k.max_blocks : 1;
-  ip.ev_begin = cfg->n_sink;
-  ip.ev_end = g.ev_end;
-  ip.units = k.units;
+  ip.T = (int32_t)x->T;
   ip.S = cfg->n_sink;
+  ip.W = cfg->window;
   ip.Bk = cfg->block_size;
-  ip.nb = (int32_t)g.nb;
+  ip.units = k.units;
+  ip.Hkv = cfg->n_kv_heads;
+  ip.tb = x->tb;
+  // the longest evicted range and the most blocks over the units (the grid's extent)
+  int64_t ev_max = 0;
+  for (int u = 0; u < k.units; ++u) {
+    const UnitGeo g = unit_geo(x->tb, u, cfg->n_kv_heads, (int32_t)x->T, cfg->n_sink, cfg->window,
+                               cfg->block_size, 0, 1, 0);
+    ev_max = std::max<int64_t>(ev_max, g.ev_end - cfg->n_sink);
+  }
+  ip.ev_max = (int32_t)ev_max;
+  ip.nb_max = (int32_t)ceil_div(ev_max, cfg->block_size);
   ip.tokens_per_cta = 2048;
   cudaError_t e = cudaMemsetAsync(ip.H64, 0, (size_t)k.units * k.D * k.D * sizeof(double), stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(ip.z64, 0, (size_t)k.units * 2 * k.D * sizeof(double), stream);
@@ -471,13 +514,12 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
   return HYB_OK;
 }
 
-int hyb_attn_attach(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T,
-                    cudaStream_t stream) {
-  HYB_RANGE;
+int attach_impl(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T,
+                const int64_t* row_T, cudaStream_t stream) {
   if (out == nullptr) return HYB_EINVAL;
   *out = nullptr;
   hyb_attn_ctx* x = nullptr;
-  const int rc = create_ctx(cfg, buf, T, &x);
+  const int rc = create_ctx(cfg, buf, T, row_T, &x);
   if (rc != HYB_OK) return rc;
   const cudaError_t e = cudaMemsetAsync(x->status, 0, sizeof(uint32_t), stream);
   if (e != cudaSuccess) {
@@ -486,6 +528,36 @@ int hyb_attn_attach(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_at
   }
   *out = x;
   return HYB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T0,
+                  cudaStream_t stream) {
+  HYB_RANGE;
+  return init_impl(out, cfg, buf, T0, nullptr, stream);
+}
+
+int hyb_attn_init_rows(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
+                       const int64_t* row_T0, cudaStream_t stream) {
+  HYB_RANGE;
+  if (row_T0 == nullptr) return HYB_EINVAL;
+  return init_impl(out, cfg, buf, 0, row_T0, stream);
+}
+
+int hyb_attn_attach(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t T,
+                    cudaStream_t stream) {
+  HYB_RANGE;
+  return attach_impl(out, cfg, buf, T, nullptr, stream);
+}
+
+int hyb_attn_attach_rows(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
+                         const int64_t* row_T, cudaStream_t stream) {
+  HYB_RANGE;
+  if (row_T == nullptr) return HYB_EINVAL;
+  return attach_impl(out, cfg, buf, 0, row_T, stream);
 }
 
 int hyb_attn_append_chunk(hyb_attn_ctx* x, const void* k_new, const void* v_new, int32_t n, cudaStream_t stream) {
@@ -499,12 +571,15 @@ int hyb_attn_append_chunk(hyb_attn_ctx* x, const void* k_new, const void* v_new,
   p.k_cache = static_cast<__nv_bfloat16*>(x->buf.k_cache);
   p.v_cache = static_cast<__nv_bfloat16*>(x->buf.v_cache);
   p.cap = x->cfg.capacity;
-  p.T = x->T;
+  p.T = (int32_t)x->T;
   p.units = x->ck.units;
+  p.Hkv = x->cfg.n_kv_heads;
   p.n = n;
+  p.tb = x->tb;
   const cudaError_t e = launch_append(p, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->T += n;
+  x->pending += n;  // their evictions are folded by the next decode or state sync
   return HYB_OK;
 }
 
@@ -515,13 +590,12 @@ int hyb_attn_append(hyb_attn_ctx* x, const void* k_new, const void* v_new, cudaS
 int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
   HYB_RANGE;
   if (x == nullptr) return HYB_EINVAL;
-  const Geometry g = geometry(x->cfg, x->T);
-  if (g.ev_end <= x->folded_end) return HYB_OK;  // nothing evicted since the last fold
-  if (g.ev_end - x->folded_end >= kFoldKernelMin) return fold_pending(x, g, stream);
-  FusedParams fp = fused_params(x, g);           // q == null: fold only
+  if (x->pending == 0) return HYB_OK;  // nothing appended since the last fold
+  if (x->pending >= kFoldKernelMin) return fold_pending(x, stream);
+  FusedParams fp = fused_params(x);   // q == null: fold only
   const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  x->folded_end = g.ev_end;
+  x->pending = 0;
   return HYB_OK;
 }
 
@@ -587,6 +661,55 @@ int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, 
   return HYB_OK;
 }
 
+size_t hyb_attn_step_layers_staging_bytes(hyb_attn_ctx* const* ctxs, int32_t n_layers) {
+  if (ctxs == nullptr || n_layers < 1) return 0;
+  size_t in = 0, out = 0;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const hyb_attn_ctx* x = ctxs[l];
+    if (x == nullptr) return 0;
+    const size_t U = (size_t)x->ck.units, D = (size_t)x->ck.D, G = (size_t)x->ck.G;
+    in += U * G * D * 2 + 2 * U * D * 2;
+    out += U * G * D * 4;
+  }
+  return align_up(in) + out;
+}
+
+int hyb_attn_step_layers_host(hyb_attn_ctx* const* ctxs, int32_t n_layers, const void* in_host, float* out_host,
+                              void* staging, size_t staging_bytes, cudaStream_t stream) {
+  HYB_RANGE;
+  if (ctxs == nullptr || n_layers < 1 || in_host == nullptr || out_host == nullptr || staging == nullptr)
+    return HYB_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(staging) & (kAlign - 1)) != 0) return HYB_EINVAL;
+  const size_t need = hyb_attn_step_layers_staging_bytes(ctxs, n_layers);
+  if (need == 0 || staging_bytes < need) return HYB_EINVAL;
+  size_t in_bytes = 0, out_bytes = 0;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const hyb_attn_ctx* x = ctxs[l];
+    if (x->T >= x->cfg.capacity) return HYB_ECAPACITY;  // nothing is enqueued when a layer is full
+    const size_t U = (size_t)x->ck.units, D = (size_t)x->ck.D, G = (size_t)x->ck.G;
+    in_bytes += U * G * D * 2 + 2 * U * D * 2;
+    out_bytes += U * G * D * 4;
+  }
+  uint8_t* din = static_cast<uint8_t*>(staging);
+  float* dout = reinterpret_cast<float*>(din + align_up(in_bytes));
+  // one copy in, every layer's decode + append back to back (chained launches), one copy out
+  if (cudaMemcpyAsync(din, in_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess) return HYB_ECUDA;
+  size_t ioff = 0, ooff = 0;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    hyb_attn_ctx* x = ctxs[l];
+    const size_t U = (size_t)x->ck.units, D = (size_t)x->ck.D, G = (size_t)x->ck.G;
+    const uint8_t* q = din + ioff;
+    const uint8_t* k = q + U * G * D * 2;
+    const uint8_t* v = k + U * D * 2;
+    const int rc = decode_impl(x, q, dout + ooff, nullptr, nullptr, nullptr, k, v, stream);
+    if (rc != HYB_OK) return rc;
+    ioff += U * G * D * 2 + 2 * U * D * 2;
+    ooff += U * G * D;
+  }
+  if (cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return HYB_ECUDA;
+  return HYB_OK;
+}
+
 int hyb_attn_decode_noalloc(hyb_attn_ctx* x, const void* q, float* out, int32_t* sel_out, cudaStream_t stream) {
   HYB_RANGE;
   if (x == nullptr) return HYB_EINVAL;
@@ -606,11 +729,16 @@ int hyb_attn_decode_noalloc(hyb_attn_ctx* x, const void* q, float* out, int32_t*
   view.buf.workspace = scratch;
   view.buf.workspace_bytes = HYB_NOALLOC_SCRATCH_BYTES;
   const int drc = decode_impl(&view, q, out, nullptr, sel_out, nullptr, nullptr, nullptr, stream);
-  x->folded_end = view.folded_end;  // the state buffers are the context's own
+  x->pending = view.pending;  // the state buffers are the context's own
   return drc;
 }
 
 int64_t hyb_attn_length(const hyb_attn_ctx* x) { return x ? x->T : -1; }
+
+int64_t hyb_attn_row_length(const hyb_attn_ctx* x, int32_t b) {
+  if (x == nullptr || b < 0 || b >= x->cfg.batch) return -1;
+  return x->T - (x->tb.ragged ? x->tb.row_lag[b] : 0);
+}
 
 int hyb_attn_status(hyb_attn_ctx* x, uint32_t* flags, int clear, cudaStream_t stream) {
   HYB_RANGE;

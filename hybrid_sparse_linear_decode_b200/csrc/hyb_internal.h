@@ -35,7 +35,7 @@ __host__ __device__ constexpr int merge_floats(int D, int C = 1) {
                                                                                : merge_floats(D, C + 1));
 }
 
-struct Geometry {        // everything a decode at length T needs, computed on the host
+struct Geometry {        // a decode at length T with the configuration's uniform budget (host: plan, sizes)
   int64_t T;
   int64_t nb;            // candidate blocks
   int64_t k_eff;         // min(top_k, nb)
@@ -44,6 +44,52 @@ struct Geometry {        // everything a decode at length T needs, computed on t
   int64_t ev_end;        // T - W when T > S + W else S
   int32_t n_sink_chunks, n_win_chunks, chunks_per_block, n_sel_chunks, chunks_per_unit;
 };
+
+constexpr int kMaxRaggedRows = 128;   // batch rows that may have lengths of their own
+constexpr int kMaxHeadBudgets = 32;   // KV heads that may have a (top_k, window) of their own
+
+// What makes one unit's length and budget differ from another's.  Row b of the
+// batch has length T - row_lag[b] (every row grows by the same appends), KV
+// head h has window head_W[h] and top-k head_k[h]; uniform when the flags are 0.
+struct UnitTables {
+  int32_t ragged, per_head;
+  int32_t row_lag[kMaxRaggedRows];
+  int32_t head_W[kMaxHeadBudgets];
+  int32_t head_k[kMaxHeadBudgets];
+};
+
+// One unit's geometry at the current step, derived on the device from the
+// launch's T, S, W, Bk, top_k, the tables and the number of appends whose
+// evictions are not yet folded (`pending`).
+struct UnitGeo {
+  int32_t T;             // this row's length
+  int32_t W, top_k;      // this head's window and top-k
+  int32_t sink_len, win_start, ev_end, nb, k_eff;
+  int32_t n_sink_chunks, n_win_chunks, n_sel_chunks;
+  int32_t fold_begin, fold_end;   // evicted positions not yet in the state
+};
+
+__host__ __device__ inline int32_t ev_end_at(int32_t T, int32_t S, int32_t W) { return T > S + W ? T - W : S; }
+
+__host__ __device__ inline UnitGeo unit_geo(const UnitTables& tb, int unit, int Hkv, int32_t T, int32_t S,
+                                            int32_t W, int32_t Bk, int32_t top_k, int32_t cpb, int32_t pending) {
+  UnitGeo g;
+  const int b = unit / Hkv, h = unit - b * Hkv;
+  g.T = T - (tb.ragged ? tb.row_lag[b] : 0);
+  g.W = tb.per_head ? tb.head_W[h] : W;
+  g.top_k = tb.per_head ? tb.head_k[h] : top_k;
+  g.sink_len = g.T < S ? g.T : S;
+  g.win_start = g.T > S ? (g.T - g.W > S ? g.T - g.W : S) : g.T;
+  g.ev_end = ev_end_at(g.T, S, g.W);
+  g.nb = g.ev_end > S ? (g.ev_end - S + Bk - 1) / Bk : 0;
+  g.k_eff = g.top_k < g.nb ? g.top_k : g.nb;
+  g.n_sink_chunks = (g.sink_len + kTile - 1) / kTile;
+  g.n_win_chunks = (g.T - g.win_start + kTile - 1) / kTile;
+  g.n_sel_chunks = g.k_eff * cpb;
+  g.fold_end = g.ev_end;
+  g.fold_begin = ev_end_at(g.T - pending > 0 ? g.T - pending : 0, S, g.W);
+  return g;
+}
 
 struct FusedParams {           // one decode (or, with q == null, the fold only) of one layer
   const __nv_bfloat16* q;       // [B][Hq][D]
@@ -55,7 +101,7 @@ struct FusedParams {           // one decode (or, with q == null, the fold only)
   float* n;                     // [units]
   __nv_bfloat16* k_cache;       // [units][cap][D]
   __nv_bfloat16* v_cache;
-  const __nv_bfloat16* k_new;   // optional token written at row T: [units][D]
+  const __nv_bfloat16* k_new;   // optional token written at each row's position T: [units][D]
   const __nv_bfloat16* v_new;
   float* scores;                // [units][max_blocks] (workspace, or the caller's buffer)
   const int32_t* sel_given;     // [units][top_k] caller's selection, or null: top-k of the scores
@@ -64,40 +110,42 @@ struct FusedParams {           // one decode (or, with q == null, the fold only)
   uint32_t* status;
   float* out;                   // [B][Hq][D]
   int64_t cap, max_blocks;
-  int64_t fold_begin, fold_end; // evicted positions not yet in the state
-  int32_t T, S, Bk, top_k, nb, k_eff;
-  int32_t sink_len, win_start, ev_end;
-  int32_t n_sink_chunks, n_win_chunks, chunks_per_block, n_sel_chunks;
-  int32_t units, G, C;          // C: CTAs (cluster size) per unit
+  int32_t T, S, W, Bk, top_k;   // T: the longest row; W, top_k: uniform budget (top_k: row stride of sel)
+  int32_t pending;              // appends whose evictions are not folded yet
+  int32_t chunks_per_block;
+  int32_t units, Hkv, G, C;     // C: CTAs (cluster size) per unit
   int32_t mstride;              // merge: floats per sending rank's slot (merge_stride)
   int32_t mslice[kMaxCluster + 1];  // merge: rank r merges outputs [mslice[r], mslice[r + 1])
   float scale;
-  uint64_t wait_ns;             // limit of every bounded wait inside the kernel
+  uint64_t wait_ns;             // limit of every bounded wait for progress inside the kernel
   uint32_t test_flags;          // HYB_TEST_* (0 in normal use)
+  UnitTables tb;
 };
 
-struct AppendParams {       // write n tokens per unit at positions [T, T + n)
+struct AppendParams {       // write n tokens per unit at each row's positions [T_b, T_b + n)
   const __nv_bfloat16* k_new; // [units][n][D]
   const __nv_bfloat16* v_new;
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
-  int64_t cap, T;
-  int32_t units, n;
+  int64_t cap;
+  int32_t T, units, Hkv, n;
+  UnitTables tb;
 };
 
-struct FoldParams {         // fold the evicted positions [fb, fe) of every unit into the state
+struct FoldParams {         // fold every unit's pending evicted positions into the state
   const __nv_bfloat16* k_cache;
   const __nv_bfloat16* v_cache;
   float* H; float* zk; float* zv; float* n; float* mu; float* var;
   int64_t cap, max_blocks;
-  int64_t fb, fe;
-  int32_t units, S, Bk;
+  int32_t T, S, W, Bk, pending;
+  int32_t units, Hkv;
+  UnitTables tb;
 };
-// pending evictions from which a decode or a state sync folds them with
+// pending appends from which a decode or a state sync folds the evictions with
 // fold_kernel (one dense pass) instead of inside the decode kernel
 constexpr int64_t kFoldKernelMin = 4;
 
-struct InitParams {
+struct InitParams {          // the state of every unit's evicted range [S, ev_end(T_b, W_h))
   const __nv_bfloat16* k_cache;
   const __nv_bfloat16* v_cache;
   float* H; float* zk; float* zv; float* n; float* mu; float* var;
@@ -105,8 +153,10 @@ struct InitParams {
   double* z64;                // [units][2][D]
   uint32_t* status;
   int64_t cap, max_blocks;
-  int64_t ev_begin, ev_end;   // evicted range [S, T0 - W)
-  int32_t units, S, Bk, nb, tokens_per_cta;
+  int32_t T, S, W, Bk;
+  int32_t units, Hkv, nb_max, ev_max;   // the largest block count and evicted length over the units
+  int32_t tokens_per_cta;
+  UnitTables tb;
 };
 
 // Launchers (kernels live in the .cu files); return cudaError_t of the launch.

@@ -199,6 +199,7 @@ struct FusedSmem {
   uint64_t scores_bar;                               // C arrivals: every rank's scores are in place
   uint64_t sel_bar;                                  // 1 arrival: the selection is known
   uint64_t merge_bar;                                // 1 arrival + the other ranks' merge bytes
+  UnitGeo geo;                                       // this unit's geometry
   int sel_state;                                     // 1 sel_cache, 2 global row (sel_row), 3 every block
   const int32_t* sel_row;
   int abort;
@@ -261,23 +262,23 @@ __device__ __forceinline__ void block_share(int nb, int C, int r, int& b0, int& 
 }
 // Does this launch select the top-k from the scores (else: the caller's row,
 // every block, or none)?
-__device__ __forceinline__ bool runs_topk(const FusedParams& p) {
-  return p.q != nullptr && p.sel_given == nullptr && p.k_eff > 0 && p.k_eff < p.nb;
+__device__ __forceinline__ bool runs_topk(const FusedParams& p, const UnitGeo& g) {
+  return p.q != nullptr && p.sel_given == nullptr && g.k_eff > 0 && g.k_eff < g.nb;
 }
 
 template <int D>
-__device__ __forceinline__ Seq make_seq(const FusedParams& p, int r) {
+__device__ __forceinline__ Seq make_seq(const FusedParams& p, const UnitGeo& g, int r) {
   Seq q;
   const int C = p.C;
-  block_share(p.nb, C, r, q.b0, q.b1);
+  block_share(g.nb, C, r, q.b0, q.b1);
   q.nS = (q.b1 - q.b0 + Geo<D>::kBlocks - 1) / Geo<D>::kBlocks;
   q.h0 = r * D / C;
   q.h1 = (r + 1) * D / C;
   q.nH = (q.h1 - q.h0 + Geo<D>::kRows - 1) / Geo<D>::kRows;
-  const int n_pre = p.n_sink_chunks + p.n_win_chunks;
+  const int n_pre = g.n_sink_chunks + g.n_win_chunks;
   if (p.q != nullptr) {
     q.nW = r < n_pre ? (n_pre - r + C - 1) / C : 0;
-    q.nX = r < p.n_sel_chunks ? (p.n_sel_chunks - r + C - 1) / C : 0;
+    q.nX = r < g.n_sel_chunks ? (g.n_sel_chunks - r + C - 1) / C : 0;
   } else {
     q.nW = q.nX = 0;
   }
@@ -294,11 +295,11 @@ __device__ __forceinline__ int seq_of_chunk(const Seq& s, int c) { return c < s.
 // Score items [*i0, *i1) of the rank hold the blocks with pending evictions
 // (empty when nothing is pending).  Computed once per launch.
 template <int D>
-__device__ __forceinline__ void fold_items(const FusedParams& p, const Seq& s, int* i0, int* i1) {
+__device__ __forceinline__ void fold_items(const FusedParams& p, const UnitGeo& g, const Seq& s, int* i0, int* i1) {
   *i0 = *i1 = 0;
-  if (p.fold_end <= p.fold_begin || s.b1 <= s.b0) return;
+  if (g.fold_end <= g.fold_begin || s.b1 <= s.b0) return;
   // positions fit in 32 bits (units x capacity < 2^31)
-  const int jb0 = (int)(p.fold_begin - p.S) / p.Bk, jb1 = (int)(p.fold_end - 1 - p.S) / p.Bk;
+  const int jb0 = (int)(g.fold_begin - p.S) / p.Bk, jb1 = (int)(g.fold_end - 1 - p.S) / p.Bk;
   const int lo = max(jb0, s.b0), hi = min(jb1, s.b1 - 1);
   if (lo > hi) return;
   *i0 = (lo - s.b0) / Geo<D>::kBlocks;
@@ -306,9 +307,9 @@ __device__ __forceinline__ void fold_items(const FusedParams& p, const Seq& s, i
 }
 // score item idx: does it hold a block with pending evictions?
 template <int D>
-__device__ __forceinline__ bool score_item_folds(const FusedParams& p, const Seq& s, int idx) {
+__device__ __forceinline__ bool score_item_folds(const FusedParams& p, const UnitGeo& g, const Seq& s, int idx) {
   int i0, i1;
-  fold_items<D>(p, s, &i0, &i1);
+  fold_items<D>(p, g, s, &i0, &i1);
   return idx >= i0 && idx < i1;
 }
 
@@ -387,8 +388,8 @@ __device__ __forceinline__ void sts_vec(float* dst, const float (&f)[CPL]) {
 // the block's score is recomputed here from the folded rows and replaces the
 // one score_item_warp stored from the old rows.
 template <int D>
-__device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx,
-                                                int stage) {
+__device__ __forceinline__ void fold_score_item(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, const Seq& s,
+                                                int unit, int idx, int stage) {
   constexpr int CPL = D / 32;
   constexpr int RB = Geo<D>::kBlocks;
   const int lane = role_tid() & 31;
@@ -396,7 +397,7 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
   const int nblk = min(RB, s.b1 - j0);
   const float* mrows = reinterpret_cast<const float*>(sm.ring[stage]);
   const float* vrows = mrows + RB * D;
-  const int jb0 = (int)(p.fold_begin - p.S) / p.Bk, jb1 = (int)(p.fold_end - 1 - p.S) / p.Bk;
+  const int jb0 = (int)(g.fold_begin - p.S) / p.Bk, jb1 = (int)(g.fold_end - 1 - p.S) / p.Bk;
   const int bl0 = max(0, jb0 - j0), bl1 = min(nblk - 1, jb1 - j0);
   float q1[CPL], q2[CPL];
   lds_vec<CPL>(&sm.qsum[0][lane * CPL], q1);
@@ -405,14 +406,14 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
   for (int bl = bl0; bl <= bl1; ++bl) {
     const int j = j0 + bl;
     const int64_t bs = p.S + (int64_t)j * p.Bk;
-    const int64_t t0 = max(bs, p.fold_begin), t1 = min(bs + p.Bk, p.fold_end);
+    const int64_t t0 = max(bs, (int64_t)g.fold_begin), t1 = min(bs + p.Bk, (int64_t)g.fold_end);
     float m[CPL], v[CPL];
     lds_vec<CPL>(mrows + bl * D + lane * CPL, m);
     lds_vec<CPL>(vrows + bl * D + lane * CPL, v);
 #pragma unroll 1
     for (int64_t t = t0; t < t1; ++t) {
       float x[CPL];
-      if (p.fold_end - p.fold_begin == 1) {
+      if (g.fold_end - g.fold_begin == 1) {
         lds_vec<CPL>(&sm.ktok[lane * CPL], x);  // staged at the start of the statistics role
       } else {
         load_bf16<CPL>(p.k_cache + ((int64_t)unit * p.cap + t) * D + lane * CPL, x);
@@ -443,7 +444,7 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
       __syncwarp();  // after score_item_warp's stores of the old score
       if (lane == 0) {
         p.scores[(int64_t)unit * p.max_blocks + j] = acc;
-        if (p.nb <= FusedSmem<D>::kGather) sm.scores[j] = acc;
+        if (g.nb <= FusedSmem<D>::kGather) sm.scores[j] = acc;
       }
     }
   }
@@ -459,8 +460,8 @@ __device__ __forceinline__ void fold_score_item(const FusedParams& p, FusedSmem<
 // own) leaves block l's score in lane l.  Rows past the item's last block hold
 // stale stage data: their sums stay in their own lanes and are not stored.
 template <int D>
-__device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx,
-                                                int stage) {
+__device__ __forceinline__ void score_item_warp(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, const Seq& s,
+                                                int unit, int idx, int stage) {
   constexpr int CPL = D / 32;
   constexpr int RB = Geo<D>::kBlocks;
   static_assert(RB == 32, "one block per lane");
@@ -495,7 +496,7 @@ __device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<
   }
   if (lane < nblk) {
     p.scores[(int64_t)unit * p.max_blocks + j0 + lane] = part[0];
-    if (p.nb <= FusedSmem<D>::kGather) sm.scores[j0 + lane] = part[0];  // this rank's share; pushed to the other ranks
+    if (g.nb <= FusedSmem<D>::kGather) sm.scores[j0 + lane] = part[0];  // this rank's share; pushed to the other ranks
   }
 }
 
@@ -504,7 +505,7 @@ __device__ __forceinline__ void score_item_warp(const FusedParams& p, FusedSmem<
 // and accumulates q'_i[r] H[r][c] into hacc (qsT[r] holds q'_0..3[r]).  With
 // one pending token (the usual case) its K and V rows come from shared memory.
 template <int D, int kFold>  // kFold: 0 none, 1 one token (ktok, vtok), 2 several (global memory)
-__device__ __forceinline__ void h_rows(const FusedParams& p, FusedSmem<D>& sm, int unit, int r0, int nrows,
+__device__ __forceinline__ void h_rows(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, int unit, int r0, int nrows,
                                        const float* hrows, float (&hacc)[kMaxGroup][D / 32]) {
   constexpr int CPL = D / 32;
   static_assert(kMaxGroup == 4, "qsT rows are one float4");
@@ -523,7 +524,7 @@ __device__ __forceinline__ void h_rows(const FusedParams& p, FusedSmem<D>& sm, i
 #pragma unroll
       for (int c = 0; c < CPL; ++c) h[c] += kr * v1[c];
     } else if (kFold == 2) {
-      for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
+      for (int64_t t = g.fold_begin; t < g.fold_end; ++t) {
         const float kr = __bfloat162float(p.k_cache[(ub + t) * D + row]);
         float vv[CPL];
         load_bf16<CPL>(p.v_cache + (ub + t) * D + lane * CPL, vv);
@@ -546,16 +547,17 @@ __device__ __forceinline__ void h_rows(const FusedParams& p, FusedSmem<D>& sm, i
 }
 
 template <int D>
-__device__ __forceinline__ void aux_h_item(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int idx, int stage,
+__device__ __forceinline__ void aux_h_item(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, const Seq& s, int unit,
+                                           int idx, int stage,
                                            float (&hacc)[kMaxGroup][D / 32]) {
   constexpr int RH = Geo<D>::kRows;
   const int r0 = s.h0 + idx * RH;
   const int nrows = min(RH, s.h1 - r0);
   const float* hrows = reinterpret_cast<const float*>(sm.ring[stage]);
-  const int64_t nf = p.fold_end - p.fold_begin;
-  if (nf == 0) h_rows<D, 0>(p, sm, unit, r0, nrows, hrows, hacc);
-  else if (nf == 1) h_rows<D, 1>(p, sm, unit, r0, nrows, hrows, hacc);
-  else h_rows<D, 2>(p, sm, unit, r0, nrows, hrows, hacc);
+  const int64_t nf = g.fold_end - g.fold_begin;
+  if (nf == 0) h_rows<D, 0>(p, g, sm, unit, r0, nrows, hrows, hacc);
+  else if (nf == 1) h_rows<D, 1>(p, g, sm, unit, r0, nrows, hrows, hacc);
+  else h_rows<D, 2>(p, g, sm, unit, r0, nrows, hrows, hacc);
 }
 
 // After every H item (aux threads): the linear partial of this rank's H rows,
@@ -564,7 +566,7 @@ __device__ __forceinline__ void aux_h_item(const FusedParams& p, FusedSmem<D>& s
 // values were loaded at the start of the role), adds zv (N_glob's count term)
 // and forms D_glob = n + q'_i . zk in linp[i][D].
 template <int D>
-__device__ void aux_finish_linear(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank,
+__device__ void aux_finish_linear(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, int unit, int rank,
                                   const float (&hacc)[kMaxGroup][D / 32], const float (&zk0)[kAuxCols<D>],
                                   const float (&zv0)[kAuxCols<D>], float n0) {
   constexpr int CPL = D / 32, NZ = kAuxCols<D>;
@@ -572,7 +574,7 @@ __device__ void aux_finish_linear(const FusedParams& p, FusedSmem<D>& sm, int un
   float zv[NZ];
   float nval = n0;
   if (rank == 0) {
-    const int64_t nf = p.fold_end - p.fold_begin;
+    const int64_t nf = g.fold_end - g.fold_begin;
     const int64_t ub = (int64_t)unit * p.cap;
 #pragma unroll
     for (int k = 0; k < NZ; ++k) {
@@ -584,7 +586,7 @@ __device__ void aux_finish_linear(const FusedParams& p, FusedSmem<D>& sm, int un
           zk += sm.ktok[c];
           zv[k] += sm.vtok[c];
         } else if (nf > 1) {
-          for (int64_t t = p.fold_begin; t < p.fold_end; ++t) {
+          for (int64_t t = g.fold_begin; t < g.fold_end; ++t) {
             zk += __bfloat162float(p.k_cache[(ub + t) * D + c]);
             zv[k] += __bfloat162float(p.v_cache[(ub + t) * D + c]);
           }
@@ -943,7 +945,7 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
 // block (k >= nb), none (k == 0), or the top-k of the unit's scores once every
 // rank's share is in place.  Rank 0 fills the caller's copy.
 template <int D>
-__device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int rank) {
+__device__ void aux_select(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, int unit, int rank) {
   const int a = role_tid() - kAttnThreads;
   int32_t* copy = (p.sel_out != nullptr && rank == 0) ? p.sel_out + (int64_t)unit * p.top_k : nullptr;
   int state = 3;
@@ -956,9 +958,9 @@ __device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int
     } else {
       state = 2;
     }
-  } else if (!runs_topk(p)) {  // no block, or every block
+  } else if (!runs_topk(p, g)) {  // no block, or every block
     if (copy)
-      for (int j = a; j < p.top_k; j += kAuxThreads) copy[j] = (p.k_eff > 0 && j < p.nb) ? j : -1;
+      for (int j = a; j < p.top_k; j += kAuxThreads) copy[j] = j < g.k_eff ? j : -1;
   } else {
     if (a == 0) {  // one decision for all statistics threads (their barrier counts must match)
       const bool ok = wait_cluster_bounded(&sm.scores_bar, 0, p.wait_ns);
@@ -970,14 +972,14 @@ __device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int
     }
     named_sync(kBarAux, kAuxThreads);
     if (sm.tk[7] != 0u) {
-      const bool glob = p.nb > FusedSmem<D>::kGather;
+      const bool glob = g.nb > FusedSmem<D>::kGather;
       const float* src = glob ? p.scores + (int64_t)unit * p.max_blocks : sm.scores;
-      int32_t* dst = p.k_eff <= kSelCache ? sm.sel_cache : p.sel + (int64_t)unit * p.top_k;
+      int32_t* dst = g.k_eff <= kSelCache ? sm.sel_cache : p.sel + (int64_t)unit * p.top_k;
       bool nan = false, done = false;
-      if (p.k_eff <= 32 && !glob) {
+      if (g.k_eff <= 32 && !glob) {
         if (a < 32) {  // one warp; the candidates go to the attention combine slots, idle until the selection is made
           bool wn;
-          const bool ok = topk_warp(sm.scores, p.nb, p.k_eff, dst, copy,
+          const bool ok = topk_warp(sm.scores, g.nb, g.k_eff, dst, copy,
                                     reinterpret_cast<unsigned long long*>(&sm.wpart[0][0]), FusedSmem<D>::kPF, wn);
           if (a == 0) {
             sm.tkw[0] = ok ? 1u : 0u;
@@ -990,12 +992,12 @@ __device__ void aux_select(const FusedParams& p, FusedSmem<D>& sm, int unit, int
       }
       if (!done) {  // more than 32 blocks, or too many candidates: the radix selection
         const TopkSmem t{sm.hist, sm.tk, &sm.tks[0][0]};
-        nan = aux_topk(t, src, glob, p.nb, p.k_eff, dst, copy);
+        nan = aux_topk(t, src, glob, g.nb, g.k_eff, dst, copy);
       }
       if (nan && a == 0) atomicOr(p.status, HYB_STATUS_NAN_SCORE);
       if (copy)
-        for (int j = p.k_eff + a; j < p.top_k; j += kAuxThreads) copy[j] = -1;
-      state = p.k_eff <= kSelCache ? 1 : 2;
+        for (int j = g.k_eff + a; j < p.top_k; j += kAuxThreads) copy[j] = -1;
+      state = g.k_eff <= kSelCache ? 1 : 2;
       row = dst;
     }
   }
@@ -1270,7 +1272,7 @@ namespace {
 // statistics item in ring order and arrives once on its stage's empty barrier
 // (the owner after its work), so that no warp falls two phases behind a stage.
 template <int D>
-__device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit, int rank) {
+__device__ void aux_role(const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, const Seq& s, int unit, int rank) {
   constexpr int CPL = D / 32;
   const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
   // a timed-out wait only stops this warp's work; it keeps visiting every item
@@ -1292,7 +1294,7 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
     }
     return have;
   };
-  const int64_t nf = p.fold_end - p.fold_begin;
+  const int64_t nf = g.fold_end - g.fold_begin;
   // rank 0's zk, zv and n, needed after the last H item: loaded now, so that
   // their round trip is not on the path at the end
   float zk0[kAuxCols<D>], zv0[kAuxCols<D>], n0 = 0.f;
@@ -1318,21 +1320,21 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
   named_sync(kBarAux, kAuxThreads);
   cluster_wait();  // every rank's barriers are initialised: remote operations are allowed from here on
   int fold_i0, fold_i1;
-  fold_items<D>(p, s, &fold_i0, &fold_i1);
+  fold_items<D>(p, g, s, &fold_i0, &fold_i1);
 #pragma unroll 1
   for (int idx = 0; idx < s.nS; ++idx) {
     const int it = seq_of_s(s, idx), stage = it % kFStages;
     const bool have = wait_item(it);
     if (have && idx % kAuxWarps == aw) {
-      if (p.q != nullptr) score_item_warp<D>(p, sm, s, unit, idx, stage);
-      if (idx >= fold_i0 && idx < fold_i1) fold_score_item<D>(p, sm, s, unit, idx, stage);
+      if (p.q != nullptr) score_item_warp<D>(p, g, sm, s, unit, idx, stage);
+      if (idx >= fold_i0 && idx < fold_i1) fold_score_item<D>(p, g, sm, s, unit, idx, stage);
       __syncwarp();
     }
     if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
   }
   named_sync(kBarAux, kAuxThreads);  // every score of this rank is in place
-  if (runs_topk(p)) {  // hand this rank's scores to every rank
-    if (p.nb <= FusedSmem<D>::kGather) {
+  if (runs_topk(p, g)) {  // hand this rank's scores to every rank
+    if (g.nb <= FusedSmem<D>::kGather) {
       // bulk copies of the share into every other rank's scores array
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       named_sync(kBarAux, kAuxThreads);
@@ -1356,7 +1358,7 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
     }
   }
 
-  if (p.q != nullptr) aux_select<D>(p, sm, unit, rank);
+  if (p.q != nullptr) aux_select<D>(p, g, sm, unit, rank);
   float hacc[kMaxGroup][CPL];
 #pragma unroll
   for (int i = 0; i < kMaxGroup; ++i)
@@ -1366,11 +1368,11 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
   for (int idx = 0; idx < s.nH; ++idx) {
     const int it = seq_of_h(s, idx), stage = it % kFStages;
     const bool have = wait_item(it);
-    if (have && (p.q != nullptr || nf > 0)) aux_h_item<D>(p, sm, s, unit, idx, stage, hacc);
+    if (have && (p.q != nullptr || nf > 0)) aux_h_item<D>(p, g, sm, s, unit, idx, stage, hacc);
     __syncwarp();
     if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAuxWarp);
   }
-  aux_finish_linear<D>(p, sm, unit, rank, hacc, zk0, zv0, n0);
+  aux_finish_linear<D>(p, g, sm, unit, rank, hacc, zk0, zv0, n0);
 }
 
 // Producer (role warp 11, lane 0): every copy of the rank, in ring order, one
@@ -1378,8 +1380,8 @@ __device__ void aux_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, i
 // a stage that held an earlier item, the stage's empty barrier must have
 // completed for that earlier item.
 template <int D>
-__device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<D>& sm, const Seq& s, int unit,
-                              int rank) {
+__device__ void producer_role(const KVMaps* tm, const FusedParams& p, const UnitGeo& g, FusedSmem<D>& sm, const Seq& s,
+                              int unit, int rank) {
   if ((threadIdx.x & 31) != 0) return;
   constexpr int RB = Geo<D>::kBlocks, RH = Geo<D>::kRows;
   const uint64_t pol = l2_evict_first();  // every copy of the ring streams data read once per launch
@@ -1416,7 +1418,7 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
   for (int i = 0; i < s.nS && ok; ++i) {
     if (!(ok = acquire())) break;
     uint64_t* bar = &sm.full_aux[stage];
-    if (p.q != nullptr || score_item_folds<D>(p, s, i)) {
+    if (p.q != nullptr || score_item_folds<D>(p, g, s, i)) {
       const uint32_t dst = smem_u32(sm.ring[stage]);
       const uint32_t bytes = (uint32_t)(min(RB, s.b1 - s.b0 - i * RB) * D * 4);
       const int64_t off = (brow + (int64_t)i * RB) * D;
@@ -1433,18 +1435,18 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
   for (int i = 0, ci = rank; i < s.nW && ok; ++i, ci += p.C) {
     if (!(ok = acquire())) break;
     int start, len;
-    if (ci < p.n_sink_chunks) {
+    if (ci < g.n_sink_chunks) {
       start = ci * kTile;
-      len = min(kTile, p.sink_len - start);
+      len = min(kTile, g.sink_len - start);
     } else {
-      start = p.win_start + (ci - p.n_sink_chunks) * kTile;
-      len = min(kTile, p.T - start);
+      start = g.win_start + (ci - g.n_sink_chunks) * kTile;
+      len = min(kTile, g.T - start);
     }
     issue_chunk<D>(tm, sm, stage, ubase, start, len, 0, pol);
     advance(false);
   }
   // H items: RH rows of H
-  const bool h_load = p.q != nullptr || p.fold_end > p.fold_begin;
+  const bool h_load = p.q != nullptr || g.fold_end > g.fold_begin;
   for (int i = 0; i < s.nH && ok; ++i) {
     if (!(ok = acquire())) break;
     uint64_t* bar = &sm.full_aux[stage];
@@ -1470,12 +1472,12 @@ __device__ void producer_role(const KVMaps* tm, const FusedParams& p, FusedSmem<
   for (int i = 0; i < s.nX && ok; ++i) {
     if (!(ok = acquire())) break;
     int jb = -1;
-    if (slot < p.k_eff) jb = st == 3 ? slot : st == 1 ? sm.sel_cache[slot] : __ldcg(sm.sel_row + slot);
+    if (slot < g.k_eff) jb = st == 3 ? slot : st == 1 ? sm.sel_cache[slot] : __ldcg(sm.sel_row + slot);
     int start = 0, len = 0;
-    if (jb >= 0 && jb < p.nb) {
+    if (jb >= 0 && jb < g.nb) {
       const int bs = p.S + jb * p.Bk;
       start = bs + piece * kTile;
-      len = max(0, min(kTile, min(bs + p.Bk, p.ev_end) - start));
+      len = max(0, min(kTile, min(bs + p.Bk, g.ev_end) - start));
     } else if (jb != -1) {
       atomicOr(p.status, HYB_STATUS_BAD_SELECTION);
     }
@@ -1616,7 +1618,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
   const int tid = threadIdx.x, warp = role_tid() >> 5;
   const int rank = (int)cluster_rank();
   const int unit = blockIdx.x / p.C;
-  const Seq s = make_seq<D>(p, rank);
+  // this unit's row length, budget and fold range (every thread, in registers;
+  // the roles read the copy thread 0 leaves in shared memory)
+  const UnitGeo g0 = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, p.top_k, p.chunks_per_block, p.pending);
+  const Seq s = make_seq<D>(p, g0, rank);
   if (warp == kProducerWarp && (tid & 31) == 0) {
     // Before the wait for the previous grid (which may still be running):
     // the rank's block statistics, its first items, are prefetched into L2.
@@ -1643,7 +1648,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     // scores_bar: the other ranks' shares arriving by bulk copy (one local
     // arrival expecting their bytes), or C arrivals when the scores go
     // through global memory
-    const bool push = runs_topk(p) && p.nb <= FusedSmem<D>::kGather;
+    sm.geo = g0;
+    const bool push = runs_topk(p, g0) && g0.nb <= FusedSmem<D>::kGather;
     mbar_init(&sm.scores_bar, push ? 1 : p.C);
     mbar_init(&sm.sel_bar, 1);
     mbar_init(&sm.merge_bar, 1);
@@ -1655,7 +1661,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
       uint32_t bytes = 0;
       for (int rr = 0; rr < p.C; ++rr) {
         int b0, b1;
-        block_share(p.nb, p.C, rr, b0, b1);
+        block_share(g0.nb, p.C, rr, b0, b1);
         if (rr != rank) bytes += (uint32_t)(((b1 - b0) * 4 + 15) & ~15);
       }
       mbar_arrive_expect_tx(&sm.scores_bar, bytes);
@@ -1673,9 +1679,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
   __syncthreads();
   cluster_arrive_relaxed();
   pdl_allow_dependents();
+  const UnitGeo& g = sm.geo;
   if (warp == kProducerWarp) {
     // the producer starts at once: it needs nothing from the lines below
-    producer_role<D>(&tm, p, sm, s, unit, rank);
+    producer_role<D>(&tm, p, g, sm, s, unit, rank);
     cluster_wait();
   } else {
     const int t = role_tid();  // 0 .. kConsumerThreads - 1
@@ -1688,7 +1695,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     static_assert(QV + D / 2 <= kConsumerThreads, "one 16-byte piece per thread");
     const int tr = t - QV, ta = t - QV - D / 4;
     const bool ld_q = p.q != nullptr && t < QV && t * 8 < p.G * D;
-    const bool ld_row = p.fold_end - p.fold_begin == 1 && tr >= 0 && tr < D / 4;
+    const bool ld_row = g.fold_end - g.fold_begin == 1 && tr >= 0 && tr < D / 4;
     const bool ld_new = p.k_new != nullptr && rank == 0 && ta >= 0 && ta < D / 4;
     uint4 raw = make_uint4(0u, 0u, 0u, 0u);
     if (ld_q) {
@@ -1696,7 +1703,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
     } else if (ld_row) {
       const int e = (tr % (D / 8)) * 8;
       raw = __ldg(reinterpret_cast<const uint4*>((tr >= D / 8 ? p.v_cache : p.k_cache) +
-                                                 ((int64_t)unit * p.cap + p.fold_begin) * D + e));
+                                                 ((int64_t)unit * p.cap + g.fold_begin) * D + e));
     } else if (ld_new) {
       const int e = (ta % (D / 8)) * 8;
       raw = __ldg(reinterpret_cast<const uint4*>((ta >= D / 8 ? p.v_new : p.k_new) + (int64_t)unit * D + e));
@@ -1721,14 +1728,14 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const __grid_consta
       }
     } else if (ld_new) {  // the decode's appended token: row T of the caches
       const int e = (ta % (D / 8)) * 8;
-      *reinterpret_cast<uint4*>((ta >= D / 8 ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T) * D + e) = raw;
+      *reinterpret_cast<uint4*>((ta >= D / 8 ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + g.T) * D + e) = raw;
     }
     named_sync(kBarConsumers, kConsumerThreads);
     if (warp < kAttnWarps) {
       if (p.q != nullptr) attn_role<D>(p, sm, s, unit);
       cluster_wait();
     } else {
-      aux_role<D>(p, sm, s, unit, rank);  // waits on the cluster barrier before its score push
+      aux_role<D>(p, g, sm, s, unit, rank);  // waits on the cluster barrier before its score push
     }
   }
   __syncthreads();  // this rank's record and linear partial are final; its ring is idle

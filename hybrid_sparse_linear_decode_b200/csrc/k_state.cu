@@ -26,20 +26,22 @@ namespace {
 // D/4 threads of 16 bytes.  A token's later eviction from the window is folded
 // into the state by the decode after it, which reads the caches.
 template <int D>
-__global__ void __launch_bounds__(D / 4) append_kernel(const AppendParams p) {
+__global__ void __launch_bounds__(D / 4) append_kernel(const __grid_constant__ AppendParams p) {
   const int unit = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;  // token j of the chunk
+  const int32_t Tb = p.T - (p.tb.ragged ? p.tb.row_lag[unit / p.Hkv] : 0);  // this row's length
   if (tid == 0) pdl_wait_primary();  // the previous decode may still read these caches' rows
   __syncthreads();
   pdl_allow_dependents();
   const bool is_v = tid >= D / 8;
   const int e = (tid % (D / 8)) * 8;
   const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + ((int64_t)unit * p.n + j) * D + e;
-  __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + p.T + j) * D + e;
+  __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + Tb + j) * D + e;
   *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
 }
 
 // ---------------------------------------------------------------- chunk fold
-// The evicted positions [fb, fe) of every unit folded into the state in one
+// The pending evicted positions [fb, fe) of every unit (each row's length and
+// each head's window give its own range) folded into the state in one
 // pass, for several pending tokens (a chunked append, or many appends between
 // decodes; SPLA "Recurrence" applied to a run of tokens is a small dense
 // update).  One CTA per unit: H += K^T V over the run (fp32 thread tiles of the
@@ -51,14 +53,17 @@ __global__ void __launch_bounds__(D / 4) append_kernel(const AppendParams p) {
 // d = mb - ma), in fp64.  The tokens of a block folded before fb are exactly
 // those before fb, as folds go in position order.
 template <int D>
-__global__ void __launch_bounds__(256) fold_kernel(const FoldParams p) {
+__global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldParams p) {
   constexpr int RT = D / 16;
   __shared__ __align__(16) float ks[32][D];
   __shared__ __align__(16) float vs[32][D];
   const int unit = blockIdx.x, tid = threadIdx.x;
+  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, p.pending);
+  const int64_t fb = g.fold_begin, fe = g.fold_end;
   if (tid == 0) pdl_wait_primary();  // the caches' rows and the state may come from the previous grid
   __syncthreads();
   pdl_allow_dependents();
+  if (fe <= fb) return;  // nothing pending in this unit (a short row)
   const int tr = tid / 16, tc = tid % 16;
   const int64_t ub = (int64_t)unit * p.cap;
   float acc[RT][RT];
@@ -67,8 +72,8 @@ __global__ void __launch_bounds__(256) fold_kernel(const FoldParams p) {
 #pragma unroll
     for (int j = 0; j < RT; ++j) acc[i][j] = 0.f;
   float zacc = 0.f;
-  for (int64_t tt = p.fb; tt < p.fe; tt += 32) {
-    const int n = (int)min((int64_t)32, p.fe - tt);
+  for (int64_t tt = fb; tt < fe; tt += 32) {
+    const int n = (int)min((int64_t)32, fe - tt);
     for (int e = tid; e < 32 * D; e += 256) {
       const int r = e / D, c = e % D;
       float kv = 0.f, vv = 0.f;
@@ -107,13 +112,13 @@ __global__ void __launch_bounds__(256) fold_kernel(const FoldParams p) {
     for (int j = 0; j < RT; ++j) H[(int64_t)(tr * RT + i) * D + tc * RT + j] += acc[i][j];
   if (tid < D) p.zk[(int64_t)unit * D + tid] += zacc;
   else if (tid < 2 * D) p.zv[(int64_t)unit * D + tid - D] += zacc;
-  if (tid == 0) p.n[unit] += (float)(p.fe - p.fb);
+  if (tid == 0) p.n[unit] += (float)(fe - fb);
   if (tid < D) {  // one channel per thread
     const __nv_bfloat16* kc = p.k_cache + ub * D + tid;
-    const int64_t j0 = (p.fb - p.S) / p.Bk, j1 = (p.fe - 1 - p.S) / p.Bk;
+    const int64_t j0 = (fb - p.S) / p.Bk, j1 = (fe - 1 - p.S) / p.Bk;
     for (int64_t j = j0; j <= j1; ++j) {
       const int64_t bs = p.S + j * p.Bk;
-      const int64_t a0 = max(bs, p.fb), a1 = min(bs + (int64_t)p.Bk, p.fe);
+      const int64_t a0 = max(bs, fb), a1 = min(bs + (int64_t)p.Bk, fe);
       const double na = (double)(a0 - bs), nb = (double)(a1 - a0);
       double sb = 0.0, qb = 0.0;
       for (int64_t t = a0; t < a1; ++t) sb += (double)__bfloat162float(kc[t * D]);
@@ -137,19 +142,23 @@ __global__ void __launch_bounds__(256) fold_kernel(const FoldParams p) {
 }
 
 // ---------------------------------------------------------------- init
-// (1) H, zk, zv over L: grid (ceil(|L| / tokens_per_cta), units).  Each CTA
+// Every unit's evicted range is L = [S, ev_end(T_b, W_h)): its row's length
+// and its head's window.
+// (1) H, zk, zv over L: grid (ceil(max |L| / tokens_per_cta), units).  Each CTA
 //     accumulates its token range in fp32 (thread tile RT x RT of the D x D
 //     outer-product sum, keys/values staged through shared memory 32 tokens at a
 //     time) and adds the result into fp64 accumulators.
 template <int D>
-__global__ void __launch_bounds__(256) init_linear_kernel(const InitParams p) {
+__global__ void __launch_bounds__(256) init_linear_kernel(const __grid_constant__ InitParams p) {
   constexpr int RT = D / 16;
   __shared__ __align__(16) float ks[32][D];
   __shared__ __align__(16) float vs[32][D];
   const int unit = blockIdx.y, tid = threadIdx.x;
   const int tr = tid / 16, tc = tid % 16;
-  const int64_t t0 = p.ev_begin + (int64_t)blockIdx.x * p.tokens_per_cta;
-  const int64_t t1 = min(t0 + (int64_t)p.tokens_per_cta, p.ev_end);
+  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
+  const int64_t t0 = p.S + (int64_t)blockIdx.x * p.tokens_per_cta;
+  const int64_t t1 = min(t0 + (int64_t)p.tokens_per_cta, (int64_t)g.ev_end);
+  if (t0 >= t1) return;  // past this unit's evicted range
   const int64_t ub = (int64_t)unit * p.cap;
   float acc[RT][RT];
 #pragma unroll
@@ -201,13 +210,14 @@ __global__ void __launch_bounds__(256) init_linear_kernel(const InitParams p) {
 // (2) block statistics: one warp per block, two passes (mean, then the mean
 //     squared deviation) in fp64.
 template <int D>
-__global__ void __launch_bounds__(256) init_stats_kernel(const InitParams p) {
+__global__ void __launch_bounds__(256) init_stats_kernel(const __grid_constant__ InitParams p) {
   constexpr int CPL = D / 32;
   const int unit = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * 8 + warp;
-  if (j >= p.nb) return;
-  const int64_t bs = p.ev_begin + (int64_t)j * p.Bk;
-  const int64_t be = min(bs + (int64_t)p.Bk, p.ev_end);
+  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
+  if (j >= g.nb) return;
+  const int64_t bs = p.S + (int64_t)j * p.Bk;
+  const int64_t be = min(bs + (int64_t)p.Bk, (int64_t)g.ev_end);
   const double cnt = (double)(be - bs);
   const __nv_bfloat16* kc = p.k_cache + (int64_t)unit * p.cap * D;
   double s[CPL], q[CPL];
@@ -234,8 +244,9 @@ __global__ void __launch_bounds__(256) init_stats_kernel(const InitParams p) {
 
 // (3) fp64 accumulators -> fp32 state; reset the status word.
 template <int D>
-__global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) {
+__global__ void __launch_bounds__(256) init_finalize_kernel(const __grid_constant__ InitParams p) {
   const int unit = blockIdx.x, tid = threadIdx.x;
+  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
   const double* H64 = p.H64 + (int64_t)unit * D * D;
   float* H = p.H + (int64_t)unit * D * D;
   for (int e = tid; e < D * D; e += 256) H[e] = (float)H64[e];
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(256) init_finalize_kernel(const InitParams p) 
     p.zv[(int64_t)unit * D + tid] = (float)p.z64[(int64_t)unit * 2 * D + D + tid];
   }
   if (tid == 0) {
-    p.n[unit] = (float)(p.ev_end - p.ev_begin);
+    p.n[unit] = (float)(g.ev_end - p.S);
     if (unit == 0) *p.status = 0u;
   }
 }
@@ -294,7 +305,7 @@ cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {
 }
 
 cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s) {
-  const int64_t ev = p.ev_end - p.ev_begin;
+  const int64_t ev = p.ev_max;
   if (ev > 0) {
     const dim3 g1((unsigned)((ev + p.tokens_per_cta - 1) / p.tokens_per_cta), p.units);
     if (D == 128)
@@ -304,8 +315,8 @@ cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (p.nb > 0) {
-    const dim3 g2((unsigned)((p.nb + 7) / 8), p.units);
+  if (p.nb_max > 0) {
+    const dim3 g2((unsigned)((p.nb_max + 7) / 8), p.units);
     if (D == 128)
       init_stats_kernel<128><<<g2, 256, 0, s>>>(p);
     else

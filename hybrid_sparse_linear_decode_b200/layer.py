@@ -12,9 +12,23 @@ from . import _abi as A
 
 
 def make_config(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, block_size: int, n_sink: int,
-                window: int, top_k: int, capacity: int, scale: float = 0.0) -> A.hyb_attn_config:
-    return A.hyb_attn_config(batch, n_q_heads, n_kv_heads, head_dim, block_size, n_sink, window, top_k,
-                             capacity, scale)
+                window: int, top_k: int, capacity: int, scale: float = 0.0, head_window=None,
+                head_top_k=None) -> A.hyb_attn_config:
+    """The C config struct.  With per-KV-head budgets (head_window, head_top_k:
+    sequences of n_kv_heads ints), `window` and `top_k` default to their
+    minimum and maximum (the sizes the buffers need)."""
+    hw = ht = None
+    if head_window is not None or head_top_k is not None:
+        assert head_window is not None and head_top_k is not None
+        assert len(head_window) == n_kv_heads and len(head_top_k) == n_kv_heads
+        window = min(window, min(head_window)) if window is not None else min(head_window)
+        top_k = max(top_k, max(head_top_k)) if top_k is not None else max(head_top_k)
+        hw = (A.c_i32 * n_kv_heads)(*[int(v) for v in head_window])
+        ht = (A.c_i32 * n_kv_heads)(*[int(v) for v in head_top_k])
+    cfg = A.hyb_attn_config(batch, n_q_heads, n_kv_heads, head_dim, block_size, n_sink, window, top_k,
+                            capacity, scale, hw, ht)
+    cfg._keep = (hw, ht)   # the arrays live as long as the struct that points at them
+    return cfg
 
 
 def _stream(stream) -> int:
@@ -73,19 +87,31 @@ class HybridAttentionLayer:
                                   self.zk.data_ptr(), self.zv.data_ptr(), self.n.data_ptr(), self.mu.data_ptr(),
                                   self.var.data_ptr(), self.workspace.data_ptr(), self.workspace.numel())
 
-    def init(self, T0: int, stream=None) -> None:
+    def init(self, T0, stream=None) -> None:
+        """Build the state of the prefilled history: T0 tokens per row, or a
+        sequence of per-row lengths."""
         if self.ctx is not None:
             A.hyb_attn_destroy(self.ctx)
         with torch.cuda.device(self.device):
-            self.ctx = A.hyb_attn_init(self.cfg, self.buffers(), T0, _stream(stream))
+            if isinstance(T0, int):
+                self.ctx = A.hyb_attn_init(self.cfg, self.buffers(), T0, _stream(stream))
+            else:
+                self.ctx = A.hyb_attn_init_rows(self.cfg, self.buffers(), list(T0), _stream(stream))
 
-    def attach(self, T: int, stream=None) -> None:
+    def attach(self, T, stream=None) -> None:
         """Bind a context to buffers that already hold the synced state of a
-        history of length T (a restored checkpoint), without rebuilding it."""
+        history of length T (or per-row lengths): a restored checkpoint,
+        without rebuilding it."""
         if self.ctx is not None:
             A.hyb_attn_destroy(self.ctx)
         with torch.cuda.device(self.device):
-            self.ctx = A.hyb_attn_attach(self.cfg, self.buffers(), T, _stream(stream))
+            if isinstance(T, int):
+                self.ctx = A.hyb_attn_attach(self.cfg, self.buffers(), T, _stream(stream))
+            else:
+                self.ctx = A.hyb_attn_attach_rows(self.cfg, self.buffers(), list(T), _stream(stream))
+
+    def row_lengths(self) -> list:
+        return [A.hyb_attn_row_length(self.ctx, b) for b in range(self.cfg.batch)]
 
     def set_wait_limit(self, ns: int) -> None:
         A.hyb_attn_set_wait_limit(self.ctx, ns)

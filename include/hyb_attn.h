@@ -41,7 +41,9 @@
  *   - Anomalies found on the device (non-finite output, denominator <= 0, an
  *     out-of-range block index in a caller-given selection, a timed-out wait)
  *     set bits in a device status word, read with hyb_attn_status().
- *   - All batch rows share the length T.  One context holds one layer.
+ *   - Batch rows share the length T unless the context was created with
+ *     per-row lengths (hyb_attn_init_rows); every row then grows by the same
+ *     appends.  One context holds one layer.
  *   - Supported: head_dim 64 or 128; group size G in {1, 2, 4};
  *     batch * n_kv_heads * capacity < 2^31.
  */
@@ -89,6 +91,16 @@ typedef struct hyb_attn_config {
   int32_t top_k;       /* k >= 0: blocks attended exactly per (b, KV head) */
   int64_t capacity;    /* rows per (b, KV head) in the KV cache, >= 1 */
   float   scale;       /* q' = q * scale; 0 selects 1/sqrt(head_dim) */
+  /* Per-KV-head budgets (host arrays of n_kv_heads entries, read when a context
+   * is created), or NULL for every head at (window, top_k): KV head h keeps
+   * window head_window[h] >= window and selects head_top_k[h] <= top_k blocks.
+   * `window` is then the smallest window (it sizes the statistics arrays) and
+   * `top_k` the largest top-k (the row length of selection arrays, whose
+   * entries past a head's own count are -1).  Both or neither; at most
+   * 32 KV heads.  (SALSA abstract: sparse-cache budgets allocated per layer;
+   * per head here, the same knob one level finer.) */
+  const int32_t* head_window;
+  const int32_t* head_top_k;
 } hyb_attn_config;
 
 /* Sizes (in elements, except where noted) of the caller-owned buffers for a
@@ -174,6 +186,16 @@ int hyb_attn_plan(const hyb_attn_config* cfg, int64_t T, int32_t n_sm, hyb_attn_
 int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
                   int64_t T0, cudaStream_t stream);
 
+/* As hyb_attn_init, with a length of its own for every batch row: row_T0 is a
+ * host array of `batch` lengths in [1, capacity] (at most 128 rows), positions
+ * [0, row_T0[b]) of row b's caches are its history, and each row's state is
+ * built over its own evicted range.  Every later append or decode step moves
+ * all rows by the same count; hyb_attn_length reports the longest row and
+ * hyb_attn_row_length each one.  A decode attends, for row b, to [0, T_b) with
+ * its own window, blocks and top-k.  Errors as hyb_attn_init. */
+int hyb_attn_init_rows(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
+                       const int64_t* row_T0, cudaStream_t stream);
+
 /* Create a context over buffers that already hold the synced state of a
  * history of length T -- the caches' positions [0, T) and H, zk, zv, n, mu,
  * var exactly as hyb_attn_sync_state left them (a checkpoint copied back by the
@@ -182,6 +204,10 @@ int hyb_attn_init(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn
  * the device status word.  Errors as hyb_attn_init. */
 int hyb_attn_attach(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
                     int64_t T, cudaStream_t stream);
+/* hyb_attn_attach for a checkpoint of a context with per-row lengths (row_T:
+ * host array of `batch` lengths, as hyb_attn_row_length reported them). */
+int hyb_attn_attach_rows(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buffers* buf,
+                         const int64_t* row_T, cudaStream_t stream);
 
 /* Append one token per unit: k_new, v_new bf16 [B][Hkv][d].  The token is
  * written at position T; then T += 1.  If the token at position T - W - 1
@@ -269,6 +295,22 @@ int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32
 int hyb_attn_step_host(hyb_attn_ctx* ctx, const void* q_host, const void* k_host,
                        const void* v_host, float* out_host, cudaStream_t stream);
 
+/* A whole decode step of several layers from host memory, with one copy in and
+ * one copy out: in_host holds, layer after layer, that layer's q (bf16
+ * [B][Hq][d]) then k and v of the appended token (bf16 [B][Hkv][d] each);
+ * out_host receives, layer after layer, the fp32 [B][Hq][d] outputs.  One
+ * cudaMemcpyAsync brings every layer's input to `staging` (caller-owned device
+ * memory, 256-byte aligned, at least hyb_attn_step_layers_staging_bytes), the
+ * layers' decode + append launches follow back to back on `stream` (chained
+ * as usual), and one cudaMemcpyAsync returns every output.  Host buffers
+ * should be pinned.  The layers may have different budgets and shapes; their
+ * contexts may share one workspace (the calls are serialised on `stream`).
+ * Errors: HYB_EINVAL, HYB_ECAPACITY (a layer is full: nothing is enqueued),
+ * HYB_ECUDA. */
+size_t hyb_attn_step_layers_staging_bytes(hyb_attn_ctx* const* ctxs, int32_t n_layers);
+int hyb_attn_step_layers_host(hyb_attn_ctx* const* ctxs, int32_t n_layers, const void* in_host, float* out_host,
+                              void* staging, size_t staging_bytes, cudaStream_t stream);
+
 /* Decode without any allocation, for callers that cannot allocate device
  * memory themselves: code that runs under an allocator it does not own (a
  * framework's caching pool, a plugin host, an embedded runtime) or that must
@@ -296,8 +338,11 @@ int hyb_attn_step_host(hyb_attn_ctx* ctx, const void* q_host, const void* k_host
 #define HYB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int hyb_attn_decode_noalloc(hyb_attn_ctx* ctx, const void* q, float* out, int32_t* sel_out, cudaStream_t stream);
 
-/* Current length T (host mirror; no device access). */
+/* Current length T (host mirror; no device access): the longest row's. */
 int64_t hyb_attn_length(const hyb_attn_ctx* ctx);
+
+/* Current length of batch row b (host mirror), or -1 for a bad argument. */
+int64_t hyb_attn_row_length(const hyb_attn_ctx* ctx, int32_t b);
 
 /* Copy the device status word to *flags (synchronises `stream`); with clear != 0
  * reset it to zero afterwards.  Returns HYB_OK or HYB_ECUDA.  The status word

@@ -34,7 +34,8 @@ def test_header_declares_the_boundary():
               "hyb_attn_workspace_size", "hyb_attn_length", "hyb_attn_status", "hyb_attn_destroy",
               "hyb_attn_strerror", "hyb_attn_query_sizes", "hyb_attn_plan", "hyb_attn_step_host",
               "hyb_attn_set_timing_events", "hyb_attn_decode_append", "hyb_attn_sync_state",
-              "hyb_attn_attach", "hyb_attn_set_wait_limit", "hyb_attn_set_test_flags"]:
+              "hyb_attn_attach", "hyb_attn_set_wait_limit", "hyb_attn_set_test_flags",
+              "hyb_attn_init_rows", "hyb_attn_attach_rows", "hyb_attn_row_length"]:
         assert n in names, n
 
 
@@ -149,3 +150,43 @@ def test_plan_cluster_size(lib, batch, want):
     c = _cfg(batch=batch, capacity=4096)
     p = H.hyb_attn_plan(c, 4096, 148)
     assert p.cluster_ctas == want and p.grid_ctas == batch * 8 * want
+
+
+def test_per_head_budgets_validated_on_the_host(lib):
+    """Per-KV-head budgets refine the config's (window, top_k): every head's
+    window at least `window` (which sizes the statistics arrays), every head's
+    top-k at most `top_k` (the selection rows' length); at most 32 KV heads."""
+    import hybrid_sparse_linear_decode_b200 as H
+    ok = H.make_config(1, 32, 8, 128, 64, 4, None, None, 40000, head_window=[1024, 2048] * 4,
+                       head_top_k=[16, 32] * 4)
+    assert (ok.window, ok.top_k) == (1024, 32)
+    s_ok = H.hyb_attn_query_sizes(ok)
+    assert s_ok.max_blocks == -(-(40000 - 4 - 1024) // 64)
+    bad = H.make_config(1, 32, 8, 128, 64, 4, None, None, 40000, head_window=[1024, 2048] * 4,
+                        head_top_k=[16, 32] * 4)
+    bad.window = 2000                       # a head below the config's window
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_query_sizes(bad)
+    bad2 = H.make_config(1, 32, 8, 128, 64, 4, None, None, 40000, head_window=[1024] * 8, head_top_k=[16] * 8)
+    bad2.top_k = 8                          # a head above the config's top-k
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_query_sizes(bad2)
+    many = H.make_config(1, 64, 64, 128, 64, 4, None, None, 4096, head_window=[64] * 64, head_top_k=[4] * 64)
+    with pytest.raises(H.HybAttnError):    # more KV heads than per-head budgets are kept for
+        H.hyb_attn_query_sizes(many)
+    half = H.make_config(1, 32, 8, 128, 64, 4, 64, 4, 4096)
+    import ctypes
+    half.head_window = (ctypes.c_int32 * 8)(*([64] * 8))   # one array without the other
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_query_sizes(half)
+
+
+def test_per_row_entry_points_reject_bad_arguments(lib):
+    import hybrid_sparse_linear_decode_b200 as H
+    c = _cfg(batch=2)
+    buf = H.hyb_attn_buffers()
+    with pytest.raises(H.HybAttnError):
+        H.hyb_attn_init_rows(c, buf, [100, 200], 0)          # null buffers
+    assert lib.hyb_attn_init_rows(None, None, None, None, None) == -1
+    assert lib.hyb_attn_attach_rows(None, None, None, None, None) == -1
+    assert lib.hyb_attn_row_length(None, 0) == -1

@@ -152,6 +152,41 @@ def test_step_host_matches_device_path():
     assert c1.layer.T == c2.layer.T
 
 
+def test_step_layers_host_matches_device_path():
+    """Several layers (different budgets) stepped from
+    one host buffer with one copy in and one copy out equal the same layers
+    stepped through the device entry point."""
+    import torch
+    import hybrid_sparse_linear_decode_b200 as H
+    kws = [dict(T0=1000, W=64, k=4), dict(T0=1000, W=100, k=6), dict(T0=1000, W=32, k=2, Bk=16)]
+    c1 = [_case(n_append=3, seed=30 + i, **kw) for i, kw in enumerate(kws)]
+    c2 = [_case(n_append=3, seed=30 + i, **kw) for i, kw in enumerate(kws)]
+    ctxs = [c.layer.ctx for c in c2]
+    nbytes = H.hyb_attn_step_layers_staging_bytes(ctxs)
+    staging = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for step in range(3):
+        qs = [c.random_q() for c in c1]
+        for c, q in zip(c2, qs):
+            c.rng.standard_normal((c.B, c.Hq, c.d))      # keep the rngs in step
+        parts, ref = [], []
+        for c, q in zip(c1, qs):
+            out, _, _ = c.decode(q, with_scores=False)
+            ref.append(out.astype(np.float32))
+            parts += [q.reshape(-1), np.ascontiguousarray(c.Kb[:, :, c.T]).reshape(-1),
+                      np.ascontiguousarray(c.Vb[:, :, c.T]).reshape(-1)]
+            c.append()
+        hin = torch.from_numpy(np.concatenate(parts).view(np.int16)).pin_memory()
+        hout = torch.empty(sum(r.size for r in ref), dtype=torch.float32).pin_memory()
+        H.hyb_attn_step_layers_host(ctxs, hin.data_ptr(), hout.data_ptr(), staging.data_ptr(), nbytes, stream)
+        torch.cuda.synchronize()
+        for c in c2:
+            c.T += 1
+        np.testing.assert_array_equal(hout.numpy(), np.concatenate([r.reshape(-1) for r in ref]))
+    assert all(c.layer.T == c.T for c in c2)
+    assert all(c.layer.status() == 0 for c in c2)
+
+
 def test_capacity_error():
     import torch
     from hybrid_sparse_linear_decode_b200 import HybAttnError
