@@ -118,7 +118,7 @@ def step_bytes_model(w, mode: str, chunk: int, T: int):
     return step_dec, step_bytes, flush
 
 
-KERNEL_SOURCES = ("k_fused.cu", "hyb_device.cuh", "hyb_internal.h")
+KERNEL_SOURCES = ("k_fused.cu", "k_common.cuh", "hyb_device.cuh", "hyb_internal.h")
 
 
 def kernel_sources_hash() -> str:

@@ -262,9 +262,13 @@ FusedParams fused_params(const hyb_attn_ctx* x) {
   fp.scale = x->scale;
   fp.wait_ns = x->wait_ns;
   fp.test_flags = x->test_flags;
-  fp.tb = x->tb;
   return fp;
 }
+
+// Does some unit have more than kStreamBlocks candidate blocks?  The most
+// blocks are those of the longest row under the smallest window, which is the
+// configuration's window (every per-head window is at least that).
+bool stream_variant(const hyb_attn_ctx* x) { return geometry(x->cfg, x->T).nb > kStreamBlocks; }
 
 // Several pending appends (a chunked append, or many appends since the last
 // fold): one dense pass of fold_kernel over every unit's evictions, so that the
@@ -322,7 +326,7 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   fp.v_new = static_cast<const __nv_bfloat16*>(v_new);
   const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
   if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
-  const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
+  const cudaError_t e = launch_fused(x->maps, fp, x->tb, stream_variant(x), x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->pending = 0;
   if (k_new != nullptr) {  // the new token's eviction, if any, is folded by the next decode
@@ -496,7 +500,7 @@ int init_impl(hyb_attn_ctx** out, const hyb_attn_config* cfg, const hyb_attn_buf
   // the longest evicted range and the most blocks over the units (the grid's extent)
   int64_t ev_max = 0;
   for (int u = 0; u < k.units; ++u) {
-    const UnitGeo g = unit_geo(x->tb, u, cfg->n_kv_heads, (int32_t)x->T, cfg->n_sink, cfg->window,
+    const UnitGeo g = unit_geo(&x->tb, u, cfg->n_kv_heads, (int32_t)x->T, cfg->n_sink, cfg->window,
                                cfg->block_size, 0, 1, 0);
     ev_max = std::max<int64_t>(ev_max, g.ev_end - cfg->n_sink);
   }
@@ -593,7 +597,7 @@ int hyb_attn_sync_state(hyb_attn_ctx* x, cudaStream_t stream) {
   if (x->pending == 0) return HYB_OK;  // nothing appended since the last fold
   if (x->pending >= kFoldKernelMin) return fold_pending(x, stream);
   FusedParams fp = fused_params(x);   // q == null: fold only
-  const cudaError_t e = launch_fused(x->maps, fp, x->ck.D, stream);
+  const cudaError_t e = launch_fused(x->maps, fp, x->tb, stream_variant(x), x->ck.D, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->pending = 0;
   return HYB_OK;

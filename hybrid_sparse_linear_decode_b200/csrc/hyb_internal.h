@@ -71,13 +71,14 @@ struct UnitGeo {
 
 __host__ __device__ inline int32_t ev_end_at(int32_t T, int32_t S, int32_t W) { return T > S + W ? T - W : S; }
 
-__host__ __device__ inline UnitGeo unit_geo(const UnitTables& tb, int unit, int Hkv, int32_t T, int32_t S,
+// tb == null: every unit at (T, W, top_k)
+__host__ __device__ inline UnitGeo unit_geo(const UnitTables* tb, int unit, int Hkv, int32_t T, int32_t S,
                                             int32_t W, int32_t Bk, int32_t top_k, int32_t cpb, int32_t pending) {
   UnitGeo g;
   const int b = unit / Hkv, h = unit - b * Hkv;
-  g.T = T - (tb.ragged ? tb.row_lag[b] : 0);
-  g.W = tb.per_head ? tb.head_W[h] : W;
-  g.top_k = tb.per_head ? tb.head_k[h] : top_k;
+  g.T = T - ((tb != nullptr && tb->ragged) ? tb->row_lag[b] : 0);
+  g.W = (tb != nullptr && tb->per_head) ? tb->head_W[h] : W;
+  g.top_k = (tb != nullptr && tb->per_head) ? tb->head_k[h] : top_k;
   g.sink_len = g.T < S ? g.T : S;
   g.win_start = g.T > S ? (g.T - g.W > S ? g.T - g.W : S) : g.T;
   g.ev_end = ev_end_at(g.T, S, g.W);
@@ -119,8 +120,13 @@ struct FusedParams {           // one decode (or, with q == null, the fold only)
   float scale;
   uint64_t wait_ns;             // limit of every bounded wait for progress inside the kernel
   uint32_t test_flags;          // HYB_TEST_* (0 in normal use)
-  UnitTables tb;
 };
+
+// The decode kernel's per-unit tables, a launch parameter of their own only in
+// the variant for contexts that have them (the uniform variant's launches stay
+// small).
+template <bool kTab> struct TabArg {};
+template <> struct TabArg<true> { UnitTables tb; };
 
 struct AppendParams {       // write n tokens per unit at each row's positions [T_b, T_b + n)
   const __nv_bfloat16* k_new; // [units][n][D]
@@ -164,7 +170,11 @@ struct InitParams {          // the state of every unit's evicted range [S, ev_e
 // for its predecessor grid before it touches memory, so stream order holds.
 // maps: K and V with 64-row boxes, then K and V with 16-row boxes.
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s);
-cudaError_t launch_fused(const CUtensorMap* maps, const FusedParams& p, int D, cudaStream_t s);
+// stream: some unit of the launch has more than kStreamBlocks candidate blocks
+// (the variant whose statistics warps keep the top-k while scoring)
+constexpr int kStreamBlocks = 512;
+cudaError_t launch_fused(const CUtensorMap* maps, const FusedParams& p, const UnitTables& tb, bool stream, int D,
+                         cudaStream_t s);
 cudaError_t prepare_fused(int D);
 // clusters of c CTAs of the decode kernel the current device can hold at once (0: none)
 int fused_max_clusters(int D, int c);

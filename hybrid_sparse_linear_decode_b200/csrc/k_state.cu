@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
   __shared__ __align__(16) float ks[32][D];
   __shared__ __align__(16) float vs[32][D];
   const int unit = blockIdx.x, tid = threadIdx.x;
-  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, p.pending);
+  const UnitGeo g = unit_geo(&p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, p.pending);
   const int64_t fb = g.fold_begin, fe = g.fold_end;
   if (tid == 0) pdl_wait_primary();  // the caches' rows and the state may come from the previous grid
   __syncthreads();
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(256) init_linear_kernel(const __grid_constant_
   __shared__ __align__(16) float vs[32][D];
   const int unit = blockIdx.y, tid = threadIdx.x;
   const int tr = tid / 16, tc = tid % 16;
-  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
+  const UnitGeo g = unit_geo(&p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
   const int64_t t0 = p.S + (int64_t)blockIdx.x * p.tokens_per_cta;
   const int64_t t1 = min(t0 + (int64_t)p.tokens_per_cta, (int64_t)g.ev_end);
   if (t0 >= t1) return;  // past this unit's evicted range
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(256) init_stats_kernel(const __grid_constant__
   constexpr int CPL = D / 32;
   const int unit = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * 8 + warp;
-  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
+  const UnitGeo g = unit_geo(&p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
   if (j >= g.nb) return;
   const int64_t bs = p.S + (int64_t)j * p.Bk;
   const int64_t be = min(bs + (int64_t)p.Bk, (int64_t)g.ev_end);
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(256) init_stats_kernel(const __grid_constant__
 template <int D>
 __global__ void __launch_bounds__(256) init_finalize_kernel(const __grid_constant__ InitParams p) {
   const int unit = blockIdx.x, tid = threadIdx.x;
-  const UnitGeo g = unit_geo(p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
+  const UnitGeo g = unit_geo(&p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, 0);
   const double* H64 = p.H64 + (int64_t)unit * D * D;
   float* H = p.H + (int64_t)unit * D * D;
   for (int e = tid; e < D * D; e += 256) H[e] = (float)H64[e];

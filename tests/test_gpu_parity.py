@@ -370,3 +370,39 @@ def test_selection_above_512_blocks(kw):
     c = _case(**kw)
     full_check(c, c.random_q())
     assert c.layer.status() == 0
+
+
+def test_distributed_selection_with_all_scores_equal():
+    """Above 512 blocks each rank selects its own share's top-k and the ranks
+    merge their candidates.  With q = 0 every score is 0: the k lowest block
+    indices must be selected (ties to the lower index, across ranks), the share
+    of a rank holds more equal keys than its gather segments (the radix
+    fallback inside the rank), and the output is the mean of V."""
+    import torch
+    c = _case(B=16, Hq=16, Hkv=4, d=64, T0=4 + 16 + 8 * 1100, Bk=8, S=4, W=16, k=16, seed=13)
+    q = np.zeros((c.B, c.Hq, c.d), dtype=np.uint16)
+    out, sel, _ = c.decode(q)
+    assert (sel == np.arange(16, dtype=np.int32)[None, None, :]).all()
+    for b, h in ((0, 0), (15, 3), (7, 2)):
+        Kf, Vf = c.unit_kv(b, h)
+        check_outputs(out[b, h * c.G:(h + 1) * c.G], np.broadcast_to(Vf.mean(axis=0), (c.G, c.d)),
+                      max_abs=1e-4, rel_l2=1e-4)
+    assert c.layer.status() == 0
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T0=600, Bk=1, S=4, W=32, k=16),                        # 564 one-token blocks: the distributed selection
+    dict(T0=600, Bk=1, S=4, W=32, k=40),                        # k > 32: the radix selection
+    dict(B=2, Hq=8, Hkv=2, d=64, T0=300, Bk=1, S=2, W=20, k=12),
+])
+def test_token_granular_exact_set(kw):
+    """Token granularity (the block size 1): the exact set is the sinks, the
+    window and the top-k evicted tokens by their group-summed score s_t; every
+    other evicted token takes the Taylor weight through the subtraction form."""
+    c = _case(**kw)
+    full_check(c, c.random_q())
+    c2 = _case(n_append=5, **kw)
+    c2.append(5)
+    full_check(c2, c2.random_q())
+    check_state(c2)
+    assert c.layer.status() == 0 and c2.layer.status() == 0

@@ -305,3 +305,37 @@ def test_population_variance():
     K = np.array([[0.0], [2.0]])
     mu, var = O.block_stats(K, O.partition(2, 0, 0, 2))
     assert mu[0, 0] == 1.0 and var[0, 0] == 1.0
+
+
+# ----------------------------------------------------------------------------- token granularity
+
+def test_block_size_one_is_token_granular_selection():
+    """Token-granular exact set (the first-order Taylor kernel for every
+    evicted token but the top ones by their own score, which keep the exact
+    kernel): at block size 1 a block is one token, its mean is the key and its
+    variance 0, so the block score is the group-summed s_t = sum_i q'_i . k_t,
+    computed here by loops over the tokens; the selection is then the k evicted
+    tokens of largest summed score (ties to the lower position), and the hybrid
+    output is the token-by-token definition with exactly those tokens exact."""
+    rng = np.random.default_rng(31)
+    T, S, W, G, d, k = 90, 3, 7, 2, 6, 9
+    q, K, V = _rand(rng, T, d, G)
+    scale = 1 / math.sqrt(d)
+    part = O.partition(T, S, W, 1)
+    assert part.nb == T - S - W
+    mu, var = O.block_stats(K, part)
+    scores = O.block_scores(q, mu, var, scale)
+    for j in range(part.nb):
+        t = S + j
+        st = 0.0
+        for i in range(G):
+            for c in range(d):
+                st += q[i, c] * scale * K[t, c]
+        assert abs(scores[j] - st) < 1e-12
+        assert np.all(var[j] == 0.0)
+    sel = O.select_blocks(scores, k)
+    order = sorted(range(part.nb), key=lambda j: (-scores[j], j))[:k]
+    assert list(sel) == sorted(order)
+    got = O.hybrid_subtract(q, K, V, part, sel, scale)
+    ref = O.brute_force_hybrid(q, K, V, T, S, W, 1, sel, scale)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
