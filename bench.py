@@ -100,13 +100,37 @@ def algorithmic_bytes(w, T):
     return decode, append
 
 
-def step_bytes_model(w, mode: str, chunk: int, T: int):
+def spec_bytes(w, T: int, n: int, union_blocks: float):
+    """Bytes per (layer, b, kv head) of n draft rows decoded together (rows at
+    lengths T .. T + n - 1) with their appends: what the rows share is counted
+    once -- the block statistics of the last row's blocks, the sinks and the
+    union of the rows' windows, the linear state, and the union of the rows'
+    selected blocks (`union_blocks`, measured) -- plus every row's q and output;
+    the appends write n cache rows, read the n tokens they evict and write the
+    state back once."""
+    d, G = w.head_dim, w.group
+    Tl = T + n - 1
+    sinks = min(w.n_sink, Tl)
+    window = Tl - max(w.n_sink, Tl - w.window) if Tl > w.n_sink else 0
+    exact = sinks + window + min(w.evicted(Tl), union_blocks * w.block_size)
+    dec = w.n_blocks(Tl) * 2 * d * 4 + exact * d * 2 * 2 + (d * d + 2 * d + 1) * 4 + n * G * d * 6
+    app = n * 4 * d + n * 4 * d + d * d * 4 + 2 * d * 4 + 4 + 2 * 2 * d * 4
+    return dec, app
+
+
+def step_bytes_model(w, mode: str, chunk: int, T: int, union_blocks=None):
     """(decode bytes, all bytes, flush L2?) of one step at length about T: every
     layer with its own budget; prefill: the chunk's rows and evicted tokens, the
-    state written back once, one decode; spec: one decode per draft row (the
-    bytes of per-row decodes)."""
+    state written back once, one decode; spec: the chunk's draft rows decoded
+    together (spec_bytes, with the measured union of their selections per layer;
+    without it, the bytes of one decode per row)."""
     step_dec = step_bytes = 0
     for l in range(w.layers):
+        if mode == "spec" and union_blocks is not None:
+            dec_b, app_b = spec_bytes(w.for_layer(l), T, chunk, union_blocks[l])
+            step_dec += w.units_per_layer * dec_b
+            step_bytes += w.units_per_layer * (dec_b + app_b)
+            continue
         dec_b, app_b = algorithmic_bytes(w.for_layer(l), T)
         if mode == "prefill":
             d = w.head_dim
@@ -278,10 +302,30 @@ class Bench:
     def launches_per_step(self):
         """Kernels per step: one fused decode launch per layer (the append's
         cache write and the fold of the previous evictions ride in it); spec:
-        one per draft token; prefill: the chunk's cache write, the dense fold of
-        the tokens it evicted (4 or more) and one decode."""
-        per = {"decode": 1, "spec": self.chunk, "prefill": 2 + (self.chunk >= 4)}[self.mode]
+        one multi-query launch per group of 4, then 2, then 1 draft rows;
+        prefill: the chunk's cache write, the dense fold of the tokens it
+        evicted (5 or more) and one decode."""
+        n = self.chunk
+        groups = n // 4 + (n % 4) // 2 + (n % 2)
+        per = {"decode": 1, "spec": groups, "prefill": 2 + (self.chunk >= 5)}[self.mode]
         return per * len(self.layers)
+
+    def union_blocks(self):
+        """Spec mode: the rows of one step decoded with their selections kept;
+        per layer, the mean over units of the number of distinct blocks the
+        rows selected (consumes one step, before any timing)."""
+        import torch
+        w, n, s = self.w, self.chunk, self.step_idx
+        res = []
+        for l, L in enumerate(self.layers):
+            wl = w.for_layer(l)
+            sel = torch.full((n, w.batch, w.n_kv_heads, wl.top_k), -1, dtype=torch.int32, device=self.device)
+            L.decode_chunk(self.q[l][s % len(self.q[l])], self.app_k[l][s * n:(s + 1) * n],
+                           self.app_v[l][s * n:(s + 1) * n], out=self.out_chunk, sel_out=sel)
+            a = sel.cpu().numpy().reshape(n, -1, wl.top_k)
+            res.append(float(np.mean([len(set(a[:, u].ravel().tolist()) - {-1}) for u in range(a.shape[1])])))
+        self.step_idx += 1
+        return res
 
 
 def run_native(args, rank, world):
@@ -294,9 +338,11 @@ def run_native(args, rank, world):
     mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
     Kk = min(K, 20) if mode == "decode" else 0  # steps of the pass timing each launch on its own
     Ke = 0 if (args.no_e2e or mode != "decode") else min(K, 20)  # steps of the end-to-end pass
-    b = Bench(w, Wm + K + Kk + Ke, device, mode, chunk)
-    T_mid = w.T0 + (Wm + K // 2) * chunk
-    step_dec, step_bytes, flush = step_bytes_model(w, mode, chunk, T_mid)
+    Kp = 1 if mode == "spec" else 0  # the step that measures the rows' union of selected blocks
+    b = Bench(w, Kp + Wm + K + Kk + Ke, device, mode, chunk)
+    union = b.union_blocks() if mode == "spec" else None
+    T_mid = w.T0 + (Kp + Wm + K // 2) * chunk
+    step_dec, step_bytes, flush = step_bytes_model(w, mode, chunk, T_mid, union)
     scratch = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if flush else None
 
     def barrier():
@@ -373,31 +419,43 @@ def run_native(args, rank, world):
     isolated = launch_bytes / (isolated_ms * 1e-3) / 1e9 if isolated_ms else None
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
-    # ---- e2e through the host-buffer entry point (pinned host q / k / v / out)
+    # ---- e2e through the whole-step host entry point: per step one copy of every
+    # layer's q / k / v in from pinned host memory, every layer's decode +
+    # append, one copy of every layer's output back (hyb_attn_step_layers_host)
     e2e = None
     if Ke > 0:
-        qh = [[t.cpu().pin_memory() for t in qs] for qs in b.q]
-        kh = [t.cpu().pin_memory() for t in b.app_k]
-        vh = [t.cpu().pin_memory() for t in b.app_v]
-        oh = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32).pin_memory()
+        import hybrid_sparse_linear_decode_b200 as H
+        ctxs = [L.ctx for L in b.layers]
+        nst = H.hyb_attn_step_layers_staging_bytes(ctxs)
+        staging = torch.empty(nst, dtype=torch.uint8, device=device)
         s0 = b.step_idx
         assert s0 + Ke <= b.n_steps
+        hin, per_layer_in = [], None
+        for i in range(Ke):  # each step's inputs, layer after layer: q, k, v (bf16 bytes), pinned
+            s = s0 + i
+            parts = []
+            for l in range(len(b.layers)):
+                parts += [b.q[l][s % len(b.q[l])].reshape(-1), b.app_k[l][s].reshape(-1), b.app_v[l][s].reshape(-1)]
+            flat = torch.cat(parts).cpu()
+            per_layer_in = flat.numel() * 2
+            hin.append(flat.pin_memory())
+        hout = torch.empty(len(b.layers) * w.batch * w.n_q_heads * w.head_dim, dtype=torch.float32).pin_memory()
+        sh = stream.cuda_stream
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
         for i in range(Ke):
-            s = b.step_idx
             evs[i][0].record(stream)
-            for l, L in enumerate(b.layers):
-                L.step_host(qh[l][s % len(qh[l])], kh[l][s], vh[l][s], oh)
+            H.hyb_attn_step_layers_host(ctxs, hin[i].data_ptr(), hout.data_ptr(), staging.data_ptr(), nst, sh)
             evs[i][1].record(stream)
             b.step_idx += 1
             if flush:
                 scratch.zero_()
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs) / Ke, world, device)
-        h2d = w.layers * (w.batch * w.n_q_heads * w.head_dim * 2 + 2 * w.batch * w.n_kv_heads * w.head_dim * 2)
-        d2h = w.layers * w.batch * w.n_q_heads * w.head_dim * 4
+        h2d = per_layer_in
+        d2h = hout.numel() * 4
         e2e = {"value": round(aggregate_steps_per_s(e2e_ms, world), 3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)}
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
+               "call": "hyb_attn_step_layers_host (one copy in, every layer's decode + append, one copy out)"}
 
     status = 0
     for L in b.layers:
@@ -421,8 +479,12 @@ def run_native(args, rank, world):
         "achieved_gbs_step": round(step_gbs, 1),
         "pct_of_hbm_peak_step": round(100 * step_gbs / hbm_peak, 2),
         "bytes_per_step": step_bytes,
+        **({"union_selected_blocks_per_unit": [round(u, 2) for u in union],
+            "bytes_model": "draft rows decoded together: shared reads counted once, the union of the rows' "
+                           "selected blocks as measured"} if union is not None else {}),
         "roofline": {"bound": "hbm",
-                     "kernel": "the fused decode kernel: one layer's decode + append (one launch)",
+                     "kernel": ("the multi-query decode kernel: one layer's draft rows decoded + appended together"
+                                if mode == "spec" else "the fused decode kernel: one layer's decode + append (one launch)"),
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
                      "traffic": measured_traffic(w.name), "bytes_per_launch": launch_bytes,

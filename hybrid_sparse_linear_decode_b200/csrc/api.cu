@@ -215,6 +215,7 @@ struct hyb_attn_ctx {
   UnitTables tb;        // per-row lengths and per-head budgets (uniform when not given)
   int device, n_sm;
   int fits[kMaxCluster + 1];  // clusters of C CTAs of the decode kernel the device holds at once
+  int fits_multi[2][kMaxCluster + 1];  // the same for the multi-query kernel with 2 and 4 rows
   float scale;
   uint64_t wait_ns;     // limit of the kernels' bounded waits for progress
   uint32_t test_flags;  // HYB_TEST_* failure injection (tests only)
@@ -337,6 +338,47 @@ int decode_impl(hyb_attn_ctx* x, const void* q, float* out, const int32_t* sel_g
   return HYB_OK;
 }
 
+// Can the multi-query kernel take nr (2 or 4) rows from the current length?
+// Uniform lengths and budgets, k <= 32, a window of at least nr - 1 tokens (the
+// rows' new tokens then lie in the shared prefix), and the last row's block
+// scores for every row fit the kernel's shared memory.
+bool multi_fits(const hyb_attn_ctx* x, int nr) {
+  const hyb_attn_config& c = x->cfg;
+  if (x->tb.ragged || x->tb.per_head) return false;
+  if (c.top_k > 32 || c.window < nr - 1) return false;
+  if (x->T + nr > c.capacity) return false;
+  const Geometry g = geometry(c, x->T + nr - 1);
+  if (g.nb > multi_score_capacity(nr)) return false;
+  const int C = cluster_ctas(x->ck.units, x->n_sm, x->fits_multi[nr == 2 ? 0 : 1]);
+  return C >= 1 && x->ck.G <= kMaxGroup;
+}
+
+// nr consecutive decode + append steps in one launch of the multi-query kernel
+// (after fold_kernel when many evictions are pending).
+int decode_multi(hyb_attn_ctx* x, int nr, const void* q, const void* k_new, const void* v_new, float* out,
+                 int32_t* sel_out, cudaStream_t stream) {
+  const int rf = fold_pending(x, stream);
+  if (rf != HYB_OK) return rf;
+  FusedParams fp = fused_params(x);
+  const Checked& k = x->ck;
+  fp.C = cluster_ctas(k.units, x->n_sm, x->fits_multi[nr == 2 ? 0 : 1]);
+  fp.mstride = multi_merge_stride(nr, k.G * k.D, fp.C);
+  for (int r = 0; r <= fp.C; ++r) fp.mslice[r] = r * (nr * k.G * k.D) / fp.C;
+  fp.q = static_cast<const __nv_bfloat16*>(q);
+  fp.out = out;
+  fp.sel_out = sel_out;
+  fp.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  fp.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  const bool timed = x->ev_begin != nullptr && x->ev_end != nullptr;
+  if (timed && cudaEventRecord(x->ev_begin, stream) != cudaSuccess) return HYB_ECUDA;
+  const cudaError_t e = launch_multi(x->maps, fp, k.D, nr, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  x->T += nr;
+  x->pending = nr;  // the state is folded to row 0's eviction edge
+  if (timed && cudaEventRecord(x->ev_end, stream) != cudaSuccess) return HYB_ECUDA;
+  return HYB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -435,7 +477,7 @@ int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t 
   x->tb = tb;
   x->device = device;
   x->n_sm = n_sm;
-  for (int c = 0; c <= kMaxCluster; ++c) x->fits[c] = 0;
+  for (int c = 0; c <= kMaxCluster; ++c) x->fits[c] = x->fits_multi[0][c] = x->fits_multi[1][c] = 0;
   x->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)k.D);
   x->wait_ns = kWaitLimit;
   x->test_flags = 0u;
@@ -451,11 +493,16 @@ int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t 
   }
   cudaError_t pe = prepare_fused(k.D);
   if (pe == cudaSuccess) pe = prepare_state(k.D);
+  if (pe == cudaSuccess) pe = prepare_multi(k.D);
   if (pe != cudaSuccess) {
     delete x;
     return cuda_fail(pe);
   }
-  for (int c = 2; c <= kMaxCluster; ++c) x->fits[c] = fused_max_clusters(k.D, c);
+  for (int c = 2; c <= kMaxCluster; ++c) {
+    x->fits[c] = fused_max_clusters(k.D, c);
+    x->fits_multi[0][c] = multi_max_clusters(k.D, 2, c);
+    x->fits_multi[1][c] = multi_max_clusters(k.D, 4, c);
+  }
   *out = x;
   return HYB_OK;
 }
@@ -621,15 +668,24 @@ int hyb_attn_decode_chunk(hyb_attn_ctx* x, const void* q, const void* k_new, con
   HYB_RANGE;
   if (x == nullptr || q == nullptr || k_new == nullptr || v_new == nullptr || out == nullptr || n < 1)
     return HYB_EINVAL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return HYB_EINVAL;
+  if (sel_out != nullptr && (reinterpret_cast<uintptr_t>(sel_out) & 3u)) return HYB_EINVAL;
   if (x->T == 0) return HYB_ESTATE;
   if (x->T + n > x->cfg.capacity) return HYB_ECAPACITY;
   const size_t U = (size_t)x->ck.units, D = (size_t)x->ck.D, G = (size_t)x->ck.G;
-  for (int32_t j = 0; j < n; ++j) {  // row j: decode at length T + j, then append token j
-    const int r = decode_impl(x, static_cast<const char*>(q) + j * U * G * D * 2, out + j * U * G * D, nullptr,
-                              sel_out == nullptr ? nullptr : sel_out + j * U * (size_t)x->cfg.top_k, nullptr,
-                              static_cast<const char*>(k_new) + j * U * D * 2,
-                              static_cast<const char*>(v_new) + j * U * D * 2, stream);
+  int32_t j = 0;
+  while (j < n) {  // rows j, j + 1, ...: decodes at lengths T + j, ..., each then appending its token
+    const int want = n - j >= 4 ? 4 : n - j >= 2 ? 2 : 1;
+    const bool multi = want > 1 && multi_fits(x, want);
+    const int nr = multi ? want : 1;
+    const char* qj = static_cast<const char*>(q) + j * U * G * D * 2;
+    const char* kj = static_cast<const char*>(k_new) + j * U * D * 2;
+    const char* vj = static_cast<const char*>(v_new) + j * U * D * 2;
+    int32_t* sj = sel_out == nullptr ? nullptr : sel_out + j * U * (size_t)x->cfg.top_k;
+    const int r = multi ? decode_multi(x, nr, qj, kj, vj, out + j * U * G * D, sj, stream)
+                        : decode_impl(x, qj, out + j * U * G * D, nullptr, sj, nullptr, kj, vj, stream);
     if (r != HYB_OK) return r;
+    j += nr;
   }
   return HYB_OK;
 }

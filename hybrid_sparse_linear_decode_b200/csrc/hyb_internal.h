@@ -149,7 +149,7 @@ struct FoldParams {         // fold every unit's pending evicted positions into 
 };
 // pending appends from which a decode or a state sync folds the evictions with
 // fold_kernel (one dense pass) instead of inside the decode kernel
-constexpr int64_t kFoldKernelMin = 4;
+constexpr int64_t kFoldKernelMin = 5;
 
 struct InitParams {          // the state of every unit's evicted range [S, ev_end(T_b, W_h))
   const __nv_bfloat16* k_cache;
@@ -179,6 +179,17 @@ cudaError_t prepare_fused(int D);
 // clusters of c CTAs of the decode kernel the current device can hold at once (0: none)
 int fused_max_clusters(int D, int c);
 cudaError_t launch_init(const InitParams& p, int D, cudaStream_t s);
+// The multi-query decode kernel (k_multi.cu): NR (2 or 4) consecutive new
+// tokens per unit in one launch.  Requirements the host checks: uniform
+// lengths and budgets, top_k <= 32, window >= NR - 1, the last row's block
+// count <= multi_score_capacity(NR); p.mstride / p.mslice computed with
+// multi_merge_stride over NR * G * D outputs.
+int multi_rows_max();
+int multi_score_capacity(int NR);
+int multi_merge_stride(int NR, int GD, int C);
+cudaError_t prepare_multi(int D);
+int multi_max_clusters(int D, int NR, int c);
+cudaError_t launch_multi(const CUtensorMap* maps, const FusedParams& p, int D, int NR, cudaStream_t s);
 cudaError_t launch_fold(const FoldParams& p, int D, cudaStream_t s);
 // per device, before the first launch: shared-memory size, cluster and carveout attributes
 cudaError_t prepare_state(int D);

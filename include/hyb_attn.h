@@ -233,7 +233,7 @@ int hyb_attn_append_chunk(hyb_attn_ctx* ctx, const void* k_new, const void* v_ne
 /* Fold every token evicted since the last decode into the state arrays, so that
  * they describe L = [S, T - W) exactly (for a checkpoint, or to read them).  A
  * no-op when nothing is pending; one launch otherwise (the dense fold pass when
- * 4 or more tokens are pending, else the decode kernel in fold-only mode).
+ * 5 or more tokens are pending, else the decode kernel in fold-only mode).
  * Errors: HYB_EINVAL, HYB_ECUDA. */
 int hyb_attn_sync_state(hyb_attn_ctx* ctx, cudaStream_t stream);
 
@@ -248,7 +248,7 @@ int hyb_attn_sync_state(hyb_attn_ctx* ctx, cudaStream_t stream);
  * the tokens evicted since the previous decode, forms the global linear term
  * phi(q)^T state, selects the top-k, attends sinks, window and selected blocks
  * exactly (split-K over the cluster, with the selected blocks' (1 + s)
- * subtraction) and merges under the shared normaliser.  When 4 or more evicted
+ * subtraction) and merges under the shared normaliser.  When 5 or more evicted
  * tokens are pending (a chunked append, or many appends since the last fold),
  * a dense fold pass over them is launched first (H += K^T V over the run, zk,
  * zv, n, and the touched blocks' statistics merged pairwise).
@@ -267,8 +267,14 @@ int hyb_attn_decode_append(hyb_attn_ctx* ctx, const void* q, const void* k_new, 
 /* n decode steps of n consecutive new tokens (speculative verification of a
  * draft of n tokens): row j decodes q[j] at length T + j -- it attends to the
  * stored history and to the chunk's tokens 0 .. j-1, with its own window, block
- * scores and top-k -- and then appends token j; T += n in all.  Identical to n
- * calls of hyb_attn_decode_append (one launch each, chained).
+ * statistics, scores and top-k -- and then appends token j; T += n in all.
+ * The result is that of n calls of hyb_attn_decode_append.  The rows go in
+ * groups of 4 (then 2, then 1) through the multi-query kernel, one launch per
+ * group: what the group's rows share (the sinks and windows, the block
+ * statistics, the linear state, the blocks several rows select) is read once.
+ * A group falls back to one launch per row when the context has per-row
+ * lengths or per-head budgets, top_k > 32, window < rows - 1, or more blocks
+ * than the kernel keeps scores for (4096 / rows per row).
  *   q       bf16 [n][B][Hq][d]     k_new, v_new  bf16 [n][B][Hkv][d]
  *   out     fp32 [n][B][Hq][d]     sel_out       int32 [n][B][Hkv][top_k] or NULL
  * Errors: HYB_EINVAL (null or misaligned pointers, n < 1), HYB_ESTATE (T == 0),

@@ -65,7 +65,8 @@ def test_all_selected_is_softmax_and_q0_is_mean():
     (dict(T0=600, Bk=32, W=64), 40),
     (dict(T0=4 + 64 + 32 * 3, Bk=32, W=64), 3),               # the first append opens a new block
     (dict(T0=601, Bk=32, W=64), 2),                           # two pending: folded inside the decode kernel
-    (dict(T0=601, Bk=32, W=64), 4),                           # four pending: the dense fold pass
+    (dict(T0=601, Bk=32, W=64), 4),                           # four pending: folded inside the decode kernel
+    (dict(T0=601, Bk=32, W=64), 5),                           # five pending: the dense fold pass
     (dict(T0=10, S=4, W=16, Bk=8), 40),                       # grows from sinks-only through eviction
     (dict(T0=200, W=0, Bk=8), 20),                            # W = 0 evicts the appended token itself
     (dict(T0=300, S=0, W=5, Bk=7, d=64), 30),
@@ -296,10 +297,15 @@ def test_append_chunk_matches_oracle(kw, n):
 
 
 @pytest.mark.parametrize("kw,n", [
-    (dict(T0=600, n_append=8), 8),
-    (dict(T0=4 + 64 + 32 * 5 - 3, n_append=6), 6),                   # the chunk completes a block
-    (dict(B=2, Hq=16, Hkv=4, T0=1500, Bk=64, W=100, k=6, n_append=5), 5),
+    (dict(T0=600, n_append=8), 8),                                    # two launches of 4 rows
+    (dict(T0=4 + 64 + 32 * 5 - 3, n_append=6), 6),                   # 4 + 2 rows; the chunk completes a block
+    (dict(B=2, Hq=16, Hkv=4, T0=1500, Bk=64, W=100, k=6, n_append=5), 5),   # 4 rows + 1
     (dict(T0=70, S=4, W=64, n_append=4), 4),                          # eviction starts inside the chunk
+    (dict(T0=2, S=4, W=16, Bk=8, n_append=4), 4),                     # the sinks fill inside the chunk
+    (dict(T0=300, S=3, W=20, Bk=1, k=12, n_append=4), 4),             # one-token blocks: E tokens in 3 blocks
+    (dict(Hq=8, Hkv=8, d=64, T0=900, Bk=16, W=40, k=5, n_append=2), 2),     # G = 1, 2 rows
+    (dict(B=2, Hq=8, Hkv=2, T0=4 + 64 + 8 * 1300, Bk=8, W=64, k=20, n_append=2), 2),  # 1300 blocks, 2 rows
+    (dict(B=4, Hq=32, Hkv=8, T0=5000, Bk=64, W=1024, k=16, n_append=4), 4),  # 32 units
 ])
 def test_decode_chunk_rows_match_oracle(kw, n):
     """Speculative verification of n draft tokens: row j is the decode at length
@@ -406,3 +412,39 @@ def test_token_granular_exact_set(kw):
     full_check(c2, c2.random_q())
     check_state(c2)
     assert c.layer.status() == 0 and c2.layer.status() == 0
+
+
+def test_decode_chunk_repeated_chunks_and_state():
+    """Speculative verification, chunk after chunk (each call folds the
+    evictions the previous chunk left pending): 5 chunks of 4 draft rows, every
+    row against the oracle at its own length, then the state."""
+    import torch
+    from harness import to_device_bf16
+    c = _case(B=2, Hq=16, Hkv=4, T0=1200, Bk=32, W=64, k=6, n_append=20, seed=17)
+    dev = c.layer.device
+    n = 4
+    for step in range(5):
+        qs = np.stack([c.random_q() for _ in range(n)])
+        kb = to_device_bf16(np.ascontiguousarray(c.Kb[:, :, c.T:c.T + n].transpose(2, 0, 1, 3)), dev)
+        vb = to_device_bf16(np.ascontiguousarray(c.Vb[:, :, c.T:c.T + n].transpose(2, 0, 1, 3)), dev)
+        sel = torch.full((n, c.B, c.Hkv, c.k), -7, dtype=torch.int32, device=dev)
+        out = c.layer.decode_chunk(to_device_bf16(qs, dev), kb, vb, sel_out=sel)
+        torch.cuda.synchronize()
+        out, sel = out.cpu().numpy().astype(np.float64), sel.cpu().numpy()
+        T0 = c.T
+        for j in range(n):
+            c.T = T0 + j
+            refs, gots = [], []
+            for b in range(c.B):
+                for h in range(c.Hkv):
+                    _, _, oscores = c.oracle_unit(qs[j], b, h)
+                    check_selection(sel[j, b, h], oscores, c.k)
+                    gsel = np.array([int(x) for x in sel[j, b, h] if x >= 0], dtype=np.int64)
+                    ref, _, _ = c.oracle_unit(qs[j], b, h, sel=gsel)
+                    refs.append(ref)
+                    gots.append(out[j, b, h * c.G:(h + 1) * c.G])
+            check_outputs(np.array(gots), np.array(refs))
+        c.T = T0 + n
+    assert c.layer.T == c.T and c.layer.status() == 0
+    check_state(c)
+    full_check(c, c.random_q())
