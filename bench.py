@@ -142,32 +142,42 @@ def step_bytes_model(w, mode: str, chunk: int, T: int, union_blocks=None):
     return step_dec, step_bytes, flush
 
 
-KERNEL_SOURCES = ("k_fused.cu", "k_common.cuh", "hyb_device.cuh", "hyb_internal.h")
+KERNEL_SOURCES = {"fused": ("k_fused.cu", "k_common.cuh", "hyb_device.cuh", "hyb_internal.h"),
+                  "multi": ("k_multi.cu", "k_common.cuh", "hyb_device.cuh", "hyb_internal.h")}
 
 
-def kernel_sources_hash() -> str:
+def kernel_sources_hash(kernel: str = "fused") -> str:
     import hashlib
     csrc = os.path.join(ROOT, "hybrid_sparse_linear_decode_b200", "csrc")
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload: str):
-    """DRAM bytes of one layer's decode kernel from the committed ncu summary of
-    this workload, if the kernel's sources are unchanged since that capture
-    (else None)."""
+def profile_name(workload: str, mode: str = "decode", chunk: int = 1) -> str:
+    """The committed ncu summary of the launch the bench's roofline is about:
+    the fused decode kernel, or (spec mode) the multi-query kernel at the
+    chunk's group size."""
+    if mode == "spec":
+        return f"multi_decode_{workload}_rows{chunk}.md"
+    return f"fused_decode_{workload}.md"
+
+
+def measured_traffic(workload: str, mode: str = "decode", chunk: int = 1):
+    """DRAM bytes of one launch of the dominant kernel from the committed ncu
+    summary of this workload, if the kernel's sources are unchanged since that
+    capture (else None)."""
     import re
-    prof = os.path.join(ROOT, "profiles", f"fused_decode_{workload}.md")
+    prof = os.path.join(ROOT, "profiles", profile_name(workload, mode, chunk))
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
     mh = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]{16})", text)
-    mt = re.search(r"traffic_bytes_per_decode:\s*(\d+)", text)
+    mt = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
     if not (mh and mt):
         return None
-    return int(mt.group(1)) if kernel_sources_hash() == mh.group(1) else None
+    return int(mt.group(1)) if kernel_sources_hash("multi" if mode == "spec" else "fused") == mh.group(1) else None
 
 
 def peaks():
@@ -487,7 +497,7 @@ def run_native(args, rank, world):
                                 if mode == "spec" else "the fused decode kernel: one layer's decode + append (one launch)"),
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
-                     "traffic": measured_traffic(w.name), "bytes_per_launch": launch_bytes,
+                     "traffic": measured_traffic(w.name, mode, chunk), "bytes_per_launch": launch_bytes,
                      "decode_bytes_per_launch": step_dec // n_launch,
                      "avg_launch_us": round(launch_ms * 1e3, 3),
                      "isolated_launch_us": round(isolated_ms * 1e3, 3) if isolated_ms else None,

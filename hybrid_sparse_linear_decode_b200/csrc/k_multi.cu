@@ -30,12 +30,17 @@
 //
 // Grid and roles as the single-token decode kernel (k_fused.cu): one cluster of
 // C CTAs per unit, 8 attention warps in 4 pairs, 3 statistics warps, 1 producer
-// lane, a ring of kMStages stages.  With NR rows the pairs split by row (NR = 2:
-// pairs 0, 1 row 0 and pairs 2, 3 row 1, alternate chunks; NR = 4: pair r row
-// r, every chunk).  The rows' G query heads each are the mma N columns of their
-// pair, their selections are made per row by the statistics warps (one warp
-// per row, as the single-token kernel does), and the merge covers NR x G x D
-// outputs.  Every wait is bounded.
+// lane, a ring of kMStages stages.  The prefix chunks take no Taylor weights, so
+// a pair runs two rows on them at once: the 8 mma N columns are rows (a, a + 1)
+// x 4 heads, all exact (NR = 2: every pair rows 0, 1, a quarter of the chunks
+// each; NR = 4: pairs 0, 1 rows 0, 1 and pairs 2, 3 rows 2, 3, alternate
+// chunks).  After the prefix a pair leaves its partial in its combine slot and
+// takes one row, with the single-token layout (4 exact + 4 Taylor columns), for
+// the E and selected chunks (NR = 2: pairs 0, 1 row 0 and pairs 2, 3 row 1,
+// alternate chunks; NR = 4: pair r row r, every chunk that row r selected).
+// Selections are made per row by the statistics warps (one warp per row, as
+// the single-token kernel does), and the merge covers NR x G x D outputs.
+// Every wait is bounded.
 #include "k_common.cuh"
 
 namespace hyb {
@@ -43,6 +48,12 @@ namespace {
 
 constexpr int kMStages = 4;
 constexpr int kMScores = 4096;  // NR rows x stride of block scores in shared memory
+// tokens the launch reads from the caches one by one: the pending evictions
+// [fold_begin, fold_end) (at most 4: more are folded by the dense fold first)
+// and the rows' E tokens after them (at most NR - 1 = 3); staged in shared
+// memory by the prologue
+constexpr int kMaxPend = 4, kMaxX = 8;
+static_assert(kMaxPend >= kFoldKernelMin - 1 && kMaxX >= kMaxPend + 3, "staged token rows");
 
 // merge slot: per row a 16-float header (per head: max, exact weight sum,
 // D_glob - D_sel), then (exact part, N_glob - N_sel) pairs of the slice
@@ -72,17 +83,19 @@ struct MultiSmem {
   static constexpr int kStageBytes = 2 * kHalf;
   static constexpr int kBoxBytes = kBoxRows * D * 2;
   static constexpr int kPF = partial_floats(D);
-  static constexpr int kRec = NR > 2 ? NR : 2;
+  static constexpr int kRec = 4;  // one slot per attention pair
   static constexpr int kBmWords = kMScores / NR / 32;
   uint8_t ring[kMStages][kStageBytes];               // 1024-byte aligned
   float scores[kMScores];                            // [NR][sstride]
   float qs[NR * kMaxGroup][D];                       // row r head i at r * 4 + i
   float qsT[D][NR * kMaxGroup];
   float qsum[NR][2][D];                              // per row: sum_i q'_i, 1/2 sum_i q'_i^2
-  alignas(16) float wpart[kRec][kPF];                // combine slots; [r] ends as row r's record
+  alignas(16) float wpart[kRec][kPF];                // top-k candidates, then the pairs' prefix partials; [r] ends as row r's record
   float linp[NR * kMaxGroup][D + 1];                 // linear partials (D_glob in rank 0)
   alignas(16) float mrecv[mmerge_floats(NR, D)];
   float zks[D];
+  alignas(16) float xk[kMaxX][D];                    // keys of [fold_begin, ev_end[NR - 1])
+  alignas(16) float xv[kMaxPend][D];                 // values of [fold_begin, fold_end)
   int32_t sel[NR][32];                               // each row's selection (k <= 32), ascending
   uint32_t selbm[NR][kBmWords];                      // each row's selection as a bitmap over blocks
   int32_t uni_j[NR * 32];                            // the union of the selections (state range only)
@@ -234,7 +247,7 @@ __device__ __forceinline__ void mfold_item(const FusedParams& p, const UnitGeo& 
 #pragma unroll 1
     for (int t = t0; t < t1; ++t) {
       float x[CPL];
-      load_bf16<CPL>(p.k_cache + ((int64_t)unit * p.cap + t) * D + lane * CPL, x);
+      lds_vec<CPL>(&sm.xk[t - t_lo][lane * CPL], x);
       const float cnt = (float)(t - bs + 1);
       const float inv = 1.f / cnt;
 #pragma unroll
@@ -301,7 +314,6 @@ __device__ __forceinline__ void mh_item(const FusedParams& p, const UnitGeo& g, 
   const int r0 = s.h0 + idx * RH;
   const int nrows = min(RH, s.h1 - r0);
   const float* hrows = reinterpret_cast<const float*>(sm.ring[stage]);
-  const int64_t ub = (int64_t)unit * p.cap;
   const bool fold = g.fold_end > g.fold_begin;
 #pragma unroll 1
   for (int rl = aw; rl < nrows; rl += kAuxWarps) {
@@ -310,10 +322,10 @@ __device__ __forceinline__ void mh_item(const FusedParams& p, const UnitGeo& g, 
     lds_vec<CPL>(hrows + rl * D + lane * CPL, h);
     if (fold) {
 #pragma unroll 1
-      for (int t = g.fold_begin; t < g.fold_end; ++t) {
-        const float kr = __bfloat162float(p.k_cache[(ub + t) * D + row]);
+      for (int t = 0; t < g.fold_end - g.fold_begin; ++t) {
+        const float kr = sm.xk[t][row];
         float vv[CPL];
-        load_bf16<CPL>(p.v_cache + (ub + t) * D + lane * CPL, vv);
+        lds_vec<CPL>(&sm.xv[t][lane * CPL], vv);
 #pragma unroll
         for (int c = 0; c < CPL; ++c) h[c] += kr * vv[c];
       }
@@ -340,15 +352,14 @@ __device__ void mfinish_linear(const FusedParams& p, const UnitGeo& g, MultiSmem
                                const float (&hacc)[NR][kMaxGroup][D / 32]) {
   constexpr int CPL = D / 32;
   const int a = role_tid() - kAttnThreads, aw = a >> 5, lane = a & 31;
-  const int64_t ub = (int64_t)unit * p.cap;
   float nval = 0.f;
   if (rank == 0) {
     for (int c = a; c < D; c += kAuxThreads) {
       float zk = p.zk[(int64_t)unit * D + c], zv = p.zv[(int64_t)unit * D + c];
       if (g.fold_end > g.fold_begin) {
-        for (int t = g.fold_begin; t < g.fold_end; ++t) {
-          zk += __bfloat162float(p.k_cache[(ub + t) * D + c]);
-          zv += __bfloat162float(p.v_cache[(ub + t) * D + c]);
+        for (int t = 0; t < g.fold_end - g.fold_begin; ++t) {
+          zk += sm.xk[t][c];
+          zv += sm.xv[t][c];
         }
         p.zk[(int64_t)unit * D + c] = zk;
         p.zv[(int64_t)unit * D + c] = zv;
@@ -489,6 +500,61 @@ __device__ void mselect(const FusedParams& p, const MultiGeo<NR>& m, MultiSmem<D
       base += __shfl_sync(kFull, incl, 31);
     }
     if (lane == 0) sm.nuni = base;
+  }
+  // Issue order: by rounds, each round taking the next C blocks of every row in
+  // turn, so that the ring's consecutive chunks of a rank (every C-th) belong
+  // to different rows and the pairs, one row each, work side by side.  A block
+  // chosen by several rows goes at its earliest place: key = min over those
+  // rows r of (i / C) (NR C) + r C + i % C, i = the block's place in row r's
+  // ascending selection (i < 32, C <= 16: keys < 256, all distinct).
+  named_sync(kBarAux, kAuxThreads);
+  const int nU = sm.nuni, C = p.C;
+  for (int i = a; i < 256; i += kAuxThreads) sm.hist[i] = 0xffffffffu;
+  named_sync(kBarAux, kAuxThreads);
+  for (int u = a; u < nU; u += kAuxThreads) {
+    const int j = sm.uni_j[u];
+    const uint32_t msk = sm.uni_m[u];
+    int key = 255;
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+      if ((msk >> r) & 1u) {
+        int i = 0;
+        for (int e = 0; e < m.k_eff[r]; ++e) i += sm.sel[r][e] < j ? 1 : 0;
+        key = min(key, (i / C) * NR * C + r * C + i % C);
+      }
+    sm.hist[key] = (uint32_t)u;
+  }
+  named_sync(kBarAux, kAuxThreads);
+  if (aw == 0) {  // compaction in key order: lane l takes keys [8 l, 8 l + 8)
+    int jj[8];
+    uint32_t mm[8], have = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t u = sm.hist[8 * lane + e];
+      jj[e] = 0;
+      mm[e] = 0u;
+      if (u != 0xffffffffu) {
+        jj[e] = sm.uni_j[u];
+        mm[e] = sm.uni_m[u];
+        have |= 1u << e;
+      }
+    }
+    const int cnt = __popc(have);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    __syncwarp();  // every entry is read before any is rewritten
+    int pos = incl - cnt;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if ((have >> e) & 1u) {
+        sm.uni_j[pos] = jj[e];
+        sm.uni_m[pos] = mm[e];
+        ++pos;
+      }
   }
 }
 
@@ -755,7 +821,10 @@ __device__ void mproducer_role(const KVMaps* tm, const FusedParams& p, const Uni
 }
 
 // ---------------------------------------------------------------- attention role
-// Pair q of the 4 handles row q * NR / 4, chunks c with c % (4 / NR) == q % (4 / NR).
+// Prefix chunks: pair q handles rows (a, a + 1), a = 2 (q / 2) for NR = 4 (0
+// for NR = 2), chunks c with c % (8 / NR) == q % (8 / NR); N column n is row
+// a + n / 4, head n % 4.  Post-selection chunks: pair q handles row q * NR / 4,
+// chunks c with c % (4 / NR) == q % (4 / NR); columns 0-3 exact, 4-7 Taylor.
 // Token t of a chunk, for row r (T_r = T + r):
 //   prefix:   exact when t < T_r;
 //   E:        exact when t >= win_start[r] or its block is in row r's
@@ -767,33 +836,65 @@ template <int D, int NR>
 __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGeo<NR>& m, MultiSmem<D, NR>& sm,
                            const MSeq& s, int unit, int rank) {
   constexpr int NT8 = D / 8, NH = NT8 / 2, KS = D / 16;
-  constexpr int kPairsPerRow = 4 / NR;
+  constexpr int kPairsPerRow = 4 / NR, kPrePairs = 8 / NR;
   const int tid = role_tid(), warp = tid >> 5, lane = tid & 31;
   const int pair = warp >> 1, half = warp & 1;
   const int row = pair / kPairsPerRow, sub = pair % kPairsPerRow;
+  const int ra = NR == 4 ? (pair >> 1) * 2 : 0, psub = pair % kPrePairs;
   const int g8 = lane >> 2, tig = lane & 3;
   const bool p_lane = g8 < 4;
   const int head = g8 & 3;
   const int mi = lane >> 3, rr = lane & 7;
   const int Tr = g.T + row;
+  const int Tpre = g.T + ra + (tig >> 1);  // the row of this lane's prefix columns 2 tig, 2 tig + 1
   const int ws = m.win_start[row];
 
   uint32_t qb[KS][2];
-  {
+  auto load_q = [&](int qrow_idx) {  // N column g8: head g8 % 4 of row qrow_idx
     const bool real = (g8 & 3) < p.G;
     const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-        p.q + (((int64_t)row * p.units + unit) * p.G + (real ? (g8 & 3) : 0)) * D);
+        p.q + (((int64_t)qrow_idx * p.units + unit) * p.G + (real ? (g8 & 3) : 0)) * D);
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       qb[kk][0] = real ? __ldg(qrow + kk * 8 + tig) : 0u;
       qb[kk][1] = real ? __ldg(qrow + kk * 8 + 4 + tig) : 0u;
     }
-  }
+  };
+  load_q(ra + (g8 >> 2));
   float O[NH][4];
 #pragma unroll
   for (int n = 0; n < NH; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
-  const bool soft_lane = tig < 2;
+  bool pre = true;                    // the prefix chunks: every column exact
+  bool soft_lane = true;              // this lane's accumulator columns take softmax weights
   float mr0 = -INFINITY, mr1 = -INFINITY, acc0 = 0.f, acc1 = 0.f;
+  // the prefix partial of rows (ra, ra + 1) into this pair's combine slot
+  // (free once the selections are made): per column its max and weight sum,
+  // then the 8 columns' D outputs
+  auto flush_prefix = [&]() {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      acc0 += __shfl_xor_sync(kFull, acc0, o);
+      acc1 += __shfl_xor_sync(kFull, acc1, o);
+    }
+    const float v0 = __shfl_sync(kFull, acc0, g8 >> 1), v1 = __shfl_sync(kFull, acc1, g8 >> 1);
+    const float m0 = __shfl_sync(kFull, mr0, g8 >> 1), m1 = __shfl_sync(kFull, mr1, g8 >> 1);
+    float* wp = sm.wpart[pair];
+    if (tig == 0 && half == 0) {
+      wp[g8] = (g8 & 1) ? m1 : m0;
+      wp[8 + g8] = (g8 & 1) ? v1 : v0;
+    }
+    float* dst = wp + 16 + g8 * D + half * (D / 2);
+#pragma unroll
+    for (int n = 0; n < NH; ++n) {
+      *reinterpret_cast<float2*>(dst + n * 8 + 2 * tig) = make_float2(O[n][0] + O[n][2], O[n][1] + O[n][3]);
+      O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+    }
+    mr0 = mr1 = -INFINITY;
+    acc0 = acc1 = 0.f;
+    pre = false;
+    soft_lane = tig < 2;
+    load_q(row);
+  };
 
   bool dead = false;
   uint32_t par = 0u;
@@ -805,6 +906,7 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       post_known = true;
       int nU = 0;
       if (!dead && mbar_wait_bounded(&sm.sel_bar, 0, p.wait_ns)) nU = sm.nuni;
+      flush_prefix();
       nchunks = s.nW + post_count(m.n_e_chunks + nU * p.chunks_per_block, rank, p.C);
       if (c >= nchunks) break;
     }
@@ -824,7 +926,8 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       }
     }
     const int4 dsc = sm.desc[stage];
-    const bool mine = (c % kPairsPerRow) == sub && (dsc.z != kKindSel || ((dsc.w >> row) & 1));
+    const bool mine = pre ? (c % kPrePairs) == psub
+                          : (c % kPairsPerRow) == sub && (dsc.z != kKindSel || ((dsc.w >> row) & 1));
     if (!mine) {
       if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
       continue;
@@ -861,7 +964,7 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
             ex = true;
             sg = 1.f;
           } else if (kind == kKindPrefix) {
-            ex = pos < Tr;
+            ex = pos < Tpre;
             sg = 0.f;
           } else {  // E: only the chunk's own positions index the bitmap
             const int blk = valid ? (pos - p.S) / p.Bk : 0;
@@ -899,7 +1002,7 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       mr0 = soft_lane ? mn0 : mr0;
       mr1 = soft_lane ? mn1 : mr1;
       const float b0 = __shfl_sync(kFull, al0, g8 >> 1), b1 = __shfl_sync(kFull, al1, g8 >> 1);
-      const float alpha = p_lane ? ((g8 & 1) ? b1 : b0) : 1.f;
+      const float alpha = (p_lane || pre) ? ((g8 & 1) ? b1 : b0) : 1.f;
       if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
@@ -991,9 +1094,35 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       O[n][2] = O[n][3] = 0.f;
     }
   };
-  // the combine slots hold the top-k candidates until the selections are made
-  if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, p.wait_ns);
-  named_sync(kBarAttn, kAttnThreads);  // every statistics warp is past the selections (sel_bar)
+  // the prefix partials of this pair's row: slots 2 X, 2 X + 1 (X = row / 2
+  // for NR = 4, the pair's post-selection index for NR = 2), this row's
+  // columns; every (slot, row) is taken by exactly one pair
+  named_sync(kBarAttn, kAttnThreads);  // every pair's prefix partial is in its slot
+  {
+    const int X = NR == 4 ? (row >> 1) : sub;
+    const int col = (row & 1) * 4 + head;
+#pragma unroll 1
+    for (int sl = 2 * X; sl < 2 * X + 2; ++sl) {
+      const float* wp = sm.wpart[sl];
+      if (p_lane) {
+        const float mp = wp[col], lp = wp[8 + col];
+        const float M = fmaxf(m_run, mp);
+        const float fa = (m_run == -INFINITY) ? 0.f : exp2f(m_run - M);
+        const float fb = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
+        l = l * fa + lp * fb;
+        m_run = M;
+        const float* src = wp + 16 + col * D + half * (D / 2);
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+          const float2 y = *reinterpret_cast<const float2*>(src + n * 8 + 2 * tig);
+          O[n][0] = (O[n][0] + O[n][2]) * fa + y.x * fb;
+          O[n][1] = (O[n][1] + O[n][3]) * fa + y.y * fb;
+          O[n][2] = O[n][3] = 0.f;
+        }
+      }
+    }
+  }
+  named_sync(kBarAttn, kAttnThreads);  // the slots are read before they are rewritten
   if constexpr (NR == 2) {  // pairs (0, 1) -> row 0 in slot 0, (2, 3) -> row 1 in slot 1
     if (sub == 1) emit(sm.wpart[row]);
     named_sync(kBarAttn, kAttnThreads);
@@ -1168,6 +1297,18 @@ __global__ void __launch_bounds__(kFThreads, 1) multi_kernel(const __grid_consta
       for (int j = 0; j < 8; ++j) {
         sm.qs[r * kMaxGroup + i][d0 + j] = qf[j];
         sm.qsT[d0 + j][r * kMaxGroup + i] = qf[j];
+      }
+    }
+    {  // the pending evictions' keys and values, the E tokens' keys
+      const int nk = (m.ev_end[NR - 1] - g.fold_begin) * (D / 8), nv = (g.fold_end - g.fold_begin) * (D / 8);
+      for (int e = t; e < nk + nv; e += kConsumerThreads) {
+        const bool isk = e < nk;
+        const int ee = isk ? e : e - nk, tok = ee / (D / 8), d0 = (ee % (D / 8)) * 8;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>((isk ? p.k_cache : p.v_cache) +
+                                                               ((int64_t)unit * p.cap + g.fold_begin + tok) * D + d0));
+        float* dst = isk ? &sm.xk[tok][d0] : &sm.xv[tok][d0];
+        *reinterpret_cast<float4*>(dst) = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(bf16_lo(raw.z), bf16_hi(raw.z), bf16_lo(raw.w), bf16_hi(raw.w));
       }
     }
     if (rank == 0 && p.k_new != nullptr)

@@ -44,20 +44,27 @@ __global__ void __launch_bounds__(D / 4) append_kernel(const __grid_constant__ A
 // each head's window give its own range) folded into the state in one
 // pass, for several pending tokens (a chunked append, or many appends between
 // decodes; SPLA "Recurrence" applied to a run of tokens is a small dense
-// update).  One CTA per unit: H += K^T V over the run (fp32 thread tiles of the
-// D x D outer-product sum, keys / values staged through shared memory 32
-// tokens at a time), zk += sum k, zv += sum v, n += count; then, per block the
-// run touches, the block's mean and population variance merged with those of
-// its new tokens by the pairwise combination of Chan, Golub and LeVeque
-// (n = na + nb, mean = ma + d nb / n, M2 = M2a + M2b + d^2 na nb / n, with
-// d = mb - ma), in fp64.  The tokens of a block folded before fb are exactly
-// those before fb, as folds go in position order.
+// update).  Two CTAs per unit, CTA h taking key channels [h D/2, (h+1) D/2):
+// its rows of H += K^T V (fp32 thread tiles of the outer-product sum, the tile
+// held in registers from before the first token; keys and values staged
+// through shared memory 32 tokens at a time, the next 32 fetched while these
+// are multiplied), its channels of zk += sum k and zv += sum v, and its
+// channels of the statistics of every block the run touches: the new tokens'
+// mean and squared deviations as fp64 sums shifted by a value near the mean
+// (the stored mean, else the block's first new key), merged with the stored
+// mean and population variance by the pairwise combination of Chan, Golub and
+// LeVeque (n = na + nb, mean = ma + d nb / n, M2 = M2a + M2b + d^2 na nb / n,
+// with d = mb - ma).  The tokens of a block folded before fb are exactly those
+// before fb, as folds go in position order.
 template <int D>
 __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldParams p) {
-  constexpr int RT = D / 16;
-  __shared__ __align__(16) float ks[32][D];
+  constexpr int DH = D / 2;                           // this CTA's key channels (rows of H)
+  constexpr int RR = DH / 16, RC = D / 16;            // thread tile of H: RR rows x RC columns
+  constexpr int KP = DH / 8, VP = D / 8, TP = KP + VP;  // 16-byte pieces per token
+  constexpr int NP = (32 * TP + 255) / 256;           // pieces per thread per 32 tokens
+  __shared__ __align__(16) float ks[32][DH];
   __shared__ __align__(16) float vs[32][D];
-  const int unit = blockIdx.x, tid = threadIdx.x;
+  const int unit = blockIdx.x, half = blockIdx.y, tid = threadIdx.x;
   const UnitGeo g = unit_geo(&p.tb, unit, p.Hkv, p.T, p.S, p.W, p.Bk, 0, 1, p.pending);
   const int64_t fb = g.fold_begin, fe = g.fold_end;
   if (tid == 0) pdl_wait_primary();  // the caches' rows and the state may come from the previous grid
@@ -65,80 +72,132 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
   pdl_allow_dependents();
   if (fe <= fb) return;  // nothing pending in this unit (a short row)
   const int tr = tid / 16, tc = tid % 16;
+  const int c0 = half * DH;
   const int64_t ub = (int64_t)unit * p.cap;
-  float acc[RT][RT];
+  float* Hrow = p.H + ((int64_t)unit * D + c0 + tr * RR) * D + tc * RC;
+  float acc[RR][RC];
 #pragma unroll
-  for (int i = 0; i < RT; ++i)
+  for (int i = 0; i < RR; ++i)
 #pragma unroll
-    for (int j = 0; j < RT; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < RC; j += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(Hrow + (int64_t)i * D + j);
+      acc[i][j] = x.x;
+      acc[i][j + 1] = x.y;
+      acc[i][j + 2] = x.z;
+      acc[i][j + 3] = x.w;
+    }
+  // statistics (threads [0, DH): key channel c0 + tid): the first block may
+  // hold tokens folded before fb
+  const int64_t j_first = (fb - p.S) / p.Bk, na_first = fb - (p.S + j_first * p.Bk);
+  const int c = c0 + tid;
+  double ma = 0.0, va = 0.0;
+  if (tid < DH && na_first > 0) {
+    const int64_t so = ((int64_t)unit * p.max_blocks + j_first) * D + c;
+    ma = (double)p.mu[so];
+    va = (double)p.var[so];
+  }
+  int64_t cur_j = -1, na = 0;
+  double shift = 0.0, s1 = 0.0, s2 = 0.0;
+  int cnt = 0;
+  auto flush = [&]() {
+    if (cnt == 0) return;
+    const int64_t so = ((int64_t)unit * p.max_blocks + cur_j) * D + c;
+    const double nb = (double)cnt, mb = shift + s1 / nb, m2b = fmax(0.0, s2 - s1 * s1 / nb);
+    double mu = mb, m2 = m2b, nn = nb;
+    if (na > 0) {
+      const double nad = (double)na, d = mb - ma;
+      nn = nad + nb;
+      mu = ma + d * nb / nn;
+      m2 = va * nad + m2b + d * d * nad * nb / nn;
+    }
+    p.mu[so] = (float)mu;
+    p.var[so] = (float)(m2 / nn);
+  };
   float zacc = 0.f;
+  uint4 pre[NP];
+  auto fetch = [&](int64_t tt) {
+    const int n = (int)min((int64_t)32, fe - tt);
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const int e = tid + q * 256, r = e / TP, x = e % TP;
+      pre[q] = make_uint4(0u, 0u, 0u, 0u);
+      if (e < 32 * TP && r < n) {
+        const __nv_bfloat16* src = x < KP ? p.k_cache + (ub + tt + r) * D + c0 + x * 8
+                                          : p.v_cache + (ub + tt + r) * D + (x - KP) * 8;
+        pre[q] = __ldg(reinterpret_cast<const uint4*>(src));
+      }
+    }
+  };
+  fetch(fb);
   for (int64_t tt = fb; tt < fe; tt += 32) {
     const int n = (int)min((int64_t)32, fe - tt);
-    for (int e = tid; e < 32 * D; e += 256) {
-      const int r = e / D, c = e % D;
-      float kv = 0.f, vv = 0.f;
-      if (r < n) {
-        kv = __bfloat162float(p.k_cache[(ub + tt + r) * D + c]);
-        vv = __bfloat162float(p.v_cache[(ub + tt + r) * D + c]);
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {  // rows past n are zero
+      const int e = tid + q * 256, r = e / TP, x = e % TP;
+      if (e < 32 * TP) {
+        float* dst = x < KP ? &ks[r][x * 8] : &vs[r][(x - KP) * 8];
+        const uint32_t w[4] = {pre[q].x, pre[q].y, pre[q].z, pre[q].w};
+        *reinterpret_cast<float4*>(dst) = make_float4(bf16_lo(w[0]), bf16_hi(w[0]), bf16_lo(w[1]), bf16_hi(w[1]));
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(bf16_lo(w[2]), bf16_hi(w[2]), bf16_lo(w[3]), bf16_hi(w[3]));
       }
-      ks[r][c] = kv;
-      vs[r][c] = vv;
     }
     __syncthreads();
+    if (tt + 32 < fe) fetch(tt + 32);
+    const int n4 = (n + 3) & ~3;
 #pragma unroll 4
-    for (int r = 0; r < 32; ++r) {
-      float a[RT], b[RT];
+    for (int r = 0; r < n4; ++r) {
+      float a[RR], b[RC];
 #pragma unroll
-      for (int i = 0; i < RT; ++i) {
-        a[i] = ks[r][tr * RT + i];
-        b[i] = vs[r][tc * RT + i];
+      for (int i = 0; i < RR; ++i) a[i] = ks[r][tr * RR + i];
+#pragma unroll
+      for (int j = 0; j < RC; j += 4) {
+        const float4 y = *reinterpret_cast<const float4*>(&vs[r][tc * RC + j]);
+        b[j] = y.x;
+        b[j + 1] = y.y;
+        b[j + 2] = y.z;
+        b[j + 3] = y.w;
       }
 #pragma unroll
-      for (int i = 0; i < RT; ++i)
+      for (int i = 0; i < RR; ++i)
 #pragma unroll
-        for (int j = 0; j < RT; ++j) acc[i][j] += a[i] * b[j];
+        for (int j = 0; j < RC; ++j) acc[i][j] += a[i] * b[j];
     }
-    if (tid < D) {
-      for (int r = 0; r < n; ++r) zacc += ks[r][tid];
-    } else if (tid < 2 * D) {
-      for (int r = 0; r < n; ++r) zacc += vs[r][tid - D];
+    if (tid < DH) {
+      for (int r = 0; r < n; ++r) {
+        const float kf = ks[r][tid];
+        zacc += kf;
+        const int64_t t = tt + r, j = (t - p.S) / p.Bk;
+        if (j != cur_j) {  // a new block: close the previous one
+          flush();
+          cur_j = j;
+          na = j == j_first ? na_first : 0;
+          shift = na > 0 ? ma : (double)kf;
+          s1 = s2 = 0.0;
+          cnt = 0;
+        }
+        const double d = (double)kf - shift;
+        s1 += d;
+        s2 += d * d;
+        ++cnt;
+      }
+    } else if (tid < 2 * DH) {
+      for (int r = 0; r < n; ++r) zacc += vs[r][c0 + tid - DH];
     }
     __syncthreads();
   }
-  float* H = p.H + (int64_t)unit * D * D;
 #pragma unroll
-  for (int i = 0; i < RT; ++i)
+  for (int i = 0; i < RR; ++i)
 #pragma unroll
-    for (int j = 0; j < RT; ++j) H[(int64_t)(tr * RT + i) * D + tc * RT + j] += acc[i][j];
-  if (tid < D) p.zk[(int64_t)unit * D + tid] += zacc;
-  else if (tid < 2 * D) p.zv[(int64_t)unit * D + tid - D] += zacc;
-  if (tid == 0) p.n[unit] += (float)(fe - fb);
-  if (tid < D) {  // one channel per thread
-    const __nv_bfloat16* kc = p.k_cache + ub * D + tid;
-    const int64_t j0 = (fb - p.S) / p.Bk, j1 = (fe - 1 - p.S) / p.Bk;
-    for (int64_t j = j0; j <= j1; ++j) {
-      const int64_t bs = p.S + j * p.Bk;
-      const int64_t a0 = max(bs, fb), a1 = min(bs + (int64_t)p.Bk, fe);
-      const double na = (double)(a0 - bs), nb = (double)(a1 - a0);
-      double sb = 0.0, qb = 0.0;
-      for (int64_t t = a0; t < a1; ++t) sb += (double)__bfloat162float(kc[t * D]);
-      const double mb = sb / nb;
-      for (int64_t t = a0; t < a1; ++t) {
-        const double d = (double)__bfloat162float(kc[t * D]) - mb;
-        qb += d * d;
-      }
-      const int64_t so = ((int64_t)unit * p.max_blocks + j) * D + tid;
-      double mu = mb, m2 = qb, nn = nb;
-      if (na > 0.0) {
-        const double ma = (double)p.mu[so], m2a = (double)p.var[so] * na, d = mb - ma;
-        nn = na + nb;
-        mu = ma + d * nb / nn;
-        m2 = m2a + qb + d * d * na * nb / nn;
-      }
-      p.mu[so] = (float)mu;
-      p.var[so] = (float)(m2 / nn);
-    }
+    for (int j = 0; j < RC; j += 4)
+      *reinterpret_cast<float4*>(Hrow + (int64_t)i * D + j) =
+          make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
+  if (tid < DH) {
+    flush();
+    p.zk[(int64_t)unit * D + c] += zacc;
+  } else if (tid < 2 * DH) {
+    p.zv[(int64_t)unit * D + c0 + tid - DH] += zacc;
   }
+  if (tid == 0 && half == 0) p.n[unit] += (float)(fe - fb);
 }
 
 // ---------------------------------------------------------------- init
@@ -278,7 +337,7 @@ cudaError_t prepare_state(int D) {
 
 cudaError_t launch_fold(const FoldParams& p, int D, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.units);
+  cfg.gridDim = dim3(p.units, 2);  // two CTAs per unit: halves of the key channels
   cfg.blockDim = dim3(256);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
