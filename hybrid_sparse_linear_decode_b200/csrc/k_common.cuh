@@ -350,7 +350,7 @@ __device__ __forceinline__ uint32_t kth_lane_max(uint32_t v, int lane, int k) {
 // strict order by value, then lower lane, then v0 before v1.
 __device__ __forceinline__ uint32_t kth_of_lane_pairs(uint32_t v0, uint32_t v1, int lane, int k) {
   int r0 = 0, r1 = 0;  // values ordered before (lane, v0) / before (lane, v1)
-#pragma unroll
+#pragma unroll 2
   for (int l = 0; l < 32; ++l) {
     const uint32_t o0 = __shfl_sync(kFull, v0, l), o1 = __shfl_sync(kFull, v1, l);
     r0 += (o0 > v0 || (o0 == v0 && l < lane)) ? 1 : 0;
@@ -374,17 +374,21 @@ __device__ __forceinline__ uint32_t kth_of_lane_pairs(uint32_t v0, uint32_t v1, 
 // bound is the k-th largest of the lanes' two largest keys (also keys, so still
 // at most the k-th largest key, and much closer to it: ~35 candidates of 2016
 // instead of ~110, whose exact ranking costs the square of their count).
+// Above 512 blocks the selection is written as short loops (its code runs
+// once per launch and is fetched cold).
 __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_t* dst, int32_t* copy,
                                           unsigned long long* cand, int cap, bool& nan_out) {
-  constexpr int kRows = 16;  // rows of 32 blocks per pass
+  constexpr int kRows = 16;  // rows of 32 blocks held in registers up to 512 blocks
   const int lane = role_tid() & 31;
   const uint32_t lt = lanemask_lt();
   uint32_t lmax = 0u;
   bool nan = false;
   int m = 0;  // candidates so far (block order)
   if (nb <= 32 * kRows) {
-    // one pass, keys in registers, loads at fixed offsets (sc holds at least
-    // 32 kRows entries; entries past nb are read but not used)
+    // keys in registers, every load issued at once (sc holds at least 32 kRows
+    // entries; entries past nb are read but not used): this path runs beside
+    // busy attention warps, where independent instructions matter more than
+    // the code's size
     uint32_t kr[kRows];
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
@@ -407,36 +411,24 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
     }
   } else {
     uint32_t lsec = 0u;  // the lane's second largest key (0, below every key, if it has one key)
-#pragma unroll 1
-    for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const int j = r0 + lane + 32 * i;
-        const float f = j < nb ? sc[j] : 0.f;
-        nan |= f != f;
-        const uint32_t u = j < nb ? float_key(f) : 0u;
-        lsec = max(lsec, min(lmax, u));
-        lmax = max(lmax, u);
-      }
+#pragma unroll 4
+    for (int j = lane; j < nb; j += 32) {
+      const float f = sc[j];
+      nan |= f != f;
+      const uint32_t u = float_key(f);
+      lsec = max(lsec, min(lmax, u));
+      lmax = max(lmax, u);
     }
     nan_out = __any_sync(kFull, nan);
     const uint32_t tau = kth_of_lane_pairs(lmax, lsec, lane, k);
 #pragma unroll 1
-    for (int r0 = 0; r0 < nb; r0 += 32 * kRows) {
-      uint32_t kr[kRows], bal[kRows];
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const int j = r0 + lane + 32 * i;
-        kr[i] = j < nb ? float_key(sc[j]) : 0u;
-        bal[i] = __ballot_sync(kFull, j < nb && kr[i] >= tau);
-      }
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const int pos = m + __popc(bal[i] & lt);
-        if (((bal[i] >> lane) & 1u) && pos < cap)
-          cand[pos] = ((unsigned long long)kr[i] << 32) | (uint32_t)~(r0 + lane + 32 * i);
-        m += __popc(bal[i]);
-      }
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t u = j < nb ? float_key(sc[j]) : 0u;
+      const uint32_t bal = __ballot_sync(kFull, j < nb && u >= tau);
+      const int pos = m + __popc(bal & lt);
+      if (((bal >> lane) & 1u) && pos < cap) cand[pos] = ((unsigned long long)u << 32) | (uint32_t)~j;
+      m += __popc(bal);
     }
   }
   if (m > cap) return false;
@@ -449,14 +441,12 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
     unsigned long long me = 0ull;
     if (c < m) {
       me = cand[c];
-      int rank = 0, o = 0;  // candidates above this one (all packed values differ)
-#pragma unroll 2
-      for (; o + 4 <= m; o += 4) {
+      int rank = 0;  // candidates above this one (all packed values differ)
+#pragma unroll 1
+      for (int o = 0; o < m; o += 2) {
         const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(&cand[o]);
-        const ulonglong2 y = *reinterpret_cast<const ulonglong2*>(&cand[o + 2]);
-        rank += (x.x > me ? 1 : 0) + (x.y > me ? 1 : 0) + (y.x > me ? 1 : 0) + (y.y > me ? 1 : 0);
+        rank += (x.x > me ? 1 : 0) + (o + 1 < m && x.y > me ? 1 : 0);
       }
-      for (; o < m; ++o) rank += cand[o] > me ? 1 : 0;
       sel = rank < k;
     }
     const uint32_t b = __ballot_sync(kFull, sel);

@@ -1191,22 +1191,19 @@ __device__ void merge_local(const FusedParams& p, FusedSmem<D>& sm, int unit, in
     const int i = e / D;
     const float* h = sm.mrecv + i;
     float M = -INFINITY;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r)
-      if (r < C) M = fmaxf(M, h[r * stride]);
+#pragma unroll 2
+    for (int r = 0; r < C; ++r) M = fmaxf(M, h[r * stride]);
     if (M == -INFINITY) M = 0.f;
     float nex = 0.f, nsub = 0.f, Dex = 0.f, Dsub = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      if (r < C) {
-        const float m = h[r * stride];
-        const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
-        const float2 v = *reinterpret_cast<const float2*>(&sm.mrecv[r * stride + 16 + 2 * (e - e0)]);
-        nex += v.x * f;
-        nsub += v.y;
-        Dex += h[r * stride + 4] * f;
-        Dsub += h[r * stride + 8];
-      }
+#pragma unroll 2
+    for (int r = 0; r < C; ++r) {
+      const float m = h[r * stride];
+      const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      const float2 v = *reinterpret_cast<const float2*>(&sm.mrecv[r * stride + 16 + 2 * (e - e0)]);
+      nex += v.x * f;
+      nsub += v.y;
+      Dex += h[r * stride + 4] * f;
+      Dsub += h[r * stride + 8];
     }
     float num, den;
     if (M >= 0.f) {
