@@ -824,7 +824,8 @@ __device__ void mproducer_role(const KVMaps* tm, const FusedParams& p, const Uni
 // Prefix chunks: pair q handles rows (a, a + 1), a = 2 (q / 2) for NR = 4 (0
 // for NR = 2), chunks c with c % (8 / NR) == q % (8 / NR); N column n is row
 // a + n / 4, head n % 4.  Post-selection chunks: pair q handles row q * NR / 4,
-// chunks c with c % (4 / NR) == q % (4 / NR); columns 0-3 exact, 4-7 Taylor.
+// and of the chunks that row takes, those whose count (in ring order) is
+// q % (4 / NR) modulo 4 / NR; columns 0-3 exact, 4-7 Taylor.
 // Token t of a chunk, for row r (T_r = T + r):
 //   prefix:   exact when t < T_r;
 //   E:        exact when t >= win_start[r] or its block is in row r's
@@ -900,6 +901,7 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
   uint32_t par = 0u;
   int nchunks = s.nW, post_base = s.nS + s.nW + s.nH;
   bool post_known = false;
+  int rcount = 0;  // post-selection chunks of this pair's row so far (every pair sees every chunk)
 #pragma unroll 1
   for (int c = 0; c < nchunks || !post_known; ++c) {
     if (c == s.nW && !post_known) {  // the selections decide the post-selection chunks
@@ -926,8 +928,14 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       }
     }
     const int4 dsc = sm.desc[stage];
-    const bool mine = pre ? (c % kPrePairs) == psub
-                          : (c % kPairsPerRow) == sub && (dsc.z != kKindSel || ((dsc.w >> row) & 1));
+    bool mine;
+    if (pre) {
+      mine = (c % kPrePairs) == psub;
+    } else {  // the row's chunks go to its pairs in turn
+      const bool has = dsc.z != kKindSel || ((dsc.w >> row) & 1);
+      mine = has && (rcount % kPairsPerRow) == sub;
+      rcount += has ? 1 : 0;
+    }
     if (!mine) {
       if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
       continue;
