@@ -441,12 +441,14 @@ __device__ __forceinline__ bool topk_warp(const float* sc, int nb, int k, int32_
     unsigned long long me = 0ull;
     if (c < m) {
       me = cand[c];
-      int rank = 0;  // candidates above this one (all packed values differ)
-#pragma unroll 1
-      for (int o = 0; o < m; o += 2) {
+      int rank = 0, o = 0;  // candidates above this one (all packed values differ)
+#pragma unroll 2
+      for (; o + 4 <= m; o += 4) {
         const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(&cand[o]);
-        rank += (x.x > me ? 1 : 0) + (o + 1 < m && x.y > me ? 1 : 0);
+        const ulonglong2 y = *reinterpret_cast<const ulonglong2*>(&cand[o + 2]);
+        rank += (x.x > me ? 1 : 0) + (x.y > me ? 1 : 0) + (y.x > me ? 1 : 0) + (y.y > me ? 1 : 0);
       }
+      for (; o < m; ++o) rank += cand[o] > me ? 1 : 0;
       sel = rank < k;
     }
     const uint32_t b = __ballot_sync(kFull, sel);

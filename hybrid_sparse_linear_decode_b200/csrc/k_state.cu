@@ -22,18 +22,24 @@ namespace hyb {
 namespace {
 
 // ---------------------------------------------------------------- append
-// Writes n tokens per unit at rows [T, T + n) of the caches: grid (units, n),
-// D/4 threads of 16 bytes.  A token's later eviction from the window is folded
-// into the state by the decode after it, which reads the caches.
+// Writes n tokens per unit at rows [T, T + n) of the caches: grid (units,
+// n / kAppendTokens<D>), 256 threads, one 16-byte piece of a key or value row
+// each.  A token's later eviction from the window is folded into the state by
+// the decode after it, which reads the caches.
 template <int D>
-__global__ void __launch_bounds__(D / 4) append_kernel(const __grid_constant__ AppendParams p) {
-  const int unit = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;  // token j of the chunk
+constexpr int kAppendTokens = 256 / (D / 4);  // tokens per CTA (D / 4 pieces per token)
+template <int D>
+__global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {
+  const int unit = blockIdx.x, tid = threadIdx.x;
+  const int j = blockIdx.y * kAppendTokens<D> + tid / (D / 4);  // token j of the chunk
   const int32_t Tb = p.T - (p.tb.ragged ? p.tb.row_lag[unit / p.Hkv] : 0);  // this row's length
   if (tid == 0) pdl_wait_primary();  // the previous decode may still read these caches' rows
   __syncthreads();
   pdl_allow_dependents();
-  const bool is_v = tid >= D / 8;
-  const int e = (tid % (D / 8)) * 8;
+  if (j >= p.n) return;
+  const int piece = tid % (D / 4);
+  const bool is_v = piece >= D / 8;
+  const int e = (piece % (D / 8)) * 8;
   const __nv_bfloat16* src = (is_v ? p.v_new : p.k_new) + ((int64_t)unit * p.n + j) * D + e;
   __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) + ((int64_t)unit * p.cap + Tb + j) * D + e;
   *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
@@ -50,11 +56,11 @@ __global__ void __launch_bounds__(D / 4) append_kernel(const __grid_constant__ A
 // through shared memory 32 tokens at a time, the next 32 fetched while these
 // are multiplied), its channels of zk += sum k and zv += sum v, and its
 // channels of the statistics of every block the run touches: the new tokens'
-// mean and squared deviations as fp64 sums shifted by a value near the mean
-// (the stored mean, else the block's first new key), merged with the stored
-// mean and population variance by the pairwise combination of Chan, Golub and
-// LeVeque (n = na + nb, mean = ma + d nb / n, M2 = M2a + M2b + d^2 na nb / n,
-// with d = mb - ma).  The tokens of a block folded before fb are exactly those
+// mean and squared deviations as fp32 sums shifted by a value near the mean
+// (the stored mean, else the block's first new key, so that the squares do not
+// cancel), merged with the stored mean and population variance in fp64 by the
+// pairwise combination of Chan, Golub and LeVeque (n = na + nb, mean = ma +
+// d nb / n, M2 = M2a + M2b + d^2 na nb / n, with d = mb - ma).  The tokens of a block folded before fb are exactly those
 // before fb, as folds go in position order.
 template <int D>
 __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldParams p) {
@@ -96,13 +102,14 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
     ma = (double)p.mu[so];
     va = (double)p.var[so];
   }
-  int64_t cur_j = -1, na = 0;
-  double shift = 0.0, s1 = 0.0, s2 = 0.0;
+  int64_t cur_j = -1, na = 0, next_bs = 0;  // the current block and the start of the next
+  float shift = 0.f, s1 = 0.f, s2 = 0.f;
   int cnt = 0;
   auto flush = [&]() {
     if (cnt == 0) return;
     const int64_t so = ((int64_t)unit * p.max_blocks + cur_j) * D + c;
-    const double nb = (double)cnt, mb = shift + s1 / nb, m2b = fmax(0.0, s2 - s1 * s1 / nb);
+    const double nb = (double)cnt, mb = (double)shift + (double)s1 / nb,
+                 m2b = fmax(0.0, (double)s2 - (double)s1 * (double)s1 / nb);
     double mu = mb, m2 = m2b, nn = nb;
     if (na > 0) {
       const double nad = (double)na, d = mb - ma;
@@ -147,8 +154,16 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
 #pragma unroll 4
     for (int r = 0; r < n4; ++r) {
       float a[RR], b[RC];
+      if constexpr (RR == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(&ks[r][tr * RR]);
+        a[0] = x.x;
+        a[1] = x.y;
+        a[2] = x.z;
+        a[3] = x.w;
+      } else {
 #pragma unroll
-      for (int i = 0; i < RR; ++i) a[i] = ks[r][tr * RR + i];
+        for (int i = 0; i < RR; ++i) a[i] = ks[r][tr * RR + i];
+      }
 #pragma unroll
       for (int j = 0; j < RC; j += 4) {
         const float4 y = *reinterpret_cast<const float4*>(&vs[r][tc * RC + j]);
@@ -166,18 +181,20 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
       for (int r = 0; r < n; ++r) {
         const float kf = ks[r][tid];
         zacc += kf;
-        const int64_t t = tt + r, j = (t - p.S) / p.Bk;
-        if (j != cur_j) {  // a new block: close the previous one
+        const int64_t t = tt + r;
+        if (cur_j < 0 || t >= next_bs) {  // a new block: close the previous one
           flush();
+          const int64_t j = (t - p.S) / p.Bk;
+          next_bs = p.S + (j + 1) * p.Bk;
           cur_j = j;
           na = j == j_first ? na_first : 0;
-          shift = na > 0 ? ma : (double)kf;
-          s1 = s2 = 0.0;
+          shift = na > 0 ? (float)ma : kf;
+          s1 = s2 = 0.f;
           cnt = 0;
         }
-        const double d = (double)kf - shift;
+        const float d = kf - shift;
         s1 += d;
-        s2 += d * d;
+        s2 = fmaf(d, d, s2);
         ++cnt;
       }
     } else if (tid < 2 * DH) {
@@ -351,8 +368,9 @@ cudaError_t launch_fold(const FoldParams& p, int D, cudaStream_t s) {
 
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.units, p.n);
-  cfg.blockDim = dim3(D / 4);
+  const int tpc = D == 128 ? kAppendTokens<128> : kAppendTokens<64>;
+  cfg.gridDim = dim3(p.units, (p.n + tpc - 1) / tpc);
+  cfg.blockDim = dim3(256);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
