@@ -91,6 +91,7 @@ struct FusedSmem {
   uint32_t tks[2][4];                                // top-k: per-warp partials / scan scratch
   uint32_t tkw[2];                                   // one-warp top-k: done, NaN seen
   int4 desc[kFStages];                               // chunk items: start, len, is_sel
+  float2 xmax[4][2][4];                              // per pair and warp: a chunk's column maxima, then the weight sums
   // A stage's items belong to one of two consumer groups.  Each group has its
   // own "full" barrier per stage and waits only for its own items, in order,
   // so it is never more than one phase ahead of a barrier it waits on (a
@@ -667,124 +668,169 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
     }
     const int4 dsc = sm.desc[stage];
     const int nvalid = have ? dsc.y : 0;
-    if (nvalid > 0) {
-      const uint32_t kb = smem_u32(sm.ring[stage]);
-      const uint32_t vb = kb + FusedSmem<D>::kHalf;
-      // ---- S^T = K Q^T: m-tile mt holds tokens 16mt .. 16mt+15, columns = heads
-      float sacc[4][4];
+    const uint32_t kb = smem_u32(sm.ring[stage]);
+    const uint32_t vb = kb + FusedSmem<D>::kHalf;
+    // ---- S^T = K Q^T for this warp's 32 tokens: m-tiles 2 half, 2 half + 1
+    // (tokens 32 half .. 32 half + 31), columns = heads.  Both warps of the
+    // pair take the same barriers whatever their waits gave (nvalid 0: nothing
+    // is computed), so a timed-out wait leaves no warp at a barrier alone.
+    float sacc[2][4];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
+    for (int mm = 0; mm < 2; ++mm) sacc[mm][0] = sacc[mm][1] = sacc[mm][2] = sacc[mm][3] = 0.f;
+    if (nvalid > 32 * half) {
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
+        for (int mm = 0; mm < 2; ++mm) {
+          const int mt = 2 * half + mm;
           uint32_t a0, a1, a2, a3;
           ldsm_x4(kb + swz<D>(mt * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)), a0, a1, a2, a3);
-          mma_16816(sacc[mt], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+          mma_16816(sacc[mm], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
         }
       }
-      // lane (g, tig): tokens 16mt + g + 8j, columns 2tig, 2tig+1, i.e. heads
-      // (2tig, 2tig+1) & 3: softmax weights in lanes tig < 2, Taylor weights
-      // 1 + s on selected tokens in lanes tig >= 2.
-      const bool sel_tok = dsc.z != 0;
-      float w[4][4];
-      float t0m = -INFINITY, t1m = -INFINITY;
+    }
+    // lane (g, tig): tokens 16mt + g + 8j, columns 2tig, 2tig+1, i.e. heads
+    // (2tig, 2tig+1) & 3: softmax weights in lanes tig < 2, Taylor weights
+    // 1 + s on selected tokens in lanes tig >= 2.
+    const bool sel_tok = dsc.z != 0;
+    float w[2][4];
+    float t0m = -INFINITY, t1m = -INFINITY;
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+    for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int t = mt * 16 + g + 8 * (q >> 1);
-          // both kinds of lanes take the same instructions (selects, no
-          // divergent branch: half the warp takes each kind)
-          const float sv = t < nvalid ? sacc[mt][q] * p.scale : 0.f;
-          const float xs = t < nvalid ? sv * kLog2e : -INFINITY;
-          const float wt = (t < nvalid && sel_tok) ? 1.f + sv : 0.f;
-          w[mt][q] = soft_lane ? xs : wt;
-          const float xm = soft_lane ? xs : -INFINITY;
-          if (q & 1) t1m = fmaxf(t1m, xm); else t0m = fmaxf(t0m, xm);
-        }
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        t0m = fmaxf(t0m, __shfl_xor_sync(kFull, t0m, o));
-        t1m = fmaxf(t1m, __shfl_xor_sync(kFull, t1m, o));
+      for (int q = 0; q < 4; ++q) {
+        const int t = (2 * half + mm) * 16 + g + 8 * (q >> 1);
+        // both kinds of lanes take the same instructions (selects, no
+        // divergent branch: half the warp takes each kind)
+        const float sv = t < nvalid ? sacc[mm][q] * p.scale : 0.f;
+        const float xs = t < nvalid ? sv * kLog2e : -INFINITY;
+        const float wt = (t < nvalid && sel_tok) ? 1.f + sv : 0.f;
+        w[mm][q] = soft_lane ? xs : wt;
+        const float xm = soft_lane ? xs : -INFINITY;
+        if (q & 1) t1m = fmaxf(t1m, xm); else t0m = fmaxf(t0m, xm);
       }
-      const float mn0 = fmaxf(mr0, t0m), mn1 = fmaxf(mr1, t1m);
-      const float al0 = (soft_lane && mn0 != -INFINITY) ? exp2f(mr0 - mn0) : 1.f;
-      const float al1 = (soft_lane && mn1 != -INFINITY) ? exp2f(mr1 - mn1) : 1.f;
-      float ws0 = 0.f, ws1 = 0.f;
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+    for (int o = 4; o < 32; o <<= 1) {
+      t0m = fmaxf(t0m, __shfl_xor_sync(kFull, t0m, o));
+      t1m = fmaxf(t1m, __shfl_xor_sync(kFull, t1m, o));
+    }
+    // the chunk's column maxima over both warps' tokens
+    if (g == 0) sm.xmax[pair][half][tig] = make_float2(t0m, t1m);
+    named_sync(kBarPair0 + pair, 64);
+    {
+      const float2 o = sm.xmax[pair][half ^ 1][tig];
+      t0m = fmaxf(t0m, o.x);
+      t1m = fmaxf(t1m, o.y);
+    }
+    const float mn0 = fmaxf(mr0, t0m), mn1 = fmaxf(mr1, t1m);
+    const float al0 = (soft_lane && mn0 != -INFINITY) ? exp2f(mr0 - mn0) : 1.f;
+    const float al1 = (soft_lane && mn1 != -INFINITY) ? exp2f(mr1 - mn1) : 1.f;
+    float ws0 = 0.f, ws1 = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float ev = exp2f(w[mt][q] - ((q & 1) ? mn1 : mn0));  // used in the softmax lanes only
-          w[mt][q] = soft_lane ? (w[mt][q] == -INFINITY ? 0.f : ev) : w[mt][q];
-          if (q & 1) ws1 += w[mt][q]; else ws0 += w[mt][q];
-        }
-      acc0 = acc0 * al0 + ws0;  // al = 1 in the Taylor lanes
-      acc1 = acc1 * al1 + ws1;
-      mr0 = soft_lane ? mn0 : mr0;
-      mr1 = soft_lane ? mn1 : mr1;
-      // rescale the softmax rows (g < 4) of O by their head's factor
-      const float b0 = __shfl_sync(kFull, al0, g >> 1), b1 = __shfl_sync(kFull, al1, g >> 1);
-      const float alpha = p_lane ? ((g & 1) ? b1 : b0) : 1.f;
-      if (__any_sync(kFull, alpha != 1.f)) {
+    for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-        for (int n = 0; n < NH; ++n) {
-          O[n][0] *= alpha;
-          O[n][1] *= alpha;
-          O[n][2] *= alpha;
-          O[n][3] *= alpha;
-        }
+      for (int q = 0; q < 4; ++q) {
+        const float ev = exp2f(w[mm][q] - ((q & 1) ? mn1 : mn0));  // used in the softmax lanes only
+        w[mm][q] = soft_lane ? (w[mm][q] == -INFINITY ? 0.f : ev) : w[mm][q];
+        if (q & 1) ws1 += w[mm][q]; else ws0 += w[mm][q];
       }
-      // ---- O += A V: A rows = weight columns (transposed 8x8 blocks), hi then lo.
-      // In a ragged chunk the rows past it have zero weights: k-steps wholly
-      // past it are skipped (rows past its 16-row boxes hold stale stage data),
-      // and in its last k-step the V fragments of rows past it, which may be
-      // unwritten cache rows, are zeroed in registers so that no 0 * NaN arises.
+    acc0 = acc0 * al0 + ws0;  // this warp's tokens only: the pair's two sums are added at the end
+    acc1 = acc1 * al1 + ws1;
+    mr0 = soft_lane ? mn0 : mr0;
+    mr1 = soft_lane ? mn1 : mr1;
+    // rescale the softmax rows (g < 4) of O by their head's factor
+    const float b0 = __shfl_sync(kFull, al0, g >> 1), b1 = __shfl_sync(kFull, al1, g >> 1);
+    const float alpha = p_lane ? ((g & 1) ? b1 : b0) : 1.f;
+    if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
-      for (int kt = 0; kt < 4; ++kt) {
-        if (kt * 16 >= nvalid) break;
-        const bool tail = kt * 16 + 16 > nvalid;  // warp-uniform
-        const int tk = kt * 16 + 2 * tig;          // rows of the low halves of b0v / b2v (b1v / b3v: + 8)
-        const uint32_t m0 = (tk < nvalid ? 0x0000ffffu : 0u) | (tk + 1 < nvalid ? 0xffff0000u : 0u);
-        const uint32_t m1 = (tk + 8 < nvalid ? 0x0000ffffu : 0u) | (tk + 9 < nvalid ? 0xffff0000u : 0u);
-        uint32_t h0, l0, h1, l1;
-        split_bf16(w[kt][0], w[kt][1], h0, l0);
-        split_bf16(w[kt][2], w[kt][3], h1, l1);
-        const uint32_t a0 = movmatrix_t(h0), a1 = movmatrix_t(l0), a2 = movmatrix_t(h1), a3 = movmatrix_t(l1);
+      for (int n = 0; n < NH; ++n) {
+        O[n][0] *= alpha;
+        O[n][1] *= alpha;
+        O[n][2] *= alpha;
+        O[n][3] *= alpha;
+      }
+    }
+    // A fragments of this warp's two k-tiles (weight columns as rows, transposed
+    // 8x8 blocks, hi then lo), handed to the other warp through the first rows
+    // of this warp's own K tokens, which nothing reads any more
+    uint32_t mf[2][4], of[2][4];  // this warp's k-tiles 2 half + mm, the other warp's
 #pragma unroll
-        for (int np = 0; np < NH / 2; ++np) {
-          uint32_t b0v, b1v, b2v, b3v;
-          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, (half * NH / 2 + np) * 2 + (mi >> 1)), b0v, b1v, b2v,
-                    b3v);
-          if (tail) {
-            b0v &= m0;
-            b1v &= m1;
-            b2v &= m0;
-            b3v &= m1;
-          }
-          mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
-          mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
+    for (int mm = 0; mm < 2; ++mm) {
+      uint32_t h0, l0, h1, l1;
+      split_bf16(w[mm][0], w[mm][1], h0, l0);
+      split_bf16(w[mm][2], w[mm][3], h1, l1);
+      mf[mm][0] = movmatrix_t(h0);
+      mf[mm][1] = movmatrix_t(l0);
+      mf[mm][2] = movmatrix_t(h1);
+      mf[mm][3] = movmatrix_t(l1);
+    }
+    {
+      constexpr uint32_t kRows32 = 32u * D * 2u;  // bytes of 32 K rows
+      const uint32_t mine_x = kb + (uint32_t)half * kRows32, theirs_x = kb + (uint32_t)(half ^ 1) * kRows32;
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm)
+        sts_u4(mine_x + (uint32_t)(mm * 512 + lane * 16), mf[mm][0], mf[mm][1], mf[mm][2], mf[mm][3]);
+      named_sync(kBarPair0 + pair, 64);
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm)
+        lds_u4(theirs_x + (uint32_t)(mm * 512 + lane * 16), of[mm][0], of[mm][1], of[mm][2], of[mm][3]);
+      // the stage's next copy (async proxy) comes after these generic writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    // ---- O += A V over the chunk's 64 tokens.  In a ragged chunk the rows
+    // past it have zero weights: k-steps wholly past it are skipped (rows past
+    // its 16-row boxes hold stale stage data), and in its last k-step the V
+    // fragments of rows past it, which may be unwritten cache rows, are zeroed
+    // in registers so that no 0 * NaN arises.
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) {
+      if (kt * 16 >= nvalid) break;
+      const bool tail = kt * 16 + 16 > nvalid;  // warp-uniform
+      const int tk = kt * 16 + 2 * tig;          // rows of the low halves of b0v / b2v (b1v / b3v: + 8)
+      const uint32_t m0 = (tk < nvalid ? 0x0000ffffu : 0u) | (tk + 1 < nvalid ? 0xffff0000u : 0u);
+      const uint32_t m1 = (tk + 8 < nvalid ? 0x0000ffffu : 0u) | (tk + 9 < nvalid ? 0xffff0000u : 0u);
+      const bool own = (kt >> 1) == half;
+      const uint32_t a0 = own ? mf[kt & 1][0] : of[kt & 1][0], a1 = own ? mf[kt & 1][1] : of[kt & 1][1];
+      const uint32_t a2 = own ? mf[kt & 1][2] : of[kt & 1][2], a3 = own ? mf[kt & 1][3] : of[kt & 1][3];
+#pragma unroll
+      for (int np = 0; np < NH / 2; ++np) {
+        uint32_t b0v, b1v, b2v, b3v;
+        ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, (half * NH / 2 + np) * 2 + (mi >> 1)), b0v, b1v, b2v, b3v);
+        if (tail) {
+          b0v &= m0;
+          b1v &= m1;
+          b2v &= m0;
+          b3v &= m1;
         }
+        mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
+        mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
       }
     }
     __syncwarp();
     if (lane == 0 && have) mbar_arrive_cnt(&sm.empty[stage], kEmptyPerAttnWarp);
   }
 
+  // each warp of a pair summed the weights of its own tokens: add the other's
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    acc0 += __shfl_xor_sync(kFull, acc0, o);
+    acc1 += __shfl_xor_sync(kFull, acc1, o);
+  }
+  if (g == 0) sm.xmax[pair][half][tig] = make_float2(acc0, acc1);
+  named_sync(kBarPair0 + pair, 64);
+  {
+    const float2 o = sm.xmax[pair][half ^ 1][tig];
+    acc0 += o.x;
+    acc1 += o.y;
+  }
   // the combine slots hold the top-k candidates until the selection is made
   // (a rank without selected chunks gets here first)
   if (!dead) mbar_wait_bounded(&sm.sel_bar, 0, p.wait_ns);
   // ---- combine the 4 pairs' partials (a tree through two shared slots: pairs
   //      2, 3 -> 0, 1, then pair 1 -> 0); pair 0 leaves the record in wpart[0].
   //      The two warps of a pair hold the same statistics and disjoint columns.
-  // per-head totals over the tokens (the lanes of one tig), then each lane takes
-  // the statistics of its O rows' head (rows g < 4 softmax, g >= 4 Taylor)
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    acc0 += __shfl_xor_sync(kFull, acc0, o);
-    acc1 += __shfl_xor_sync(kFull, acc1, o);
-  }
+  // each lane takes the statistics of its O rows' head (rows g < 4 softmax,
+  // g >= 4 Taylor); the per-head totals are in every lane of a tig
   float m_run, l, ds;
   {
     const int src = p_lane ? (head >> 1) : 2 + (head >> 1);
