@@ -638,8 +638,10 @@ __device__ void attn_role(const FusedParams& p, FusedSmem<D>& sm, const Seq& s, 
   float mr0 = -INFINITY, mr1 = -INFINITY, acc0 = 0.f, acc1 = 0.f;
 
   // Chunk items go to the attention warp pairs in turn (chunk c to pair c % 4):
-  // both warps of the pair compute the chunk's scores and weights, each the
-  // PV product for half of the head dimension.  Every attention warp waits for
+  // each warp of the pair scores and weighs its own 32 of the chunk's tokens,
+  // and each computes the PV product of all 64 tokens for half of the head
+  // dimension (the weights cross between the two warps through shared
+  // memory).  Every attention warp waits for
   // every chunk item in ring order and arrives on its stage's empty barrier
   // (the owner after its work), so that no warp falls two phases behind a
   // stage; a timed-out wait only stops this warp's work.

@@ -61,8 +61,11 @@ __host__ __device__ constexpr int mmerge_stride(int NR, int GD, int C) {
   return 16 * NR + ((2 * ((NR * GD + C - 1) / C) + 3) & ~3);
 }
 __host__ __device__ constexpr int mmerge_floats_for(int NR, int D, int C) { return C * mmerge_stride(NR, kMaxGroup * D, C); }
+// at most 8 CTAs per unit (the merge slots of larger clusters would take the
+// shared memory of the attention pairs' exchange buffers)
+constexpr int kMultiMaxCluster = 8;
 __host__ __device__ constexpr int mmerge_floats(int NR, int D, int C = 1) {
-  return C > kMaxCluster ? 0
+  return C > kMultiMaxCluster ? 0
                          : (mmerge_floats_for(NR, D, C) > mmerge_floats(NR, D, C + 1) ? mmerge_floats_for(NR, D, C)
                                                                                        : mmerge_floats(NR, D, C + 1));
 }
@@ -105,6 +108,9 @@ struct MultiSmem {
   uint32_t tks[2][4];
   uint32_t tkw[2 * NR];
   int4 desc[kMStages];                               // chunk items: start, len, kind, row mask
+  float2 xmax[4][2][4];                              // per pair and warp: a chunk's column maxima
+  float2 xacc[2][4][2][4];                           // per pair and warp: the weight sums at the prefix's end, at the end
+  uint4 xfrag[8][2][32];                             // per attention warp: its two k-tiles' PV weight fragments
   uint64_t full_attn[kMStages];
   uint64_t full_aux[kMStages];
   uint64_t empty[kMStages];
@@ -877,6 +883,14 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       acc0 += __shfl_xor_sync(kFull, acc0, o);
       acc1 += __shfl_xor_sync(kFull, acc1, o);
     }
+    // each warp of the pair summed its own tokens: add the other's
+    if (g8 == 0) sm.xacc[0][pair][half][tig] = make_float2(acc0, acc1);
+    named_sync(kBarPair0 + pair, 64);
+    {
+      const float2 o = sm.xacc[0][pair][half ^ 1][tig];
+      acc0 += o.x;
+      acc1 += o.y;
+    }
     const float v0 = __shfl_sync(kFull, acc0, g8 >> 1), v1 = __shfl_sync(kFull, acc1, g8 >> 1);
     const float m0 = __shfl_sync(kFull, mr0, g8 >> 1), m1 = __shfl_sync(kFull, mr1, g8 >> 1);
     float* wp = sm.wpart[pair];
@@ -941,110 +955,142 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
       continue;
     }
     const int nvalid = have ? dsc.y : 0;
-    if (nvalid > 0) {
-      const uint32_t kb = smem_u32(sm.ring[stage]);
-      const uint32_t vb = kb + MultiSmem<D, NR>::kHalf;
-      float sacc[4][4];
+    const uint32_t kb = smem_u32(sm.ring[stage]);
+    const uint32_t vb = kb + MultiSmem<D, NR>::kHalf;
+    // S^T = K Q^T for this warp's 32 tokens (m-tiles 2 half, 2 half + 1); both
+    // warps of the pair take the same barriers whatever their waits gave
+    float sacc[2][4];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
+    for (int mm = 0; mm < 2; ++mm) sacc[mm][0] = sacc[mm][1] = sacc[mm][2] = sacc[mm][3] = 0.f;
+    if (nvalid > 32 * half) {
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
+        for (int mm = 0; mm < 2; ++mm) {
+          const int mt = 2 * half + mm;
           uint32_t a0, a1, a2, a3;
           ldsm_x4(kb + swz<D>(mt * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)), a0, a1, a2, a3);
-          mma_16816(sacc[mt], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+          mma_16816(sacc[mm], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
         }
       }
-      const int kind = dsc.z, start = dsc.x;
-      float w[4][4];
-      float t0m = -INFINITY, t1m = -INFINITY;
+    }
+    const int kind = dsc.z, start = dsc.x;
+    float w[2][4];
+    float t0m = -INFINITY, t1m = -INFINITY;
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+    for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int t = mt * 16 + g8 + 8 * (q >> 1);
-          const int pos = start + t;
-          const bool valid = t < nvalid;
-          bool ex;
-          float sg;
-          if (kind == kKindSel) {
-            ex = true;
-            sg = 1.f;
-          } else if (kind == kKindPrefix) {
-            ex = pos < Tpre;
-            sg = 0.f;
-          } else {  // E: only the chunk's own positions index the bitmap
-            const int blk = valid ? (pos - p.S) / p.Bk : 0;
-            const bool in_win = pos >= ws;
-            const bool chosen = valid && ((sm.selbm[row][blk >> 5] >> (blk & 31)) & 1u);
-            ex = pos < Tr && (in_win || chosen);
-            sg = (pos < Tr && !in_win && !chosen) ? -1.f : 0.f;
-          }
-          const float sv = valid ? sacc[mt][q] * p.scale : 0.f;
-          const float xs = (valid && ex) ? sv * kLog2e : -INFINITY;
-          const float wt = valid ? sg * (1.f + sv) : 0.f;
-          w[mt][q] = soft_lane ? xs : wt;
-          const float xm = soft_lane ? xs : -INFINITY;
-          if (q & 1) t1m = fmaxf(t1m, xm); else t0m = fmaxf(t0m, xm);
+      for (int q = 0; q < 4; ++q) {
+        const int t = (2 * half + mm) * 16 + g8 + 8 * (q >> 1);
+        const int pos = start + t;
+        const bool valid = t < nvalid;
+        bool ex;
+        float sg;
+        if (kind == kKindSel) {
+          ex = true;
+          sg = 1.f;
+        } else if (kind == kKindPrefix) {
+          ex = pos < Tpre;
+          sg = 0.f;
+        } else {  // E: only the chunk's own positions index the bitmap
+          const int blk = valid ? (pos - p.S) / p.Bk : 0;
+          const bool in_win = pos >= ws;
+          const bool chosen = valid && ((sm.selbm[row][blk >> 5] >> (blk & 31)) & 1u);
+          ex = pos < Tr && (in_win || chosen);
+          sg = (pos < Tr && !in_win && !chosen) ? -1.f : 0.f;
         }
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        t0m = fmaxf(t0m, __shfl_xor_sync(kFull, t0m, o));
-        t1m = fmaxf(t1m, __shfl_xor_sync(kFull, t1m, o));
-      }
-      const float mn0 = fmaxf(mr0, t0m), mn1 = fmaxf(mr1, t1m);
-      const float al0 = (soft_lane && mn0 != -INFINITY) ? exp2f(mr0 - mn0) : 1.f;
-      const float al1 = (soft_lane && mn1 != -INFINITY) ? exp2f(mr1 - mn1) : 1.f;
-      float ws0 = 0.f, ws1 = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float ev = exp2f(w[mt][q] - ((q & 1) ? mn1 : mn0));
-          w[mt][q] = soft_lane ? (w[mt][q] == -INFINITY ? 0.f : ev) : w[mt][q];
-          if (q & 1) ws1 += w[mt][q]; else ws0 += w[mt][q];
-        }
-      acc0 = acc0 * al0 + ws0;
-      acc1 = acc1 * al1 + ws1;
-      mr0 = soft_lane ? mn0 : mr0;
-      mr1 = soft_lane ? mn1 : mr1;
-      const float b0 = __shfl_sync(kFull, al0, g8 >> 1), b1 = __shfl_sync(kFull, al1, g8 >> 1);
-      const float alpha = (p_lane || pre) ? ((g8 & 1) ? b1 : b0) : 1.f;
-      if (__any_sync(kFull, alpha != 1.f)) {
-#pragma unroll
-        for (int n = 0; n < NH; ++n) {
-          O[n][0] *= alpha;
-          O[n][1] *= alpha;
-          O[n][2] *= alpha;
-          O[n][3] *= alpha;
-        }
+        const float sv = valid ? sacc[mm][q] * p.scale : 0.f;
+        const float xs = (valid && ex) ? sv * kLog2e : -INFINITY;
+        const float wt = valid ? sg * (1.f + sv) : 0.f;
+        w[mm][q] = soft_lane ? xs : wt;
+        const float xm = soft_lane ? xs : -INFINITY;
+        if (q & 1) t1m = fmaxf(t1m, xm); else t0m = fmaxf(t0m, xm);
       }
 #pragma unroll
-      for (int kt = 0; kt < 4; ++kt) {
-        if (kt * 16 >= nvalid) break;
-        const bool tail = kt * 16 + 16 > nvalid;
-        const int tk = kt * 16 + 2 * tig;
-        const uint32_t m0 = (tk < nvalid ? 0x0000ffffu : 0u) | (tk + 1 < nvalid ? 0xffff0000u : 0u);
-        const uint32_t m1 = (tk + 8 < nvalid ? 0x0000ffffu : 0u) | (tk + 9 < nvalid ? 0xffff0000u : 0u);
-        uint32_t h0, l0, h1, l1;
-        split_bf16(w[kt][0], w[kt][1], h0, l0);
-        split_bf16(w[kt][2], w[kt][3], h1, l1);
-        const uint32_t a0 = movmatrix_t(h0), a1 = movmatrix_t(l0), a2 = movmatrix_t(h1), a3 = movmatrix_t(l1);
+    for (int o = 4; o < 32; o <<= 1) {
+      t0m = fmaxf(t0m, __shfl_xor_sync(kFull, t0m, o));
+      t1m = fmaxf(t1m, __shfl_xor_sync(kFull, t1m, o));
+    }
+    // the chunk's column maxima over both warps' tokens
+    if (g8 == 0) sm.xmax[pair][half][tig] = make_float2(t0m, t1m);
+    named_sync(kBarPair0 + pair, 64);
+    {
+      const float2 o = sm.xmax[pair][half ^ 1][tig];
+      t0m = fmaxf(t0m, o.x);
+      t1m = fmaxf(t1m, o.y);
+    }
+    const float mn0 = fmaxf(mr0, t0m), mn1 = fmaxf(mr1, t1m);
+    const float al0 = (soft_lane && mn0 != -INFINITY) ? exp2f(mr0 - mn0) : 1.f;
+    const float al1 = (soft_lane && mn1 != -INFINITY) ? exp2f(mr1 - mn1) : 1.f;
+    float ws0 = 0.f, ws1 = 0.f;
 #pragma unroll
-        for (int np = 0; np < NH / 2; ++np) {
-          uint32_t b0v, b1v, b2v, b3v;
-          ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, (half * NH / 2 + np) * 2 + (mi >> 1)), b0v, b1v, b2v,
-                    b3v);
-          if (tail) {
-            b0v &= m0;
-            b1v &= m1;
-            b2v &= m0;
-            b3v &= m1;
-          }
-          mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
-          mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
+    for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float ev = exp2f(w[mm][q] - ((q & 1) ? mn1 : mn0));
+        w[mm][q] = soft_lane ? (w[mm][q] == -INFINITY ? 0.f : ev) : w[mm][q];
+        if (q & 1) ws1 += w[mm][q]; else ws0 += w[mm][q];
+      }
+    acc0 = acc0 * al0 + ws0;  // this warp's tokens only: the pair's two sums are added at the end
+    acc1 = acc1 * al1 + ws1;
+    mr0 = soft_lane ? mn0 : mr0;
+    mr1 = soft_lane ? mn1 : mr1;
+    const float b0 = __shfl_sync(kFull, al0, g8 >> 1), b1 = __shfl_sync(kFull, al1, g8 >> 1);
+    const float alpha = (p_lane || pre) ? ((g8 & 1) ? b1 : b0) : 1.f;
+    if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+      for (int n = 0; n < NH; ++n) {
+        O[n][0] *= alpha;
+        O[n][1] *= alpha;
+        O[n][2] *= alpha;
+        O[n][3] *= alpha;
+      }
+    }
+    // this warp's PV weight fragments to the other warp of the pair
+    uint32_t mf[2][4], of[2][4];
+#pragma unroll
+    for (int mm = 0; mm < 2; ++mm) {
+      uint32_t h0, l0, h1, l1;
+      split_bf16(w[mm][0], w[mm][1], h0, l0);
+      split_bf16(w[mm][2], w[mm][3], h1, l1);
+      mf[mm][0] = movmatrix_t(h0);
+      mf[mm][1] = movmatrix_t(l0);
+      mf[mm][2] = movmatrix_t(h1);
+      mf[mm][3] = movmatrix_t(l1);
+      sm.xfrag[warp][mm][lane] = make_uint4(mf[mm][0], mf[mm][1], mf[mm][2], mf[mm][3]);
+    }
+    named_sync(kBarPair0 + pair, 64);
+#pragma unroll
+    for (int mm = 0; mm < 2; ++mm) {
+      const uint4 x = sm.xfrag[warp ^ 1][mm][lane];
+      of[mm][0] = x.x;
+      of[mm][1] = x.y;
+      of[mm][2] = x.z;
+      of[mm][3] = x.w;
+    }
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) {
+      if (kt * 16 >= nvalid) break;
+      const bool tail = kt * 16 + 16 > nvalid;
+      const int tk = kt * 16 + 2 * tig;
+      const uint32_t m0 = (tk < nvalid ? 0x0000ffffu : 0u) | (tk + 1 < nvalid ? 0xffff0000u : 0u);
+      const uint32_t m1 = (tk + 8 < nvalid ? 0x0000ffffu : 0u) | (tk + 9 < nvalid ? 0xffff0000u : 0u);
+      const bool own = (kt >> 1) == half;
+      const uint32_t a0 = own ? mf[kt & 1][0] : of[kt & 1][0], a1 = own ? mf[kt & 1][1] : of[kt & 1][1];
+      const uint32_t a2 = own ? mf[kt & 1][2] : of[kt & 1][2], a3 = own ? mf[kt & 1][3] : of[kt & 1][3];
+#pragma unroll
+      for (int np = 0; np < NH / 2; ++np) {
+        uint32_t b0v, b1v, b2v, b3v;
+        ldsm_x4_t(vb + swz<D>(kt * 16 + (mi & 1) * 8 + rr, (half * NH / 2 + np) * 2 + (mi >> 1)), b0v, b1v, b2v,
+                  b3v);
+        if (tail) {
+          b0v &= m0;
+          b1v &= m1;
+          b2v &= m0;
+          b3v &= m1;
         }
+        mma_16816(O[2 * np], a0, a1, a2, a3, b0v, b1v);
+        mma_16816(O[2 * np + 1], a0, a1, a2, a3, b2v, b3v);
       }
     }
     __syncwarp();
@@ -1055,6 +1101,13 @@ __device__ void mattn_role(const FusedParams& p, const UnitGeo& g, const MultiGe
   for (int o = 4; o < 32; o <<= 1) {
     acc0 += __shfl_xor_sync(kFull, acc0, o);
     acc1 += __shfl_xor_sync(kFull, acc1, o);
+  }
+  if (g8 == 0) sm.xacc[1][pair][half][tig] = make_float2(acc0, acc1);
+  named_sync(kBarPair0 + pair, 64);
+  {
+    const float2 o = sm.xacc[1][pair][half ^ 1][tig];
+    acc0 += o.x;
+    acc1 += o.y;
   }
   float m_run, l, ds;
   {
@@ -1394,6 +1447,7 @@ cudaError_t prepare_multi(int D) {
 }
 
 int multi_max_clusters(int D, int NR, int c) {
+  if (c > kMultiMaxCluster) return 0;  // the merge slots are sized for at most this many ranks
   if (NR == 2) return D == 128 ? multi_clusters<128, 2>(c) : multi_clusters<64, 2>(c);
   return D == 128 ? multi_clusters<128, 4>(c) : multi_clusters<64, 4>(c);
 }
