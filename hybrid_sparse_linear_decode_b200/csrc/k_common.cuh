@@ -493,9 +493,10 @@ __device__ __forceinline__ unsigned long long bitonic_step(unsigned long long v,
 }
 // Sort the warp's 32 values descending (lane 0 the largest).
 __device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long v, int lane) {
-#pragma unroll 1
+  // straight-line network (15 steps): it runs once per scored item
+#pragma unroll
   for (int k = 2; k <= 32; k <<= 1)
-#pragma unroll 1
+#pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1) v = bitonic_step(v, lane, j, (lane & k) == 0);
   return v;
 }
@@ -505,7 +506,7 @@ __device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long 
 __device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long a, unsigned long long b, int lane) {
   const unsigned long long br = shfl_u64(b, 31 - lane);
   unsigned long long v = a > br ? a : br;
-#pragma unroll 1
+#pragma unroll
   for (int j = 16; j > 0; j >>= 1) v = bitonic_step(v, lane, j, true);
   return v;
 }
