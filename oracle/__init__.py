@@ -15,6 +15,8 @@ from .hybrid import (  # noqa: F401
     block_stats,
     block_scores,
     select_blocks,
+    strided_blocks,
+    select_blocks_strided,
     exact_mask,
     hybrid_direct,
     hybrid_subtract,

@@ -39,7 +39,12 @@ Readings where the pages are silent (the plainest reading the rest supports):
   selects every block;
 * R6 the Taylor kernel is exp(s) ~ 1 + s with the same scaled s, no clamp;
 * R7 one normaliser: exact weights exp(s_t), linear weights (1 + s_t), one sum in
-  the denominator.
+  the denominator;
+* R8 strided block selection (SPLA, table of contents: the section's heading
+  only): a fixed stride of always-exact blocks -- the last block of every
+  `stride` consecutive candidate blocks -- plus the top-k among the rest.  The
+  page gives no definition, so this is one reading of the heading, not the
+  page's method; it is pinned to its own definition only.
 
 Pins (tests/test_oracle_pins.py): every function here is pinned by at least one
 check that does not retype it -- all-selected equals full softmax, empty exact
@@ -141,6 +146,24 @@ def select_blocks(scores: np.ndarray, k: int) -> np.ndarray:
     nb = scores.shape[0]
     order = sorted(range(nb), key=lambda j: (-scores[j], j))
     return np.array(sorted(order[: min(k, nb)]), dtype=np.int64)
+
+
+def strided_blocks(nb: int, stride: int) -> np.ndarray:
+    """The always-exact blocks of strided block selection (R8): the last block
+    of every group of `stride` consecutive candidate blocks, j % stride ==
+    stride - 1 (none when stride > nb; every block when stride == 1)."""
+    return np.array([j for j in range(nb) if j % stride == stride - 1], dtype=np.int64)
+
+
+def select_blocks_strided(scores: np.ndarray, k: int, stride: int) -> np.ndarray:
+    """Strided block selection (R8): the strided blocks, plus the top-k by
+    score among the other blocks (larger score first, ties to the lower
+    index); ascending."""
+    nb = scores.shape[0]
+    fixed = set(int(j) for j in strided_blocks(nb, stride))
+    rest = [j for j in range(nb) if j not in fixed]
+    order = sorted(rest, key=lambda j: (-scores[j], j))
+    return np.array(sorted(fixed | set(order[: min(k, len(rest))])), dtype=np.int64)
 
 
 def exact_mask(part: Partition, sel) -> np.ndarray:

@@ -251,6 +251,52 @@ def test_topk_against_exhaustive_search():
             assert got == best[1], (scores, k, got, best)
 
 
+def test_strided_selection_by_exhaustive_search():
+    """Strided block selection (R8, one reading of a heading the page leaves
+    empty): the strided blocks are range(stride - 1, nb, stride); the rest of
+    the selection is, among all subsets of the other blocks of the right
+    size, the one with the largest score sum, ties to the lexicographically
+    smallest index tuple."""
+    rng = np.random.default_rng(21)
+    for trial in range(50):
+        nb = int(rng.integers(0, 10))
+        scores = rng.integers(-3, 4, nb).astype(float)      # many ties
+        for stride in range(1, nb + 3):
+            fixed = list(range(stride - 1, nb, stride))
+            assert list(O.strided_blocks(nb, stride)) == fixed
+            others = [j for j in range(nb) if j not in fixed]
+            for k in range(0, nb + 2):
+                got = tuple(O.select_blocks_strided(scores, k, stride))
+                kk = min(k, len(others))
+                best = None
+                for sub in itertools.combinations(others, kk):
+                    key = (-sum(scores[list(sub)]), sub)
+                    if best is None or key < best:
+                        best = key
+                assert got == tuple(sorted(fixed + list(best[1]))), (scores, k, stride, got)
+
+
+def test_strided_selection_special_cases():
+    """A stride past the block count is plain top-k; stride 1 selects every
+    block, and the hybrid output then equals full softmax."""
+    rng = np.random.default_rng(22)
+    scores = rng.standard_normal(40)
+    for k in (0, 3, 39, 50):
+        assert list(O.select_blocks_strided(scores, k, 41)) == list(O.select_blocks(scores, k))
+    T, S, W, Bk, d, G = 300, 4, 32, 16, 16, 2
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    q = rng.standard_normal((G, d))
+    part = O.partition(T, S, W, Bk)
+    scale = 1 / math.sqrt(d)
+    mu, var = O.block_stats(K, part)
+    sc = O.block_scores(q, mu, var, scale)
+    sel = O.select_blocks_strided(sc, 2, 1)
+    assert list(sel) == list(range(part.nb))
+    np.testing.assert_allclose(O.hybrid_subtract(q, K, V, part, sel, scale), O.full_softmax(q, K, V, T, scale),
+                               rtol=1e-12, atol=1e-12)
+
+
 # ----------------------------------------------------------------------------- state / recurrence
 
 def test_linear_state_by_loops():
