@@ -26,6 +26,7 @@ from ._abi import (  # noqa: F401
     hyb_attn_decode_append,
     hyb_attn_decode_chunk,
     hyb_attn_decode_with_selection,
+    hyb_attn_decode_strided,
     hyb_attn_step_host,
     hyb_attn_step_layers_staging_bytes,
     hyb_attn_step_layers_host,

@@ -77,6 +77,7 @@ SIGNATURES = [
     ("hyb_attn_decode_append", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_chunk", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     ("hyb_attn_decode_with_selection", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("hyb_attn_decode_strided", ctypes.c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp]),
     ("hyb_attn_step_host", ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("hyb_attn_step_layers_staging_bytes", c_sz, [ctypes.POINTER(c_vp), c_i32]),
     ("hyb_attn_step_layers_host", ctypes.c_int, [ctypes.POINTER(c_vp), c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
@@ -217,6 +218,11 @@ def hyb_attn_decode_chunk(ctx: int, q: int, k_new: int, v_new: int, n: int, out:
 def hyb_attn_decode_with_selection(ctx: int, q: int, sel: int, out: int, stream: int) -> None:
     _check("hyb_attn_decode_with_selection",
            load_library().hyb_attn_decode_with_selection(ctx, q, sel, out, stream))
+
+
+def hyb_attn_decode_strided(ctx: int, q: int, k_top: int, stride: int, out: int, sel_out: int, stream: int) -> None:
+    _check("hyb_attn_decode_strided",
+           load_library().hyb_attn_decode_strided(ctx, q, k_top, stride, out, sel_out, stream))
 
 
 def hyb_attn_step_host(ctx: int, q_host: int, k_host, v_host, out_host: int, stream: int) -> None:

@@ -16,8 +16,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhyb_attn.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["api.cu", "k_fused.cu", "k_multi.cu", "k_state.cu"]
-HEADERS = ["hyb_device.cuh", "hyb_internal.h", "k_common.cuh"]
+SOURCES = ["api.cu", "k_fused.cu", "k_multi.cu", "k_select.cu", "k_state.cu"]
+HEADERS = ["hyb_device.cuh", "hyb_internal.h", "k_common.cuh", "k_select.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 

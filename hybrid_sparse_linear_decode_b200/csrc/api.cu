@@ -16,6 +16,7 @@
 
 #include "../../include/hyb_attn.h"
 #include "hyb_internal.h"
+#include "k_select.h"
 
 using namespace hyb;
 
@@ -494,6 +495,7 @@ int create_ctx(const hyb_attn_config* cfg, const hyb_attn_buffers* buf, int64_t 
   cudaError_t pe = prepare_fused(k.D);
   if (pe == cudaSuccess) pe = prepare_state(k.D);
   if (pe == cudaSuccess) pe = prepare_multi(k.D);
+  if (pe == cudaSuccess) pe = prepare_strided_select(k.D);
   if (pe != cudaSuccess) {
     delete x;
     return cuda_fail(pe);
@@ -695,6 +697,47 @@ int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32
   HYB_RANGE;
   if (sel == nullptr) return HYB_EINVAL;
   return decode_impl(ctx, q, out, sel, nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+int hyb_attn_decode_strided(hyb_attn_ctx* x, const void* q, int32_t k_top, int32_t stride, float* out,
+                            int32_t* sel_out, cudaStream_t stream) {
+  HYB_RANGE;
+  if (x == nullptr || q == nullptr || out == nullptr || stride < 1 || k_top < 0) return HYB_EINVAL;
+  if (x->tb.ragged || x->tb.per_head) return HYB_EINVAL;  // one length and one budget for every unit
+  if (!aligned16(q) || (sel_out != nullptr && (reinterpret_cast<uintptr_t>(sel_out) & 3u))) return HYB_EINVAL;
+  const Geometry g = geometry(x->cfg, x->T);
+  const int64_t nb = g.nb, n_fixed = nb / stride;
+  const int64_t n_sel = n_fixed + std::min<int64_t>(k_top, nb - n_fixed);
+  if (n_sel > x->cfg.top_k) return HYB_EINVAL;  // the selection row holds top_k blocks
+  const size_t smem = strided_select_smem(x->ck.D, (int)nb);
+  if (nb > 0 && smem == 0) return HYB_EINVAL;
+  // the block statistics must hold every evicted token before they are scored
+  int rc = hyb_attn_sync_state(x, stream);
+  if (rc != HYB_OK) return rc;
+  int32_t* sel = x->w<int32_t>(x->ws.sel);
+  if (nb > 0) {
+    StridedSelParams sp{};
+    sp.q = static_cast<const __nv_bfloat16*>(q);
+    sp.mu = x->buf.mu;
+    sp.var = x->buf.var;
+    sp.sel = sel;
+    sp.sel_copy = sel_out;
+    sp.status = x->status;
+    sp.max_blocks = x->ck.max_blocks > 0 ? x->ck.max_blocks : 1;
+    sp.units = x->ck.units;
+    sp.nb = (int32_t)nb;
+    sp.G = x->ck.G;
+    sp.k = k_top;
+    sp.stride = stride;
+    sp.width = x->cfg.top_k;
+    sp.scale = x->cfg.scale;
+    const cudaError_t e = launch_strided_select(sp, x->ck.D, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  } else if (sel_out != nullptr && x->cfg.top_k > 0) {
+    if (cudaMemsetAsync(sel_out, 0xff, (size_t)x->ck.units * x->cfg.top_k * sizeof(int32_t), stream) != cudaSuccess)
+      return HYB_ECUDA;
+  }
+  return decode_impl(x, q, out, nb > 0 ? sel : nullptr, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 int hyb_attn_step_host(hyb_attn_ctx* x, const void* q_host, const void* k_host, const void* v_host,

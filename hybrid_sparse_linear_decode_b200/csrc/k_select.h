@@ -1,0 +1,27 @@
+// Strided block selection (a separate kernel ahead of the decode).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace hyb {
+
+struct StridedSelParams {
+  const __nv_bfloat16* q;   // [units][G][D]
+  const float* mu;          // [units][max_blocks][D] block means (every eviction folded)
+  const float* var;         // [units][max_blocks][D] block population variances
+  int32_t* sel;             // [units][width]: the selection, ascending, -1 padded
+  int32_t* sel_copy;        // optional second copy of sel (the caller's), or null
+  uint32_t* status;         // status word: HYB_STATUS_NAN_SCORE
+  int64_t max_blocks;
+  int32_t units, nb, G, k, stride, width;
+  float scale;
+};
+
+// Dynamic shared memory the kernel needs for nb candidate blocks (0: too many).
+size_t strided_select_smem(int D, int nb);
+cudaError_t prepare_strided_select(int D);
+cudaError_t launch_strided_select(const StridedSelParams& p, int D, cudaStream_t s);
+
+}  // namespace hyb

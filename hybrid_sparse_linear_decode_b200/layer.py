@@ -163,6 +163,20 @@ class HybridAttentionLayer:
         A.hyb_attn_decode_with_selection(self.ctx, q.data_ptr(), sel.data_ptr(), out.data_ptr(), _stream(stream))
         return out
 
+    def decode_strided(self, q: torch.Tensor, k_top: int, stride: int, out: torch.Tensor | None = None,
+                       sel_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Decode with strided block selection: the last block of every `stride`
+        candidate blocks always exact, plus the top-k_top of the others."""
+        c = self.cfg
+        assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.shape == (c.batch, c.n_q_heads, c.head_dim)
+        if out is None:
+            out = torch.empty((c.batch, c.n_q_heads, c.head_dim), dtype=torch.float32, device=q.device)
+        if sel_out is not None:
+            assert sel_out.dtype == torch.int32 and sel_out.shape == (c.batch, c.n_kv_heads, c.top_k)
+        A.hyb_attn_decode_strided(self.ctx, q.data_ptr(), int(k_top), int(stride), out.data_ptr(), _ptr(sel_out),
+                                  _stream(stream))
+        return out
+
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
         c = self.cfg
         for t in (k_new, v_new):

@@ -290,6 +290,27 @@ int hyb_attn_decode_chunk(hyb_attn_ctx* ctx, const void* q, const void* k_new, c
 int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32_t* sel,
                                    float* out, cudaStream_t stream);
 
+/* Decode with strided block selection ("SPLA: Block Sparse Plus Linear
+ * Attention for Long Context Modeling", table of contents: "Strided block
+ * selection" -- the page gives the heading only; the reading implemented
+ * here is a fixed stride of always-exact blocks): the last block of every
+ * `stride` consecutive candidate blocks (index j with j % stride == stride - 1)
+ * is exact, and the top-k_top blocks by the usual score among the others (ties
+ * to the lower index) are added.  The union replaces the top-k as the decode's
+ * selection; the rest of the decode is hyb_attn_decode's.
+ *   q       bf16 [B][Hq][d], device, 16-byte aligned;  out fp32 [B][Hq][d].
+ *   k_top   >= 0;  stride >= 1 (stride 1: every block; stride > nb: plain top-k).
+ *   sel_out optional int32 [B][Hkv][top_k] (device): the selection, ascending,
+ *           -1 padded.
+ * The configuration's top_k must hold the union (nb / stride + min(k_top,
+ * the other blocks)), else HYB_EINVAL; so must one length and one budget for
+ * every unit (no per-row lengths, no per-head budgets).  Folds the pending
+ * evictions first (hyb_attn_sync_state), then one selection launch that
+ * reads the block statistics, then the decode.  Scores that are NaN raise
+ * HYB_STATUS_NAN_SCORE. */
+int hyb_attn_decode_strided(hyb_attn_ctx* ctx, const void* q, int32_t k_top, int32_t stride, float* out,
+                            int32_t* sel_out, cudaStream_t stream);
+
 /* One decode + append step from host memory, for callers whose inputs and
  * outputs live on the host: copies q_host (bf16 [B][Hq][d]) and k_host, v_host
  * (bf16 [B][Hkv][d]) to device staging space in the workspace, runs
