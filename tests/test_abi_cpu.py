@@ -39,11 +39,11 @@ def test_header_declares_the_boundary():
         assert n in names, n
 
 
-def test_documented_departures_from_the_scope_table_signatures():
-    """Two documented departures from the survey's sketch of the boundary: the
-    status call takes (ctx, uint32_t* flags, int clear, stream), and the
-    buffers hold no open-block running sums (the open block's mean / variance
-    rows are updated in place)."""
+def test_documented_departures_from_the_first_boundary_sketch():
+    """Two departures from the first sketch of the boundary, documented in the
+    header: the status call takes (ctx, uint32_t* flags, int clear, stream),
+    and the buffers hold no open-block running sums (the open block's mean /
+    variance rows are updated in place)."""
     src = open(HEADER).read()
     flat = re.sub(r"\s+", " ", re.sub(r"/\*.*?\*/", "", src, flags=re.S))
     assert "int hyb_attn_status(hyb_attn_ctx* ctx, uint32_t* flags, int clear, cudaStream_t stream);" in flat

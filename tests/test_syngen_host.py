@@ -133,9 +133,9 @@ def test_layer_budgets_view():
     assert base.for_layer(5) is base
 
 
-def test_algorithmic_bytes_match_the_scope_table():
+def test_algorithmic_bytes_match_the_per_head_figures():
     """The benchmark's algorithmic bytes per (layer, b) at the workloads' prefill
-    length, against the per-KV-head figures of the survey's scope table: exact
+    length, against the method's per-KV-head bytes written out by hand: exact
     KV 2052 x 128 x 4, statistics nb x 2 x 128 x 4, state (128^2 + 2 x 128 + 1) x 4,
     q + out 4 x 128 x 6."""
     import bench
