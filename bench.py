@@ -19,6 +19,7 @@ step time is the max over ranks ("scaling": "weak").
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -50,10 +51,12 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (smaller instances for profiling)")
-    ap.add_argument("--mode", default="decode", choices=["decode", "spec", "prefill"],
+    ap.add_argument("--mode", default="decode", choices=["decode", "spec", "prefill", "strided"],
                     help="decode: one decode + append per layer and step; spec: hyb_attn_decode_chunk of "
                          "--chunk draft tokens per layer and step; prefill: hyb_attn_append_chunk of --chunk "
-                         "tokens, then one decode, per layer and step")
+                         "tokens, then one decode, per layer and step; strided: hyb_attn_decode_strided "
+                         "(stride --chunk, the workload's top-k among the other blocks), then one append, "
+                         "per layer and step")
     ap.add_argument("--chunk", type=int, default=4)
     return ap.parse_args()
 
@@ -126,6 +129,19 @@ def step_bytes_model(w, mode: str, chunk: int, T: int, union_blocks=None):
     without it, the bytes of one decode per row)."""
     step_dec = step_bytes = 0
     for l in range(w.layers):
+        if w.head_budgets or mode == "strided":
+            wl = w.for_layer(l)
+            for h in range(w.n_kv_heads):
+                wh = wl.for_head(h)
+                if mode == "strided":  # the union selection, and the statistics read again by its launch
+                    nb = wh.n_blocks(T)
+                    wh = dataclasses.replace(wh, top_k=nb // chunk + min(wh.top_k, nb - nb // chunk))
+                dec_b, app_b = algorithmic_bytes(wh, T)
+                if mode == "strided":
+                    dec_b += wh.n_blocks(T) * 2 * wh.head_dim * 4
+                step_dec += w.batch * dec_b
+                step_bytes += w.batch * (dec_b + app_b)
+            continue
         if mode == "spec" and union_blocks is not None:
             dec_b, app_b = spec_bytes(w.for_layer(l), T, chunk, union_blocks[l])
             step_dec += w.units_per_layer * dec_b
@@ -169,6 +185,8 @@ def measured_traffic(workload: str, mode: str = "decode", chunk: int = 1):
     summary of this workload, if the kernel's sources are unchanged since that
     capture (else None)."""
     import re
+    if mode not in ("decode", "spec"):  # several kernels per step: no single launch's capture applies
+        return None
     prof = os.path.join(ROOT, "profiles", profile_name(workload, mode, chunk))
     if not os.path.exists(prof):
         return None
@@ -252,12 +270,19 @@ class Bench:
         self.w, self.device = w, device
         self.n_steps = n_steps
         self.mode, self.chunk = mode, (chunk if mode != "decode" else 1)
-        n_app = self.n_steps * self.chunk
+        n_app = self.n_steps * (self.chunk if mode in ("spec", "prefill") else 1)  # strided: chunk is the stride
 
-        def cfg_of(l):  # the layer's own top-k and window when budgets vary by layer
+        def cfg_of(l):  # the layer's own top-k and window when budgets vary by layer (or by KV head)
             wl = w.for_layer(l)
-            return make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, wl.window,
-                               wl.top_k, w.T0 + n_app)
+            heads = [wl.for_head(h) for h in range(w.n_kv_heads)]
+            top_k = max(wh.top_k for wh in heads)
+            if self.mode == "strided":  # the selection row holds the strided blocks and the top-k
+                nb = w.n_blocks(w.T0 + n_app)
+                top_k = nb // self.chunk + min(top_k, nb - nb // self.chunk)
+            hw = [wh.window for wh in heads] if w.head_budgets else None
+            hk = [wh.top_k for wh in heads] if w.head_budgets else None
+            return make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink,
+                               min(wh.window for wh in heads), top_k, w.T0 + n_app, head_window=hw, head_top_k=hk)
 
         ws_bytes = max(HybridAttentionLayer.workspace_bytes(cfg_of(l)) for l in range(w.layers))
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device)   # shared: one stream
@@ -302,6 +327,9 @@ class Bench:
             if self.mode == "spec":
                 L.decode_chunk(q, self.app_k[l][s * n:(s + 1) * n], self.app_v[l][s * n:(s + 1) * n],
                                out=self.out_chunk)
+            elif self.mode == "strided":
+                L.decode_strided(q, self.w.for_layer(l).top_k, n, out=self.out)
+                L.append(self.app_k[l][s], self.app_v[l][s])
             elif self.mode == "prefill":
                 L.append_chunk(self.app_k[l][s], self.app_v[l][s])
                 L.decode(q, out=self.out)
@@ -314,10 +342,12 @@ class Bench:
         cache write and the fold of the previous evictions ride in it); spec:
         one multi-query launch per group of 4, then 2, then 1 draft rows;
         prefill: the chunk's cache write, the dense fold of the tokens it
-        evicted (5 or more) and one decode."""
+        evicted (5 or more) and one decode; strided: the fold of the previous
+        eviction (a fold-only decode launch), the selection, the decode and the
+        append's cache write."""
         n = self.chunk
         groups = n // 4 + (n % 4) // 2 + (n % 2)
-        per = {"decode": 1, "spec": groups, "prefill": 2 + (self.chunk >= 5)}[self.mode]
+        per = {"decode": 1, "spec": groups, "prefill": 2 + (self.chunk >= 5), "strided": 4}[self.mode]
         return per * len(self.layers)
 
     def union_blocks(self):
@@ -494,7 +524,11 @@ def run_native(args, rank, world):
                            "selected blocks as measured"} if union is not None else {}),
         "roofline": {"bound": "hbm",
                      "kernel": ("the multi-query decode kernel: one layer's draft rows decoded + appended together"
-                                if mode == "spec" else "the fused decode kernel: one layer's decode + append (one launch)"),
+                                if mode == "spec" else
+                                "one layer's launches, averaged: the fold, the strided selection, the decode, the append"
+                                if mode == "strided" else
+                                "one layer's launches, averaged: the chunk's cache write, the dense fold, the decode"
+                                if mode == "prefill" else "the fused decode kernel: one layer's decode + append (one launch)"),
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
                      "traffic": measured_traffic(w.name, mode, chunk), "bytes_per_launch": launch_bytes,
@@ -700,9 +734,10 @@ def workload_config(w, mode: str, chunk: int, world: int, flush: bool) -> dict:
         "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context_T0": w.T0, "block": w.block_size,
         "sinks": w.n_sink, "window": w.window, "top_k": w.top_k,
         **({"layer_budgets_k_W": [list(x) for x in w.layer_budgets]} if w.layer_budgets else {}),
+        **({"head_budgets_k_W": [list(x) for x in w.head_budgets]} if w.head_budgets else {}),
         "l2": "flushed between timed steps (512 MB write)" if flush else "step data >> L2 (no flush)",
         "parallelism": f"replicas x{world} (independent units per GPU)",
-        **({"mode": mode, "chunk": chunk} if mode != "decode" else {}),
+        **({"mode": mode, "stride": chunk} if mode == "strided" else {"mode": mode, "chunk": chunk} if mode != "decode" else {}),
     }
 
 
@@ -711,6 +746,10 @@ def run_reference(args, rank, world):
     overrides = {"layers": args.layers} if args.layers else {}
     w = C.get_workload(args.workload, **overrides)
     mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
+    if mode == "strided":
+        print(json.dumps({"impl": "reference", "unavailable": "the oracle arm times decode, spec and prefill steps; "
+                          "strided selection is checked against the oracle in the tests, not timed"}), flush=True)
+        return
     pool = OraclePool(w)
     try:
         per = args.cpu_sample_seconds / max(1, args.steps)
@@ -759,7 +798,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_native(args, rank, world)
-    if rank == 0 and not args.no_cpu_baseline and world == 1:
+    if rank == 0 and not args.no_cpu_baseline and world == 1 and args.mode != "strided":  # (the oracle's step is decode + append with the plain top-k)
         from syngen import configs as C
         overrides = {"layers": args.layers} if args.layers else {}
         w = C.get_workload(args.workload, **overrides)

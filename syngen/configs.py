@@ -39,6 +39,9 @@ class Workload:
     # per-layer (top_k, window), cycled over the layers; empty: every layer has
     # top_k and window above
     layer_budgets: tuple = ()
+    # per-KV-head (top_k, window), cycled over the KV heads; empty: every head
+    # has the layer's budget
+    head_budgets: tuple = ()
 
     def for_layer(self, layer: int) -> "Workload":
         """The workload as layer `layer` sees it: its own top-k and window when
@@ -48,6 +51,14 @@ class Workload:
             return self
         k, win = self.layer_budgets[layer % len(self.layer_budgets)]
         return dataclasses.replace(self, top_k=k, window=win, layer_budgets=())
+
+    def for_head(self, h: int) -> "Workload":
+        """The workload as KV head `h` sees it: its own top-k and window when the
+        budgets vary by head."""
+        if not self.head_budgets:
+            return self
+        k, win = self.head_budgets[h % len(self.head_budgets)]
+        return dataclasses.replace(self, top_k=k, window=win, head_budgets=())
 
     @property
     def group(self) -> int:
@@ -112,6 +123,17 @@ WORKLOADS = {
                                           block_size=64, n_sink=4, window=1024, top_k=16, steps=1,
                                           head_scale=True,
                                           layer_budgets=((8, 512), (16, 1024), (24, 1536), (32, 2048))),
+    # per-KV-head budgets (k, W) varying over the 8 KV heads of every layer
+    "llama8b_32layers_b8_32k_head_budgets": _w(name="llama8b_32layers_b8_32k_head_budgets", batch=8, layers=32,
+                                               n_q_heads=32, n_kv_heads=8, head_dim=128, T0=32768,
+                                               block_size=64, n_sink=4, window=512, top_k=32, steps=1,
+                                               head_scale=True,
+                                               head_budgets=((8, 512), (16, 1024), (24, 1536), (32, 2048))),
+    # token-granular exact set: blocks of one token, the top 1024 tokens exact
+    # (the same exact budget as 16 blocks of 64)
+    "llama8b_32k_layer_tokens": _w(name="llama8b_32k_layer_tokens", batch=1, layers=1, n_q_heads=32,
+                                   n_kv_heads=8, head_dim=128, T0=32768, block_size=1, n_sink=4,
+                                   window=1024, top_k=1024, steps=1, n_planted=8),
     "llama8b_32layers_b4_128k": _w(name="llama8b_32layers_b4_128k", batch=4, layers=32,
                                    n_q_heads=32, n_kv_heads=8, head_dim=128, T0=131072,
                                    block_size=64, n_sink=4, window=2048, top_k=32, steps=1,

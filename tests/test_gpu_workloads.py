@@ -1,4 +1,4 @@
-"""Parity at the full sizes of the five synthetic workloads, in the launch
+"""Parity at the full sizes of the synthetic workloads, in the launch
 configuration the benchmark times: device caches are filled by the device
 generator, the oracle regenerates the same units on the host (bit-identical
 generator twins, see test_gpu_syngen.py) for sampled units."""
@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle as O
-from harness import bits_to_f64, check_outputs, check_selection, to_device_bf16, OUT_MAX_ABS, OUT_REL_L2, STATE_REL
+from harness import bits_to_f64, check_outputs, check_selection, to_device_bf16, OUT_MAX_ABS, OUT_REL_L2, SEL_TIE, STATE_REL
 from syngen import configs as C
 from syngen import host as SH
 
@@ -25,8 +25,12 @@ class WorkloadLayer:
         w = w.for_layer(layer)  # the layer's own top-k and window when budgets vary by layer
         self.w, self.l = w, layer
         self.n_app = w.capacity - w.T0 if n_app is None else n_app
-        cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window,
-                          w.top_k, w.T0 + self.n_app)
+        heads = [w.for_head(h) for h in range(w.n_kv_heads)]  # per-head budgets, when the workload has them
+        self.k_max = max(wh.top_k for wh in heads)
+        cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink,
+                          min(wh.window for wh in heads), self.k_max, w.T0 + self.n_app,
+                          head_window=[wh.window for wh in heads] if w.head_budgets else None,
+                          head_top_k=[wh.top_k for wh in heads] if w.head_budgets else None)
         self.layer = HybridAttentionLayer(cfg, device)
         self.tables = SD.DeviceTables(w, layer, self.layer.device)
         SD.fill_kv(w, self.tables, self.layer.k_cache, self.layer.v_cache, 0, w.T0)
@@ -47,7 +51,7 @@ class WorkloadLayer:
     def decode(self, qb):
         import torch
         dev = self.layer.device
-        sel = torch.full((self.w.batch, self.w.n_kv_heads, self.w.top_k), -7, dtype=torch.int32, device=dev)
+        sel = torch.full((self.w.batch, self.w.n_kv_heads, self.k_max), -7, dtype=torch.int32, device=dev)
         out = self.layer.decode(to_device_bf16(qb, dev), sel_out=sel)
         torch.cuda.synchronize()
         return out.cpu().numpy().astype(np.float64), sel.cpu().numpy()
@@ -64,15 +68,17 @@ class WorkloadLayer:
     def check_units(self, qb, units, out, sel):
         w = self.w
         G = w.group
-        part = O.partition(self.T, w.n_sink, w.window, w.block_size)
         refs, gots, ndiff = [], [], 0
         for (b, h) in units:
+            wh = w.for_head(h)  # the head's own budget
+            part = O.partition(self.T, w.n_sink, wh.window, w.block_size)
             K, V = self.host_unit(b, h)
             K, V = K[:self.T], V[:self.T]
             q = bits_to_f64(qb)[b, h * G:(h + 1) * G]
             mu, var = O.block_stats(K, part)
             scores = O.block_scores(q, mu, var, self.scale)
-            ndiff += check_selection(sel[b, h], scores, w.top_k)
+            assert all(j == -1 for j in sel[b, h][wh.top_k:])
+            ndiff += check_selection(sel[b, h][:wh.top_k], scores, wh.top_k)
             gsel = np.array([j for j in sel[b, h] if j >= 0])
             refs.append(O.hybrid_subtract(q, K, V, part, gsel, self.scale))
             gots.append(out[b, h * G:(h + 1) * G])
@@ -80,10 +86,10 @@ class WorkloadLayer:
 
     def check_state(self, units):
         w = self.w
-        part = O.partition(self.T, w.n_sink, w.window, w.block_size)
         L = self.layer
         L.sync_state()  # fold the evictions since the last decode
         for (b, h) in units:
+            part = O.partition(self.T, w.n_sink, w.for_head(h).window, w.block_size)
             K, V = self.host_unit(b, h)
             K, V = K[:self.T], V[:self.T]
             H, zk, zv, n = O.linear_state(K, V, part)
@@ -180,6 +186,78 @@ def test_llama8b_32layers_b4_128k_sampled(layer, units):
     out, sel = wl.decode(qb)
     wl.check_units(qb, units, out, sel)
     assert wl.layer.status() == 0
+
+
+def test_llama8b_32layers_b8_32k_head_budgets_sampled():
+    """Per-KV-head budgets at full size: the 8 KV heads of a layer cycle through
+    (k, W) = (8, 512), (16, 1024), (24, 1536), (32, 2048); units of every budget
+    and both batch ends against the oracle with their own head's budget, then
+    the state after an append."""
+    w = C.get_workload("llama8b_32layers_b8_32k_head_budgets")
+    wl = WorkloadLayer(w, 5, n_app=1)
+    units = [(0, 0), (7, 1), (3, 2), (5, 3), (1, 7)]
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    wl.check_units(qb, units, out, sel)
+    wl.append(0)
+    wl.check_state(units[:2])
+    assert wl.layer.status() == 0
+
+
+def test_llama8b_32k_layer_tokens_every_unit():
+    """Token-granular exact set at full size: blocks of one token (31.7 K
+    candidates per unit), the top 1024 tokens exact; every unit against the
+    oracle."""
+    w = C.get_workload("llama8b_32k_layer_tokens")
+    wl = WorkloadLayer(w, 0, n_app=0)
+    qb = wl.q_bits(0)
+    out, sel = wl.decode(qb)
+    wl.check_units(qb, [(0, h) for h in range(w.n_kv_heads)], out, sel)
+    assert wl.layer.status() == 0
+
+
+def test_llama8b_32layers_b8_32k_strided_sampled():
+    """Strided block selection at full size (stride 16 over 496 candidate
+    blocks: 31 always-exact blocks, plus the top 16 of the others), in the
+    bench's configuration: the selection row sized for the union."""
+    import torch
+    from hybrid_sparse_linear_decode_b200 import HybridAttentionLayer, make_config
+    import syngen.device as SD
+    w = C.get_workload("llama8b_32layers_b8_32k")
+    stride, k_top = 16, 16
+    nb = w.n_blocks(w.T0)
+    width = nb // stride + min(k_top, nb - nb // stride)
+    SD.build()
+    cfg = make_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.n_sink, w.window, width, w.T0)
+    L = HybridAttentionLayer(cfg, "cuda")
+    tables = SD.DeviceTables(w, 3, L.device)
+    SD.fill_kv(w, tables, L.k_cache, L.v_cache, 0, w.T0)
+    L.init(w.T0)
+    qb = SH.q_bits(w, 3, 0)
+    sel = torch.full((w.batch, w.n_kv_heads, width), -7, dtype=torch.int32, device=L.device)
+    out = L.decode_strided(to_device_bf16(qb, L.device), k_top, stride, sel_out=sel)
+    torch.cuda.synchronize()
+    out, sel = out.cpu().numpy().astype(np.float64), sel.cpu().numpy()
+    assert L.status() == 0
+    scale = 1 / math.sqrt(w.head_dim)
+    part = O.partition(w.T0, w.n_sink, w.window, w.block_size)
+    refs, gots = [], []
+    for (b, h) in [(0, 0), (7, 7), (3, 5)]:
+        K, V = SH.kv_f64(w, tables.host, b, h, 0, w.T0)
+        q = bits_to_f64(qb)[b, h * w.group:(h + 1) * w.group]
+        mu, var = O.block_stats(K, part)
+        scores = O.block_scores(q, mu, var, scale)
+        want = set(int(j) for j in O.select_blocks_strided(scores, k_top, stride))
+        got = [int(j) for j in sel[b, h]]
+        assert got == sorted(got) and len(got) == width and set(O.strided_blocks(part.nb, stride)) <= set(got)
+        fixed = set(int(j) for j in O.strided_blocks(part.nb, stride))
+        others = np.sort(np.array([scores[j] for j in range(part.nb) if j not in fixed]))[::-1]
+        kth = others[k_top - 1]
+        for j in set(got) ^ want:
+            assert abs(scores[j] - kth) <= SEL_TIE * max(1.0, abs(kth)), (j, scores[j], kth)
+        refs.append(O.hybrid_subtract(q, K, V, part, np.array(got, dtype=np.int64), scale))
+        gots.append(out[b, h * w.group:(h + 1) * w.group])
+    check_outputs(np.array(gots), np.array(refs))
 
 
 def test_llama8b_256k_256_steps_every_unit():
