@@ -7,20 +7,31 @@
 // ascending, is handed to the decode as its selection, so the exact part and
 // the subtraction of the selected blocks' linear terms are the decode's own.
 //
-// One CTA per unit: the group's q' sums, the score of every candidate block
-// from its mean and variance rows (one warp per block, lanes over channels),
-// the top-k by repeated block-wide maxima of packed (key << 32 | ~index)
-// words, the union as a bitmap, compacted in block order by one warp.  This is
-// a separate launch that reads the block statistics once more; it serves a
-// selection rule the pages only name, not the decode step's hot path.
+// One CTA per unit.  The unit's mean and variance rows are prefetched into L2
+// before the wait for the previous grid (L2 is the point of coherence, so a
+// row that grid still writes is current there).  Scoring: the group's q' sums
+// stay in registers, every warp takes 8 rows per step with one 16-byte load of
+// the mean and one of the variance per lane (16 loads in flight per lane), and
+// reduces the 8 rows' partial sums at once.  The scores of the non-strided
+// blocks are stored compacted (c = j - (j + 1) / stride, which keeps block
+// order, so ties to the lower compacted index are ties to the lower block).
+// Top-k: up to 32, one warp's bound-and-rank selection (the decode kernel's);
+// above 32, or when too many keys tie at the bound, k rounds of block-wide
+// maxima of packed (key << 32 | ~index) words.  The union is a bitmap,
+// compacted in block order by one warp.  This is a separate launch that reads
+// the block statistics once more; it serves a selection rule the pages only
+// name, not the decode step's hot path.
 
-#include "hyb_device.cuh"
+#include "k_common.cuh"
 #include "k_select.h"
 
 namespace hyb {
 namespace {
 
-constexpr int kSelThreads = 256, kSelWarps = kSelThreads / 32;
+constexpr int kSelThreads = 512, kSelWarps = kSelThreads / 32;
+constexpr int kSelSteps = 8;      // rows per lane per step (loads in flight: 2 per row)
+constexpr int kSelCap = 256;      // candidates at the bound the one-warp selection ranks
+constexpr int kSelMinRows = 512;  // the one-warp selection reads 512 scores when it has fewer
 
 __device__ __forceinline__ unsigned long long shfl_xor_u64s(unsigned long long v, int m) {
   const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
@@ -30,16 +41,31 @@ __device__ __forceinline__ unsigned long long shfl_xor_u64s(unsigned long long v
 
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __grid_constant__ StridedSelParams p) {
+  constexpr int LPR = D / 4;       // lanes per row (one float4 of channels each)
+  constexpr int RPW = 32 / LPR;    // rows per warp per load
+  static_assert(D % 4 == 0 && 32 % LPR == 0, "a row is a whole number of 16-byte lane slices within a warp");
+  constexpr int kRowsPerIter = RPW * kSelSteps;
   extern __shared__ __align__(16) uint8_t sel_smem[];
-  float* q1 = reinterpret_cast<float*>(sel_smem);      // sum_i q'_i
-  float* q2 = q1 + D;                                    // 1/2 sum_i q'_i^2
-  float* sc = q2 + D;                                    // [nb] block scores
-  uint32_t* bm = reinterpret_cast<uint32_t*>(sc + ((p.nb + 3) & ~3));  // [ceil(nb / 32)] selected blocks
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(sel_smem);  // [kSelCap]
+  float* q1 = reinterpret_cast<float*>(cand + kSelCap);                       // sum_i q'_i
+  float* q2 = q1 + D;                                                           // 1/2 sum_i q'_i^2
+  float* csc = q2 + D;                                      // [max(nc, 512)] scores of the non-strided blocks
+  const int nb = p.nb, stride = p.stride, words = (nb + 31) >> 5;
+  const int n_fixed = nb / stride, nc = nb - n_fixed;
+  const int ncp = ((nc > kSelMinRows ? nc : kSelMinRows) + 3) & ~3;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(csc + ncp);   // [words] selected blocks
   __shared__ unsigned long long red[kSelWarps];
-  __shared__ uint32_t nan_seen;
+  __shared__ int32_t selc[32];
+  __shared__ uint32_t nan_seen, warp_ok;
   const int unit = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nb = p.nb, words = (nb + 31) >> 5;
+  const int64_t row0 = (int64_t)unit * p.max_blocks;
   if (tid == 0) {
+    const int64_t bytes = (int64_t)nb * D * 4;
+    for (int64_t o = 0; o < bytes; o += 32768) {
+      const uint32_t n = (uint32_t)(bytes - o < 32768 ? bytes - o : 32768);
+      bulk_prefetch_l2(reinterpret_cast<const char*>(p.mu + row0 * D) + o, n);
+      bulk_prefetch_l2(reinterpret_cast<const char*>(p.var + row0 * D) + o, n);
+    }
     pdl_wait_primary();  // the statistics and q may come from the previous grid
     nan_seen = 0u;
   }
@@ -57,52 +83,105 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
   }
   for (int w = tid; w < words; w += kSelThreads) bm[w] = 0u;
   __syncthreads();
-  // scores: q'.mu_j + 1/2 q'^2 . var_j summed over the group's heads
-  for (int j = warp; j < nb; j += kSelWarps) {
-    const float* mu = p.mu + ((int64_t)unit * p.max_blocks + j) * D;
-    const float* var = p.var + ((int64_t)unit * p.max_blocks + j) * D;
-    float acc = 0.f;
-#pragma unroll
-    for (int c = lane; c < D; c += 32) acc += q1[c] * mu[c] + q2[c] * var[c];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      sc[j] = acc;
-      if (acc != acc) nan_seen = 1u;
-    }
-  }
-  // the strided blocks are always taken
-  for (int j = p.stride - 1 + tid * p.stride; j < nb; j += kSelThreads * p.stride) atomicOr(&bm[j >> 5], 1u << (j & 31));
-  __syncthreads();
-  // top-k among the others: k rounds of the largest packed word below the last
-  const int n_fixed = nb / p.stride;
-  const int kk = min(p.k, nb - n_fixed);
-  unsigned long long last = ~0ull;
+  // scores q'.mu_j + 1/2 q'^2 . var_j summed over the group's heads
+  const int sub = lane / LPR, cl = lane % LPR;
+  const float4 a1 = *reinterpret_cast<const float4*>(q1 + 4 * cl);
+  const float4 a2 = *reinterpret_cast<const float4*>(q2 + 4 * cl);
+  bool nan = false;
 #pragma unroll 1
-  for (int it = 0; it < kk; ++it) {
-    unsigned long long best = 0ull;
-    for (int j = tid; j < nb; j += kSelThreads) {
-      if (j % p.stride == p.stride - 1) continue;
-      const unsigned long long v = ((unsigned long long)float_key(sc[j]) << 32) | (uint32_t)~(uint32_t)j;
-      if (v < last && v > best) best = v;
-    }
+  for (int j0 = warp * kRowsPerIter; j0 < nb; j0 += kSelWarps * kRowsPerIter) {
+    float4 m[kSelSteps], v[kSelSteps];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long y = shfl_xor_u64s(best, o);
-      best = y > best ? y : best;
+    for (int s = 0; s < kSelSteps; ++s) {
+      const int j = j0 + s * RPW + sub;
+      if (j < nb) {
+        const int64_t off = (row0 + j) * D + 4 * cl;
+        m[s] = __ldg(reinterpret_cast<const float4*>(p.mu + off));
+        v[s] = __ldg(reinterpret_cast<const float4*>(p.var + off));
+      } else {
+        m[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+        v[s] = m[s];
+      }
     }
-    if (lane == 0) red[warp] = best;
-    __syncthreads();
-    best = red[0];
+    float acc[kSelSteps];
 #pragma unroll
-    for (int w = 1; w < kSelWarps; ++w) best = red[w] > best ? red[w] : best;
-    last = best;
-    if (tid == 0 && best != 0ull) {  // (a candidate always remains: kk <= the other blocks)
-      const int j = (int)~(uint32_t)best;
-      bm[j >> 5] |= 1u << (j & 31);
+    for (int s = 0; s < kSelSteps; ++s)
+      acc[s] = a1.x * m[s].x + a1.y * m[s].y + a1.z * m[s].z + a1.w * m[s].w + a2.x * v[s].x + a2.y * v[s].y +
+               a2.z * v[s].z + a2.w * v[s].w;
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1)
+#pragma unroll
+      for (int s = 0; s < kSelSteps; ++s) acc[s] += __shfl_xor_sync(0xffffffffu, acc[s], o);
+    if (cl == 0) {
+#pragma unroll
+      for (int s = 0; s < kSelSteps; ++s) {
+        const int j = j0 + s * RPW + sub;
+        if (j < nb) {
+          nan |= acc[s] != acc[s];
+          if (j % stride != stride - 1) csc[j - (j + 1) / stride] = acc[s];
+        }
+      }
     }
-    __syncthreads();  // red is rewritten next round; the bitmap is complete after the last
   }
+  if (nan) nan_seen = 1u;
+  // the strided blocks are always taken
+  for (int64_t j = stride - 1 + (int64_t)tid * stride; j < nb; j += (int64_t)kSelThreads * stride)
+    atomicOr(&bm[j >> 5], 1u << (j & 31));
+  __syncthreads();
+  // top-k among the others (compacted index c is block c + c / (stride - 1))
+  const int kk = min(p.k, nc);
+  if (kk == nc) {  // every other block
+    for (int c = tid; c < nc; c += kSelThreads) {
+      const int j = c + c / (stride - 1);
+      atomicOr(&bm[j >> 5], 1u << (j & 31));
+    }
+  } else if (kk > 0) {
+    bool ok = false;
+    if (kk <= 32) {
+      if (warp == 0) {
+        bool wn;
+        const bool r = topk_warp(csc, nc, kk, selc, nullptr, cand, kSelCap, wn);
+        __syncwarp();
+        if (r && lane < kk) {
+          const int c = selc[lane];
+          const int j = c + c / (stride - 1);
+          atomicOr(&bm[j >> 5], 1u << (j & 31));
+        }
+        if (lane == 0) warp_ok = r ? 1u : 0u;
+      }
+      __syncthreads();
+      ok = warp_ok != 0u;
+    }
+    if (!ok) {  // k rounds of the largest packed word below the last
+      unsigned long long last = ~0ull;
+#pragma unroll 1
+      for (int it = 0; it < kk; ++it) {
+        unsigned long long best = 0ull;
+        for (int c = tid; c < nc; c += kSelThreads) {
+          const unsigned long long w = ((unsigned long long)float_key(csc[c]) << 32) | (uint32_t)~(uint32_t)c;
+          if (w < last && w > best) best = w;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long y = shfl_xor_u64s(best, o);
+          best = y > best ? y : best;
+        }
+        if (lane == 0) red[warp] = best;
+        __syncthreads();
+        best = red[0];
+#pragma unroll
+        for (int w = 1; w < kSelWarps; ++w) best = red[w] > best ? red[w] : best;
+        last = best;
+        if (tid == 0 && best != 0ull) {  // (a candidate always remains: kk < nc)
+          const int c = (int)~(uint32_t)best;
+          const int j = c + c / (stride - 1);
+          bm[j >> 5] |= 1u << (j & 31);
+        }
+        __syncthreads();  // red is rewritten next round; the bitmap is complete after the last
+      }
+    }
+  }
+  __syncthreads();
   // the union in block order, -1 padded to the row width
   if (warp == 0) {
     int32_t* row = p.sel + (int64_t)unit * p.width;
@@ -143,7 +222,8 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
 }  // namespace
 
 size_t strided_select_smem(int D, int nb) {
-  const size_t bytes = (size_t)(2 * D + ((nb + 3) & ~3)) * 4 + (size_t)((nb + 31) / 32) * 4;
+  const size_t rows = (size_t)((nb > kSelMinRows ? nb : kSelMinRows) + 3) & ~(size_t)3;
+  const size_t bytes = (size_t)kSelCap * 8 + (2 * (size_t)D + rows) * 4 + (size_t)((nb + 31) / 32) * 4;
   return bytes <= 200 * 1024 ? bytes : 0;
 }
 

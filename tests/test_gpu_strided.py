@@ -83,3 +83,48 @@ def test_strided_selection_arguments_are_checked():
         with pytest.raises(HybAttnError):
             c.layer.decode_strided(q, k_top, stride)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("nbk,k_top,stride,d", [
+    (300, 40, 5, 128),    # k above 32: the selection by rounds of block-wide maxima
+    (700, 16, 50, 128),   # 686 non-strided blocks: the one-warp selection above 512 scores
+    (520, 32, 3, 64),     # k = 32, head dimension 64, 347 candidates
+])
+def test_strided_selection_wide_k_and_many_blocks(nbk, k_top, stride, d):
+    S, W, Bk = 4, 64, 8
+    T0 = S + nbk * Bk + W + 5  # a ragged last block
+    nb = (T0 - S - W + Bk - 1) // Bk
+    width = nb // stride + min(k_top, nb - nb // stride)
+    c = Case(B=1, Hq=4, Hkv=1, d=d, T0=T0, Bk=Bk, S=S, W=W, k=width, seed=34)
+    _check(c, c.random_q(), k_top, stride)
+
+
+@pytest.mark.parametrize("nbk,k_top,stride", [
+    (600, 10, 7),   # 515 candidates tie: more than the one-warp selection ranks, above 512
+    (400, 24, 9),   # 356 candidates tie, below 512
+])
+def test_strided_selection_all_scores_equal(nbk, k_top, stride):
+    """q = 0 makes every score 0: the strided blocks and the k lowest other
+    block indices, exactly; every token weighs 1, so the output is the mean of V."""
+    import torch
+    from harness import to_device_bf16
+    S, W, Bk = 4, 16, 8
+    nb = nbk
+    width = nb // stride + k_top
+    c = Case(B=2, Hq=4, Hkv=2, d=64, T0=S + nbk * Bk + W, Bk=Bk, S=S, W=W, k=width, seed=35)
+    dev = c.layer.device
+    q = to_device_bf16(np.zeros((c.B, c.Hq, c.d), dtype=np.uint16), dev)
+    sel = torch.full((c.B, c.Hkv, c.k), -7, dtype=torch.int32, device=dev)
+    out = c.layer.decode_strided(q, k_top, stride, sel_out=sel)
+    torch.cuda.synchronize()
+    out, sel = out.cpu().numpy().astype(np.float64), sel.cpu().numpy()
+    assert c.layer.status() == 0
+    fixed = [j for j in range(nb) if j % stride == stride - 1]
+    others = [j for j in range(nb) if j % stride != stride - 1]
+    want = sorted(fixed + others[:k_top])
+    for b in range(c.B):
+        for h in range(c.Hkv):
+            assert list(sel[b, h]) == want
+            _, Vf = c.unit_kv(b, h)
+            check_outputs(out[b, h * c.G:(h + 1) * c.G], np.broadcast_to(Vf.mean(axis=0), (c.G, c.d)),
+                          max_abs=1e-4, rel_l2=1e-4)
