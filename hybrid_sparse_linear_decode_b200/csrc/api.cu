@@ -731,6 +731,7 @@ int hyb_attn_decode_strided(hyb_attn_ctx* x, const void* q, int32_t k_top, int32
     sp.stride = stride;
     sp.width = x->cfg.top_k;
     sp.scale = x->scale;  // resolved (1/sqrt(d) when the configuration gives 0)
+    sp.parts = strided_select_parts((int)nb, x->ck.units, x->n_sm);
     const cudaError_t e = launch_strided_select(sp, x->ck.D, stream);
     if (e != cudaSuccess) return cuda_fail(e);
   } else if (sel_out != nullptr && x->cfg.top_k > 0) {

@@ -7,14 +7,19 @@
 // ascending, is handed to the decode as its selection, so the exact part and
 // the subtraction of the selected blocks' linear terms are the decode's own.
 //
-// One CTA per unit.  The unit's mean and variance rows are prefetched into L2
-// before the wait for the previous grid (L2 is the point of coherence, so a
-// row that grid still writes is current there).  Scoring: the group's q' sums
-// stay in registers, every warp takes 8 rows per step with one 16-byte load of
-// the mean and one of the variance per lane (16 loads in flight per lane), and
-// reduces the 8 rows' partial sums at once.  The scores of the non-strided
-// blocks are stored compacted (c = j - (j + 1) / stride, which keeps block
-// order, so ties to the lower compacted index are ties to the lower block).
+// One cluster of `parts` CTAs per unit (as many as fill the SMs once, at most
+// 8), each scoring a contiguous share of the blocks.  A CTA's mean and
+// variance rows are prefetched into L2 before the wait for the previous grid
+// (L2 is the point of coherence, so a row that grid still writes is current
+// there).  Scoring: every warp takes 8 rows per step with one 16-byte load of
+// the mean and one of the variance per lane (16 loads in flight per lane; the
+// first step's loads are issued before the group's q' sums are formed, so the
+// two round trips overlap), and reduces the 8 rows' partial sums at once.
+// The scores of the non-strided blocks are stored compacted into the shared
+// memory of the cluster's first CTA (c = j - (j + 1) / stride, which keeps
+// block order, so ties to the lower compacted index are ties to the lower
+// block); two cluster barriers bracket these stores (every CTA has started;
+// every score is in place).  The first CTA then selects.
 // Top-k: up to 32, one warp's bound-and-rank selection (the decode kernel's);
 // above 32, or when too many keys tie at the bound, k rounds of block-wide
 // maxima of packed (key << 32 | ~index) words.  The union is a bitmap,
@@ -32,6 +37,15 @@ constexpr int kSelThreads = 512, kSelWarps = kSelThreads / 32;
 constexpr int kSelSteps = 8;      // rows per lane per step (loads in flight: 2 per row)
 constexpr int kSelCap = 256;      // candidates at the bound the one-warp selection ranks
 constexpr int kSelMinRows = 512;  // the one-warp selection reads 512 scores when it has fewer
+
+// every thread of every CTA of the cluster arrives, then waits (release /
+// acquire: shared-memory stores into other CTAs before it are visible after it)
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive;\n\tbarrier.cluster.wait;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 
 __device__ __forceinline__ unsigned long long shfl_xor_u64s(unsigned long long v, int m) {
   const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
@@ -57,44 +71,32 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
   __shared__ unsigned long long red[kSelWarps];
   __shared__ int32_t selc[32];
   __shared__ uint32_t nan_seen, warp_ok;
-  const int unit = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int parts = p.parts, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int unit = blockIdx.x / parts;
+  const int part = parts > 1 ? (int)cluster_rank() : 0;
+  const int share = (nb + parts - 1) / parts;
+  const int r0 = min(nb, part * share), r1 = min(nb, r0 + share);
   const int64_t row0 = (int64_t)unit * p.max_blocks;
   if (tid == 0) {
-    const int64_t bytes = (int64_t)nb * D * 4;
+    const int64_t first = (row0 + r0) * D * 4, bytes = (int64_t)(r1 - r0) * D * 4;
     for (int64_t o = 0; o < bytes; o += 32768) {
       const uint32_t n = (uint32_t)(bytes - o < 32768 ? bytes - o : 32768);
-      bulk_prefetch_l2(reinterpret_cast<const char*>(p.mu + row0 * D) + o, n);
-      bulk_prefetch_l2(reinterpret_cast<const char*>(p.var + row0 * D) + o, n);
+      bulk_prefetch_l2(reinterpret_cast<const char*>(p.mu) + first + o, n);
+      bulk_prefetch_l2(reinterpret_cast<const char*>(p.var) + first + o, n);
     }
     pdl_wait_primary();  // the statistics and q may come from the previous grid
     nan_seen = 0u;
   }
   __syncthreads();
   pdl_allow_dependents();
-  for (int c = tid; c < D; c += kSelThreads) {
-    float a = 0.f, b = 0.f;
-    for (int i = 0; i < p.G; ++i) {
-      const float v = __bfloat162float(p.q[((int64_t)unit * p.G + i) * D + c]) * p.scale;
-      a += v;
-      b += 0.5f * v * v;
-    }
-    q1[c] = a;
-    q2[c] = b;
-  }
-  for (int w = tid; w < words; w += kSelThreads) bm[w] = 0u;
-  __syncthreads();
   // scores q'.mu_j + 1/2 q'^2 . var_j summed over the group's heads
   const int sub = lane / LPR, cl = lane % LPR;
-  const float4 a1 = *reinterpret_cast<const float4*>(q1 + 4 * cl);
-  const float4 a2 = *reinterpret_cast<const float4*>(q2 + 4 * cl);
-  bool nan = false;
-#pragma unroll 1
-  for (int j0 = warp * kRowsPerIter; j0 < nb; j0 += kSelWarps * kRowsPerIter) {
-    float4 m[kSelSteps], v[kSelSteps];
+  float4 m[kSelSteps], v[kSelSteps];
+  auto load_rows = [&](int j0) {
 #pragma unroll
     for (int s = 0; s < kSelSteps; ++s) {
       const int j = j0 + s * RPW + sub;
-      if (j < nb) {
+      if (j < r1) {
         const int64_t off = (row0 + j) * D + 4 * cl;
         m[s] = __ldg(reinterpret_cast<const float4*>(p.mu + off));
         v[s] = __ldg(reinterpret_cast<const float4*>(p.var + off));
@@ -103,6 +105,28 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
         v[s] = m[s];
       }
     }
+  };
+  int j0 = r0 + warp * kRowsPerIter;
+  load_rows(j0);
+  for (int c = tid; c < D; c += kSelThreads) {
+    float a = 0.f, b = 0.f;
+    for (int i = 0; i < p.G; ++i) {
+      const float x = __bfloat162float(p.q[((int64_t)unit * p.G + i) * D + c]) * p.scale;
+      a += x;
+      b += 0.5f * x * x;
+    }
+    q1[c] = a;
+    q2[c] = b;
+  }
+  for (int w = tid; w < words; w += kSelThreads) bm[w] = 0u;
+  if (parts > 1) cluster_sync_all();  // every CTA of the cluster has started before its shared memory is written
+  else __syncthreads();
+  const float4 a1 = *reinterpret_cast<const float4*>(q1 + 4 * cl);
+  const float4 a2 = *reinterpret_cast<const float4*>(q2 + 4 * cl);
+  const uint32_t csc_first = parts > 1 ? map_rank(smem_u32(csc), 0u) : 0u;  // csc in the first CTA
+  bool nan = false;
+#pragma unroll 1
+  while (true) {
     float acc[kSelSteps];
 #pragma unroll
     for (int s = 0; s < kSelSteps; ++s)
@@ -116,14 +140,25 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
 #pragma unroll
       for (int s = 0; s < kSelSteps; ++s) {
         const int j = j0 + s * RPW + sub;
-        if (j < nb) {
+        if (j < r1) {
           nan |= acc[s] != acc[s];
-          if (j % stride != stride - 1) csc[j - (j + 1) / stride] = acc[s];
+          if (j % stride != stride - 1) {
+            const int c = j - (j + 1) / stride;
+            if (part == 0) csc[c] = acc[s];
+            else st_cluster_f32(csc_first + 4u * (uint32_t)c, acc[s]);
+          }
         }
       }
     }
+    j0 += kSelWarps * kRowsPerIter;
+    if (j0 >= r1) break;
+    load_rows(j0);
   }
   if (nan) nan_seen = 1u;
+  if (parts > 1) cluster_sync_all();  // every score is in the first CTA
+  else __syncthreads();
+  if (tid == 0 && nan_seen) atomicOr(p.status, HYB_STATUS_NAN_SCORE);
+  if (part != 0) return;
   // the strided blocks are always taken
   for (int64_t j = stride - 1 + (int64_t)tid * stride; j < nb; j += (int64_t)kSelThreads * stride)
     atomicOr(&bm[j >> 5], 1u << (j & 31));
@@ -216,10 +251,17 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
       if (copy) copy[e] = -1;
     }
   }
-  if (tid == 0 && nan_seen) atomicOr(p.status, HYB_STATUS_NAN_SCORE);
 }
 
 }  // namespace
+
+int strided_select_parts(int nb, int units, int n_sm) {
+  int parts = n_sm / (units > 0 ? units : 1);
+  parts = parts < kSelMaxParts ? parts : kSelMaxParts;
+  const int by_rows = (nb + 63) / 64;  // at least 64 blocks a CTA
+  parts = parts < by_rows ? parts : by_rows;
+  return parts > 1 ? parts : 1;
+}
 
 size_t strided_select_smem(int D, int nb) {
   const size_t rows = (size_t)((nb > kSelMinRows ? nb : kSelMinRows) + 3) & ~(size_t)3;
@@ -234,15 +276,20 @@ cudaError_t prepare_strided_select(int D) {
 
 cudaError_t launch_strided_select(const StridedSelParams& p, int D, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.units);
+  if (p.parts < 1 || p.parts > kSelMaxParts) return cudaErrorInvalidValue;
+  cfg.gridDim = dim3((unsigned)p.units * (unsigned)p.parts);
   cfg.blockDim = dim3(kSelThreads);
   cfg.dynamicSmemBytes = strided_select_smem(D, p.nb);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)p.parts;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.parts > 1 ? 2 : 1;
   if (D == 128) return cudaLaunchKernelEx(&cfg, strided_select_kernel<128>, p);
   return cudaLaunchKernelEx(&cfg, strided_select_kernel<64>, p);
 }

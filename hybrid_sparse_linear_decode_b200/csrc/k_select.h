@@ -16,9 +16,15 @@ struct StridedSelParams {
   uint32_t* status;         // status word: HYB_STATUS_NAN_SCORE
   int64_t max_blocks;
   int32_t units, nb, G, k, stride, width;
+  int32_t parts;            // CTAs (one cluster) per unit, 1..kSelMaxParts
   float scale;
 };
 
+constexpr int kSelMaxParts = 8;  // a portable cluster size
+
+// CTAs per unit: as many as fill the device's n_sm SMs once, at most 8, each
+// with at least 64 blocks.
+int strided_select_parts(int nb, int units, int n_sm);
 // Dynamic shared memory the kernel needs for nb candidate blocks (0: too many).
 size_t strided_select_smem(int D, int nb);
 cudaError_t prepare_strided_select(int D);
