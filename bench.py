@@ -342,12 +342,13 @@ class Bench:
         cache write and the fold of the previous evictions ride in it); spec:
         one multi-query launch per group of 4, then 2, then 1 draft rows;
         prefill: the chunk's cache write, the dense fold of the tokens it
-        evicted (5 or more) and one decode; strided: the fold of the previous
-        eviction (a fold-only decode launch), the selection, the decode and the
-        append's cache write."""
+        evicted (5 or more) and one decode; strided: the selection (which
+        scores the block holding the previous step's eviction from its rows
+        folded on the fly), the decode (which folds that eviction into the
+        state) and the append's cache write."""
         n = self.chunk
         groups = n // 4 + (n % 4) // 2 + (n % 2)
-        per = {"decode": 1, "spec": groups, "prefill": 2 + (self.chunk >= 5), "strided": 4}[self.mode]
+        per = {"decode": 1, "spec": groups, "prefill": 2 + (self.chunk >= 5), "strided": 3}[self.mode]
         return per * len(self.layers)
 
     def union_blocks(self):
@@ -525,7 +526,7 @@ def run_native(args, rank, world):
         "roofline": {"bound": "hbm",
                      "kernel": ("the multi-query decode kernel: one layer's draft rows decoded + appended together"
                                 if mode == "spec" else
-                                "one layer's launches, averaged: the fold, the strided selection, the decode, the append"
+                                "one layer's launches, averaged: the strided selection, the decode, the append"
                                 if mode == "strided" else
                                 "one layer's launches, averaged: the chunk's cache write, the dense fold, the decode"
                                 if mode == "prefill" else "the fused decode kernel: one layer's decode + append (one launch)"),

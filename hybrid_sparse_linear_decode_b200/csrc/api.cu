@@ -711,8 +711,10 @@ int hyb_attn_decode_strided(hyb_attn_ctx* x, const void* q, int32_t k_top, int32
   if (n_sel > x->cfg.top_k) return HYB_EINVAL;  // the selection row holds top_k blocks
   const size_t smem = strided_select_smem(x->ck.D, (int)nb);
   if (nb > 0 && smem == 0) return HYB_EINVAL;
-  // the block statistics must hold every evicted token before they are scored
-  int rc = hyb_attn_sync_state(x, stream);
+  // Several pending evictions are folded by one dense pass first; a few (the
+  // previous step's) are folded by the selection launch for its scores and by
+  // the decode into the state, as in a plain decode.
+  int rc = fold_pending(x, stream);
   if (rc != HYB_OK) return rc;
   int32_t* sel = x->w<int32_t>(x->ws.sel);
   if (nb > 0) {
@@ -732,6 +734,12 @@ int hyb_attn_decode_strided(hyb_attn_ctx* x, const void* q, int32_t k_top, int32
     sp.width = x->cfg.top_k;
     sp.scale = x->scale;  // resolved (1/sqrt(d) when the configuration gives 0)
     sp.parts = strided_select_parts((int)nb, x->ck.units, x->n_sm);
+    sp.k_cache = static_cast<const __nv_bfloat16*>(x->buf.k_cache);
+    sp.cap = x->cfg.capacity;
+    sp.S = x->cfg.n_sink;
+    sp.Bk = x->cfg.block_size;
+    sp.fold_end = ev_end_at((int32_t)x->T, x->cfg.n_sink, x->cfg.window);
+    sp.fold_begin = ev_end_at((int32_t)(x->T - x->pending > 0 ? x->T - x->pending : 0), x->cfg.n_sink, x->cfg.window);
     const cudaError_t e = launch_strided_select(sp, x->ck.D, stream);
     if (e != cudaSuccess) return cuda_fail(e);
   } else if (sel_out != nullptr && x->cfg.top_k > 0) {

@@ -19,7 +19,11 @@
 // memory of the cluster's first CTA (c = j - (j + 1) / stride, which keeps
 // block order, so ties to the lower compacted index are ties to the lower
 // block); two cluster barriers bracket these stores (every CTA has started;
-// every score is in place).  The first CTA then selects.
+// every score is in place).  A block that holds evictions not yet folded into
+// the statistics (the previous step's, usually one token) is scored from its
+// rows folded in registers one token at a time by Welford's update, the
+// decode's own fold, which the decode that follows writes back.  The first
+// CTA then selects.
 // Top-k: up to 32, one warp's bound-and-rank selection (the decode kernel's);
 // above 32, or when too many keys tie at the bound, k rounds of block-wide
 // maxima of packed (key << 32 | ~index) words.  The union is a bitmap,
@@ -124,7 +128,18 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
   const float4 a1 = *reinterpret_cast<const float4*>(q1 + 4 * cl);
   const float4 a2 = *reinterpret_cast<const float4*>(q2 + 4 * cl);
   const uint32_t csc_first = parts > 1 ? map_rank(smem_u32(csc), 0u) : 0u;  // csc in the first CTA
+  // blocks [jb0, jb1] hold evictions not yet folded (none: jb0 > jb1)
+  const bool folds = p.fold_end > p.fold_begin;
+  const int jb0 = folds ? (p.fold_begin - p.S) / p.Bk : 1, jb1 = folds ? (p.fold_end - 1 - p.S) / p.Bk : 0;
   bool nan = false;
+  auto put = [&](int j, float sc) {  // one score: the NaN flag, and the compacted slot of a non-strided block
+    nan |= sc != sc;
+    if (j % stride != stride - 1) {
+      const int c = j - (j + 1) / stride;
+      if (part == 0) csc[c] = sc;
+      else st_cluster_f32(csc_first + 4u * (uint32_t)c, sc);
+    }
+  };
 #pragma unroll 1
   while (true) {
     float acc[kSelSteps];
@@ -140,19 +155,55 @@ __global__ void __launch_bounds__(kSelThreads) strided_select_kernel(const __gri
 #pragma unroll
       for (int s = 0; s < kSelSteps; ++s) {
         const int j = j0 + s * RPW + sub;
-        if (j < r1) {
-          nan |= acc[s] != acc[s];
-          if (j % stride != stride - 1) {
-            const int c = j - (j + 1) / stride;
-            if (part == 0) csc[c] = acc[s];
-            else st_cluster_f32(csc_first + 4u * (uint32_t)c, acc[s]);
-          }
-        }
+        if (j < r1 && (j < jb0 || j > jb1)) put(j, acc[s]);
       }
     }
     j0 += kSelWarps * kRowsPerIter;
     if (j0 >= r1) break;
     load_rows(j0);
+  }
+  // the blocks with pending evictions in this CTA's share, one warp each
+  // (lanes [0, LPR): four channels each)
+#pragma unroll 1
+  for (int j = max(jb0, r0) + warp; j <= min(jb1, r1 - 1); j += kSelWarps) {
+    float sc = 0.f;
+    if (sub == 0) {
+      const int64_t bs = p.S + (int64_t)j * p.Bk;
+      const int64_t t0 = bs > p.fold_begin ? bs : (int64_t)p.fold_begin;
+      const int64_t t1 = bs + p.Bk < p.fold_end ? bs + p.Bk : (int64_t)p.fold_end;
+      float mm[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (t0 > bs) {  // the tokens [bs, t0) are in the stored rows
+        const int64_t off = (row0 + j) * D + 4 * cl;
+        const float4 a = __ldg(reinterpret_cast<const float4*>(p.mu + off));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(p.var + off));
+        mm[0] = a.x; mm[1] = a.y; mm[2] = a.z; mm[3] = a.w;
+        vv[0] = b.x; vv[1] = b.y; vv[2] = b.z; vv[3] = b.w;
+      }
+#pragma unroll 1
+      for (int64_t t = t0; t < t1; ++t) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p.k_cache + ((int64_t)unit * p.cap + t) * D + 4 * cl);
+        const float x[4] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y)};
+        const float cnt = (float)(t - bs + 1);
+        const float inv = 1.f / cnt;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (t == bs) {  // the block's first token
+            mm[c] = x[c];
+            vv[c] = 0.f;
+          } else {
+            const float delta = x[c] - mm[c];
+            const float m1 = mm[c] + delta * inv;
+            vv[c] = (vv[c] * (cnt - 1.f) + delta * (x[c] - m1)) * inv;
+            mm[c] = m1;
+          }
+        }
+      }
+      sc = a1.x * mm[0] + a1.y * mm[1] + a1.z * mm[2] + a1.w * mm[3] + a2.x * vv[0] + a2.y * vv[1] + a2.z * vv[2] +
+           a2.w * vv[3];
+    }
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+    if (lane == 0) put(j, sc);
   }
   if (nan) nan_seen = 1u;
   if (parts > 1) cluster_sync_all();  // every score is in the first CTA

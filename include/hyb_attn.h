@@ -304,10 +304,12 @@ int hyb_attn_decode_with_selection(hyb_attn_ctx* ctx, const void* q, const int32
  *           -1 padded.
  * The configuration's top_k must hold the union (nb / stride + min(k_top,
  * the other blocks)), else HYB_EINVAL; so must one length and one budget for
- * every unit (no per-row lengths, no per-head budgets).  Folds the pending
- * evictions first (hyb_attn_sync_state), then one selection launch that
- * reads the block statistics, then the decode.  Scores that are NaN raise
- * HYB_STATUS_NAN_SCORE. */
+ * every unit (no per-row lengths, no per-head budgets).  Launches: one
+ * selection launch that reads the block statistics (a block holding evictions
+ * not folded yet, at most 4 tokens, is scored from its statistics with them
+ * folded in registers), then the decode, which folds them into the state as
+ * hyb_attn_decode does; 5 or more pending evictions are first folded by one
+ * dense pass.  Scores that are NaN raise HYB_STATUS_NAN_SCORE. */
 int hyb_attn_decode_strided(hyb_attn_ctx* ctx, const void* q, int32_t k_top, int32_t stride, float* out,
                             int32_t* sel_out, cudaStream_t stream);
 

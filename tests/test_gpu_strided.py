@@ -128,3 +128,21 @@ def test_strided_selection_all_scores_equal(nbk, k_top, stride):
             _, Vf = c.unit_kv(b, h)
             check_outputs(out[b, h * c.G:(h + 1) * c.G], np.broadcast_to(Vf.mean(axis=0), (c.G, c.d)),
                           max_abs=1e-4, rel_l2=1e-4)
+
+
+@pytest.mark.parametrize("appends,Bk,d", [(1, 16, 128), (3, 4, 64), (4, 4, 128), (2, 1, 64)])
+def test_strided_selection_folds_pending_evictions(appends, Bk, d):
+    """One to four appends since the last fold (a decode step's usual case):
+    the selection launch scores the blocks that hold them from rows folded on
+    the fly, and the decode folds them into the state.  The first pending token
+    is the last of its block, so the ones after it open a new block (with
+    blocks of one token, every pending token is a block of its own)."""
+    from harness import check_state
+    S, W, nblk = 4, 64, 300
+    T0 = S + W + nblk * Bk + (Bk - 1)
+    nb = (T0 + appends - W - S + Bk - 1) // Bk
+    k_top, stride = 6, 5
+    c = Case(B=1, Hq=4, Hkv=2, d=d, T0=T0, Bk=Bk, S=S, W=W, k=nb // stride + k_top, n_append=appends, seed=36)
+    _check(c, c.random_q(), k_top, stride, appends=appends)
+    assert c.layer.status() == 0
+    check_state(c)
