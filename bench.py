@@ -560,7 +560,7 @@ def _oracle_unit_inputs(w, unit_id: int, max_appends: int):
     """Inputs of unit `unit_id` of the workload (layers cycle first, so that
     units of different per-layer budgets and head scales are sampled): its keys
     and values for [0, T0 + max_appends), the step-0 query of its group, and its
-    layer's (window, top_k)."""
+    (window, top_k): its layer's, or its KV head's when the budgets vary by head."""
     from syngen import host as SH
     layer, j = unit_id % w.layers, unit_id // w.layers
     wl = w.for_layer(layer)
@@ -568,13 +568,19 @@ def _oracle_unit_inputs(w, unit_id: int, max_appends: int):
     tb = SH.LayerTables(wl, layer)
     q_all = SH.bf16_bits_to_f64(SH.q_bits(wl, layer, 0))
     K, V = SH.kv_f64(wl, tb, b, h, 0, w.T0 + max_appends)
-    return K, V, np.ascontiguousarray(q_all[b, h * w.group:(h + 1) * w.group]), wl.window, wl.top_k
+    wh = wl.for_head(h)
+    return K, V, np.ascontiguousarray(q_all[b, h * w.group:(h + 1) * w.group]), wh.window, wh.top_k
 
 
-def _oracle_sample_unit(e, seconds: float):
+def _oracle_sample_unit(e, seconds: float, stride=None):
     """Decode + append pairs on one unit for about `seconds` of timed work; when
     its prepared tokens are used up it starts again from T0 (the rebuild is not
-    timed).  Returns (pairs, decode seconds, append seconds)."""
+    timed).  With `stride`, the decode takes the strided selection: the block
+    scores from the unit's statistics, the strided blocks plus the top-k of the
+    others, then the decode given that selection (which scores the blocks once
+    more, as the unit's decode always does).  Returns (pairs, decode seconds,
+    append seconds)."""
+    O = e["O"]
     t_dec = t_app = 0.0
     n = 0
     while t_dec + t_app < seconds:
@@ -582,7 +588,13 @@ def _oracle_sample_unit(e, seconds: float):
             e["u"], e["pos"] = e["fresh"](), 0
         u, pos = e["u"], e["pos"]
         t0 = time.perf_counter()
-        u.decode(e["q"])
+        if stride is None:
+            u.decode(e["q"])
+        else:
+            mu, var = u.stats()
+            nb = mu.shape[0]
+            sc = O.block_scores(e["q"], mu, var, u.scale) if nb else np.zeros(0)
+            u.decode(e["q"], sel=O.select_blocks_strided(sc, u.k, stride))
         t1 = time.perf_counter()
         u.append(e["K"][e["T0"] + pos], e["V"][e["T0"] + pos])
         t2 = time.perf_counter()
@@ -618,14 +630,14 @@ def _oracle_worker(conn, spec: dict):
         return O.OracleUnit(K[:T0], V[:T0], spec["S"], spec["W"], spec["Bk"], spec["k"], spec["scale"],
                             capacity=T)
 
-    e = {"fresh": fresh, "u": fresh(), "K": K, "V": V, "q": q, "T0": T0, "n_app": T - T0, "pos": 0}
+    e = {"fresh": fresh, "u": fresh(), "K": K, "V": V, "q": q, "T0": T0, "n_app": T - T0, "pos": 0, "O": O}
     conn.send("ready")
     try:
         while True:
             msg = conn.recv()
             if msg is None:
                 break
-            conn.send(_oracle_sample_unit(e, msg))
+            conn.send(_oracle_sample_unit(e, *msg))   # (seconds, stride or None)
     finally:
         del K, V, buf, e
         shm.close()
@@ -691,13 +703,14 @@ class OraclePool:
         """All workers time `seconds` of decode + append pairs at once.  Returns
         (seconds per full step, extrapolated from the timed units; pairs timed)."""
         for c in self.conns:
-            c.send(seconds)
+            c.send((seconds, chunk if mode == "strided" else None))
         res = [c.recv() for c in self.conns]
         rate = 0.0   # unit steps per second, all workers together
         pairs = 0
         for n, td, ta in res:
             dd, aa = td / n, ta / n
-            per_unit_step = {"decode": dd + aa, "spec": chunk * (dd + aa), "prefill": chunk * aa + dd}[mode]
+            per_unit_step = {"decode": dd + aa, "spec": chunk * (dd + aa), "prefill": chunk * aa + dd,
+                             "strided": dd + aa}[mode]
             rate += 1.0 / per_unit_step
             pairs += n
         units_per_step = self.w.layers * self.w.units_per_layer
@@ -706,7 +719,8 @@ class OraclePool:
     def describe(self, pairs: int, mode: str, chunk: int) -> str:
         w = self.w
         what = {"decode": "decode + append", "spec": f"{chunk} x (decode + append)",
-                "prefill": f"{chunk} appends + decode"}[mode]
+                "prefill": f"{chunk} appends + decode",
+                "strided": f"strided selection (stride {chunk}) + decode + append"}[mode]
         return (f"extrapolated from {self.units} units: {pairs} timed decode + append pairs on whole "
                 f"(layer, b, kv-head) units at {w.T0}+ tokens, {self.workers} single-threaded worker processes "
                 f"at once, each with its own copy of one of the {self.units} units; a step = {what} per unit, "
@@ -747,10 +761,6 @@ def run_reference(args, rank, world):
     overrides = {"layers": args.layers} if args.layers else {}
     w = C.get_workload(args.workload, **overrides)
     mode, chunk = args.mode, (args.chunk if args.mode != "decode" else 1)
-    if mode == "strided":
-        print(json.dumps({"impl": "reference", "unavailable": "the oracle arm times decode, spec and prefill steps; "
-                          "strided selection is checked against the oracle in the tests, not timed"}), flush=True)
-        return
     pool = OraclePool(w)
     try:
         per = args.cpu_sample_seconds / max(1, args.steps)
@@ -799,7 +809,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_native(args, rank, world)
-    if rank == 0 and not args.no_cpu_baseline and world == 1 and args.mode != "strided":  # (the oracle's step is decode + append with the plain top-k)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
         from syngen import configs as C
         overrides = {"layers": args.layers} if args.layers else {}
         w = C.get_workload(args.workload, **overrides)

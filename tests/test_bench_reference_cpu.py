@@ -22,7 +22,7 @@ def _run(*extra):
     return json.loads(lines[0])
 
 
-@pytest.mark.parametrize("mode", ["decode", "spec", "prefill"])
+@pytest.mark.parametrize("mode", ["decode", "spec", "prefill", "strided"])
 def test_reference_arm_line(mode):
     import bench
     from syngen import configs as C
@@ -39,7 +39,8 @@ def test_reference_arm_line(mode):
     _, _, flush = bench.step_bytes_model(w, mode, chunk, w.T0)
     assert j["config"] == bench.workload_config(w, mode, chunk, 1, flush)
     if mode != "decode":
-        assert ("4 x (decode + append)" if mode == "spec" else "4 appends + decode") in cb["sample"]
+        assert {"spec": "4 x (decode + append)", "prefill": "4 appends + decode",
+                "strided": "strided selection (stride 4) + decode + append"}[mode] in cb["sample"]
 
 
 def test_oracle_pool_keeps_timing_past_its_prepared_tokens():
